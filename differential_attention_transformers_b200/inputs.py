@@ -1,0 +1,143 @@
+"""Seeded synthetic inputs for the differential attention workloads.
+
+This module only draws random numbers and arranges them in the layouts the
+library takes; it holds none of the method's arithmetic.  Both the CUDA path
+(tests, bench) and the fp64 oracle consume what it returns.
+
+Workloads (shapes, value distributions):
+
+  v1_tiny      V1 layout, fp32: B1 H1 Lq=Lk=128 d32 dv64, causal, all N(0,1),
+               lambda from lq/lk in R^32 ~ N(0, 0.1) at layer 1.
+  noise_probe  fp32, 64 independent instances of the tutorial's toy
+               construction ("差分注意力", Step 1 / Step 3): q ~ N(0,1) in d=64,
+               1000 keys ~ N(0,1) with key 0 = 5q, an independent second map
+               (Q2, K2 ~ N(0,1)), V = the 1000x1000 identity, lambda = 0.5.
+               Laid out as V1 with B=64, H=1, Lq=1, Lk=1000, non-causal.
+  v1_prefill   V1, bf16: B8 H16 (Hkv16) N4096 d64 dv128, causal,
+               N(0,1)/sqrt(64), layer 12, RMSNorm eps 1e-5.
+  v2_prefill   V2, bf16: B2 Hq64 Hkv8 N8192 D128, causal, N(0,1)/sqrt(128),
+               layer 24.
+  v2_decode    V2 single-token decode, bf16: B16 Hq64 Hkv8 T65536 D128,
+               N(0,1)/sqrt(128), layer 24.
+  v1_decode    the same decode shape in the V1 layout: 32 heads over 8 KV
+               heads, Q1/Q2/K1/K2 width 64, V width 128.
+
+bf16 tensors are drawn in fp32 and rounded to bf16 (round-to-nearest-even);
+the oracle receives those rounded values.  lq/lk are fp32 N(0,1)*0.1 with the
+QK width as their length.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    layout: str            # "v1" | "v2" | "v1_decode" | "v2_decode"
+    dtype: torch.dtype
+    B: int
+    H: int                 # V1: heads; V2: Q heads (pairs = H // 2)
+    Hkv: int
+    Lq: int
+    Lk: int
+    d: int                 # QK contraction width
+    dv: int                # value width
+    causal: bool
+    layer: int             # lambda_init layer (1-based); 0 = explicit lambda
+    rmsnorm: bool
+    std: float
+    seed: int
+    explicit_lambda: float | None = None
+
+    @property
+    def pairs(self) -> int:
+        return self.H // 2 if self.layout.startswith("v2") else self.H
+
+
+WORKLOADS = {
+    "v1_tiny": Workload("v1_tiny", "v1", torch.float32, 1, 1, 1, 128, 128, 32, 64,
+                        True, 1, False, 1.0, 1001),
+    "noise_probe": Workload("noise_probe", "v1", torch.float32, 64, 1, 1, 1, 1000, 64, 1000,
+                            False, 0, False, 1.0, 1002, explicit_lambda=0.5),
+    "v1_prefill": Workload("v1_prefill", "v1", torch.bfloat16, 8, 16, 16, 4096, 4096, 64, 128,
+                           True, 12, True, 1.0 / math.sqrt(64), 1003),
+    "v2_prefill": Workload("v2_prefill", "v2", torch.bfloat16, 2, 64, 8, 8192, 8192, 128, 128,
+                           True, 24, False, 1.0 / math.sqrt(128), 1004),
+    "v2_decode": Workload("v2_decode", "v2_decode", torch.bfloat16, 16, 64, 8, 1, 65536, 128, 128,
+                          True, 24, False, 1.0 / math.sqrt(128), 1005),
+    "v1_decode": Workload("v1_decode", "v1_decode", torch.bfloat16, 16, 32, 8, 1, 65536, 64, 128,
+                          True, 24, False, 1.0 / math.sqrt(64), 1006),
+}
+
+
+def with_shape(w: Workload, **kw) -> Workload:
+    """A copy of ``w`` with some fields replaced (smaller parity cases)."""
+    d = dict(w.__dict__)
+    d.update(kw)
+    return Workload(**d)
+
+
+def _randn(gen, shape, std, dtype, device):
+    x = torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(dtype)
+
+
+def lambda_params(w: Workload, device="cpu", seed_offset: int = 0):
+    """lq1, lk1, lq2, lk2 [pairs, d] fp32 ~ N(0, 0.1)."""
+    gen = torch.Generator(device=device).manual_seed(w.seed * 7 + 13 + seed_offset)
+    return tuple(_randn(gen, (w.pairs, w.d), 0.1, torch.float32, device) for _ in range(4))
+
+
+def make(w: Workload, device="cpu"):
+    """Draw the attention inputs of workload ``w`` on ``device``.
+
+    Returns a dict.  V1: q1, k1, q2, k2, v.  V2: q, k, v.  Decode layouts drop
+    the query length axis (q [B, H, d]).
+    """
+    gen = torch.Generator(device=device).manual_seed(w.seed)
+    dt, std = w.dtype, w.std
+    if w.name == "noise_probe":
+        n, N, d = w.B, w.Lk, w.d
+        q1 = _randn(gen, (n, 1, 1, d), 1.0, torch.float32, device)
+        k1 = _randn(gen, (n, 1, N, d), 1.0, torch.float32, device)
+        k1[:, 0, 0, :] = 5.0 * q1[:, 0, 0, :]
+        q2 = _randn(gen, (n, 1, 1, d), 1.0, torch.float32, device)
+        k2 = _randn(gen, (n, 1, N, d), 1.0, torch.float32, device)
+        v = torch.eye(N, dtype=torch.float32, device=device).expand(n, 1, N, N).contiguous()
+        return {"q1": q1, "k1": k1, "q2": q2, "k2": k2, "v": v}
+    if w.layout == "v1":
+        return {
+            "q1": _randn(gen, (w.B, w.H, w.Lq, w.d), std, dt, device),
+            "k1": _randn(gen, (w.B, w.Hkv, w.Lk, w.d), std, dt, device),
+            "q2": _randn(gen, (w.B, w.H, w.Lq, w.d), std, dt, device),
+            "k2": _randn(gen, (w.B, w.Hkv, w.Lk, w.d), std, dt, device),
+            "v": _randn(gen, (w.B, w.Hkv, w.Lk, w.dv), std, dt, device),
+        }
+    if w.layout == "v2":
+        return {
+            "q": _randn(gen, (w.B, w.H, w.Lq, w.d), std, dt, device),
+            "k": _randn(gen, (w.B, w.Hkv, w.Lk, w.d), std, dt, device),
+            "v": _randn(gen, (w.B, w.Hkv, w.Lk, w.dv), std, dt, device),
+        }
+    if w.layout == "v2_decode":
+        return {
+            "q": _randn(gen, (w.B, w.H, w.d), std, dt, device),
+            "k": _randn(gen, (w.B, w.Hkv, w.Lk, w.d), std, dt, device),
+            "v": _randn(gen, (w.B, w.Hkv, w.Lk, w.dv), std, dt, device),
+        }
+    if w.layout == "v1_decode":
+        return {
+            "q1": _randn(gen, (w.B, w.H, w.d), std, dt, device),
+            "k1": _randn(gen, (w.B, w.Hkv, w.Lk, w.d), std, dt, device),
+            "q2": _randn(gen, (w.B, w.H, w.d), std, dt, device),
+            "k2": _randn(gen, (w.B, w.Hkv, w.Lk, w.d), std, dt, device),
+            "v": _randn(gen, (w.B, w.Hkv, w.Lk, w.dv), std, dt, device),
+        }
+    raise ValueError(w.layout)
