@@ -1,0 +1,467 @@
+#!/usr/bin/env python3
+"""Benchmark of the differential attention forward on B200.
+
+One step = the whole hot path for one batch of the primary workload: the
+per-head lambda kernel, then the prefill kernel (default workload: V2 causal
+prefill, B2 Hq64 Hkv8 N8192 D128 bf16, layer 24).  The other hot-path
+workloads (V1 prefill with RMSNorm, V2 64k decode, V1-layout 64k decode fused
+and unfused) are timed the same way and reported under "secondary".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl reference] [--no-cpu-baseline] [--no-secondary]
+
+All inputs are synthetic (seeded, on the device), larger than L2, so no L2
+flush is needed between timed steps.  Device times come from CUDA events on
+the launching stream; for N > 1 (torchrun) each rank runs its own batch
+(weak scaling, no collective on the data path) and rank 0 reports the max
+time over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import differential_attention_transformers_b200 as da  # noqa: E402
+from differential_attention_transformers_b200 import inputs  # noqa: E402
+
+METRIC = "diff-attn fwd prefill TFLOP/s & decode KV GB/s on 1 B200 (% of roofline)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- work counts
+def causal_pairs(Lq: int, Lk: int, causal: bool) -> int:
+    """Number of (query, key) pairs a row-softmax sees (bottom-right causal mask)."""
+    if not causal:
+        return Lq * Lk
+    off = Lk - Lq
+    tot = 0
+    # rows i see min(Lk, max(0, i + off + 1)) keys; sum in closed form by ranges
+    lo = max(0, -off)                      # first row that sees >= 1 key
+    hi = min(Lq, Lk - off)                 # rows [lo, hi) see i + off + 1 keys
+    if hi > lo:
+        tot += (hi - lo) * (off + 1) + (hi - 1 + lo) * (hi - lo) // 2
+    if Lq > max(hi, lo):
+        tot += (Lq - max(hi, lo)) * Lk     # rows that see every key
+    return tot
+
+
+def prefill_flops(w) -> int:
+    """Executed-minimum FLOP: two QK^T and two PV products per diff head."""
+    nc = causal_pairs(w.Lq, w.Lk, w.causal)
+    if w.layout == "v2":
+        return nc * 4 * w.d * w.H * w.B          # H = Q heads; each map 2d (QK) + 2dv (PV), dv == d
+    return nc * (4 * w.d + 4 * w.dv) * w.H * w.B
+
+
+def decode_bytes(w) -> int:
+    """Algorithmic bytes of one decode step: the K and V caches read once."""
+    per_key = (w.d + w.dv) * 2 if w.layout == "v2_decode" else (2 * w.d + w.dv) * 2
+    return w.B * w.Hkv * w.Lk * per_key
+
+
+# ----------------------------------------------------------------------------- peaks / clocks
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workloads
+class Prefill:
+    def __init__(self, w, device):
+        self.w = w
+        self.x = inputs.make(w, device=device)
+        self.lp = inputs.lambda_params(w, device=device)
+        self.init = da.lambda_init(w.layer)
+        self.lam = torch.empty(w.pairs, dtype=torch.float32, device=device)
+        out_h = w.pairs
+        self.out = torch.empty((w.B, out_h, w.Lq, w.dv), dtype=w.dtype, device=device)
+        self.launches_per_step = 2
+        self.k_start = torch.cuda.Event(enable_timing=True)
+        self.k_end = torch.cuda.Event(enable_timing=True)
+
+    def step(self, ev=None):
+        w, x = self.w, self.x
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        if ev is not None:
+            ev[0].record()
+        if w.layout == "v2":
+            da.fwd_v2(x["q"], x["k"], x["v"], self.lam, causal=w.causal, out=self.out)
+        else:
+            da.fwd_v1(x["q1"], x["k1"], x["q2"], x["k2"], x["v"], self.lam, causal=w.causal,
+                      rmsnorm=w.rmsnorm, eps=1e-5, out=self.out)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        return prefill_flops(self.w) / 1e12, "TFLOP/s"
+
+    def host_call(self, host):
+        w = self.w
+        lam = da.compute_lambda(*host["lp"], self.init)
+        if w.layout == "v2":
+            return da.fwd_v2(host["q"], host["k"], host["v"], lam, causal=w.causal)
+        return da.fwd_v1(host["q1"], host["k1"], host["q2"], host["k2"], host["v"], lam, causal=w.causal,
+                         rmsnorm=w.rmsnorm, eps=1e-5)
+
+
+class Decode:
+    def __init__(self, w, device, fused=True):
+        self.w = w
+        self.fused = fused
+        self.x = inputs.make(w, device=device)
+        self.lp = inputs.lambda_params(w, device=device)
+        self.init = da.lambda_init(w.layer)
+        self.lam = torch.empty(w.pairs, dtype=torch.float32, device=device)
+        self.out = torch.empty((w.B, w.pairs, w.dv), dtype=w.dtype, device=device)
+        self.ws = torch.empty(da.decode_workspace_size(w.B, w.Hkv, w.Lk, w.dv), dtype=torch.uint8, device=device)
+        passes = 1 if (w.layout == "v2_decode" or fused) else 2
+        self.launches_per_step = 2 + passes
+
+    def step(self, ev=None):
+        w, x = self.w, self.x
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        if ev is not None:
+            ev[0].record()
+        if w.layout == "v2_decode":
+            da.decode_v2(x["q"], x["k"], x["v"], self.lam, out=self.out, workspace=self.ws)
+        else:
+            da.decode_v1(x["q1"], x["k1"], x["q2"], x["k2"], x["v"], self.lam, fused=self.fused, out=self.out,
+                         workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        b = decode_bytes(self.w)
+        if self.w.layout == "v1_decode" and not self.fused:
+            b += self.w.B * self.w.Hkv * self.w.Lk * self.w.dv * 2   # V read a second time
+        return b / 1e9, "GB/s"
+
+    def host_call(self, host):
+        w = self.w
+        lam = da.compute_lambda(*host["lp"], self.init)
+        if w.layout == "v2_decode":
+            return da.decode_v2(host["q"], host["k"], host["v"], lam)
+        return da.decode_v1(host["q1"], host["k1"], host["q2"], host["k2"], host["v"], lam, fused=self.fused)
+
+
+def make_runner(name, device):
+    w = inputs.WORKLOADS[name.replace("_unfused", "")]
+    if w.layout in ("v1", "v2"):
+        return Prefill(w, device)
+    return Decode(w, device, fused=not name.endswith("_unfused"))
+
+
+def describe(name):
+    w = inputs.WORKLOADS[name.replace("_unfused", "")]
+    d = {"workload": name, "layout": w.layout, "B": w.B, "heads": w.H, "kv_heads": w.Hkv, "Lq": w.Lq, "Lk": w.Lk,
+         "d": w.d, "dv": w.dv, "causal": w.causal, "layer": w.layer, "rmsnorm": w.rmsnorm,
+         "l2": "inputs larger than L2 (126 MB): no flush between steps"}
+    if name.endswith("_unfused"):
+        d["mode"] = "two passes, V read twice (comparison)"
+    return d
+
+
+# ----------------------------------------------------------------------------- timing
+def time_runner(r, steps, warmup, dist_on):
+    for _ in range(warmup):
+        r.step()
+    torch.cuda.synchronize()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(steps):
+        r.step(kev[i])
+    end.record()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / steps
+    return total_ms, kern_ms
+
+
+def max_over_ranks(x, dist_on):
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def e2e_measure(r, steps):
+    """Same metric through the public API with pinned HOST buffers: the
+    host->device copies of the step's inputs and the device->host copy of its
+    output are inside the timed region."""
+    host = {k: v.cpu().pin_memory() for k, v in r.x.items()}
+    host["lp"] = [t.cpu().pin_memory() for t in r.lp]
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if k != "lp")
+    h2d += sum(t.numel() * t.element_size() for t in host["lp"])
+    out = r.host_call(host)                     # warm-up (pinned output buffers cached)
+    d2h = out.numel() * out.element_size()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    s.record()
+    for _ in range(steps):
+        out = r.host_call(host)
+    e.record()
+    torch.cuda.synchronize()
+    wall = (time.perf_counter() - t0) * 1e3 / steps
+    dev_ms = s.elapsed_time(e) / steps
+    ms = max(wall, dev_ms)
+    work, unit = r.work()
+    del host
+    return {"value": work / (ms / 1e3), "unit": unit, "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def roofline(r, kern_ms, peaks):
+    work, unit = r.work()
+    if unit == "TFLOP/s":
+        ach = work / (kern_ms / 1e3)
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": None, "peak_kind": f"{peaks['source']} burst cuBLAS bf16",
+                "kernel_ms": kern_ms}
+    ach = work / (kern_ms / 1e3)
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": None,
+            "peak_kind": f"{peaks['source']} HBM copy", "kernel_ms": kern_ms}
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+def cpu_oracle_run(name, budget_s=12.0):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload.
+
+    Prefill: whole (batch, head) slices over all rows; decode: whole (batch,
+    KV head) groups.  The work done is counted with the same convention as
+    the GPU metric and divided by the measured time."""
+    import numpy as np
+    from oracle import diffattn as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    w = inputs.WORKLOADS[name.replace("_unfused", "")]
+    x = inputs.make(w, device="cpu") if w.layout in ("v1", "v2") else None
+    lam = np.full(w.pairs, 0.5)
+    done_work, t_total, n = 0.0, 0.0, 0
+    if w.layout in ("v1", "v2"):
+        per_slice = prefill_flops(w) / (w.B * w.pairs) / 1e12
+        units = [(b, h) for h in range(w.pairs) for b in range(w.B)]
+        for b, h in units:
+            t0 = time.perf_counter()
+            if w.layout == "v2":
+                g = (2 * h) // (w.H // w.Hkv)
+                orc.diffattn_v2(x["q"][b:b + 1, 2 * h:2 * h + 2], x["k"][b:b + 1, g:g + 1],
+                                x["v"][b:b + 1, g:g + 1], lam[h:h + 1], causal=w.causal)
+            else:
+                g = h // (w.H // w.Hkv)
+                s = lambda t, hh: t[b:b + 1, hh:hh + 1]  # noqa: E731
+                orc.diffattn_v1(s(x["q1"], h), s(x["k1"], g), s(x["q2"], h), s(x["k2"], g), s(x["v"], g),
+                                lam[h:h + 1], causal=w.causal, rms=w.rmsnorm)
+            t_total += time.perf_counter() - t0
+            done_work += per_slice
+            n += 1
+            if t_total >= budget_s:
+                break
+        unit = "TFLOP/s"
+        sample = f"{n} of {w.B * w.pairs} (batch, head) slices, all {w.Lq} rows, fp64 NumPy"
+    else:
+        gen = torch.Generator().manual_seed(w.seed)
+        grp = w.H // w.Hkv
+        per_group = decode_bytes(w) / (w.B * w.Hkv) / 1e9
+        for b in range(w.B):
+            for g in range(w.Hkv):
+                if w.layout == "v2_decode":
+                    q = (torch.randn(1, grp, w.d, generator=gen) * w.std).to(torch.bfloat16)
+                    kc = (torch.randn(1, 1, w.Lk, w.d, generator=gen) * w.std).to(torch.bfloat16)
+                    vc = (torch.randn(1, 1, w.Lk, w.dv, generator=gen) * w.std).to(torch.bfloat16)
+                    t0 = time.perf_counter()
+                    orc.decode_v2(q, kc, vc, lam[: grp // 2])
+                else:
+                    q1 = (torch.randn(1, grp, w.d, generator=gen) * w.std).to(torch.bfloat16)
+                    k1 = (torch.randn(1, 1, w.Lk, w.d, generator=gen) * w.std).to(torch.bfloat16)
+                    vc = (torch.randn(1, 1, w.Lk, w.dv, generator=gen) * w.std).to(torch.bfloat16)
+                    t0 = time.perf_counter()
+                    orc.decode_v1(q1, k1, q1, k1, vc, lam[:grp])
+                t_total += time.perf_counter() - t0
+                done_work += per_group
+                n += 1
+                if t_total >= budget_s:
+                    break
+            if t_total >= budget_s:
+                break
+        unit = "GB/s"
+        sample = f"{n} of {w.B * w.Hkv} (batch, KV head) groups, full cache, fp64 NumPy"
+    return {"value": done_work / t_total, "unit": unit, "cores": int(cores), "kind": "oracle", "sample": sample,
+            "seconds": t_total}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="v2_prefill",
+                    choices=["v2_prefill", "v1_prefill", "v2_decode", "v1_decode", "v1_decode_unfused"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = inputs.WORKLOADS[args.workload.replace("_unfused", "")]
+
+    if args.impl == "reference":
+        # The reference arm is the fp64 CPU oracle, on rank 0 only.
+        if rank != 0:
+            return 0
+        steps = max(1, args.steps)
+        res = [cpu_oracle_run(args.workload, budget_s=max(2.0, 60.0 / (steps + args.warmup)))
+               for _ in range(steps + max(0, args.warmup))][args.warmup:] or [None]
+        vals = [r["value"] for r in res]
+        v = statistics.median(vals)
+        cb = dict(res[-1])
+        cb["value"] = v
+        unit = cb["unit"]
+        work_unit = prefill_flops(w) / 1e12 if unit == "TFLOP/s" else decode_bytes(w) / 1e9
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": work_unit / v * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": describe(args.workload), "cpu_baseline": cb,
+                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    peaks = measured_peaks()
+
+    r = make_runner(args.workload, device)
+    with ClockSampler(local) as clk:
+        total_ms, kern_ms = time_runner(r, args.steps, args.warmup, dist_on)
+    total_ms = max_over_ranks(total_ms, dist_on)
+    ms = total_ms / args.steps
+    work, unit = r.work()
+    value = work * world / (ms / 1e3)
+    rf = roofline(r, kern_ms, peaks)
+
+    secondary = {}
+    if not args.no_secondary and rank == 0 and not dist_on:
+        names = ["v1_prefill", "v2_decode", "v1_decode", "v1_decode_unfused", "v2_prefill"]
+        for name in names:
+            if name == args.workload:
+                continue
+            r2 = make_runner(name, device)
+            t2, k2 = time_runner(r2, max(3, args.steps // 2), args.warmup, False)
+            wk, un = r2.work()
+            secondary[name] = {"value": wk / (t2 / max(3, args.steps // 2) / 1e3), "unit": un,
+                               "ms_per_step": t2 / max(3, args.steps // 2), "roofline": roofline(r2, k2, peaks),
+                               "config": describe(name)}
+            del r2
+            torch.cuda.empty_cache()
+
+    e2e = e2e_measure(r, max(2, min(args.steps, 5)))
+    e2e["value"] *= world
+
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(d) inputs on device)",
+            "config": dict(describe(args.workload), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+            "roofline": rf, "e2e": e2e, "gpu_launches": r.launches_per_step * args.steps,
+            "clocks": clk.summary()}
+    if secondary:
+        line["secondary"] = secondary
+    if rank == 0 and not args.no_cpu_baseline and not dist_on:
+        line["cpu_baseline"] = cpu_oracle_run(args.workload)
+    if rank == 0:
+        print(json.dumps(line))
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,226 @@
-"""B200-native differential attention forward (placeholder; binding follows)."""
+"""B200-native differential attention forward: thin Python binding of libdiffattn.so.
+
+The operation is O = (softmax(Q1 K1^T/sqrt(d)) - lambda softmax(Q2 K2^T/sqrt(d))) V
+with lambda = exp(lq1.lk1) - exp(lq2.lk2) + lambda_init ("差分注意力" tutorial,
+sections 差分思路, Step 2 and Step 4).  Every step runs in the CUDA kernels
+of ``libdiffattn.so`` (C ABI in ``include/diffattn.h``); this module only
+marshals torch tensors (device memory, the current stream) into that ABI.
+There is no CPU fallback: if the library is missing, every call raises.
+
+Inputs may be CUDA tensors (results stay on the device) or CPU tensors (they
+are copied to the current CUDA device, the kernels run there, and the result
+is copied back: the end-to-end path).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdiffattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5, -6
+F32, BF16 = 0, 1
+
+EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffattn_fwd_v1", "diffattn_fwd_v2",
+           "diffattn_decode_workspace_size", "diffattn_decode_v2", "diffattn_decode_v1", "diffattn_last_error",
+           "diffattn_last_status", "diffattn_set_wait_limit_ns"]
+
+_lib = None
+
+
+class DiffAttnError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"diffattn error {code}: {msg}")
+        self.code = code
+
+
+def load():
+    """Load libdiffattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m differential_attention_transformers_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, D, Z, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double, ctypes.c_size_t, ctypes.c_ulonglong
+    sig = {
+        "diffattn_version": (ctypes.c_char_p, []),
+        "diffattn_lambda_init": (D, [I]),
+        "diffattn_lambda": (I, [P, P, P, P, I, I, D, P, P]),
+        "diffattn_fwd_v1": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P]),
+        "diffattn_fwd_v2": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, P]),
+        "diffattn_decode_workspace_size": (Z, [I, I, I, I]),
+        "diffattn_decode_v2": (I, [P, P, P, P, P, I, I, I, I, I, I, P, Z, P]),
+        "diffattn_decode_v1": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]),
+        "diffattn_last_error": (ctypes.c_char_p, []),
+        "diffattn_last_status": (I, [P]),
+        "diffattn_set_wait_limit_ns": (None, [U]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    env = os.environ.get("DIFFATTN_WAIT_LIMIT_NS")
+    if env:
+        L.diffattn_set_wait_limit_ns(int(env))
+    _lib = L
+    return L
+
+
+def _check(code):
+    if code != OK:
+        raise DiffAttnError(code, load().diffattn_last_error().decode())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+def _prep(tensors):
+    """Move CPU inputs to the current CUDA device; report whether we did."""
+    host = any(t.device.type == "cpu" for t in tensors)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = []
+    for t in tensors:
+        if t.device.type == "cpu":
+            t = t.pin_memory().to(dev, non_blocking=True) if not t.is_pinned() else t.to(dev, non_blocking=True)
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        out.append(t)
+    return host, out
+
+
+def _finish(host, out):
+    if not host:
+        return out
+    res = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    res.copy_(out, non_blocking=True)
+    torch.cuda.current_stream().synchronize()
+    return res
+
+
+# ----------------------------------------------------------------------------
+def version() -> str:
+    return load().diffattn_version().decode()
+
+
+def lambda_init(layer: int) -> float:
+    """0.8 - 0.6 exp(-0.3 (layer - 1)), layer counted from 1."""
+    return float(load().diffattn_lambda_init(int(layer)))
+
+
+def compute_lambda(lq1, lk1, lq2, lk2, lam_init: float, out=None):
+    """Per-head lambda (f32 [H]) from f32 [H, dim] parameters, on the GPU."""
+    host, (lq1, lk1, lq2, lk2) = _prep([lq1, lk1, lq2, lk2])
+    H, dim = lq1.shape
+    for t in (lq1, lk1, lq2, lk2):
+        if t.dtype != torch.float32 or tuple(t.shape) != (H, dim):
+            raise ValueError("lq1, lk1, lq2, lk2 must be float32 [H, dim]")
+    if out is None:
+        out = torch.empty(H, dtype=torch.float32, device=lq1.device)
+    _check(load().diffattn_lambda(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), H, dim, float(lam_init),
+                                  _ptr(out), _stream()))
+    return _finish(host, out)
+
+
+def fwd_v1(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5, out=None):
+    """V1 layout: q1,q2 [B,H,Lq,d]; k1,k2 [B,Hkv,Lk,d]; v [B,Hkv,Lk,dv]; lam f32 [H]."""
+    host, (q1, k1, q2, k2, v, lam) = _prep([q1, k1, q2, k2, v, lam])
+    B, H, Lq, d = q1.shape
+    Hkv, Lk, dv = k1.shape[1], k1.shape[2], v.shape[3]
+    dt = _dtype_code(q1)
+    if out is None:
+        out = torch.empty((B, H, Lq, dv), dtype=q1.dtype, device=q1.device)
+    _check(load().diffattn_fwd_v1(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(v), _ptr(lam), _ptr(out), dt,
+                                  B, H, Hkv, Lq, Lk, d, dv, int(causal), int(rmsnorm), float(eps), _stream()))
+    return _finish(host, out)
+
+
+def fwd_v2(q, k, v, lam, causal=True, out=None):
+    """V2 layout: q [B,Hq,Lq,D]; k,v [B,Hkv,Lk,D]; lam f32 [Hq/2] -> [B,Hq/2,Lq,D]."""
+    host, (q, k, v, lam) = _prep([q, k, v, lam])
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, Hq // 2, Lq, D), dtype=q.dtype, device=q.device)
+    _check(load().diffattn_fwd_v2(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), dt, B, Hq, Hkv, Lq, Lk, D,
+                                  int(causal), _stream()))
+    return _finish(host, out)
+
+
+def decode_workspace_size(B: int, Hkv: int, T: int, dv: int = 128) -> int:
+    return int(load().diffattn_decode_workspace_size(B, Hkv, T, dv))
+
+
+_ws_cache = {}
+
+
+def _workspace(nbytes, device):
+    key = (device.index, )
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def decode_v2(q, kc, vc, lam, out=None, workspace=None):
+    """Single-token V2 decode: q [B,Hq,D]; kc,vc [B,Hkv,T,D]; lam [Hq/2] -> [B,Hq/2,D]."""
+    host, (q, kc, vc, lam) = _prep([q, kc, vc, lam])
+    B, Hq, D = q.shape
+    Hkv, T = kc.shape[1], kc.shape[2]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=q.dtype, device=q.device)
+    need = decode_workspace_size(B, Hkv, T, D)
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check(load().diffattn_decode_v2(_ptr(q), _ptr(kc), _ptr(vc), _ptr(lam), _ptr(out), dt, B, Hq, Hkv, T, D,
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream()))
+    return _finish(host, out)
+
+
+def decode_v1(q1, k1, q2, k2, v, lam, fused=True, out=None, workspace=None):
+    """Single-token V1-layout decode: q1,q2 [B,H,d]; k1,k2 [B,Hkv,T,d]; v [B,Hkv,T,dv] -> [B,H,dv]."""
+    host, (q1, k1, q2, k2, v, lam) = _prep([q1, k1, q2, k2, v, lam])
+    B, H, d = q1.shape
+    Hkv, T, dv = k1.shape[1], k1.shape[2], v.shape[3]
+    dt = _dtype_code(q1)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q1.dtype, device=q1.device)
+    need = decode_workspace_size(B, Hkv, T, dv)
+    ws = workspace if workspace is not None else _workspace(need, q1.device)
+    _check(load().diffattn_decode_v1(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(v), _ptr(lam), _ptr(out), dt,
+                                     B, H, Hkv, T, d, dv, int(fused), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream()))
+    return _finish(host, out)
+
+
+def last_status() -> int:
+    """Synchronise the current stream and read/clear the device status word."""
+    return int(load().diffattn_last_status(_stream()))
+
+
+def last_error() -> str:
+    return load().diffattn_last_error().decode()
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load().diffattn_set_wait_limit_ns(int(ns))

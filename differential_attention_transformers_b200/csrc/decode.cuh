@@ -1,0 +1,370 @@
+// decode.cuh -- single-token differential attention decode over a KV cache.
+//
+// HBM-bound: every cached K and V element is read exactly once for all query
+// heads of its KV group and for both maps ("差分注意力" tutorial, section V1
+// 到 V2 的 diff: V2 doubles the Q heads over the same KV heads so that one KV
+// load serves more queries; V1 is charged with loading the V cache twice,
+// which the fused V1 mode here avoids by reading K1, K2 and V once).
+//
+// Split-KV: the (batch, KV head, 64-key block) space is cut into equal
+// contiguous ranges, one per CTA (grid = a multiple of the SM count), so every
+// CTA streams the same number of bytes.  A CTA emits one partial record per
+// (batch, KV head) segment of its range: for each of the 8 query columns the
+// running max m (log2 units), the sum l and the unnormalised output O[128].
+// The combine kernel merges the records of each query head (log-sum-exp) and
+// applies O = O1/l1 - lambda * O2/l2.
+//
+// Inner product per 16-key slice and warp, on mma.sync m16n8k16 (bf16, f32
+// accumulate) with the keys as M so that the 8 query columns fill N = 8:
+//   S^T[16 keys x 8 cols]  = K[16 x 128] . Qcols^T[128 x 8]
+//   O^T[128 x 8]          += V^T[128 x 16] . P^T[16 x 8]
+// P^T goes from the C-fragment layout to the B-fragment layout with
+// movmatrix.trans.  Query columns: V2 = the G <= 8 Q heads of the group
+// (pair p = columns 2p, 2p+1); V1 = columns 0..3 map 1 of the group's heads
+// and 4..7 map 2, against K = [K1 | K2] (block-diagonal query operand).
+#pragma once
+
+#include "common.cuh"
+
+namespace da {
+
+constexpr int DEC_KB = 64;                  // keys per block (one pipeline stage)
+constexpr int DEC_CONSUMERS = 4;            // consumer warps, 16 keys of each block each
+constexpr int DEC_THREADS = 32 * (DEC_CONSUMERS + 1);
+constexpr int DEC_REC = 8 * 2 + 8 * 128;    // floats per partial record: m[8], l[8], O[8][128]
+constexpr int DEC_TILE_BYTES = DEC_KB * 128 * 2;  // one 64-key x 128-wide bf16 tile (two 8 KB boxes)
+
+struct DecodeArgs {
+  const __nv_bfloat16* q1;  // V2: q [B,Hq,128]; V1: q1 [B,H,64]
+  const __nv_bfloat16* q2;  // V1: q2 [B,H,64]; V2: unused
+  float* ws;                // partial records
+  int B, Hq, Hkv, T;        // Hq: V2 Q heads, V1 heads
+  int v1;                   // layout
+  int maps;                 // bit0: map 1 columns, bit1: map 2 columns (V1 unfused passes)
+  int grid;                 // CTAs
+  int maxseg;               // partial slots per CTA
+  long long nblk;           // 64-key blocks per (batch, KV head)
+  long long total;          // B * Hkv * nblk
+  float scale_log2;         // log2(e) / sqrt(d)
+  Watch watch;
+};
+
+__host__ __device__ __forceinline__ long long dec_blk_start(long long i, long long total, int grid) {
+  return i * total / grid;
+}
+
+template <int NST>
+struct DecSmem {
+  alignas(1024) uint8_t k[NST][DEC_TILE_BYTES];
+  alignas(1024) uint8_t v[NST][DEC_TILE_BYTES];
+  float mo[DEC_CONSUMERS][8][128];
+  float mm[DEC_CONSUMERS][8];
+  float ml[DEC_CONSUMERS][8];
+  alignas(8) uint64_t full[NST];
+  uint64_t empty[NST];
+  int abort_flag;
+};
+
+// Byte offset of element (row, 16-byte chunk) inside a 128-byte-swizzled box
+// of 128-byte rows (TMA SWIZZLE_128B, box base 1024-byte aligned).
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ bool bar_any(bool pred) {
+  // Barrier over the consumer warps (named barrier 1) with an OR reduction,
+  // so that all of them take the same abort decision.
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(DEC_CONSUMERS * 32)
+      : "memory");
+  return r != 0;
+}
+
+template <int NST>
+__global__ void __launch_bounds__(DEC_THREADS)
+decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
+                    const __grid_constant__ CUtensorMap tmV, DecodeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  DecSmem<NST>& S = *reinterpret_cast<DecSmem<NST>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &S.abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(smem_u32(&S.full[i]), 1);
+      mbar_init(smem_u32(&S.empty[i]), DEC_CONSUMERS);
+    }
+    S.abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  const long long lo = dec_blk_start(blockIdx.x, a.total, a.grid);
+  const long long hi = dec_blk_start(blockIdx.x + 1, a.total, a.grid);
+  const bool load_k2 = a.v1 ? (a.maps & 2) != 0 : true;
+  const bool load_k1 = a.v1 ? (a.maps & 1) != 0 : true;
+
+  if (warp == DEC_CONSUMERS) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK1);
+      tma_prefetch_desc(&tmV);
+      if (a.v1) tma_prefetch_desc(&tmK2);
+      long long issued_last[NST];
+      for (int i = 0; i < NST; ++i) issued_last[i] = -1;
+      bool ok = true;
+      for (long long x = lo; x < hi; ++x) {
+        const long long it = x - lo;
+        const int st = (int)(it % NST);
+        const long long use = it / NST;
+        if (use > 0 && !wait_bar(smem_u32(&S.empty[st]), (uint32_t)((use - 1) & 1), abort_flag, a.watch)) {
+          ok = false;
+          break;
+        }
+        const long long bg = x / a.nblk;
+        const int key0 = (int)((x % a.nblk) * DEC_KB);
+        const uint32_t fb = smem_u32(&S.full[st]);
+        uint32_t bytes = DEC_TILE_BYTES;  // V
+        if (a.v1) bytes += (load_k1 ? DEC_TILE_BYTES / 2 : 0) + (load_k2 ? DEC_TILE_BYTES / 2 : 0);
+        else bytes += DEC_TILE_BYTES;
+        mbar_expect_tx(fb, bytes);
+        const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
+        if (a.v1) {
+          if (load_k1) tma_load_3d(kd, &tmK1, fb, 0, key0, (int)bg);
+          if (load_k2) tma_load_3d(kd + DEC_TILE_BYTES / 2, &tmK2, fb, 0, key0, (int)bg);
+        } else {
+          tma_load_3d(kd, &tmK1, fb, 0, key0, (int)bg);
+          tma_load_3d(kd + DEC_TILE_BYTES / 2, &tmK1, fb, 64, key0, (int)bg);
+        }
+        tma_load_3d(vd, &tmV, fb, 0, key0, (int)bg);
+        tma_load_3d(vd + DEC_TILE_BYTES / 2, &tmV, fb, 64, key0, (int)bg);
+        issued_last[st] = use;
+      }
+      (void)ok;
+      // Every copy issued must have landed before the CTA may exit.
+      for (int i = 0; i < NST; ++i)
+        if (issued_last[i] >= 0) drain_bar(smem_u32(&S.full[i]), (uint32_t)(issued_last[i] & 1), a.watch.status);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers --
+  const int w = warp;                 // 16-key slice of each block
+  const int col0 = 2 * (lane & 3);    // this thread's two query columns
+  const int grp = a.v1 ? a.Hq / a.Hkv : a.Hq / a.Hkv;
+  const int seg_first_bg = (int)(lo / a.nblk);
+  // V1 single-map passes load only one K half: skip the other half's k-steps.
+  const int kk_lo = (a.v1 && !load_k1) ? 4 : 0;
+  const int kk_hi = (a.v1 && !load_k2) ? 4 : 8;
+  bool aborted = false;
+  long long x = lo;
+  while (x < hi) {
+    const long long bg = x / a.nblk;
+    const long long seg_end = min(hi, (bg + 1) * a.nblk);
+    const int b = (int)(bg / a.Hkv), g = (int)(bg % a.Hkv);
+
+    // query operand (B fragments) for the 8 columns: n = lane / 4
+    uint32_t qb[8][2];
+    {
+      const int n = lane >> 2;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t v0 = 0u, v1r = 0u;
+        const int dim = 16 * (kk & 3) + 2 * (lane & 3);
+        if (a.v1) {
+          // columns 0..3: map 1 (dims of K1 = k-steps 0..3); 4..7: map 2 (k-steps 4..7)
+          const bool m2 = n >= 4;
+          const int hl = n & 3;
+          const bool active = (kk >= 4) == m2 && hl < grp && (m2 ? (a.maps & 2) : (a.maps & 1));
+          if (active) {
+            const __nv_bfloat16* qp = (m2 ? a.q2 : a.q1) + ((size_t)b * a.Hq + g * grp + hl) * 64;
+            v0 = *reinterpret_cast<const uint32_t*>(qp + dim);
+            v1r = *reinterpret_cast<const uint32_t*>(qp + dim + 8);
+          }
+        } else if (n < grp) {
+          const __nv_bfloat16* qp = a.q1 + ((size_t)b * a.Hq + g * grp + n) * 128 + 64 * (kk >> 2);
+          v0 = *reinterpret_cast<const uint32_t*>(qp + dim);
+          v1r = *reinterpret_cast<const uint32_t*>(qp + dim + 8);
+        }
+        qb[kk][0] = v0;
+        qb[kk][1] = v1r;
+      }
+    }
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+    for (; x < seg_end; ++x) {
+      const long long it = x - lo;
+      const int st = (int)(it % NST);
+      bool ok = true;
+      if (lane == 0) ok = wait_bar(smem_u32(&S.full[st]), (uint32_t)((it / NST) & 1), abort_flag, a.watch);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) { aborted = true; break; }
+
+      const uint32_t kb = smem_u32(S.k[st]), vb = smem_u32(S.v[st]);
+      const int r0 = 16 * w;
+      // S^T = K . Q^T
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        if (kk < kk_lo || kk >= kk_hi) continue;
+        const int row = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int chunk = 2 * (kk & 3) + (lane >> 4);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kb + (kk >> 2) * (DEC_TILE_BYTES / 2) + swz(row, chunk), a0, a1, a2, a3);
+        mma16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+      }
+      // mask the ragged tail of the cache
+      const int key_lo = (int)((x % a.nblk) * DEC_KB) + r0 + (lane >> 2);
+      const bool v_lo = key_lo < a.T, v_hi = key_lo + 8 < a.T;
+      float xs[4];
+      xs[0] = v_lo ? s[0] * a.scale_log2 : -INFINITY;
+      xs[1] = v_lo ? s[1] * a.scale_log2 : -INFINITY;
+      xs[2] = v_hi ? s[2] * a.scale_log2 : -INFINITY;
+      xs[3] = v_hi ? s[3] * a.scale_log2 : -INFINITY;
+      float mx0 = fmaxf(xs[0], xs[2]), mx1 = fmaxf(xs[1], xs[3]);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+      const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = ex2(m_run[0] - mu0), al1 = ex2(m_run[1] - mu1);
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+      const float p0 = ex2(xs[0] - mu0), p1 = ex2(xs[1] - mu1);
+      const float p2 = ex2(xs[2] - mu0), p3 = ex2(xs[3] - mu1);
+      l_run[0] = l_run[0] * al0 + p0 + p2;
+      l_run[1] = l_run[1] * al1 + p1 + p3;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[i][0] *= al0; acc[i][2] *= al0;
+        acc[i][1] *= al1; acc[i][3] *= al1;
+      }
+      const uint32_t pb0 = movm_t(pack_bf16(p0, p1));
+      const uint32_t pb1 = movm_t(pack_bf16(p2, p3));
+      // O^T += V^T . P^T
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int mi = lane >> 3;
+        const int row = r0 + (lane & 7) + (mi >> 1) * 8;
+        const int chunk = 2 * (mt & 3) + (mi & 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vb + (mt >> 2) * (DEC_TILE_BYTES / 2) + swz(row, chunk), a0, a1, a2, a3);
+        mma16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.empty[st]));
+    }
+
+    // ---- merge the four warps' states of this segment into one record ----
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], o);
+      l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], o);
+    }
+    if (lane < 4) {
+      S.mm[w][col0] = m_run[0]; S.mm[w][col0 + 1] = m_run[1];
+      S.ml[w][col0] = l_run[0]; S.ml[w][col0 + 1] = l_run[1];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int dv = 16 * mt + (lane >> 2);
+      S.mo[w][col0][dv] = acc[mt][0];
+      S.mo[w][col0 + 1][dv] = acc[mt][1];
+      S.mo[w][col0][dv + 8] = acc[mt][2];
+      S.mo[w][col0 + 1][dv + 8] = acc[mt][3];
+    }
+    if (bar_any(aborted || *abort_flag)) break;
+    {
+      const int t = threadIdx.x;  // 0..127: output dv index, all 8 columns
+      float* rec = a.ws + ((size_t)blockIdx.x * a.maxseg + (size_t)(bg - seg_first_bg)) * DEC_REC;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < DEC_CONSUMERS; ++ww) M = fmaxf(M, S.mm[ww][c]);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float o = 0.f, l = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < DEC_CONSUMERS; ++ww) {
+          const float f = ex2(S.mm[ww][c] - Mu);
+          o += S.mo[ww][c][t] * f;
+          l += S.ml[ww][c] * f;
+        }
+        rec[16 + c * 128 + t] = o;
+        if (t == 0) { rec[c] = M; rec[8 + c] = l; }
+      }
+    }
+    if (bar_any(false)) break;  // records read from smem before the next segment overwrites it
+  }
+}
+
+struct CombineArgs {
+  const float* ws;
+  const float* lambda;
+  __nv_bfloat16* out;  // V2: [B, Hq/2, 128]; V1: [B, H, 128]
+  int B, Hq, Hkv, v1;
+  int grid, maxseg;
+  long long nblk, total;
+  int two_pass;        // V1 unfused: map 2 records live in a second workspace half
+  size_t half_floats;  // offset of the second half
+};
+
+// One CTA (128 threads = the value width) per (batch, output head).
+__global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
+  const int t = threadIdx.x;
+  const int Hout = a.v1 ? a.Hq : a.Hq / 2;
+  const int b = blockIdx.x / Hout, h = blockIdx.x % Hout;
+  const int grp = a.Hq / a.Hkv;
+  int g, c1, c2;
+  if (a.v1) { g = h / grp; c1 = h % grp; c2 = 4 + h % grp; }
+  else { g = (2 * h) / grp; c1 = (2 * h) % grp; c2 = c1 + 1; }
+  const long long bg = (long long)b * a.Hkv + g;
+  const long long x0 = bg * a.nblk, x1 = x0 + a.nblk;
+
+  // CTAs whose block range overlaps [x0, x1)
+  long long i0 = a.total > 0 ? x0 * a.grid / a.total : 0;
+  while (i0 > 0 && dec_blk_start(i0, a.total, a.grid) > x0) --i0;
+  while (i0 + 1 < a.grid && dec_blk_start(i0 + 1, a.total, a.grid) <= x0) ++i0;
+
+  float res[2];
+  for (int mp = 0; mp < 2; ++mp) {
+    const int c = mp == 0 ? c1 : c2;
+    const float* base = a.ws + ((a.two_pass && mp == 1) ? a.half_floats : 0);
+    float M = -INFINITY;
+    for (long long i = i0; i < a.grid && dec_blk_start(i, a.total, a.grid) < x1; ++i) {
+      const long long s = dec_blk_start(i, a.total, a.grid);
+      if (dec_blk_start(i + 1, a.total, a.grid) <= x0 || s >= x1) continue;
+      const float* rec = base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
+      M = fmaxf(M, rec[c]);
+    }
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float o = 0.f, l = 0.f;
+    for (long long i = i0; i < a.grid && dec_blk_start(i, a.total, a.grid) < x1; ++i) {
+      const long long s = dec_blk_start(i, a.total, a.grid);
+      if (dec_blk_start(i + 1, a.total, a.grid) <= x0 || s >= x1) continue;
+      const float* rec = base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
+      const float f = ex2(rec[c] - Mu);
+      o += rec[16 + c * 128 + t] * f;
+      l += rec[8 + c] * f;
+    }
+    res[mp] = l > 0.f ? o / l : 0.f;
+  }
+  const float lam = a.lambda[h];
+  a.out[((size_t)b * Hout + h) * 128 + t] = __float2bfloat16_rn(res[0] - lam * res[1]);
+}
+
+}  // namespace da

@@ -1,0 +1,387 @@
+// diffattn.cu -- C ABI of libdiffattn.so (declared in include/diffattn.h).
+//
+// Host side: argument validation (before any launch), TMA tensor-map
+// encoding, launch configuration, the device status word.  All device work
+// lives in the kernels included below; nothing here computes on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/diffattn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "lambda_simt.cuh"
+#include "prefill_sm100.cuh"
+
+using namespace da;
+
+// Device status word (timeouts of bounded waits), one per device.
+__device__ unsigned g_diffattn_status;
+
+namespace {
+
+thread_local std::string t_last_error;
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int ok() {
+  t_last_error.clear();
+  return DIFFATTN_OK;
+}
+
+#define CUDA_TRY(expr)                                                                  \
+  do {                                                                                  \
+    cudaError_t e_ = (expr);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(DIFFATTN_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));   \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  unsigned* status = nullptr;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+template <int DQK>
+constexpr size_t prefill_smem() { return sizeof(PfSmem<DQK>) + 1024; }
+constexpr int kDecNst = 2;
+constexpr size_t decode_smem() { return sizeof(DecSmem<kDecNst>) + 1024; }
+constexpr int kDecCtasPerSm = 2;
+
+// Per-device set-up: SM count, status word address, kernel attributes,
+// tensor-map encoder.  Called with the target device current.
+int device_setup(DeviceInfo** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(DIFFATTN_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (major != 10 || minor != 0)
+      return fail(DIFFATTN_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                  major, minor);
+    CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_diffattn_status));
+    d.status = static_cast<unsigned*>(p);
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)prefill_smem<64>()));
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)prefill_smem<128>()));
+    CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)decode_smem()));
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      CUDA_TRY(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn)
+        return fail(DIFFATTN_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.init = true;
+  }
+  *out = &d;
+  return DIFFATTN_OK;
+}
+
+Watch make_watch(const DeviceInfo* d) { return Watch{d->status, g_wait_limit_ns.load()}; }
+
+// 3-D bf16 tensor map over a contiguous [Z, Y, X] tensor, box {64, box_y, 1},
+// 128-byte swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap* m, const void* base, int X, long long Y, long long Z, int box_y) {
+  cuuint64_t dims[3] = {(cuuint64_t)X, (cuuint64_t)Y, (cuuint64_t)Z};
+  cuuint64_t strides[2] = {(cuuint64_t)X * 2, (cuuint64_t)X * 2 * (cuuint64_t)Y};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_y, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DIFFATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DIFFATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_bf16_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
+  return DIFFATTN_OK;
+}
+
+float log2e_over_sqrt(int d) { return (float)(1.4426950408889634 / std::sqrt((double)d)); }
+
+int launch_simt(const SimtArgs& a, cudaStream_t s) {
+  if (a.Lq == 0 || a.B == 0 || a.Hout == 0) return ok();
+  if ((long long)a.B * a.Hout > 65535) return fail(DIFFATTN_ERR_UNSUPPORTED, "B * heads > 65535 on the f32 path");
+  dim3 grid((unsigned)a.Lq, (unsigned)(a.B * a.Hout));
+  simt_forward_kernel<<<grid, SIMT_THREADS, 0, s>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
+                   const float* lambda, void* out, int B, int Hout, int Hq, int Hkv, int Lq, int Lk, int dqk,
+                   bool v1, int causal, int rms, float eps, cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  if (Lq == 0 || B == 0 || Hout == 0) return ok();
+  CUtensorMap mq1, mq2, mk1, mk2, mv;
+  // Q maps: V2 reads both maps from one tensor [B*Hq, Lq, dqk]
+  if (int e = make_map(&mq1, q1, dqk, Lq, (long long)B * Hq, PF_BM)) return e;
+  if (int e = make_map(&mq2, q2, dqk, Lq, (long long)B * Hq, PF_BM)) return e;
+  const long long Lk_map = Lk > 0 ? Lk : 1;  // a zero extent is not encodable; Lk == 0 launches no loads
+  if (int e = make_map(&mk1, k1, dqk, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+  if (int e = make_map(&mk2, k2, dqk, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+  if (int e = make_map(&mv, v, PF_DV, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+  PrefillArgs a;
+  a.lambda = lambda;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.B = B; a.Hout = Hout; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk;
+  a.v1 = v1 ? 1 : 0;
+  a.causal = causal ? 1 : 0;
+  a.rms = rms ? 1 : 0;
+  a.eps = eps;
+  a.scale_log2 = log2e_over_sqrt(dqk);
+  a.n_rb = (Lq + PF_BM - 1) / PF_BM;
+  a.watch = make_watch(dev);
+  const long long units = (long long)a.n_rb * B * Hout;
+  if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
+  if (dqk == 64)
+    prefill_kernel<64><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+  else
+    prefill_kernel<128><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+struct DecodePlan {
+  int grid = 1;
+  int maxseg = 1;
+  long long nblk = 0, total = 0;
+  size_t bytes_per_pass = 0;
+};
+
+DecodePlan plan_decode(int sms, int B, int Hkv, int T) {
+  DecodePlan p;
+  p.nblk = ((long long)T + DEC_KB - 1) / DEC_KB;
+  p.total = (long long)B * Hkv * p.nblk;
+  long long g = (long long)sms * kDecCtasPerSm;
+  if (g > p.total) g = p.total;
+  if (g < 1) g = 1;
+  p.grid = (int)g;
+  const long long per = (p.total + p.grid - 1) / p.grid;
+  p.maxseg = p.nblk > 0 ? (int)((per + p.nblk - 1) / p.nblk + 1) : 1;
+  p.bytes_per_pass = (size_t)p.grid * p.maxseg * DEC_REC * sizeof(float);
+  return p;
+}
+
+int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
+                  const float* lambda, void* out, int B, int Hq, int Hkv, int T, bool v1, int fused, void* ws,
+                  size_t ws_bytes, cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  if (B == 0) return ok();
+  const DecodePlan p = plan_decode(dev->sms, B, Hkv, T);
+  const int passes = (v1 && !fused) ? 2 : 1;
+  const size_t need = p.bytes_per_pass * passes;
+  if (p.total > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(DIFFATTN_ERR_WORKSPACE, "decode workspace %zu B < required %zu B", ws_bytes, need);
+  if (p.total > 0 && !aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  if (p.total > 0) {
+    CUtensorMap mk1, mk2, mv;
+    const int dk = v1 ? 64 : 128;
+    if (int e = make_map(&mk1, k1, dk, T, (long long)B * Hkv, DEC_KB)) return e;
+    if (int e = make_map(&mk2, v1 ? k2 : k1, dk, T, (long long)B * Hkv, DEC_KB)) return e;
+    if (int e = make_map(&mv, v, 128, T, (long long)B * Hkv, DEC_KB)) return e;
+    DecodeArgs a;
+    a.q1 = static_cast<const __nv_bfloat16*>(q1);
+    a.q2 = static_cast<const __nv_bfloat16*>(v1 ? q2 : q1);
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T = T;
+    a.v1 = v1 ? 1 : 0;
+    a.grid = p.grid; a.maxseg = p.maxseg; a.nblk = p.nblk; a.total = p.total;
+    a.scale_log2 = log2e_over_sqrt(dk);
+    a.watch = make_watch(dev);
+    for (int pass = 0; pass < passes; ++pass) {
+      a.maps = passes == 1 ? 3 : (1 << pass);
+      a.ws = static_cast<float*>(ws) + (size_t)pass * (p.bytes_per_pass / sizeof(float));
+      decode_split_kernel<kDecNst><<<p.grid, DEC_THREADS, decode_smem(), s>>>(mk1, mk2, mv, a);
+      CUDA_TRY(cudaGetLastError());
+    }
+  }
+  CombineArgs c;
+  c.ws = static_cast<const float*>(ws);
+  c.lambda = lambda;
+  c.out = static_cast<__nv_bfloat16*>(out);
+  c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.v1 = v1 ? 1 : 0;
+  c.grid = p.grid; c.maxseg = p.maxseg; c.nblk = p.nblk; c.total = p.total;
+  c.two_pass = passes == 2 ? 1 : 0;
+  c.half_floats = p.bytes_per_pass / sizeof(float);
+  const int Hout = v1 ? Hq : Hq / 2;
+  decode_combine_kernel<<<(unsigned)(B * Hout), 128, 0, s>>>(c);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+}  // namespace
+
+// ============================================================================
+extern "C" {
+
+const char* diffattn_version(void) { return "diffattn 0.1 sm_100a"; }
+
+double diffattn_lambda_init(int layer) {
+  if (layer < 1) return NAN;
+  return 0.8 - 0.6 * std::exp(-0.3 * (double)(layer - 1));
+}
+
+const char* diffattn_last_error(void) { return t_last_error.c_str(); }
+
+void diffattn_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns); }
+
+int diffattn_last_status(void* stream) {
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  unsigned v = 0;
+  CUDA_TRY(cudaMemcpy(&v, dev->status, sizeof(v), cudaMemcpyDeviceToHost));
+  const unsigned zero = 0;
+  CUDA_TRY(cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice));
+  if (v & STATUS_TIMEOUT) return fail(DIFFATTN_ERR_TIMEOUT, "a bounded device wait expired");
+  return ok();
+}
+
+int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2, int heads, int dim,
+                    double lambda_init, float* lambda_out, void* stream) {
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !lambda_out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (heads < 1 || dim < 1) return fail(DIFFATTN_ERR_INVALID_ARG, "heads and dim must be >= 1");
+  const int threads = 128;
+  lambda_kernel<<<(heads + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      lq1, lk1, lq2, lk2, heads, dim, lambda_init, lambda_out);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+int diffattn_fwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                    const float* lambda, void* out, diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk,
+                    int d, int dv, int causal, int rmsnorm, float eps, void* stream) {
+  if (B < 0 || H < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || d < 1 || dv < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d Lq=%d Lk=%d d=%d dv=%d)", B, H, Hkv, Lq,
+                Lk, d, dv);
+  if (H % Hkv) return fail(DIFFATTN_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+  if (!q1 || !k1 || !q2 || !k2 || !v || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (rmsnorm && !(eps >= 0.f)) return fail(DIFFATTN_ERR_INVALID_ARG, "eps must be >= 0");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DIFFATTN_F32) {
+    if (d > SIMT_MAXD || dv > SIMT_MAXCOL * SIMT_THREADS)
+      return fail(DIFFATTN_ERR_UNSUPPORTED, "f32 path supports d <= %d, dv <= %d", SIMT_MAXD,
+                  SIMT_MAXCOL * SIMT_THREADS);
+    SimtArgs a{static_cast<const float*>(q1), static_cast<const float*>(q2), static_cast<const float*>(k1),
+               static_cast<const float*>(k2), static_cast<const float*>(v), lambda, static_cast<float*>(out),
+               B, H, H, Hkv, Lq, Lk, d, dv, 0, causal ? 1 : 0, rmsnorm ? 1 : 0, eps,
+               (float)(1.0 / std::sqrt((double)d))};
+    return launch_simt(a, s);
+  }
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (!(d == 64 || d == 128) || dv != 128)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 V1 path needs d in {64,128} and dv == 128 (got d=%d dv=%d)", d, dv);
+  if (int e = check_bf16_ptrs({q1, k1, q2, k2, v, out})) return e;
+  return launch_prefill(q1, q2, k1, k2, v, lambda, out, B, H, H, Hkv, Lq, Lk, d, true, causal, rmsnorm, eps, s);
+}
+
+int diffattn_fwd_v2(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                    diffattn_dtype dtype, int B, int Hq, int Hkv, int Lq, int Lk, int D, int causal,
+                    void* stream) {
+  if (B < 0 || Hq < 2 || Hkv < 1 || Lq < 0 || Lk < 0 || D < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d Lq=%d Lk=%d D=%d)", B, Hq, Hkv, Lq, Lk, D);
+  if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (!q || !k || !v || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DIFFATTN_F32) {
+    if (D > SIMT_MAXD) return fail(DIFFATTN_ERR_UNSUPPORTED, "f32 path supports D <= %d", SIMT_MAXD);
+    SimtArgs a{static_cast<const float*>(q), static_cast<const float*>(q), static_cast<const float*>(k),
+               static_cast<const float*>(k), static_cast<const float*>(v), lambda, static_cast<float*>(out),
+               B, Hq / 2, Hq, Hkv, Lq, Lk, D, D, 1, causal ? 1 : 0, 0, 0.f, (float)(1.0 / std::sqrt((double)D))};
+    return launch_simt(a, s);
+  }
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (D != 128) return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 V2 path needs D == 128 (got %d)", D);
+  if (int e = check_bf16_ptrs({q, k, v, out})) return e;
+  return launch_prefill(q, q, k, k, v, lambda, out, B, Hq / 2, Hq, Hkv, Lq, Lk, 128, false, causal, 0, 0.f, s);
+}
+
+size_t diffattn_decode_workspace_size(int B, int Hkv, int T, int dv) {
+  (void)dv;
+  if (B < 0 || Hkv < 1 || T < 0) return 0;
+  DeviceInfo* dev = nullptr;
+  if (device_setup(&dev)) return 0;
+  return plan_decode(dev->sms, B, Hkv, T).bytes_per_pass * 2;  // room for the two-pass V1 comparison
+}
+
+int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const float* lambda, void* out,
+                       diffattn_dtype dtype, int B, int Hq, int Hkv, int T, int D, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (B < 0 || Hq < 2 || Hkv < 1 || T < 0 || D < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d T=%d D=%d)", B, Hq, Hkv, T, D);
+  if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (!q || !kc || !vc || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DIFFATTN_F32)
+    return diffattn_fwd_v2(q, kc, vc, lambda, out, dtype, B, Hq, Hkv, 1, T, D, 1, stream);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (D != 128 || Hq / Hkv > 8)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 decode needs D == 128 and Hq/Hkv <= 8 (D=%d Hq=%d Hkv=%d)", D, Hq,
+                Hkv);
+  if (int e = check_bf16_ptrs({q, kc, vc, out})) return e;
+  return launch_decode(q, nullptr, kc, nullptr, vc, lambda, out, B, Hq, Hkv, T, false, 1, ws, ws_bytes, s);
+}
+
+int diffattn_decode_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                       const float* lambda, void* out, diffattn_dtype dtype, int B, int H, int Hkv, int T, int d,
+                       int dv, int fused, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 0 || H < 1 || Hkv < 1 || T < 0 || d < 1 || dv < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d T=%d d=%d dv=%d)", B, H, Hkv, T, d, dv);
+  if (H % Hkv) return fail(DIFFATTN_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+  if (!q1 || !k1 || !q2 || !k2 || !v || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DIFFATTN_F32)
+    return diffattn_fwd_v1(q1, k1, q2, k2, v, lambda, out, dtype, B, H, Hkv, 1, T, d, dv, 1, 0, 0.f, stream);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (d != 64 || dv != 128 || H / Hkv > 4)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 V1 decode needs d == 64, dv == 128, H/Hkv <= 4");
+  if (int e = check_bf16_ptrs({q1, k1, q2, k2, v, out})) return e;
+  return launch_decode(q1, q2, k1, k2, v, lambda, out, B, H, Hkv, T, true, fused, ws, ws_bytes, s);
+}
+
+}  // extern "C"

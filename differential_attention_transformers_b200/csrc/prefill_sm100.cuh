@@ -1,0 +1,371 @@
+// prefill_sm100.cuh -- causal differential attention prefill on tcgen05.
+//
+// One CTA computes 128 query rows of one output head, for both maps:
+//   S_m = Q_m K_m^T          (tcgen05.mma, A and B from shared memory, D in TMEM)
+//   P_m = exp(S_m/sqrt(d) - rowmax_m), l_m = rowsum(P_m)   (online, per map)
+//   O_m += P_m V             (tcgen05.mma, A = P_m from TMEM, B = V from smem)
+//   out = O_1 / l_1 - lambda * O_2 / l_2  [then RMSNorm]     (epilogue)
+// ("差分注意力" tutorial, section 差分思路 and Step 2; V1/V2 layouts from
+// its section V1 到 V2 的 diff.)  Each K/V tile is loaded once by TMA and
+// serves both maps: in V2 both maps share K and V; in V1 the tile holds K1,
+// K2 and the shared V.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax of map 1 (thread i <-> query row i <-> TMEM lane i)
+//   warps 4-7  softmax of map 2
+//   warp  8    TMA producer; allocates / frees TMEM
+//   warp  9    MMA issuer (one thread)
+// TMEM (512 columns): S1 [0,128) S2 [128,256) O1 [256,384) O2 [384,512).
+// P_m (bf16, 64 columns) overwrites the first half of S_m after the softmax
+// has read S_m; the MMA issuer orders "PV_m(j) then S_m(j+1)" so the tensor
+// pipe reads P_m before it writes the next S_m.
+// Shared memory: Q1, Q2 tiles, then NS stages of {K tile(s), V tile}; every
+// tile is a set of 128-row x 128-byte boxes in the TMA 128-byte swizzle,
+// which is the canonical K-major (Q, K) / MN-major (V) UMMA layout.
+#pragma once
+
+#include "common.cuh"
+
+namespace da {
+
+constexpr int PF_BM = 128;        // query rows per CTA
+constexpr int PF_BN = 128;        // keys per tile
+constexpr int PF_DV = 128;        // value width
+constexpr int PF_NS = 2;          // K/V pipeline stages
+constexpr int PF_THREADS = 320;
+constexpr int PF_BOX = 128 * 128; // bytes of one 128-row x 64-element bf16 box
+constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+struct PrefillArgs {
+  const float* lambda;
+  __nv_bfloat16* out;   // [B, Hout, Lq, 128]
+  int B, Hout, Hq, Hkv, Lq, Lk;
+  int v1;               // layout: 1 = V1 (q1/q2, k1/k2 tensors), 0 = V2 (pairs of Q heads)
+  int causal, rms;
+  float eps, scale_log2;
+  int n_rb;             // row blocks per head
+  Watch watch;
+};
+
+template <int DQK>
+struct PfSmem {
+  static constexpr int QTILE = PF_BM * DQK * 2;  // bytes of one Q tile
+  alignas(1024) uint8_t q[2][QTILE];
+  alignas(1024) uint8_t k[PF_NS][2 * PF_BOX];   // V2: K tile (2 boxes); V1: K1 box, K2 box
+  alignas(1024) uint8_t v[PF_NS][2 * PF_BOX];   // V tile, dv 0-63 box then 64-127 box
+  float l[2][PF_BM];
+  float ss[2][PF_BM];
+  alignas(8) uint64_t q_full;
+  uint64_t kv_full[PF_NS];
+  uint64_t kv_empty[PF_NS];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_final;
+  uint64_t xl;      // epilogue exchange of l (256 arrivals)
+  uint64_t xs;      // epilogue exchange of RMS partial sums (256 arrivals)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          const Watch& w) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, w);
+  return __shfl_sync(0xffffffffu, ok, 0);
+}
+
+template <int DQK>
+__global__ void __launch_bounds__(PF_THREADS, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
+               const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
+               const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
+  static_assert(DQK == 64 || DQK == 128, "QK width 64 or 128");
+  constexpr int QBOXES = DQK / 64;
+  extern __shared__ uint8_t smem_raw[];
+  PfSmem<DQK>& S = *reinterpret_cast<PfSmem<DQK>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &S.abort_flag;
+
+  // ---- work unit: heaviest row blocks first (causal) ----
+  const int BH = a.B * a.Hout;
+  const int rb = a.n_rb - 1 - (int)(blockIdx.x / BH);
+  const int bh = (int)(blockIdx.x % BH);
+  const int b = bh / a.Hout, h = bh % a.Hout;
+  const int r0 = rb * PF_BM;
+  int qh1, qh2, g;
+  if (a.v1) { qh1 = qh2 = h; g = h / (a.Hq / a.Hkv); }
+  else { qh1 = 2 * h; qh2 = 2 * h + 1; g = qh1 / (a.Hq / a.Hkv); }
+  const int zq1 = b * a.Hq + qh1, zq2 = b * a.Hq + qh2, zkv = b * a.Hkv + g;
+  // keys visible to the last row of the block
+  long long kend = a.causal ? (long long)min(r0 + PF_BM, a.Lq) - 1 + (a.Lk - a.Lq) + 1 : a.Lk;
+  kend = max(0LL, min(kend, (long long)a.Lk));
+  const int nT = (int)((kend + PF_BN - 1) / PF_BN);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&S.q_full), 1);
+    for (int i = 0; i < PF_NS; ++i) {
+      mbar_init(smem_u32(&S.kv_full[i]), 1);
+      mbar_init(smem_u32(&S.kv_empty[i]), 1);
+    }
+    for (int m = 0; m < 2; ++m) {
+      mbar_init(smem_u32(&S.s_full[m]), 1);
+      mbar_init(smem_u32(&S.p_full[m]), 128);
+    }
+    mbar_init(smem_u32(&S.o_final), 1);
+    mbar_init(smem_u32(&S.xl), 256);
+    mbar_init(smem_u32(&S.xs), 256);
+    mbar_init(smem_u32(&S.drain), 1);
+    S.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(&S.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0 && nT > 0) {
+      tma_prefetch_desc(&tmK1);
+      tma_prefetch_desc(&tmV);
+      const uint32_t qb = smem_u32(&S.q_full);
+      mbar_expect_tx(qb, 2 * PfSmem<DQK>::QTILE);
+      for (int x = 0; x < QBOXES; ++x) {
+        tma_load_3d(smem_u32(S.q[0]) + x * PF_BOX, &tmQ1, qb, 64 * x, r0, zq1);
+        tma_load_3d(smem_u32(S.q[1]) + x * PF_BOX, &tmQ2, qb, 64 * x, r0, zq2);
+      }
+      int last_use[PF_NS];
+      for (int i = 0; i < PF_NS; ++i) last_use[i] = -1;
+      bool ok = true;
+      for (int j = 0; j < nT; ++j) {
+        const int st = j % PF_NS, use = j / PF_NS;
+        if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(&S.kv_full[st]);
+        mbar_expect_tx(fb, 4 * PF_BOX);
+        const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
+        if (a.v1) {
+          tma_load_3d(kd, &tmK1, fb, 0, j * PF_BN, zkv);
+          tma_load_3d(kd + PF_BOX, &tmK2, fb, 0, j * PF_BN, zkv);
+        } else {
+          tma_load_3d(kd, &tmK1, fb, 0, j * PF_BN, zkv);
+          tma_load_3d(kd + PF_BOX, &tmK1, fb, 64, j * PF_BN, zkv);
+        }
+        tma_load_3d(vd, &tmV, fb, 0, j * PF_BN, zkv);
+        tma_load_3d(vd + PF_BOX, &tmV, fb, 64, j * PF_BN, zkv);
+        last_use[st] = use;
+      }
+      (void)ok;
+      // Every copy issued must have landed before the CTA may exit (returns at
+      // once when the consumer has already seen the phase).
+      drain_bar(qb, 0, a.watch.status);
+      for (int i = 0; i < PF_NS; ++i)
+        if (last_use[i] >= 0) drain_bar(smem_u32(&S.kv_full[i]), last_use[i] & 1, a.watch.status);
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0 && nT > 0) {
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, PF_BN, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, PF_DV, true);
+      const uint32_t tS[2] = {tmem + 0, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 384};
+      const uint32_t sq[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
+      bool ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
+      auto issue_qk = [&](int m, int j) {
+        const int st = j % PF_NS;
+        const uint32_t kb = smem_u32(S.k[st]) + (a.v1 ? m * PF_BOX : 0);
+#pragma unroll
+        for (int s = 0; s < DQK / 16; ++s) {
+          const uint32_t off = (s >> 2) * PF_BOX + (s & 3) * 32;
+          mma_ss(tS[m], umma_desc(sq[m] + off, 16, 1024), umma_desc(kb + off, 16, 1024), IDESC_QK, s > 0);
+        }
+        mma_commit(smem_u32(&S.s_full[m]));
+      };
+      auto issue_pv = [&](int m, int j) {
+        const int st = j % PF_NS;
+        const uint32_t vb = smem_u32(S.v[st]);
+#pragma unroll
+        for (int s = 0; s < PF_BN / 16; ++s)
+          mma_ts(tO[m], tS[m] + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, (j > 0 || s > 0));
+      };
+      if (ok) {
+        tc_fence_after();
+        ok = wait_bar(smem_u32(&S.kv_full[0]), 0, abort_flag, a.watch);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          issue_qk(1, 0);
+        }
+      }
+      for (int j = 0; ok && j < nT; ++j) {
+        const int st = j % PF_NS;
+        const bool more = j + 1 < nT;
+        if (!(ok = wait_bar(smem_u32(&S.p_full[0]), j & 1, abort_flag, a.watch))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!(ok = wait_bar(smem_u32(&S.kv_full[(j + 1) % PF_NS]), ((j + 1) / PF_NS) & 1, abort_flag, a.watch)))
+            break;
+          tc_fence_after();
+          issue_qk(0, j + 1);
+        }
+        if (!(ok = wait_bar(smem_u32(&S.p_full[1]), j & 1, abort_flag, a.watch))) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(smem_u32(&S.kv_empty[st]));
+        if (more) issue_qk(1, j + 1);
+      }
+      if (ok) mma_commit(smem_u32(&S.o_final));
+      // Every MMA issued must have completed before TMEM is freed.
+      mma_commit(smem_u32(&S.drain));
+      drain_bar(smem_u32(&S.drain), 0, a.watch.status);
+    }
+  } else {
+    // ------------------------------------------------- softmax (two groups) --
+    const int m = warp >> 2;                 // map
+    const int wq = warp & 3;                 // TMEM lane quadrant
+    const int r = threadIdx.x & 127;         // row within the block
+    const int rg = r0 + r;                   // query row
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + m * 128;
+    // last visible key of this row
+    const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nT; ++j) {
+      if (!(ok = warp_wait(smem_u32(&S.s_full[m]), j & 1, abort_flag, a.watch))) break;
+      tc_fence_after();
+      float s[PF_BN];
+      {
+        uint32_t rr[PF_BN];
+#pragma unroll
+        for (int c = 0; c < PF_BN / 32; ++c) tmem_ld32p(tS + c * 32, rr + c * 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < PF_BN; ++i) s[i] = __uint_as_float(rr[i]);
+      }
+      const long long lim = lastk - (long long)j * PF_BN;   // columns > lim are masked
+      if (lim < PF_BN - 1) {
+#pragma unroll
+        for (int c = 0; c < PF_BN; ++c)
+          if (c > lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < PF_BN; ++c) mx = fmaxf(mx, s[c]);
+      const float mxs = mx * a.scale_log2;
+      float alpha = 1.f;
+      if (mxs > m_run + PF_RESCALE_THRESHOLD) {
+        if (m_run != -INFINITY && j > 0) alpha = ex2(m_run - mxs);
+        m_run = mxs;
+      }
+      const float mu = m_run == -INFINITY ? 0.f : m_run;
+      float sum = 0.f;
+      uint32_t pk[PF_BN / 2];
+#pragma unroll
+      for (int c = 0; c < PF_BN; c += 2) {
+        const float p0 = ex2(fmaf(s[c], a.scale_log2, -mu));
+        const float p1 = ex2(fmaf(s[c + 1], a.scale_log2, -mu));
+        sum += p0 + p1;
+        pk[c / 2] = pack_bf16(p0, p1);
+      }
+      l_run = l_run * alpha + sum;
+      // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs it
+      // (rows whose alpha is 1 multiply by 1).
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        // O_m(j-1) is complete: S_m(j) was committed after PV_m(j-1).
+        const uint32_t tO = tmem + lane_off + 256 + m * 128;
+#pragma unroll
+        for (int c = 0; c < PF_DV / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32p(tO + c * 32, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          tmem_st32p(tO + c * 32, rr);
+        }
+      }
+      tmem_st32p(tS, pk);
+      tmem_st32p(tS + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&S.p_full[m]));
+    }
+
+    // --------------------------------------------------------- epilogue --
+    // Rows that saw no key (l == 0) output zeros.
+    const float lam = a.lambda[h];
+    __nv_bfloat16* orow = a.out + (((size_t)b * a.Hout + h) * a.Lq + rg) * PF_DV + m * 64;
+    float y[64];
+    bool have = false;
+    if (ok && nT > 0) {
+      S.l[m][r] = l_run;
+      mbar_arrive(smem_u32(&S.xl));
+      ok = warp_wait(smem_u32(&S.xl), 0, abort_flag, a.watch) &&
+           warp_wait(smem_u32(&S.o_final), 0, abort_flag, a.watch);
+      if (ok) {
+        tc_fence_after();
+        const float l1 = S.l[0][r], l2 = S.l[1][r];
+        const float c1 = l1 > 0.f ? 1.f / l1 : 0.f;
+        const float c2 = l2 > 0.f ? lam / l2 : 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t o1[32], o2[32];
+          tmem_ld32p(tmem + lane_off + 256 + m * 64 + c * 32, o1);
+          tmem_ld32p(tmem + lane_off + 384 + m * 64 + c * 32, o2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            y[c * 32 + i] = __uint_as_float(o1[i]) * c1 - __uint_as_float(o2[i]) * c2;
+        }
+        have = true;
+        if (a.rms) {
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) ss = fmaf(y[i], y[i], ss);
+          S.ss[m][r] = ss;
+          mbar_arrive(smem_u32(&S.xs));
+          ok = warp_wait(smem_u32(&S.xs), 0, abort_flag, a.watch);
+          have = ok;
+          if (ok) {
+            const float rs = rsqrtf((S.ss[0][r] + S.ss[1][r]) / (float)PF_DV + a.eps);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) y[i] *= rs;
+          }
+        }
+      }
+    } else if (nT == 0) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) y[i] = 0.f;
+      have = true;
+    }
+    if (have && rg < a.Lq) {
+#pragma unroll
+      for (int i = 0; i < 64; i += 8) {
+        uint4 v;
+        v.x = pack_bf16(y[i + 0], y[i + 1]);
+        v.y = pack_bf16(y[i + 2], y[i + 3]);
+        v.z = pack_bf16(y[i + 4], y[i + 5]);
+        v.w = pack_bf16(y[i + 6], y[i + 7]);
+        *reinterpret_cast<uint4*>(orow + i) = v;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace da

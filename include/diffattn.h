@@ -1,0 +1,161 @@
+/*
+ * diffattn.h -- C ABI of libdiffattn.so, the B200 (sm_100a) differential
+ * attention forward.
+ *
+ * The operation (sources cited by page title and section):
+ *
+ *   A1 = softmax(Q1 K1^T / sqrt(d)),  A2 = softmax(Q2 K2^T / sqrt(d))
+ *   O  = (A1 - lambda * A2) V
+ *       "差分注意力" tutorial (aiknowledge.cn), section 差分思路 and
+ *       二、从零实现 Step 2; the paper note "Understanding Differential
+ *       Transformer Unchains Pretrained Self-Attentions", section 关键设计.
+ *   lambda = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init
+ *       "差分注意力" tutorial, section 差分思路 and Step 4 (λ 参数化).
+ *   lambda_init = 0.8 - 0.6 exp(-0.3 (layer - 1))
+ *       "Differential Transformer：用“差分降噪”重塑LLM注意力机制" (mcipr.com),
+ *       section 3 工程实践.
+ *   V1 layout (half-width Q/K per head, one V, optional per-head RMSNorm) and
+ *   V2 layout (Q heads doubled over shared KV heads, no norm)
+ *       "差分注意力" tutorial, section V1 到 V2 的 diff.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, last dimension contiguous, no padding.
+ *     The shapes are given per argument.  "bf16" is IEEE bfloat16, "f32" IEEE
+ *     binary32.  Output precision equals input precision; all arithmetic is
+ *     fp32 (lambda: fp64) whatever the input type.
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library
+ *     keeps no reference after the call and allocates no device memory.  Work
+ *     is queued asynchronously on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream); the call returns before the GPU finishes.
+ *   - Every bf16 tensor must start on a 16-byte boundary and its row
+ *     (last-dimension) length in bytes must be a multiple of 16 (tensor-map
+ *     copies require it); violations return DIFFATTN_ERR_MISALIGNED before
+ *     any launch.
+ *   - Causal masking is bottom-right aligned: query row i sees key j iff
+ *     j <= i + (Lk - Lq).  A row that sees no key outputs zeros.
+ *   - Errors: every argument error is reported before anything is launched,
+ *     as a negative status; diffattn_last_error() then describes it.  No C++
+ *     exception crosses this boundary.  A device-side bounded wait that runs
+ *     out does not fault the GPU: the kernel records DIFFATTN_ERR_TIMEOUT in a
+ *     device status word, releases what it holds and returns; read it with
+ *     diffattn_last_status().
+ */
+#ifndef DIFFATTN_H_
+#define DIFFATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DIFFATTN_API __attribute__((visibility("default")))
+#else
+#define DIFFATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { DIFFATTN_F32 = 0, DIFFATTN_BF16 = 1 } diffattn_dtype;
+
+enum {
+  DIFFATTN_OK = 0,
+  DIFFATTN_ERR_INVALID_ARG = -1, /* null pointer, negative size, head counts that do not divide */
+  DIFFATTN_ERR_UNSUPPORTED = -2, /* valid but not implemented (e.g. bf16 with an unsupported width) */
+  DIFFATTN_ERR_MISALIGNED = -3,  /* pointer or row length not 16-byte aligned (bf16 paths) */
+  DIFFATTN_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed; message has the CUDA error */
+  DIFFATTN_ERR_TIMEOUT = -5,     /* a bounded device wait expired (read via diffattn_last_status) */
+  DIFFATTN_ERR_WORKSPACE = -6    /* workspace pointer null or smaller than required */
+};
+
+/* Library version string, e.g. "diffattn 0.1 sm_100a". */
+DIFFATTN_API const char* diffattn_version(void);
+
+/* lambda_init for a 1-based layer index: 0.8 - 0.6*exp(-0.3*(layer-1)).
+ * Returns NaN for layer < 1.  Host-only, no GPU needed.
+ * Source: "Differential Transformer" (mcipr.com), section 3 工程实践. */
+DIFFATTN_API double diffattn_lambda_init(int layer);
+
+/* lambda[h] = exp(lq1[h].lk1[h]) - exp(lq2[h].lk2[h]) + lambda_init, h < heads.
+ *   lq1, lk1, lq2, lk2 : device f32 [heads, dim]
+ *   lambda_out         : device f32 [heads]
+ * Dot products are sequential fp64 sums, exp is fp64, the result is rounded
+ * once to f32.  heads, dim >= 1.
+ * Source: "差分注意力" tutorial, Step 4 (λ 参数化). */
+DIFFATTN_API int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                    int heads, int dim, double lambda_init, float* lambda_out, void* stream);
+
+/* V1-layout forward ("差分注意力" tutorial, section V1 到 V2 的 diff).
+ *   q1, q2 : [B, H,   Lq, d]      k1, k2 : [B, Hkv, Lk, d]
+ *   v      : [B, Hkv, Lk, dv]     lambda : device f32 [H]
+ *   out    : [B, H,   Lq, dv]     (same dtype as the inputs)
+ * Head h reads KV head h / (H / Hkv); H % Hkv == 0 required.
+ * rmsnorm != 0 applies y = x / sqrt(mean(x^2) + eps) over dv per row (unit
+ * weight) to the difference output.
+ * bf16: tensor-core path, requires d in {64, 128} and dv == 128.
+ * f32 : exact-softmax SIMT path, any d <= 256, dv <= 4096.
+ * Lq == 0 or B == 0 is a no-op; Lk == 0 writes zeros. */
+DIFFATTN_API int diffattn_fwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                    const float* lambda, void* out, diffattn_dtype dtype,
+                    int B, int H, int Hkv, int Lq, int Lk, int d, int dv,
+                    int causal, int rmsnorm, float eps, void* stream);
+
+/* V2-layout forward (same section).
+ *   q      : [B, Hq,  Lq, D]      k, v : [B, Hkv, Lk, D]
+ *   lambda : device f32 [Hq/2]    out  : [B, Hq/2, Lq, D]
+ * Diff pair h = Q heads (2h, 2h+1) = (map 1, map 2); both read KV head
+ * 2h / (Hq / Hkv).  Requires Hq even, Hq % Hkv == 0 and (Hq/Hkv) even so that
+ * a pair never straddles two KV groups.
+ * bf16: tensor-core path, D == 128.  f32: SIMT path, D <= 256. */
+DIFFATTN_API int diffattn_fwd_v2(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                    diffattn_dtype dtype, int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                    int causal, void* stream);
+
+/* Bytes of device workspace diffattn_decode_v2 / diffattn_decode_v1 need for
+ * a batch of B sequences, Hkv KV heads, cache length T and value width dv on
+ * the current device.  The caller allocates it (any alignment >= 16 B). */
+DIFFATTN_API size_t diffattn_decode_workspace_size(int B, int Hkv, int T, int dv);
+
+/* Single-token V2 decode over a KV cache (tutorial section V1 到 V2 的 diff:
+ * doubled Q heads, K/V read once per KV group for both maps).
+ *   q      : [B, Hq, D]           kc, vc : [B, Hkv, T, D]  (bf16)
+ *   lambda : device f32 [Hq/2]    out    : [B, Hq/2, D]
+ *   ws     : device workspace of ws_bytes >= diffattn_decode_workspace_size(B, Hkv, T, D)
+ * The new token sees every cached key.  bf16: D == 128 and Hq/Hkv in
+ * {2,4,6,8}.  f32: routed to the SIMT path (no workspace used).  Two launches
+ * (split-KV partials, then a combine) on `stream`. */
+DIFFATTN_API int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const float* lambda, void* out,
+                       diffattn_dtype dtype, int B, int Hq, int Hkv, int T, int D,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Single-token V1-layout decode: q1, q2 [B, H, d]; k1, k2 [B, Hkv, T, d];
+ * v [B, Hkv, T, dv]; lambda [H]; out [B, H, dv].  bf16: d == 64, dv == 128,
+ * H/Hkv <= 4.  K1, K2 and V are each read once for both maps (fused).
+ * fused == 0 instead runs the two maps as two passes that each read V (the
+ * "V cache loaded twice" behaviour the tutorial attributes to V1), for
+ * comparison only. */
+DIFFATTN_API int diffattn_decode_v1(const void* q1, const void* k1, const void* q2, const void* k2,
+                       const void* v, const float* lambda, void* out, diffattn_dtype dtype,
+                       int B, int H, int Hkv, int T, int d, int dv, int fused,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Message of the last error returned on this host thread ("" if none). */
+DIFFATTN_API const char* diffattn_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: DIFFATTN_OK, DIFFATTN_ERR_TIMEOUT if a kernel's bounded
+ * wait expired since the last call, or DIFFATTN_ERR_CUDA if the stream
+ * reports an error. */
+DIFFATTN_API int diffattn_last_status(void* stream);
+
+/* Upper bound, in nanoseconds, of every device-side wait (mbarrier phases
+ * between warps of one CTA).  Default 2e9 (2 s).  0 makes any wait that is
+ * not already satisfied expire at once (used to test the timeout path).
+ * Applies to launches made after the call, process-wide. */
+DIFFATTN_API void diffattn_set_wait_limit_ns(unsigned long long ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIFFATTN_H_ */

@@ -1,0 +1,88 @@
+"""The C ABI library without a GPU: it loads, exports every declared symbol,
+and rejects bad arguments before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import differential_attention_transformers_b200 as da
+from differential_attention_transformers_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "diffattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return da.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(diffattn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_symbols() == sorted(da.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    # and nothing else of ours leaks out (hidden visibility for internals)
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", da.LIB_PATH], capture_output=True, text=True).stdout
+    ours = sorted({l.split()[-1] for l in out.splitlines() if l.split()[-1].startswith("diffattn_")})
+    assert ours == declared_symbols()
+
+
+def test_version_and_lambda_init(L):
+    assert "sm_100a" in da.version()
+    assert da.lambda_init(1) == pytest.approx(0.2, abs=1e-15)
+    import math
+    for l in (1, 2, 12, 24):
+        assert da.lambda_init(l) == 0.8 - 0.6 * math.exp(-0.3 * (l - 1))
+    assert math.isnan(da.lambda_init(0))
+
+
+def test_argument_errors_before_any_device_call(L):
+    P = ctypes.c_void_p(64)  # never dereferenced: validation fails first
+    s = ctypes.c_void_p(0)
+    # Hq odd
+    assert L.diffattn_fwd_v2(P, P, P, P, P, da.BF16, 1, 3, 1, 8, 8, 128, 1, s) == da.ERR_INVALID_ARG
+    # a pair straddling two KV groups (Hq/Hkv odd)
+    assert L.diffattn_fwd_v2(P, P, P, P, P, da.BF16, 1, 6, 2, 8, 8, 128, 1, s) == da.ERR_INVALID_ARG
+    assert "Hq" in da.last_error()
+    # null pointer
+    assert L.diffattn_fwd_v2(None, P, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, s) == da.ERR_INVALID_ARG
+    # negative sizes
+    assert L.diffattn_fwd_v1(P, P, P, P, P, P, P, da.BF16, 1, 2, 1, -1, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_INVALID_ARG
+    # H not a multiple of Hkv
+    assert L.diffattn_fwd_v1(P, P, P, P, P, P, P, da.BF16, 1, 3, 2, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_INVALID_ARG
+    # unknown dtype
+    assert L.diffattn_fwd_v2(P, P, P, P, P, 7, 1, 4, 2, 8, 8, 128, 1, s) == da.ERR_INVALID_ARG
+    # unsupported bf16 widths
+    assert L.diffattn_fwd_v2(P, P, P, P, P, da.BF16, 1, 4, 2, 8, 8, 96, 1, s) == da.ERR_UNSUPPORTED
+    assert L.diffattn_fwd_v1(P, P, P, P, P, P, P, da.BF16, 1, 2, 1, 8, 8, 32, 128, 1, 0, 1e-5, s) == da.ERR_UNSUPPORTED
+    # misaligned bf16 pointer (16-byte rule of tensor-map copies)
+    Pm = ctypes.c_void_p(66)
+    assert L.diffattn_fwd_v2(Pm, P, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, s) == da.ERR_MISALIGNED
+    # lambda: bad sizes / null
+    assert L.diffattn_lambda(P, P, P, P, 0, 8, 0.2, P, s) == da.ERR_INVALID_ARG
+    assert L.diffattn_lambda(None, P, P, P, 2, 8, 0.2, P, s) == da.ERR_INVALID_ARG
+    # decode
+    assert L.diffattn_decode_v2(P, P, P, P, P, da.BF16, 1, 5, 1, 64, 128, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    assert L.diffattn_decode_v2(P, P, P, P, P, da.BF16, 1, 32, 2, 64, 128, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+    assert L.diffattn_decode_v1(P, P, P, P, P, P, P, da.BF16, 1, 16, 2, 64, 64, 128, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+
+
+def test_binding_has_no_cpu_fallback(monkeypatch):
+    """With the library missing, the product path raises instead of computing elsewhere."""
+    monkeypatch.setattr(da, "_lib", None)
+    monkeypatch.setattr(da, "LIB_PATH", "/nonexistent/libdiffattn.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        da.load()
