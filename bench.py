@@ -379,7 +379,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the batch size of the workload (smaller profiling cases)")
     args = ap.parse_args()
+    if args.batch is not None:
+        base = args.workload.replace("_unfused", "")
+        inputs.WORKLOADS[base] = inputs.with_shape(inputs.WORKLOADS[base], B=args.batch)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -442,8 +448,10 @@ def main():
             del r2
             torch.cuda.empty_cache()
 
-    e2e = e2e_measure(r, max(2, min(args.steps, 5)))
-    e2e["value"] *= world
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_measure(r, max(2, min(args.steps, 5)))
+        e2e["value"] *= world
 
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

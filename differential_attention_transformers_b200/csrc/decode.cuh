@@ -253,8 +253,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
         acc[i][0] *= al0; acc[i][2] *= al0;
         acc[i][1] *= al1; acc[i][3] *= al1;
       }
-      const uint32_t pb0 = movm_t(pack_bf16(p0, p1));
-      const uint32_t pb1 = movm_t(pack_bf16(p2, p3));
+      // P = P_hi + P_lo in bf16 (see the prefill kernel): residual MMAs keep
+      // the map difference accurate when lambda is near 1.
+      const uint32_t h01 = pack_bf16(p0, p1), h23 = pack_bf16(p2, p3);
+      const uint32_t pb0 = movm_t(h01);
+      const uint32_t pb1 = movm_t(h23);
+      const uint32_t pr0 = movm_t(pack_bf16(p0 - __uint_as_float(h01 << 16), p1 - __uint_as_float(h01 & 0xFFFF0000u)));
+      const uint32_t pr1 = movm_t(pack_bf16(p2 - __uint_as_float(h23 << 16), p3 - __uint_as_float(h23 & 0xFFFF0000u)));
       // O^T += V^T . P^T
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
@@ -264,6 +269,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
         uint32_t a0, a1, a2, a3;
         ldsm_x4_t(vb + (mt >> 2) * (DEC_TILE_BYTES / 2) + swz(row, chunk), a0, a1, a2, a3);
         mma16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+        mma16816(acc[mt], a0, a1, a2, a3, pr0, pr1);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[st]));
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
     res[mp] = l > 0.f ? o / l : 0.f;
   }
   const float lam = a.lambda[h];
-  a.out[((size_t)b * Hout + h) * 128 + t] = __float2bfloat16_rn(res[0] - lam * res[1]);
+  a.out[((size_t)b * Hout + h) * 128 + t] = __float2bfloat16_rn(__fsub_rn(res[0], __fmul_rn(lam, res[1])));
 }
 
 }  // namespace da

@@ -298,8 +298,11 @@ int diffattn_fwd_v1(const void* q1, const void* k1, const void* q2, const void* 
     return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d Lq=%d Lk=%d d=%d dv=%d)", B, H, Hkv, Lq,
                 Lk, d, dv);
   if (H % Hkv) return fail(DIFFATTN_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
-  if (!q1 || !k1 || !q2 || !k2 || !v || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   if (rmsnorm && !(eps >= 0.f)) return fail(DIFFATTN_ERR_INVALID_ARG, "eps must be >= 0");
+  if (B == 0 || Lq == 0) return ok();  // nothing to compute; pointers may be null
+  if (!q1 || !q2 || !lambda || !out || (Lk > 0 && (!k1 || !k2 || !v)))
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (Lk == 0) k1 = k2 = v = q1;  // never read: no key is visible
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == DIFFATTN_F32) {
     if (d > SIMT_MAXD || dv > SIMT_MAXCOL * SIMT_THREADS)
@@ -325,7 +328,9 @@ int diffattn_fwd_v2(const void* q, const void* k, const void* v, const float* la
     return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d Lq=%d Lk=%d D=%d)", B, Hq, Hkv, Lq, Lk, D);
   if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
     return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
-  if (!q || !k || !v || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (B == 0 || Lq == 0) return ok();  // nothing to compute; pointers may be null
+  if (!q || !lambda || !out || (Lk > 0 && (!k || !v))) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (Lk == 0) k = v = q;  // never read: no key is visible
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == DIFFATTN_F32) {
     if (D > SIMT_MAXD) return fail(DIFFATTN_ERR_UNSUPPORTED, "f32 path supports D <= %d", SIMT_MAXD);
@@ -355,7 +360,9 @@ int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const floa
     return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d T=%d D=%d)", B, Hq, Hkv, T, D);
   if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
     return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
-  if (!q || !kc || !vc || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (B == 0) return ok();
+  if (!q || !lambda || !out || (T > 0 && (!kc || !vc))) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (T == 0) kc = vc = q;  // never read: the cache is empty
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == DIFFATTN_F32)
     return diffattn_fwd_v2(q, kc, vc, lambda, out, dtype, B, Hq, Hkv, 1, T, D, 1, stream);
@@ -373,7 +380,10 @@ int diffattn_decode_v1(const void* q1, const void* k1, const void* q2, const voi
   if (B < 0 || H < 1 || Hkv < 1 || T < 0 || d < 1 || dv < 1)
     return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d T=%d d=%d dv=%d)", B, H, Hkv, T, d, dv);
   if (H % Hkv) return fail(DIFFATTN_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
-  if (!q1 || !k1 || !q2 || !k2 || !v || !lambda || !out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (B == 0) return ok();
+  if (!q1 || !q2 || !lambda || !out || (T > 0 && (!k1 || !k2 || !v)))
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (T == 0) k1 = k2 = v = q1;  // never read: the cache is empty
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == DIFFATTN_F32)
     return diffattn_fwd_v1(q1, k1, q2, k2, v, lambda, out, dtype, B, H, Hkv, 1, T, d, dv, 1, 0, 0.f, stream);

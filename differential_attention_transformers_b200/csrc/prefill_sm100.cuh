@@ -16,9 +16,10 @@
 //   warp  8    TMA producer; allocates / frees TMEM
 //   warp  9    MMA issuer (one thread)
 // TMEM (512 columns): S1 [0,128) S2 [128,256) O1 [256,384) O2 [384,512).
-// P_m (bf16, 64 columns) overwrites the first half of S_m after the softmax
-// has read S_m; the MMA issuer orders "PV_m(j) then S_m(j+1)" so the tensor
-// pipe reads P_m before it writes the next S_m.
+// P_m is stored as two bf16 halves, P_hi in columns [0,64) and the residual
+// P_lo = P - P_hi in [64,128) of S_m, after the softmax has read S_m; both
+// accumulate into O_m.  The MMA issuer orders "PV_m(j) then S_m(j+1)" so the
+// tensor pipe reads P_m before it writes the next S_m.
 // Shared memory: Q1, Q2 tiles, then NS stages of {K tile(s), V tile}; every
 // tile is a set of 128-row x 128-byte boxes in the TMA 128-byte swizzle,
 // which is the canonical K-major (Q, K) / MN-major (V) UMMA layout.
@@ -195,6 +196,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 #pragma unroll
         for (int s = 0; s < PF_BN / 16; ++s)
           mma_ts(tO[m], tS[m] + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, (j > 0 || s > 0));
+#pragma unroll
+        for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
+          mma_ts(tO[m], tS[m] + 64 + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, 1);
       };
       if (ok) {
         tc_fence_after();
@@ -268,14 +272,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         m_run = mxs;
       }
       const float mu = m_run == -INFINITY ? 0.f : m_run;
+      // P = P_hi + P_lo, both bf16: the residual keeps ~16 bits of P, so the
+      // difference O1/l1 - lambda*O2/l2 does not amplify P's rounding when the
+      // two maps are close and lambda is near 1.
       float sum = 0.f;
-      uint32_t pk[PF_BN / 2];
+      uint32_t pk[PF_BN / 2], pl[PF_BN / 2];
 #pragma unroll
       for (int c = 0; c < PF_BN; c += 2) {
         const float p0 = ex2(fmaf(s[c], a.scale_log2, -mu));
         const float p1 = ex2(fmaf(s[c + 1], a.scale_log2, -mu));
         sum += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
+        const uint32_t hi = pack_bf16(p0, p1);
+        pk[c / 2] = hi;
+        pl[c / 2] = pack_bf16(p0 - __uint_as_float(hi << 16), p1 - __uint_as_float(hi & 0xFFFF0000u));
       }
       l_run = l_run * alpha + sum;
       // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs it
@@ -295,6 +304,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       }
       tmem_st32p(tS, pk);
       tmem_st32p(tS + 32, pk + 32);
+      tmem_st32p(tS + 64, pl);
+      tmem_st32p(tS + 96, pl + 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&S.p_full[m]));
@@ -324,7 +335,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            y[c * 32 + i] = __uint_as_float(o1[i]) * c1 - __uint_as_float(o2[i]) * c2;
+            y[c * 32 + i] = __fsub_rn(__fmul_rn(__uint_as_float(o1[i]), c1), __fmul_rn(__uint_as_float(o2[i]), c2));
         }
         have = true;
         if (a.rms) {
