@@ -72,9 +72,9 @@ def test_v1_prefill_full_sampled(v1_prefill):
         ref = orc.diffattn_v1(sl(x["q1"]), sl(x["k1"]), sl(x["q2"]), sl(x["k2"]), sl(x["v"]), lref[h:h + 1],
                               causal=True, rms=True, eps=1e-5)
         assert rel_err(out[b:b + 1, h:h + 1], ref) <= BF16_TOL, (b, h)
-    # RMSNorm: every row has mean square ms/(ms+eps) < 1, close to 1 here
+    # RMSNorm: every row's mean square is ms/(ms+eps) <= 1 (bf16 output rounding aside)
     msq = (out.float() ** 2).mean(dim=-1)
-    assert torch.all(msq < 1.02) and torch.all(msq > 0.9)
+    assert torch.all(msq <= 1.0 + 2e-2)
 
 
 def test_v2_decode_full_all_heads():
