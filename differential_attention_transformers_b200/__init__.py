@@ -27,7 +27,7 @@ F32, BF16 = 0, 1
 
 EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffattn_fwd_v1", "diffattn_fwd_v2",
            "diffattn_decode_workspace_size", "diffattn_decode_v2", "diffattn_decode_v1", "diffattn_last_error",
-           "diffattn_last_status", "diffattn_set_wait_limit_ns"]
+           "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc"]
 
 _lib = None
 
@@ -60,6 +60,7 @@ def load():
         "diffattn_last_error": (ctypes.c_char_p, []),
         "diffattn_last_status": (I, [P]),
         "diffattn_set_wait_limit_ns": (None, [U]),
+        "diffattn_decode_v2_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

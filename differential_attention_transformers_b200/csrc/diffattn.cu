@@ -252,6 +252,32 @@ int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2
   return ok();
 }
 
+// Scratch for diffattn_decode_v2_noalloc: split-KV partial records of the
+// decode, for callers that cannot allocate device memory.  One copy per
+// device, reserved when the library is loaded and kept until exit.  Host code
+// must not pass `g_noalloc_scratch` itself to a kernel (on the host it names a
+// stand-in, not device memory): it uses the address looked up below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DIFFATTN_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Once per device, with that device current: the device address of the scratch.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(DIFFATTN_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(DIFFATTN_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DIFFATTN_OK;
+}
+
 }  // namespace
 
 // ============================================================================
@@ -372,6 +398,25 @@ int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const floa
                 Hkv);
   if (int e = check_bf16_ptrs({q, kc, vc, out})) return e;
   return launch_decode(q, nullptr, kc, nullptr, vc, lambda, out, B, Hq, Hkv, T, false, 1, ws, ws_bytes, s);
+}
+
+int diffattn_decode_v2_noalloc(const void* q, const void* kc, const void* vc, const float* lambda, void* out,
+                               diffattn_dtype dtype, int B, int Hq, int Hkv, int T, int D, void* stream) {
+  if (B < 0 || Hq < 2 || Hkv < 1 || T < 0 || D < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d T=%d D=%d)", B, Hq, Hkv, T, D);
+  if (dtype == DIFFATTN_BF16 && B > 0) {
+    DeviceInfo* dev = nullptr;
+    if (int e = device_setup(&dev)) return e;
+    const size_t need = plan_decode(dev->sms, B, Hkv, T).bytes_per_pass;
+    if (need > DIFFATTN_NOALLOC_SCRATCH_BYTES)
+      return fail(DIFFATTN_ERR_UNSUPPORTED,
+                  "decode needs %zu B of partial records, above the %u B scratch of the no-allocation entry point",
+                  need, (unsigned)DIFFATTN_NOALLOC_SCRATCH_BYTES);
+  }
+  void* scratch = nullptr;
+  if (int e = noalloc_scratch(&scratch)) return e;
+  return diffattn_decode_v2(q, kc, vc, lambda, out, dtype, B, Hq, Hkv, T, D, scratch,
+                            DIFFATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int diffattn_decode_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,

@@ -154,6 +154,34 @@ DIFFATTN_API int diffattn_last_status(void* stream);
  * Applies to launches made after the call, process-wide. */
 DIFFATTN_API void diffattn_set_wait_limit_ns(unsigned long long ns);
 
+/* Maximum scratch, in bytes, that diffattn_decode_v2_noalloc can use. */
+#define DIFFATTN_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* Single-token V2 decode that allocates nothing and takes no workspace.
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot call cudaMalloc, e.g. code running inside a memory pool or an
+ * allocator hook that must not re-enter the allocator, or a runtime that owns
+ * all device memory and hands this library only its tensors.
+ * Arguments, layouts and results are those of diffattn_decode_v2 without
+ * `ws` / `ws_bytes`: the split-KV partial records live instead in a scratch
+ * array of DIFFATTN_NOALLOC_SCRATCH_BYTES (4 MiB) that the library reserves in
+ * device memory on every GPU that loads it, until the process exits.
+ *   - Sizes whose partial records need more than that (see
+ *     diffattn_decode_workspace_size; about 2.5 MB for 16 sequences x 8 KV
+ *     heads x 65536 tokens) return DIFFATTN_ERR_UNSUPPORTED before any launch.
+ *   - The first call on a device does a one-time set-up on that device (the
+ *     scratch address and kernel attributes are looked up); make that first
+ *     call before any stream capture.
+ *   - Every call on a device shares the one scratch array, and it keeps the
+ *     last call's contents.  Nothing in it needs to start at zero: each call
+ *     writes every record it later reads.  Calls that can overlap on the GPU
+ *     (different streams without ordering between them) race on the scratch
+ *     and produce wrong results; serialise them on one stream.
+ *   - No cudaMalloc, cudaFree or any other allocating call is made. */
+DIFFATTN_API int diffattn_decode_v2_noalloc(const void* q, const void* kc, const void* vc, const float* lambda,
+                                            void* out, diffattn_dtype dtype, int B, int Hq, int Hkv, int T,
+                                            int D, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
