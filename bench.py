@@ -250,11 +250,18 @@ def time_runner(r, steps, warmup, dist_on):
 
 
 def max_over_ranks(x, dist_on):
+    """Max of a per-rank time over all ranks (the slowest rank sets the step time)."""
     if not dist_on:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(work_per_rank, world, ms_per_step):
+    """Whole-job throughput: every rank processes its own batch (weak scaling)."""
+    return work_per_rank * world / (ms_per_step / 1e3)
 
 
 def e2e_measure(r, steps):
@@ -430,7 +437,7 @@ def main():
     total_ms = max_over_ranks(total_ms, dist_on)
     ms = total_ms / args.steps
     work, unit = r.work()
-    value = work * world / (ms / 1e3)
+    value = aggregate(work, world, ms)
     rf = roofline(r, kern_ms, peaks)
 
     secondary = {}
