@@ -22,6 +22,11 @@
 
 using namespace da;
 
+// |1 - lambda| below which the prefill keeps the bf16 residual of P (see PrefillArgs).
+#ifndef DIFFATTN_RESID_TAU
+#define DIFFATTN_RESID_TAU 0.25f
+#endif
+
 // Device status word (timeouts of bounded waits), one per device.
 __device__ unsigned g_diffattn_status;
 
@@ -173,6 +178,7 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.eps = eps;
   a.scale_log2 = log2e_over_sqrt(dqk);
   a.n_rb = (Lq + PF_BM - 1) / PF_BM;
+  a.resid_tau = DIFFATTN_RESID_TAU;
   a.watch = make_watch(dev);
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");

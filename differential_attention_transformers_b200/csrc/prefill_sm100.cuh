@@ -45,6 +45,12 @@ struct PrefillArgs {
   int causal, rms;
   float eps, scale_log2;
   int n_rb;             // row blocks per head
+  // Precision policy: P is stored as bf16 P_hi plus a bf16 residual P_lo (a
+  // second PV MMA) for heads with |1 - lambda| < resid_tau.  The difference
+  // O1/l1 - lambda*O2/l2 amplifies P's bf16 rounding (2^-9) by about
+  // (1+|lambda|)/|1-lambda| when the two maps are alike; below resid_tau that
+  // factor would exceed ~8 and the residual restores ~2^-17.
+  float resid_tau;
   Watch watch;
 };
 
@@ -77,7 +83,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 template <int DQK>
-__global__ void __launch_bounds__(PF_THREADS, 1)
+__global__ void __maxnreg__(200)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
                const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
@@ -179,6 +185,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       const uint32_t tS[2] = {tmem + 0, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
       const uint32_t sq[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
+      const bool resid = fabsf(1.f - a.lambda[h]) < a.resid_tau;
       bool ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
       auto issue_qk = [&](int m, int j) {
         const int st = j % PF_NS;
@@ -196,9 +203,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 #pragma unroll
         for (int s = 0; s < PF_BN / 16; ++s)
           mma_ts(tO[m], tS[m] + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, (j > 0 || s > 0));
+        if (resid) {
 #pragma unroll
-        for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
-          mma_ts(tO[m], tS[m] + 64 + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, 1);
+          for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
+            mma_ts(tO[m], tS[m] + 64 + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, 1);
+        }
       };
       if (ok) {
         tc_fence_after();
@@ -240,6 +249,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     const int rg = r0 + r;                   // query row
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + m * 128;
+    const bool resid = fabsf(1.f - a.lambda[h]) < a.resid_tau;
     // last visible key of this row
     const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
     float m_run = -INFINITY, l_run = 0.f;
@@ -262,9 +272,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         for (int c = 0; c < PF_BN; ++c)
           if (c > lim) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      // row max: four independent 3-input max chains (short dependency chains)
+      float mx;
+      {
+        float c0 = s[0], c1 = s[1], c2 = s[2], c3 = s[3];
 #pragma unroll
-      for (int c = 1; c < PF_BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 4; c < PF_BN; c += 8) {
+          c0 = fmax3(c0, s[c], s[c + 1]);
+          c1 = fmax3(c1, s[c + 2], s[c + 3]);
+          c2 = fmax3(c2, s[c + 4], s[c + 5]);
+          c3 = fmax3(c3, s[c + 6], s[c + 7]);
+        }
+        mx = fmax3(c0, c1, fmaxf(c2, c3));
+      }
       const float mxs = mx * a.scale_log2;
       float alpha = 1.f;
       if (mxs > m_run + PF_RESCALE_THRESHOLD) {
@@ -272,20 +292,38 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         m_run = mxs;
       }
       const float mu = m_run == -INFINITY ? 0.f : m_run;
-      // P = P_hi + P_lo, both bf16: the residual keeps ~16 bits of P, so the
-      // difference O1/l1 - lambda*O2/l2 does not amplify P's rounding when the
-      // two maps are close and lambda is near 1.
-      float sum = 0.f;
-      uint32_t pk[PF_BN / 2], pl[PF_BN / 2];
+      // P = P_hi (+ P_lo), bf16.  With the residual P_lo = P - P_hi the MMA sees
+      // ~16 bits of P, so O1/l1 - lambda*O2/l2 does not amplify P's rounding
+      // when lambda is near 1 (see resid in PrefillArgs).
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nm2 = make_float2(-mu, -mu);
+      const float2 neg1 = make_float2(-1.f, -1.f);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // Two halves of 64 keys; each half's P words go to TMEM as soon as they
+      // are ready (keeps register pressure down; the stores are asynchronous).
 #pragma unroll
-      for (int c = 0; c < PF_BN; c += 2) {
-        const float p0 = ex2(fmaf(s[c], a.scale_log2, -mu));
-        const float p1 = ex2(fmaf(s[c + 1], a.scale_log2, -mu));
-        sum += p0 + p1;
-        const uint32_t hi = pack_bf16(p0, p1);
-        pk[c / 2] = hi;
-        pl[c / 2] = pack_bf16(p0 - __uint_as_float(hi << 16), p1 - __uint_as_float(hi & 0xFFFF0000u));
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32], pl[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = half * 64 + 2 * i;
+          const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
+          const float2 p = make_float2(ex2(x.x), ex2(x.y));
+          acc[i & 3] = __fadd2_rn(acc[i & 3], p);
+          const uint32_t hi = pack_bf16(p.x, p.y);
+          pk[i] = hi;
+          if (resid) {
+            const float2 h = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
+            const float2 lo = __ffma2_rn(h, neg1, p);   // p - h, exact
+            pl[i] = pack_bf16(lo.x, lo.y);
+          }
+        }
+        tmem_st32p(tS + half * 32, pk);
+        if (resid) tmem_st32p(tS + 64 + half * 32, pl);
       }
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a03 = __fadd2_rn(a01, a23);
+      const float sum = a03.x + a03.y;
       l_run = l_run * alpha + sum;
       // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs it
       // (rows whose alpha is 1 multiply by 1).
@@ -302,10 +340,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           tmem_st32p(tO + c * 32, rr);
         }
       }
-      tmem_st32p(tS, pk);
-      tmem_st32p(tS + 32, pk + 32);
-      tmem_st32p(tS + 64, pl);
-      tmem_st32p(tS + 96, pl + 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&S.p_full[m]));
