@@ -166,6 +166,12 @@ __device__ __forceinline__ void tmem_st32p(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8p(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // UMMA shared-memory matrix descriptor (sm_100 format): start address,
 // leading/stride byte offsets (16-byte units), version 1 at bits 46-47,
 // swizzle mode at bits 61-63 (2 = 128-byte swizzle).

@@ -83,7 +83,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 template <int DQK>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
                const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
@@ -299,14 +299,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       const float2 nm2 = make_float2(-mu, -mu);
       const float2 neg1 = make_float2(-1.f, -1.f);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      // Two halves of 64 keys; each half's P words go to TMEM as soon as they
-      // are ready (keeps register pressure down; the stores are asynchronous).
+      // Chunks of 16 keys; each chunk's P words go to TMEM as soon as they are
+      // ready (keeps register pressure down; the stores are asynchronous).
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32], pl[32];
+      for (int ch = 0; ch < PF_BN / 16; ++ch) {
+        uint32_t pk[8], pl[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = half * 64 + 2 * i;
+        for (int i = 0; i < 8; ++i) {
+          const int c = ch * 16 + 2 * i;
           const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
           const float2 p = make_float2(ex2(x.x), ex2(x.y));
           acc[i & 3] = __fadd2_rn(acc[i & 3], p);
@@ -318,8 +318,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
             pl[i] = pack_bf16(lo.x, lo.y);
           }
         }
-        tmem_st32p(tS + half * 32, pk);
-        if (resid) tmem_st32p(tS + 64 + half * 32, pl);
+        tmem_st8p(tS + ch * 8, pk);
+        if (resid) tmem_st8p(tS + 64 + ch * 8, pl);
       }
       const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
       const float2 a03 = __fadd2_rn(a01, a23);
