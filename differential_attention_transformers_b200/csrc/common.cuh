@@ -71,6 +71,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          const Watch& w) {
   if (mbar_test(bar, parity)) return true;
+  if (w.limit != 0) {
+    // Fast path: a few hardware-suspending polls before touching the clock.
+    for (int i = 0; i < 8; ++i)
+      if (mbar_try(bar, parity)) return true;
+  }
   const uint64_t t0 = globaltimer();
   while (true) {
     if (*abort_flag) return false;

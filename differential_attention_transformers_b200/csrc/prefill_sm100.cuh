@@ -15,26 +15,32 @@
 //   warps 4-7  softmax of map 2
 //   warp  8    TMA producer; allocates / frees TMEM
 //   warp  9    MMA issuer (one thread)
-// TMEM (512 columns): S1 [0,128) S2 [128,256) O1 [256,384) O2 [384,512).
-// P_m is stored as two bf16 halves, P_hi in columns [0,64) and the residual
-// P_lo = P - P_hi in [64,128) of S_m, after the softmax has read S_m; both
-// accumulate into O_m.  The MMA issuer orders "PV_m(j) then S_m(j+1)" so the
-// tensor pipe reads P_m before it writes the next S_m.
-// Shared memory: Q1, Q2 tiles, then NS stages of {K tile(s), V tile}; every
-// tile is a set of 128-row x 128-byte boxes in the TMA 128-byte swizzle,
-// which is the canonical K-major (Q, K) / MN-major (V) UMMA layout.
+// Keys are processed in tiles of 64.  TMEM (512 columns) holds two S buffers
+// per map -- S1[0] [0,64) S1[1] [64,128) S2[0] [128,192) S2[1] [192,256) --
+// and the accumulators O1 [256,384) O2 [384,512).  While a map's softmax works
+// on tile j in one buffer, the tensor pipe computes S for tile j+1 into the
+// other, so each map's softmax runs back to back.  P_m(j) is written over
+// S_m(j) as bf16 P_hi in the buffer's columns [0,32) and, for heads that need
+// it, the bf16 residual P_lo = P - P_hi in [32,64); both accumulate into O_m.
+// The MMA issuer orders "PV_m(j) then S_m(j+2)" into the same buffer, so the
+// tensor pipe reads P_m(j) before it overwrites it.
+// Shared memory: Q1, Q2 tiles (128 rows), then NS stages of {K tile(s), V
+// tile} of 64 keys; every tile is a set of boxes of 128-byte rows in the TMA
+// 128-byte swizzle, which is the canonical K-major (Q, K) / MN-major (V) UMMA
+// layout.
 #pragma once
 
 #include "common.cuh"
 
 namespace da {
 
-constexpr int PF_BM = 128;        // query rows per CTA
-constexpr int PF_BN = 128;        // keys per tile
-constexpr int PF_DV = 128;        // value width
-constexpr int PF_NS = 2;          // K/V pipeline stages
+constexpr int PF_BM = 128;         // query rows per CTA
+constexpr int PF_BN = 64;          // keys per tile
+constexpr int PF_DV = 128;         // value width
+constexpr int PF_NS = 4;           // K/V pipeline stages
 constexpr int PF_THREADS = 320;
-constexpr int PF_BOX = 128 * 128; // bytes of one 128-row x 64-element bf16 box
+constexpr int PF_QBOX = 128 * 128; // bytes of one 128-row x 64-element bf16 box (Q)
+constexpr int PF_KBOX = 64 * 128;  // bytes of one 64-row x 64-element bf16 box (K, V)
 constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 struct PrefillArgs {
@@ -58,15 +64,16 @@ template <int DQK>
 struct PfSmem {
   static constexpr int QTILE = PF_BM * DQK * 2;  // bytes of one Q tile
   alignas(1024) uint8_t q[2][QTILE];
-  alignas(1024) uint8_t k[PF_NS][2 * PF_BOX];   // V2: K tile (2 boxes); V1: K1 box, K2 box
-  alignas(1024) uint8_t v[PF_NS][2 * PF_BOX];   // V tile, dv 0-63 box then 64-127 box
+  alignas(1024) uint8_t k[PF_NS][2 * PF_KBOX];   // V2: K tile (dims 0-63 box, 64-127 box); V1: K1 box, K2 box
+  alignas(1024) uint8_t v[PF_NS][2 * PF_KBOX];   // V tile, dv 0-63 box then 64-127 box
   float l[2][PF_BM];
   float ss[2][PF_BM];
   alignas(8) uint64_t q_full;
   uint64_t kv_full[PF_NS];
   uint64_t kv_empty[PF_NS];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[2][2];  // [map][buffer]
+  uint64_t p_full[2][2];
+  uint64_t o_done[2];     // PV_m(j) complete (one phase per tile)
   uint64_t o_final;
   uint64_t xl;      // epilogue exchange of l (256 arrivals)
   uint64_t xs;      // epilogue exchange of RMS partial sums (256 arrivals)
@@ -109,6 +116,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
   long long kend = a.causal ? (long long)min(r0 + PF_BM, a.Lq) - 1 + (a.Lk - a.Lq) + 1 : a.Lk;
   kend = max(0LL, min(kend, (long long)a.Lk));
   const int nT = (int)((kend + PF_BN - 1) / PF_BN);
+  const bool resid = fabsf(1.f - a.lambda[h]) < a.resid_tau;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&S.q_full), 1);
@@ -117,8 +125,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       mbar_init(smem_u32(&S.kv_empty[i]), 1);
     }
     for (int m = 0; m < 2; ++m) {
-      mbar_init(smem_u32(&S.s_full[m]), 1);
-      mbar_init(smem_u32(&S.p_full[m]), 128);
+      for (int bb = 0; bb < 2; ++bb) {
+        mbar_init(smem_u32(&S.s_full[m][bb]), 1);
+        mbar_init(smem_u32(&S.p_full[m][bb]), 128);
+      }
+      mbar_init(smem_u32(&S.o_done[m]), 1);
     }
     mbar_init(smem_u32(&S.o_final), 1);
     mbar_init(smem_u32(&S.xl), 256);
@@ -144,33 +155,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       const uint32_t qb = smem_u32(&S.q_full);
       mbar_expect_tx(qb, 2 * PfSmem<DQK>::QTILE);
       for (int x = 0; x < QBOXES; ++x) {
-        tma_load_3d(smem_u32(S.q[0]) + x * PF_BOX, &tmQ1, qb, 64 * x, r0, zq1);
-        tma_load_3d(smem_u32(S.q[1]) + x * PF_BOX, &tmQ2, qb, 64 * x, r0, zq2);
+        tma_load_3d(smem_u32(S.q[0]) + x * PF_QBOX, &tmQ1, qb, 64 * x, r0, zq1);
+        tma_load_3d(smem_u32(S.q[1]) + x * PF_QBOX, &tmQ2, qb, 64 * x, r0, zq2);
       }
       int last_use[PF_NS];
       for (int i = 0; i < PF_NS; ++i) last_use[i] = -1;
-      bool ok = true;
       for (int j = 0; j < nT; ++j) {
         const int st = j % PF_NS, use = j / PF_NS;
-        if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) {
-          ok = false;
-          break;
-        }
+        if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
         const uint32_t fb = smem_u32(&S.kv_full[st]);
-        mbar_expect_tx(fb, 4 * PF_BOX);
+        mbar_expect_tx(fb, 4 * PF_KBOX);
         const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
         if (a.v1) {
           tma_load_3d(kd, &tmK1, fb, 0, j * PF_BN, zkv);
-          tma_load_3d(kd + PF_BOX, &tmK2, fb, 0, j * PF_BN, zkv);
+          tma_load_3d(kd + PF_KBOX, &tmK2, fb, 0, j * PF_BN, zkv);
         } else {
           tma_load_3d(kd, &tmK1, fb, 0, j * PF_BN, zkv);
-          tma_load_3d(kd + PF_BOX, &tmK1, fb, 64, j * PF_BN, zkv);
+          tma_load_3d(kd + PF_KBOX, &tmK1, fb, 64, j * PF_BN, zkv);
         }
         tma_load_3d(vd, &tmV, fb, 0, j * PF_BN, zkv);
-        tma_load_3d(vd + PF_BOX, &tmV, fb, 64, j * PF_BN, zkv);
+        tma_load_3d(vd + PF_KBOX, &tmV, fb, 64, j * PF_BN, zkv);
         last_use[st] = use;
       }
-      (void)ok;
       // Every copy issued must have landed before the CTA may exit (returns at
       // once when the consumer has already seen the phase).
       drain_bar(qb, 0, a.watch.status);
@@ -182,59 +188,60 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     if (lane == 0 && nT > 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, PF_BN, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, PF_DV, true);
-      const uint32_t tS[2] = {tmem + 0, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 384};
-      const uint32_t sq[2] = {smem_u32(S.q[0]), smem_u32(S.q[1])};
-      const bool resid = fabsf(1.f - a.lambda[h]) < a.resid_tau;
-      bool ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
+      const uint32_t sq0 = smem_u32(S.q[0]), sq1 = smem_u32(S.q[1]);
+      auto tS = [&](int m, int bb) { return tmem + (uint32_t)(m * 128 + bb * 64); };
       auto issue_qk = [&](int m, int j) {
         const int st = j % PF_NS;
-        const uint32_t kb = smem_u32(S.k[st]) + (a.v1 ? m * PF_BOX : 0);
+        const uint32_t kb = smem_u32(S.k[st]) + (a.v1 ? m * PF_KBOX : 0);
+        const uint32_t qb = m ? sq1 : sq0;
+        const uint32_t d = tS(m, j & 1);
 #pragma unroll
         for (int s = 0; s < DQK / 16; ++s) {
-          const uint32_t off = (s >> 2) * PF_BOX + (s & 3) * 32;
-          mma_ss(tS[m], umma_desc(sq[m] + off, 16, 1024), umma_desc(kb + off, 16, 1024), IDESC_QK, s > 0);
+          const uint32_t kin = (s & 3) * 32;
+          mma_ss(d, umma_desc(qb + (s >> 2) * PF_QBOX + kin, 16, 1024),
+                 umma_desc(kb + (s >> 2) * PF_KBOX + kin, 16, 1024), IDESC_QK, s > 0);
         }
-        mma_commit(smem_u32(&S.s_full[m]));
+        mma_commit(smem_u32(&S.s_full[m][j & 1]));
       };
       auto issue_pv = [&](int m, int j) {
-        const int st = j % PF_NS;
-        const uint32_t vb = smem_u32(S.v[st]);
+        const uint32_t vb = smem_u32(S.v[j % PF_NS]);
+        const uint32_t p = tS(m, j & 1), o = tmem + 256 + m * 128;
 #pragma unroll
         for (int s = 0; s < PF_BN / 16; ++s)
-          mma_ts(tO[m], tS[m] + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, (j > 0 || s > 0));
+          mma_ts(o, p + s * 8, umma_desc(vb + s * 2048, PF_KBOX, 1024), IDESC_PV, (j > 0 || s > 0));
         if (resid) {
 #pragma unroll
           for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
-            mma_ts(tO[m], tS[m] + 64 + s * 8, umma_desc(vb + s * 2048, PF_BOX, 1024), IDESC_PV, 1);
+            mma_ts(o, p + 32 + s * 8, umma_desc(vb + s * 2048, PF_KBOX, 1024), IDESC_PV, 1);
         }
+        mma_commit(smem_u32(&S.o_done[m]));
       };
-      if (ok) {
+      auto kv_ready = [&](int j) {
+        return wait_bar(smem_u32(&S.kv_full[j % PF_NS]), (j / PF_NS) & 1, abort_flag, a.watch);
+      };
+      bool ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
+      for (int j0 = 0; ok && j0 < 2 && j0 < nT; ++j0) {
+        if (!(ok = kv_ready(j0))) break;
         tc_fence_after();
-        ok = wait_bar(smem_u32(&S.kv_full[0]), 0, abort_flag, a.watch);
-        if (ok) {
-          tc_fence_after();
-          issue_qk(0, 0);
-          issue_qk(1, 0);
-        }
+        issue_qk(0, j0);
+        issue_qk(1, j0);
       }
       for (int j = 0; ok && j < nT; ++j) {
-        const int st = j % PF_NS;
-        const bool more = j + 1 < nT;
-        if (!(ok = wait_bar(smem_u32(&S.p_full[0]), j & 1, abort_flag, a.watch))) break;
+        const int bb = j & 1, ph = (j >> 1) & 1;
+        const bool more = j + 2 < nT;
+        if (!(ok = wait_bar(smem_u32(&S.p_full[0][bb]), ph, abort_flag, a.watch))) break;
         tc_fence_after();
         issue_pv(0, j);
         if (more) {
-          if (!(ok = wait_bar(smem_u32(&S.kv_full[(j + 1) % PF_NS]), ((j + 1) / PF_NS) & 1, abort_flag, a.watch)))
-            break;
+          if (!(ok = kv_ready(j + 2))) break;
           tc_fence_after();
-          issue_qk(0, j + 1);
+          issue_qk(0, j + 2);
         }
-        if (!(ok = wait_bar(smem_u32(&S.p_full[1]), j & 1, abort_flag, a.watch))) break;
+        if (!(ok = wait_bar(smem_u32(&S.p_full[1][bb]), ph, abort_flag, a.watch))) break;
         tc_fence_after();
         issue_pv(1, j);
-        mma_commit(smem_u32(&S.kv_empty[st]));
-        if (more) issue_qk(1, j + 1);
+        mma_commit(smem_u32(&S.kv_empty[j % PF_NS]));
+        if (more) issue_qk(1, j + 2);
       }
       if (ok) mma_commit(smem_u32(&S.o_final));
       // Every MMA issued must have completed before TMEM is freed.
@@ -248,20 +255,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     const int r = threadIdx.x & 127;         // row within the block
     const int rg = r0 + r;                   // query row
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + m * 128;
-    const bool resid = fabsf(1.f - a.lambda[h]) < a.resid_tau;
+    const uint32_t tO = tmem + lane_off + 256 + m * 128;
     // last visible key of this row
     const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    const float2 neg1 = make_float2(-1.f, -1.f);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nT; ++j) {
-      if (!(ok = warp_wait(smem_u32(&S.s_full[m]), j & 1, abort_flag, a.watch))) break;
+      const int bb = j & 1;
+      const uint32_t tS = tmem + lane_off + m * 128 + bb * 64;
+      if (!(ok = warp_wait(smem_u32(&S.s_full[m][bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
       tc_fence_after();
       float s[PF_BN];
       {
         uint32_t rr[PF_BN];
-#pragma unroll
-        for (int c = 0; c < PF_BN / 32; ++c) tmem_ld32p(tS + c * 32, rr + c * 32);
+        tmem_ld32p(tS, rr);
+        tmem_ld32p(tS + 32, rr + 32);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < PF_BN; ++i) s[i] = __uint_as_float(rr[i]);
@@ -272,12 +282,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         for (int c = 0; c < PF_BN; ++c)
           if (c > lim) s[c] = -INFINITY;
       }
-      // row max: four independent 3-input max chains (short dependency chains)
+      // row max: four independent 3-input max chains
       float mx;
       {
-        float c0 = s[0], c1 = s[1], c2 = s[2], c3 = s[3];
+        float c0 = fmaxf(s[0], s[1]), c1 = fmaxf(s[2], s[3]), c2 = fmaxf(s[4], s[5]), c3 = fmaxf(s[6], s[7]);
 #pragma unroll
-        for (int c = 4; c < PF_BN; c += 8) {
+        for (int c = 8; c < PF_BN; c += 8) {
           c0 = fmax3(c0, s[c], s[c + 1]);
           c1 = fmax3(c1, s[c + 2], s[c + 3]);
           c2 = fmax3(c2, s[c + 4], s[c + 5]);
@@ -292,12 +302,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         m_run = mxs;
       }
       const float mu = m_run == -INFINITY ? 0.f : m_run;
-      // P = P_hi (+ P_lo), bf16.  With the residual P_lo = P - P_hi the MMA sees
-      // ~16 bits of P, so O1/l1 - lambda*O2/l2 does not amplify P's rounding
-      // when lambda is near 1 (see resid in PrefillArgs).
-      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
       const float2 nm2 = make_float2(-mu, -mu);
-      const float2 neg1 = make_float2(-1.f, -1.f);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       // Chunks of 16 keys; each chunk's P words go to TMEM as soon as they are
       // ready (keeps register pressure down; the stores are asynchronous).
@@ -313,23 +318,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           const uint32_t hi = pack_bf16(p.x, p.y);
           pk[i] = hi;
           if (resid) {
-            const float2 h = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
-            const float2 lo = __ffma2_rn(h, neg1, p);   // p - h, exact
+            const float2 hf = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
+            const float2 lo = __ffma2_rn(hf, neg1, p);   // p - hi, exact
             pl[i] = pack_bf16(lo.x, lo.y);
           }
         }
         tmem_st8p(tS + ch * 8, pk);
-        if (resid) tmem_st8p(tS + 64 + ch * 8, pl);
+        if (resid) tmem_st8p(tS + 32 + ch * 8, pl);
       }
       const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
       const float2 a03 = __fadd2_rn(a01, a23);
-      const float sum = a03.x + a03.y;
-      l_run = l_run * alpha + sum;
-      // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs it
-      // (rows whose alpha is 1 multiply by 1).
+      l_run = l_run * alpha + (a03.x + a03.y);
+      // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs
+      // it (rows whose alpha is 1 multiply by 1).  O_m must be complete first:
+      // wait for PV_m(j-1) (o_done phase j-1; PV_m(j-2) is known complete since
+      // S_m(j) was issued after it, so the parity is unambiguous).
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        // O_m(j-1) is complete: S_m(j) was committed after PV_m(j-1).
-        const uint32_t tO = tmem + lane_off + 256 + m * 128;
+        if (!(ok = warp_wait(smem_u32(&S.o_done[m]), (j - 1) & 1, abort_flag, a.watch))) break;
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < PF_DV / 32; ++c) {
           uint32_t rr[32];
@@ -342,7 +348,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&S.p_full[m]));
+      mbar_arrive(smem_u32(&S.p_full[m][bb]));
     }
 
     // --------------------------------------------------------- epilogue --
