@@ -22,8 +22,10 @@
 // other, so each map's softmax runs back to back.  P_m(j) is written over
 // S_m(j) as bf16 P_hi in the buffer's columns [0,32) and, for heads that need
 // it, the bf16 residual P_lo = P - P_hi in [32,64); both accumulate into O_m.
-// The MMA issuer orders "PV_m(j) then S_m(j+2)" into the same buffer, so the
-// tensor pipe reads P_m(j) before it overwrites it.
+// Per tile the MMA issuer orders PV_1(j), PV_2(j), then S_1(j+2), S_2(j+2):
+// each S write lands in the buffer its map's PV(j) just read, in issue order
+// (so P_m(j) is read before it is overwritten), and with another group in
+// between so the pipe does not stall on that write-after-read.
 // Shared memory: Q1, Q2 tiles (128 rows), then NS stages of {K tile(s), V
 // tile} of 64 keys; every tile is a set of boxes of 128-byte rows in the TMA
 // 128-byte swizzle, which is the canonical K-major (Q, K) / MN-major (V) UMMA
@@ -188,31 +190,35 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     if (lane == 0 && nT > 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, PF_BN, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, PF_DV, true);
-      const uint32_t sq0 = smem_u32(S.q[0]), sq1 = smem_u32(S.q[1]);
-      auto tS = [&](int m, int bb) { return tmem + (uint32_t)(m * 128 + bb * 64); };
+      // Descriptor words computed once; per MMA only the low word moves.
+      constexpr uint32_t HI = umma_desc_hi(1024);
+      constexpr uint32_t KSTAGE = (2 * PF_KBOX) >> 4;          // stage stride in 16-byte units
+      const uint32_t q_lo0 = umma_desc_lo(smem_u32(S.q[0]), 16), q_lo1 = umma_desc_lo(smem_u32(S.q[1]), 16);
+      const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16);
+      const uint32_t v_lo0 = umma_desc_lo(smem_u32(S.v[0]), PF_KBOX);
+      const uint32_t km_off = a.v1 ? (PF_KBOX >> 4) : 0u;         // V1: K2 box follows the K1 box
       auto issue_qk = [&](int m, int j) {
-        const int st = j % PF_NS;
-        const uint32_t kb = smem_u32(S.k[st]) + (a.v1 ? m * PF_KBOX : 0);
-        const uint32_t qb = m ? sq1 : sq0;
-        const uint32_t d = tS(m, j & 1);
+        const uint32_t klo = k_lo0 + (uint32_t)(j % PF_NS) * KSTAGE + (m ? km_off : 0u);
+        const uint32_t qlo = m ? q_lo1 : q_lo0;
+        const uint32_t d = tmem + (uint32_t)(m * 128 + (j & 1) * 64);
 #pragma unroll
         for (int s = 0; s < DQK / 16; ++s) {
-          const uint32_t kin = (s & 3) * 32;
-          mma_ss(d, umma_desc(qb + (s >> 2) * PF_QBOX + kin, 16, 1024),
-                 umma_desc(kb + (s >> 2) * PF_KBOX + kin, 16, 1024), IDESC_QK, s > 0);
+          const uint32_t qo = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+          const uint32_t ko = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+          mma_ss_w(d, qlo + qo, HI, klo + ko, HI, IDESC_QK, s > 0);
         }
         mma_commit(smem_u32(&S.s_full[m][j & 1]));
       };
       auto issue_pv = [&](int m, int j) {
-        const uint32_t vb = smem_u32(S.v[j % PF_NS]);
-        const uint32_t p = tS(m, j & 1), o = tmem + 256 + m * 128;
+        const uint32_t vlo = v_lo0 + (uint32_t)(j % PF_NS) * KSTAGE;
+        const uint32_t p = tmem + (uint32_t)(m * 128 + (j & 1) * 64), o = tmem + 256 + m * 128;
 #pragma unroll
         for (int s = 0; s < PF_BN / 16; ++s)
-          mma_ts(o, p + s * 8, umma_desc(vb + s * 2048, PF_KBOX, 1024), IDESC_PV, (j > 0 || s > 0));
+          mma_ts_w(o, p + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, (j > 0 || s > 0));
         if (resid) {
 #pragma unroll
           for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
-            mma_ts(o, p + 32 + s * 8, umma_desc(vb + s * 2048, PF_KBOX, 1024), IDESC_PV, 1);
+            mma_ts_w(o, p + 32 + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, 1);
         }
         mma_commit(smem_u32(&S.o_done[m]));
       };
@@ -228,20 +234,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       }
       for (int j = 0; ok && j < nT; ++j) {
         const int bb = j & 1, ph = (j >> 1) & 1;
-        const bool more = j + 2 < nT;
+        // PV of both maps first, then S(j+2) of both maps: every QK writes a
+        // buffer whose last reader (PV_m(j)) has a whole group between them,
+        // so the tensor pipe does not stall on the write-after-read.
         if (!(ok = wait_bar(smem_u32(&S.p_full[0][bb]), ph, abort_flag, a.watch))) break;
         tc_fence_after();
         issue_pv(0, j);
-        if (more) {
-          if (!(ok = kv_ready(j + 2))) break;
-          tc_fence_after();
-          issue_qk(0, j + 2);
-        }
         if (!(ok = wait_bar(smem_u32(&S.p_full[1][bb]), ph, abort_flag, a.watch))) break;
         tc_fence_after();
         issue_pv(1, j);
         mma_commit(smem_u32(&S.kv_empty[j % PF_NS]));
-        if (more) issue_qk(1, j + 2);
+        if (j + 2 < nT) {
+          if (!(ok = kv_ready(j + 2))) break;
+          tc_fence_after();
+          issue_qk(0, j + 2);
+          issue_qk(1, j + 2);
+        }
       }
       if (ok) mma_commit(smem_u32(&S.o_final));
       // Every MMA issued must have completed before TMEM is freed.
