@@ -249,6 +249,15 @@ def time_runner(r, steps, warmup, dist_on):
     return total_ms, kern_ms
 
 
+def keep_busy(r, seconds):
+    """Run untimed steps for about `seconds` (device time)."""
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(8):
+            r.step()
+        torch.cuda.synchronize()
+
+
 def max_over_ranks(x, dist_on):
     """Max of a per-rank time over all ranks (the slowest rank sets the step time)."""
     if not dist_on:
@@ -433,7 +442,11 @@ def main():
 
     r = make_runner(args.workload, device)
     with ClockSampler(local) as clk:
+        # untimed steps before and after keep the GPU under load long enough
+        # (>= ~0.4 s each side) for the 200 ms clock samples to cover the timed steps
+        keep_busy(r, 0.4)
         total_ms, kern_ms = time_runner(r, args.steps, args.warmup, dist_on)
+        keep_busy(r, 0.4)
     total_ms = max_over_ranks(total_ms, dist_on)
     ms = total_ms / args.steps
     work, unit = r.work()
