@@ -303,3 +303,21 @@ def test_decode_v1_small(case, fused):
     out = da.decode_v1(q1, k1, q2, k2, v, lam, fused=bool(fused))
     ref = orc.decode_v1(q1, k1, q2, k2, v, lam.cpu().numpy())
     assert rel_err(out, ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("lam_value", [0.97, 1.0, 1.03, 0.74, 1.26])
+def test_bf16_near_unit_lambda_with_similar_maps(lam_value):
+    """The hardest case for bf16 P: near-uniform, nearly identical maps and lambda
+    close to 1, where O1/l1 - lambda*O2/l2 cancels.  0.97/1.0/1.03 take the residual
+    path; 0.74/1.26 sit just outside its threshold and use bf16 P alone."""
+    g = torch.Generator(device="cpu").manual_seed(int(lam_value * 1000))
+    s = 1 / math.sqrt(128)
+    q1 = torch.randn(1, 1, 1024, 128, generator=g) * s
+    q2 = q1 + 0.05 * s * torch.randn(1, 1, 1024, 128, generator=g)       # map 2 close to map 1
+    q = torch.cat([q1, q2], dim=1).to(torch.bfloat16).to(DEV)
+    k = bf16(1, 1, 1024, 128, g=g, std=s)
+    v = bf16(1, 1, 1024, 128, g=g, std=s)
+    lam = torch.tensor([lam_value], device=DEV)
+    out = da.fwd_v2(q, k, v, lam, causal=True)
+    ref = orc.diffattn_v2(q, k, v, np.array([lam_value]), causal=True)
+    assert rel_err(out, ref) <= BF16_TOL
