@@ -10,11 +10,12 @@
 // serves both maps: in V2 both maps share K and V; in V1 the tile holds K1,
 // K2 and the shared V.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3  softmax of map 1 (thread i <-> query row i <-> TMEM lane i)
 //   warps 4-7  softmax of map 2
 //   warp  8    TMA producer; allocates / frees TMEM
-//   warp  9    MMA issuer (one thread)
+//   warp  9    PV issuer (one thread)
+//   warp 10    QK issuer (one thread)
 // Keys are processed in tiles of 64.  TMEM (512 columns) holds two S buffers
 // per map -- S1[0] [0,64) S1[1] [64,128) S2[0] [128,192) S2[1] [192,256) --
 // and the accumulators O1 [256,384) O2 [384,512).  While a map's softmax works
@@ -22,10 +23,11 @@
 // other, so each map's softmax runs back to back.  P_m(j) is written over
 // S_m(j) as bf16 P_hi in the buffer's columns [0,32) and, for heads that need
 // it, the bf16 residual P_lo = P - P_hi in [32,64); both accumulate into O_m.
-// Per tile the MMA issuer orders PV_1(j), PV_2(j), then S_1(j+2), S_2(j+2):
-// each S write lands in the buffer its map's PV(j) just read, in issue order
-// (so P_m(j) is read before it is overwritten), and with another group in
-// between so the pipe does not stall on that write-after-read.
+// The tensor pipe takes MMAs from a very shallow queue, so a single issuing
+// thread that stops to test a barrier leaves it idle.  Two issuers keep it
+// fed: one issues PV_m(j) when P_m(j) is stored, the other issues S_m(j+2)
+// into the buffer PV_m(j) read, once that PV has completed (s_free); each
+// one's waits overlap the other's MMAs.
 // Shared memory: Q1, Q2 tiles (128 rows), then NS stages of {K tile(s), V
 // tile} of 64 keys; every tile is a set of boxes of 128-byte rows in the TMA
 // 128-byte swizzle, which is the canonical K-major (Q, K) / MN-major (V) UMMA
@@ -40,7 +42,7 @@ constexpr int PF_BM = 128;         // query rows per CTA
 constexpr int PF_BN = 64;          // keys per tile
 constexpr int PF_DV = 128;         // value width
 constexpr int PF_NS = 4;           // K/V pipeline stages
-constexpr int PF_THREADS = 320;
+constexpr int PF_THREADS = 352;
 constexpr int PF_QBOX = 128 * 128; // bytes of one 128-row x 64-element bf16 box (Q)
 constexpr int PF_KBOX = 64 * 128;  // bytes of one 64-row x 64-element bf16 box (K, V)
 constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -71,15 +73,17 @@ struct PfSmem {
   float l[2][PF_BM];
   float ss[2][PF_BM];
   alignas(8) uint64_t q_full;
-  uint64_t kv_full[PF_NS];
+  uint64_t k_full[PF_NS];
+  uint64_t v_full[PF_NS];
   uint64_t kv_empty[PF_NS];
   uint64_t s_full[2][2];  // [map][buffer]
   uint64_t p_full[2][2];
+  uint64_t s_free[2][2];  // PV_m of the buffer's last tile complete: S may be overwritten
   uint64_t o_done[2];     // PV_m(j) complete (one phase per tile)
   uint64_t o_final;
   uint64_t xl;      // epilogue exchange of l (256 arrivals)
   uint64_t xs;      // epilogue exchange of RMS partial sums (256 arrivals)
-  uint64_t drain;
+  uint64_t drain[2];      // per issuer: all its MMAs complete
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -123,20 +127,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&S.q_full), 1);
     for (int i = 0; i < PF_NS; ++i) {
-      mbar_init(smem_u32(&S.kv_full[i]), 1);
+      mbar_init(smem_u32(&S.k_full[i]), 1);
+      mbar_init(smem_u32(&S.v_full[i]), 1);
       mbar_init(smem_u32(&S.kv_empty[i]), 1);
     }
     for (int m = 0; m < 2; ++m) {
       for (int bb = 0; bb < 2; ++bb) {
         mbar_init(smem_u32(&S.s_full[m][bb]), 1);
         mbar_init(smem_u32(&S.p_full[m][bb]), 128);
+        mbar_init(smem_u32(&S.s_free[m][bb]), 1);
       }
       mbar_init(smem_u32(&S.o_done[m]), 1);
+      mbar_init(smem_u32(&S.drain[m]), 1);
     }
     mbar_init(smem_u32(&S.o_final), 1);
     mbar_init(smem_u32(&S.xl), 256);
     mbar_init(smem_u32(&S.xs), 256);
-    mbar_init(smem_u32(&S.drain), 1);
     S.abort_flag = 0;
     mbar_fence_init();
   }
@@ -165,96 +171,97 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       for (int j = 0; j < nT; ++j) {
         const int st = j % PF_NS, use = j / PF_NS;
         if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
-        const uint32_t fb = smem_u32(&S.kv_full[st]);
-        mbar_expect_tx(fb, 4 * PF_KBOX);
+        const uint32_t kb = smem_u32(&S.k_full[st]), vb = smem_u32(&S.v_full[st]);
         const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
+        mbar_expect_tx(kb, 2 * PF_KBOX);
         if (a.v1) {
-          tma_load_3d(kd, &tmK1, fb, 0, j * PF_BN, zkv);
-          tma_load_3d(kd + PF_KBOX, &tmK2, fb, 0, j * PF_BN, zkv);
+          tma_load_3d(kd, &tmK1, kb, 0, j * PF_BN, zkv);
+          tma_load_3d(kd + PF_KBOX, &tmK2, kb, 0, j * PF_BN, zkv);
         } else {
-          tma_load_3d(kd, &tmK1, fb, 0, j * PF_BN, zkv);
-          tma_load_3d(kd + PF_KBOX, &tmK1, fb, 64, j * PF_BN, zkv);
+          tma_load_3d(kd, &tmK1, kb, 0, j * PF_BN, zkv);
+          tma_load_3d(kd + PF_KBOX, &tmK1, kb, 64, j * PF_BN, zkv);
         }
-        tma_load_3d(vd, &tmV, fb, 0, j * PF_BN, zkv);
-        tma_load_3d(vd + PF_KBOX, &tmV, fb, 64, j * PF_BN, zkv);
+        mbar_expect_tx(vb, 2 * PF_KBOX);
+        tma_load_3d(vd, &tmV, vb, 0, j * PF_BN, zkv);
+        tma_load_3d(vd + PF_KBOX, &tmV, vb, 64, j * PF_BN, zkv);
         last_use[st] = use;
       }
       // Every copy issued must have landed before the CTA may exit (returns at
       // once when the consumer has already seen the phase).
       drain_bar(qb, 0, a.watch.status);
       for (int i = 0; i < PF_NS; ++i)
-        if (last_use[i] >= 0) drain_bar(smem_u32(&S.kv_full[i]), last_use[i] & 1, a.watch.status);
+        if (last_use[i] >= 0) {
+          drain_bar(smem_u32(&S.k_full[i]), last_use[i] & 1, a.watch.status);
+          drain_bar(smem_u32(&S.v_full[i]), last_use[i] & 1, a.watch.status);
+        }
     }
-  } else if (warp == 9) {
-    // ---------------------------------------------------------- MMA issuer --
+  } else if (warp >= 9) {
+    // --------------------------------------------------------- MMA issuers --
     if (lane == 0 && nT > 0) {
-      constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, PF_BN, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, PF_DV, true);
       // Descriptor words computed once; per MMA only the low word moves.
       constexpr uint32_t HI = umma_desc_hi(1024);
       constexpr uint32_t KSTAGE = (2 * PF_KBOX) >> 4;          // stage stride in 16-byte units
-      const uint32_t q_lo0 = umma_desc_lo(smem_u32(S.q[0]), 16), q_lo1 = umma_desc_lo(smem_u32(S.q[1]), 16);
-      const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16);
-      const uint32_t v_lo0 = umma_desc_lo(smem_u32(S.v[0]), PF_KBOX);
-      const uint32_t km_off = a.v1 ? (PF_KBOX >> 4) : 0u;         // V1: K2 box follows the K1 box
-      auto issue_qk = [&](int m, int j) {
-        const uint32_t klo = k_lo0 + (uint32_t)(j % PF_NS) * KSTAGE + (m ? km_off : 0u);
-        const uint32_t qlo = m ? q_lo1 : q_lo0;
-        const uint32_t d = tmem + (uint32_t)(m * 128 + (j & 1) * 64);
+      const int issuer = warp - 9;                             // 0: PV, 1: QK
+      bool ok = true;
+      if (issuer == 0) {
+        // PV_1(j), PV_2(j) as soon as the softmax has stored each map's P.
+        constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, PF_DV, true);
+        const uint32_t v_lo0 = umma_desc_lo(smem_u32(S.v[0]), PF_KBOX);
+        for (int j = 0; ok && j < nT; ++j) {
+          const int bb = j & 1, ph = (j >> 1) & 1;
+          const uint32_t vlo = v_lo0 + (uint32_t)(j % PF_NS) * KSTAGE;
+          if (!(ok = wait_bar(smem_u32(&S.v_full[j % PF_NS]), (j / PF_NS) & 1, abort_flag, a.watch))) break;
+          for (int m = 0; m < 2; ++m) {
+            if (!(ok = wait_bar(smem_u32(&S.p_full[m][bb]), ph, abort_flag, a.watch))) break;
+            tc_fence_after();
+            const uint32_t p = tmem + (uint32_t)(m * 128 + bb * 64), o = tmem + 256 + m * 128;
 #pragma unroll
-        for (int s = 0; s < DQK / 16; ++s) {
-          const uint32_t qo = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
-          const uint32_t ko = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
-          mma_ss_w(d, qlo + qo, HI, klo + ko, HI, IDESC_QK, s > 0);
+            for (int s = 0; s < PF_BN / 16; ++s)
+              mma_ts_w(o, p + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, (j > 0 || s > 0));
+            if (resid) {
+#pragma unroll
+              for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
+                mma_ts_w(o, p + 32 + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, 1);
+            }
+            mma_commit(smem_u32(&S.o_done[m]));
+            mma_commit(smem_u32(&S.s_free[m][bb]));
+          }
+          if (!ok) break;
+          // The stage's K was read by S(j), complete before P(j) existed.
+          mma_commit(smem_u32(&S.kv_empty[j % PF_NS]));
         }
-        mma_commit(smem_u32(&S.s_full[m][j & 1]));
-      };
-      auto issue_pv = [&](int m, int j) {
-        const uint32_t vlo = v_lo0 + (uint32_t)(j % PF_NS) * KSTAGE;
-        const uint32_t p = tmem + (uint32_t)(m * 128 + (j & 1) * 64), o = tmem + 256 + m * 128;
+        if (ok) mma_commit(smem_u32(&S.o_final));
+      } else {
+        // S_m(j) once K(j) has landed and, for j >= 2, PV_m(j-2) -- the last
+        // reader of the buffer -- has completed.
+        constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, PF_BN, false);
+        const uint32_t q_lo0 = umma_desc_lo(smem_u32(S.q[0]), 16), q_lo1 = umma_desc_lo(smem_u32(S.q[1]), 16);
+        const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16);
+        const uint32_t km_off = a.v1 ? (PF_KBOX >> 4) : 0u;         // V1: K2 box follows the K1 box
+        ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
+        for (int j = 0; ok && j < nT; ++j) {
+          const int bb = j & 1;
+          if (!(ok = wait_bar(smem_u32(&S.k_full[j % PF_NS]), (j / PF_NS) & 1, abort_flag, a.watch))) break;
+          for (int m = 0; m < 2; ++m) {
+            if (j >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[m][bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch)))
+              break;
+            tc_fence_after();
+            const uint32_t klo = k_lo0 + (uint32_t)(j % PF_NS) * KSTAGE + (m ? km_off : 0u);
+            const uint32_t qlo = m ? q_lo1 : q_lo0;
+            const uint32_t d = tmem + (uint32_t)(m * 128 + bb * 64);
 #pragma unroll
-        for (int s = 0; s < PF_BN / 16; ++s)
-          mma_ts_w(o, p + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, (j > 0 || s > 0));
-        if (resid) {
-#pragma unroll
-          for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
-            mma_ts_w(o, p + 32 + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, 1);
+            for (int s = 0; s < DQK / 16; ++s) {
+              const uint32_t qo = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+              const uint32_t ko = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+              mma_ss_w(d, qlo + qo, HI, klo + ko, HI, IDESC_QK, s > 0);
+            }
+            mma_commit(smem_u32(&S.s_full[m][bb]));
+          }
         }
-        mma_commit(smem_u32(&S.o_done[m]));
-      };
-      auto kv_ready = [&](int j) {
-        return wait_bar(smem_u32(&S.kv_full[j % PF_NS]), (j / PF_NS) & 1, abort_flag, a.watch);
-      };
-      bool ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
-      for (int j0 = 0; ok && j0 < 2 && j0 < nT; ++j0) {
-        if (!(ok = kv_ready(j0))) break;
-        tc_fence_after();
-        issue_qk(0, j0);
-        issue_qk(1, j0);
       }
-      for (int j = 0; ok && j < nT; ++j) {
-        const int bb = j & 1, ph = (j >> 1) & 1;
-        // PV of both maps first, then S(j+2) of both maps: every QK writes a
-        // buffer whose last reader (PV_m(j)) has a whole group between them,
-        // so the tensor pipe does not stall on the write-after-read.
-        if (!(ok = wait_bar(smem_u32(&S.p_full[0][bb]), ph, abort_flag, a.watch))) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        if (!(ok = wait_bar(smem_u32(&S.p_full[1][bb]), ph, abort_flag, a.watch))) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        mma_commit(smem_u32(&S.kv_empty[j % PF_NS]));
-        if (j + 2 < nT) {
-          if (!(ok = kv_ready(j + 2))) break;
-          tc_fence_after();
-          issue_qk(0, j + 2);
-          issue_qk(1, j + 2);
-        }
-      }
-      if (ok) mma_commit(smem_u32(&S.o_final));
-      // Every MMA issued must have completed before TMEM is freed.
-      mma_commit(smem_u32(&S.drain));
-      drain_bar(smem_u32(&S.drain), 0, a.watch.status);
+      // Every MMA this thread issued must have completed before TMEM is freed.
+      mma_commit(smem_u32(&S.drain[issuer]));
+      drain_bar(smem_u32(&S.drain[issuer]), 0, a.watch.status);
     }
   } else {
     // ------------------------------------------------- softmax (two groups) --
@@ -340,7 +347,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs
       // it (rows whose alpha is 1 multiply by 1).  O_m must be complete first:
       // wait for PV_m(j-1) (o_done phase j-1; PV_m(j-2) is known complete since
-      // S_m(j) was issued after it, so the parity is unambiguous).
+      // S_m(j) was issued only after s_free showed it, so the parity is
+      // unambiguous).
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
         if (!(ok = warp_wait(smem_u32(&S.o_done[m]), (j - 1) & 1, abort_flag, a.watch))) break;
         tc_fence_after();
