@@ -95,6 +95,40 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __shfl_sync(0xffffffffu, ok, 0);
 }
 
+// P = 2^(s*scale_log2 - mu) for the 64 keys of one row, stored over S in TMEM
+// as bf16 P_hi (columns [0,32)) and, with RESID, the bf16 residual P - P_hi
+// (columns [32,64)); returns the row sum of P in f32.  Chunks of 16 keys: each
+// chunk's words go to TMEM as soon as they are ready (keeps register pressure
+// down; the stores are asynchronous).
+template <bool RESID>
+__device__ __forceinline__ float pf_exp_store(const float (&s)[PF_BN], float2 sc2, float2 nm2, uint32_t tS) {
+  const float2 neg1 = make_float2(-1.f, -1.f);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int ch = 0; ch < PF_BN / 16; ++ch) {
+    uint32_t pk[8], pl[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = ch * 16 + 2 * i;
+      const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
+      const float2 p = make_float2(ex2(x.x), ex2(x.y));
+      acc[i & 3] = __fadd2_rn(acc[i & 3], p);
+      const uint32_t hi = pack_bf16(p.x, p.y);
+      pk[i] = hi;
+      if (RESID) {
+        const float2 hf = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
+        const float2 lo = __ffma2_rn(hf, neg1, p);   // p - hi, exact
+        pl[i] = pack_bf16(lo.x, lo.y);
+      }
+    }
+    tmem_st8p(tS + ch * 8, pk);
+    if (RESID) tmem_st8p(tS + 32 + ch * 8, pl);
+  }
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 a03 = __fadd2_rn(a01, a23);
+  return a03.x + a03.y;
+}
+
 template <int DQK>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
@@ -274,7 +308,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     // last visible key of this row
     const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-    const float2 neg1 = make_float2(-1.f, -1.f);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nT; ++j) {
@@ -318,32 +351,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       }
       const float mu = m_run == -INFINITY ? 0.f : m_run;
       const float2 nm2 = make_float2(-mu, -mu);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      // Chunks of 16 keys; each chunk's P words go to TMEM as soon as they are
-      // ready (keeps register pressure down; the stores are asynchronous).
-#pragma unroll
-      for (int ch = 0; ch < PF_BN / 16; ++ch) {
-        uint32_t pk[8], pl[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = ch * 16 + 2 * i;
-          const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
-          const float2 p = make_float2(ex2(x.x), ex2(x.y));
-          acc[i & 3] = __fadd2_rn(acc[i & 3], p);
-          const uint32_t hi = pack_bf16(p.x, p.y);
-          pk[i] = hi;
-          if (resid) {
-            const float2 hf = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
-            const float2 lo = __ffma2_rn(hf, neg1, p);   // p - hi, exact
-            pl[i] = pack_bf16(lo.x, lo.y);
-          }
-        }
-        tmem_st8p(tS + ch * 8, pk);
-        if (resid) tmem_st8p(tS + 32 + ch * 8, pl);
-      }
-      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-      const float2 a03 = __fadd2_rn(a01, a23);
-      l_run = l_run * alpha + (a03.x + a03.y);
+      // The residual choice is per head: branch once per tile, so each
+      // variant's exp loop is one straight-line block the scheduler can
+      // interleave across key pairs.
+      const float rowsum = resid ? pf_exp_store<true>(s, sc2, nm2, tS) : pf_exp_store<false>(s, sc2, nm2, tS);
+      l_run = l_run * alpha + rowsum;
       // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs
       // it (rows whose alpha is 1 multiply by 1).  O_m must be complete first:
       // wait for PV_m(j-1) (o_done phase j-1; PV_m(j-2) is known complete since
