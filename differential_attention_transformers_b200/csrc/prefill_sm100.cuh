@@ -59,7 +59,7 @@ struct PrefillArgs {
   // second PV MMA) for heads with |1 - lambda| < resid_tau.  The difference
   // O1/l1 - lambda*O2/l2 amplifies P's bf16 rounding (2^-9) by about
   // (1+|lambda|)/|1-lambda| when the two maps are alike; below resid_tau that
-  // factor would exceed ~8 and the residual restores ~2^-17.
+  // factor would exceed ~12 and the residual restores ~2^-17.
   float resid_tau;
   Watch watch;
 };

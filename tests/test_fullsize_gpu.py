@@ -11,7 +11,7 @@ import torch
 import differential_attention_transformers_b200 as da
 from differential_attention_transformers_b200 import inputs
 from oracle import diffattn as orc
-from tests.test_parity_gpu import BF16_TOL, DEV, lam_gpu_and_ref, rel_err
+from tests.test_parity_gpu import BF16_TOL, DEV, PREFILL_RESID_TAU, lam_gpu_and_ref, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -109,7 +109,7 @@ def test_v1_decode_full_sampled():
                 assert np.max(np.abs(out[b:b + 1, hs] - ref)) <= BF16_TOL * np.max(np.abs(ref)), (fused, b, g)
 
 
-def _hardest_heads(lref, tau=0.25):
+def _hardest_heads(lref, tau=PREFILL_RESID_TAU):
     """The head nearest lambda = 1 (residual path, largest amplification) and the
     non-residual head nearest the threshold (bf16-only path, largest amplification)."""
     d = np.abs(1.0 - lref.astype(np.float64))

@@ -305,11 +305,16 @@ def test_decode_v1_small(case, fused):
     assert rel_err(out, ref) <= BF16_TOL
 
 
-@pytest.mark.parametrize("lam_value", [0.97, 1.0, 1.03, 0.74, 1.26])
+# |1 - lambda| below which the prefill keeps the bf16 residual of P
+PREFILL_RESID_TAU = 0.15
+
+
+@pytest.mark.parametrize("lam_value", [0.97, 1.0, 1.03, 0.86, 1.14, 0.84, 1.16, 0.74, 1.26])
 def test_bf16_near_unit_lambda_with_similar_maps(lam_value):
     """The hardest case for bf16 P: near-uniform, nearly identical maps and lambda
-    close to 1, where O1/l1 - lambda*O2/l2 cancels.  0.97/1.0/1.03 take the residual
-    path; 0.74/1.26 sit just outside its threshold and use bf16 P alone."""
+    close to 1, where O1/l1 - lambda*O2/l2 cancels.  0.97/1.0/1.03 and 0.86/1.14 take
+    the residual path; 0.84/1.16 sit just outside its threshold (|1 - lambda| = 0.16)
+    and use bf16 P alone, as do 0.74/1.26."""
     g = torch.Generator(device="cpu").manual_seed(int(lam_value * 1000))
     s = 1 / math.sqrt(128)
     q1 = torch.randn(1, 1, 1024, 128, generator=g) * s
