@@ -70,6 +70,7 @@ struct PfSmem {
   alignas(1024) uint8_t q[2][QTILE];
   alignas(1024) uint8_t k[PF_NS][2 * PF_KBOX];   // V2: K tile (dims 0-63 box, 64-127 box); V1: K1 box, K2 box
   alignas(1024) uint8_t v[PF_NS][2 * PF_KBOX];   // V tile, dv 0-63 box then 64-127 box
+  alignas(16) uint8_t stage[8][16 * 128];          // per softmax warp: 16 output rows of 64 bf16 (epilogue)
   float l[2][PF_BM];
   float ss[2][PF_BM];
   alignas(8) uint64_t q_full;
@@ -382,7 +383,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     // --------------------------------------------------------- epilogue --
     // Rows that saw no key (l == 0) output zeros.
     const float lam = a.lambda[h];
-    __nv_bfloat16* orow = a.out + (((size_t)b * a.Hout + h) * a.Lq + rg) * PF_DV + m * 64;
     float y[64];
     bool have = false;
     if (ok && nT > 0) {
@@ -426,15 +426,39 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       for (int i = 0; i < 64; ++i) y[i] = 0.f;
       have = true;
     }
-    if (have && rg < a.Lq) {
+    // Coalesced output: each thread holds 64 columns (128 bytes) of its own
+    // row, so storing them directly would touch 32 lines per warp
+    // instruction.  Instead the warp stages 16 rows at a time in its shared
+    // buffer (16-byte chunks XOR-swizzled by row, conflict-free both ways) and
+    // writes them back as 4 rows x 128 contiguous bytes per instruction.
+    have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;   // warp-uniform (ok is)
+    if (have) {
+      uint8_t* st = S.stage[warp];
+      const int row_w0 = r0 + wq * 32;                    // first row of this warp
+      __nv_bfloat16* obase = a.out + (((size_t)b * a.Hout + h) * a.Lq) * PF_DV + m * 64;
 #pragma unroll
-      for (int i = 0; i < 64; i += 8) {
-        uint4 v;
-        v.x = pack_bf16(y[i + 0], y[i + 1]);
-        v.y = pack_bf16(y[i + 2], y[i + 3]);
-        v.z = pack_bf16(y[i + 4], y[i + 5]);
-        v.w = pack_bf16(y[i + 6], y[i + 7]);
-        *reinterpret_cast<uint4*>(orow + i) = v;
+      for (int half = 0; half < 2; ++half) {
+        if ((lane >> 4) == half) {
+          const int rr = lane & 15;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 v;
+            v.x = pack_bf16(y[8 * c + 0], y[8 * c + 1]);
+            v.y = pack_bf16(y[8 * c + 2], y[8 * c + 3]);
+            v.z = pack_bf16(y[8 * c + 4], y[8 * c + 5]);
+            v.w = pack_bf16(y[8 * c + 6], y[8 * c + 7]);
+            *reinterpret_cast<uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4)) = v;
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = 4 * i + (lane >> 3), c = lane & 7;
+          const int row = row_w0 + 16 * half + rr;
+          const uint4 v = *reinterpret_cast<const uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4));
+          if (row < a.Lq) *reinterpret_cast<uint4*>(obase + (size_t)row * PF_DV + c * 8) = v;
+        }
+        __syncwarp();
       }
     }
   }
