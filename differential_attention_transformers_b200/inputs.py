@@ -141,3 +141,37 @@ def make(w: Workload, device="cpu"):
             "v": _randn(gen, (w.B, w.Hkv, w.Lk, w.dv), std, dt, device),
         }
     raise ValueError(w.layout)
+
+
+def paged_cache(kc, vc, page_size: int, seed: int, spare_pages: int = 3, lens=None):
+    """Scatter contiguous caches kc, vc [B, Hkv, T, D] into a shuffled pool of
+    token-major pages [num_pages, page_size, Hkv, D] (the serving layout).
+
+    Sequence b keeps its first lens[b] tokens (default: all T) in
+    ceil(lens[b] / page_size) pages drawn at random from the pool; spare pages
+    and the unused rows of each sequence's last page hold NaN, so a reader that
+    touches anything outside a sequence shows it.  Returns (k_pages, v_pages,
+    block_table [B, max_pages] int32, seq_lens [B] int32) on kc's device.
+    Pure data movement: no arithmetic of the method.
+    """
+    B, Hkv, T, D = kc.shape
+    lens = [T] * B if lens is None else [int(x) for x in lens]
+    need = [-(-n // page_size) for n in lens]
+    max_pages = max(1, -(-T // page_size))
+    num_pages = sum(need) + spare_pages
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=gen).tolist()
+    kp = torch.full((num_pages, page_size, Hkv, D), float("nan"), dtype=kc.dtype, device=kc.device)
+    vp = torch.full_like(kp, float("nan"))
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        for i in range(need[b]):
+            pid = perm[nxt]
+            nxt += 1
+            table[b, i] = pid
+            t0, t1 = i * page_size, min((i + 1) * page_size, lens[b])
+            kp[pid, : t1 - t0] = kc[b, :, t0:t1].transpose(0, 1)
+            vp[pid, : t1 - t0] = vc[b, :, t0:t1].transpose(0, 1)
+    return kp, vp, table.to(kc.device), torch.tensor(lens, dtype=torch.int32, device=kc.device)
+

@@ -234,6 +234,50 @@ def decode_v2(q, kc, vc, lam, batches=None, pairs=None) -> np.ndarray:
     return out[:, :, 0, :]
 
 
+def gather_pages(pages, table_row, n: int) -> np.ndarray:
+    """The first ``n`` cached tokens of one sequence, read from a page pool.
+
+    pages [num_pages, page_size, Hkv, D] (token-major pages: each page holds
+    page_size consecutive tokens, every KV head of a token side by side);
+    table_row lists the sequence's page ids in token order.  Returns
+    [Hkv, n, D] fp64.
+    """
+    pages = _f64(pages)
+    ps = pages.shape[1]
+    npg = -(-n // ps)
+    if npg == 0:
+        return np.zeros((pages.shape[2], 0, pages.shape[3]))
+    toks = np.concatenate([pages[int(p)] for p in np.asarray(table_row)[:npg]], axis=0)[:n]
+    return np.transpose(toks, (1, 0, 2))
+
+
+def decode_v2_paged(q, k_pages, v_pages, block_table, seq_lens, lam) -> np.ndarray:
+    """Single-token V2 decode of B sequences whose K/V caches live in a shared
+    pool of fixed-size pages, each sequence with its own length.
+
+    Serving layout (the tutorial's V1 到 V2 的 diff section names the
+    vLLM/SGLang integration; the pages give no layout, so this follows the
+    common token-major page pool): k_pages, v_pages [num_pages, page_size,
+    Hkv, D]; block_table [B, max_pages] page ids; seq_lens [B].  Sequence b is
+    its first seq_lens[b] tokens in page order, and its output is
+    ``decode_v2`` against exactly that cache (a length of 0 gives zeros).
+    Returns [B, Hq/2, D] fp64.
+    """
+    q = _f64(q)
+    bt = np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table)
+    sl = np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens)
+    B, Hq, D = q.shape
+    out = np.zeros((B, Hq // 2, D))
+    for b in range(B):
+        n = max(0, int(sl[b]))
+        if n == 0:
+            continue
+        kc = gather_pages(k_pages, bt[b], n)[None]
+        vc = gather_pages(v_pages, bt[b], n)[None]
+        out[b] = decode_v2(q[b:b + 1], kc, vc, lam)[0]
+    return out
+
+
 def decode_v1(q1, k1, q2, k2, v, lam, batches=None, heads=None) -> np.ndarray:
     """Single-token V1-layout decode: q1,q2 [B,H,d]; k1,k2 [B,Hkv,T,d]; v [B,Hkv,T,dv]."""
     q1, q2 = _f64(q1), _f64(q2)
