@@ -210,7 +210,47 @@ class Decode:
         return da.decode_v1(host["q1"], host["k1"], host["q2"], host["k2"], host["v"], lam, fused=self.fused)
 
 
+PAGE_SIZE = 16   # paged decode secondary: 16-token pages
+
+
+class PagedDecode:
+    """The V2 decode workload with its caches in a shuffled pool of 16-token pages."""
+
+    def __init__(self, w, device):
+        self.w = w
+        x = inputs.make(w, device=device)
+        kp, vp, bt, sl = inputs.paged_cache(x["k"], x["v"], PAGE_SIZE, seed=w.seed)
+        del x["k"], x["v"]
+        self.x = {"q": x["q"], "k_pages": kp, "v_pages": vp, "block_table": bt, "seq_lens": sl}
+        self.lp = inputs.lambda_params(w, device=device)
+        self.init = da.lambda_init(w.layer)
+        self.lam = torch.empty(w.pairs, dtype=torch.float32, device=device)
+        self.out = torch.empty((w.B, w.pairs, w.dv), dtype=w.dtype, device=device)
+        self.ws = torch.empty(da.decode_paged_workspace_size(w.B, w.Hkv), dtype=torch.uint8, device=device)
+        self.launches_per_step = 3
+
+    def step(self, ev=None):
+        x = self.x
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        if ev is not None:
+            ev[0].record()
+        da.decode_v2_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"], self.lam,
+                           out=self.out, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        return decode_bytes(self.w) / 1e9, "GB/s"
+
+    def host_call(self, host):
+        lam = da.compute_lambda(*host["lp"], self.init)
+        return da.decode_v2_paged(host["q"], host["k_pages"], host["v_pages"], host["block_table"],
+                                  host["seq_lens"], lam)
+
+
 def make_runner(name, device):
+    if name == "v2_decode_paged":
+        return PagedDecode(inputs.WORKLOADS["v2_decode"], device)
     w = inputs.WORKLOADS[name.replace("_unfused", "")]
     if w.layout in ("v1", "v2"):
         return Prefill(w, device)
@@ -218,12 +258,14 @@ def make_runner(name, device):
 
 
 def describe(name):
-    w = inputs.WORKLOADS[name.replace("_unfused", "")]
+    w = inputs.WORKLOADS[name.replace("_unfused", "").replace("_paged", "")]
     d = {"workload": name, "layout": w.layout, "B": w.B, "heads": w.H, "kv_heads": w.Hkv, "Lq": w.Lq, "Lk": w.Lk,
          "d": w.d, "dv": w.dv, "causal": w.causal, "layer": w.layer, "rmsnorm": w.rmsnorm,
          "l2": "inputs larger than L2 (126 MB): no flush between steps"}
     if name.endswith("_unfused"):
         d["mode"] = "two passes, V read twice (comparison)"
+    if name.endswith("_paged"):
+        d["mode"] = f"paged: shuffled pool of {PAGE_SIZE}-token pages [num_pages, {PAGE_SIZE}, Hkv, 128], block table"
     return d
 
 
@@ -336,7 +378,8 @@ def cpu_oracle_run(name, budget_s=12.0):
         cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
     except Exception:
         cores = len(os.sched_getaffinity(0))
-    w = inputs.WORKLOADS[name.replace("_unfused", "")]
+    paged = name == "v2_decode_paged"
+    w = inputs.WORKLOADS[name.replace("_unfused", "").replace("_paged", "")]
     x = inputs.make(w, device="cpu") if w.layout in ("v1", "v2") else None
     lam = np.full(w.pairs, 0.5)
     done_work, t_total, n = 0.0, 0.0, 0
@@ -371,8 +414,13 @@ def cpu_oracle_run(name, budget_s=12.0):
                     q = (torch.randn(1, grp, w.d, generator=gen) * w.std).to(torch.bfloat16)
                     kc = (torch.randn(1, 1, w.Lk, w.d, generator=gen) * w.std).to(torch.bfloat16)
                     vc = (torch.randn(1, 1, w.Lk, w.dv, generator=gen) * w.std).to(torch.bfloat16)
-                    t0 = time.perf_counter()
-                    orc.decode_v2(q, kc, vc, lam[: grp // 2])
+                    if paged:
+                        kp, vp, bt, sl = inputs.paged_cache(kc, vc, PAGE_SIZE, seed=b * w.Hkv + g)
+                        t0 = time.perf_counter()
+                        orc.decode_v2_paged(q, kp, vp, bt, sl, lam[: grp // 2])
+                    else:
+                        t0 = time.perf_counter()
+                        orc.decode_v2(q, kc, vc, lam[: grp // 2])
                 else:
                     q1 = (torch.randn(1, grp, w.d, generator=gen) * w.std).to(torch.bfloat16)
                     k1 = (torch.randn(1, 1, w.Lk, w.d, generator=gen) * w.std).to(torch.bfloat16)
@@ -399,7 +447,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="v2_prefill",
-                    choices=["v2_prefill", "v1_prefill", "v2_decode", "v1_decode", "v1_decode_unfused"])
+                    choices=["v2_prefill", "v1_prefill", "v2_decode", "v2_decode_paged", "v1_decode",
+                             "v1_decode_unfused"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
@@ -465,7 +514,7 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        names = ["v1_prefill", "v2_decode", "v1_decode", "v1_decode_unfused", "v2_prefill"]
+        names = ["v1_prefill", "v2_decode", "v2_decode_paged", "v1_decode", "v1_decode_unfused", "v2_prefill"]
         for name in names:
             if name == args.workload:
                 continue

@@ -27,7 +27,8 @@ F32, BF16 = 0, 1
 
 EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffattn_fwd_v1", "diffattn_fwd_v2",
            "diffattn_decode_workspace_size", "diffattn_decode_v2", "diffattn_decode_v1", "diffattn_last_error",
-           "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc"]
+           "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc",
+           "diffattn_decode_paged_workspace_size", "diffattn_decode_v2_paged"]
 
 _lib = None
 
@@ -61,6 +62,8 @@ def load():
         "diffattn_last_status": (I, [P]),
         "diffattn_set_wait_limit_ns": (None, [U]),
         "diffattn_decode_v2_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P]),
+        "diffattn_decode_paged_workspace_size": (Z, [I, I]),
+        "diffattn_decode_v2_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -195,6 +198,31 @@ def decode_v2(q, kc, vc, lam, out=None, workspace=None):
     ws = workspace if workspace is not None else _workspace(need, q.device)
     _check(load().diffattn_decode_v2(_ptr(q), _ptr(kc), _ptr(vc), _ptr(lam), _ptr(out), dt, B, Hq, Hkv, T, D,
                                      _ptr(ws), ws.numel() * ws.element_size(), _stream()))
+    return _finish(host, out)
+
+
+def decode_paged_workspace_size(B: int, Hkv: int) -> int:
+    return int(load().diffattn_decode_paged_workspace_size(B, Hkv))
+
+
+def decode_v2_paged(q, k_pages, v_pages, block_table, seq_lens, lam, out=None, workspace=None):
+    """Paged, variable-length V2 decode: q [B,Hq,128]; k_pages, v_pages [num_pages, page_size, Hkv, 128];
+    block_table int32 [B, max_pages]; seq_lens int32 [B]; lam [Hq/2] -> [B, Hq/2, 128]."""
+    host, (q, k_pages, v_pages, block_table, seq_lens, lam) = _prep([q, k_pages, v_pages, block_table, seq_lens,
+                                                                      lam])
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=q.dtype, device=q.device)
+    need = decode_paged_workspace_size(B, Hkv)
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check(load().diffattn_decode_v2_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                           _ptr(seq_lens), _ptr(lam), _ptr(out), dt, B, Hq, Hkv, num_pages,
+                                           page_size, block_table.shape[1], _ptr(ws),
+                                           ws.numel() * ws.element_size(), _stream()))
     return _finish(host, out)
 
 

@@ -14,6 +14,17 @@
 // The combine kernel merges the records of each query head (log-sum-exp) and
 // applies O = O1/l1 - lambda * O2/l2.
 //
+// Paged, variable-length mode (V2): the caches are a pool of token-major pages
+// [num_pages, page_size, Hkv, 128] addressed through a block table, and each
+// sequence has its own length.  Every CTA first builds, in shared memory, the
+// prefix of 64-key blocks over the sequences (block counts times Hkv), so the
+// same equal split of the flattened block space applies; a CTA's record for
+// segment (b, g) goes to slot CTA + b*Hkv + g, which is unique along the
+// staircase of CTA ranges and bounded by grid + B*Hkv.  Tiles come in by a 4-D
+// tensor map over the pool (one box per page part of the block).  Cache rows
+// past a sequence's length are masked and their V rows zeroed in shared memory
+// before the PV product, since a page's unused rows may hold anything.
+//
 // Inner product per 16-key slice and warp, on mma.sync m16n8k16 (bf16, f32
 // accumulate) with the keys as M so that the 8 query columns fill N = 8:
 //   S^T[16 keys x 8 cols]  = K[16 x 128] . Qcols^T[128 x 8]
@@ -33,6 +44,7 @@ constexpr int DEC_CONSUMERS = 4;            // consumer warps, 16 keys of each b
 constexpr int DEC_THREADS = 32 * (DEC_CONSUMERS + 1);
 constexpr int DEC_REC = 8 * 2 + 8 * 128;    // floats per partial record: m[8], l[8], O[8][128]
 constexpr int DEC_TILE_BYTES = DEC_KB * 128 * 2;  // one 64-key x 128-wide bf16 tile (two 8 KB boxes)
+constexpr int DEC_MAXB = 2048;              // paged mode: most sequences per launch
 
 struct DecodeArgs {
   const __nv_bfloat16* q1;  // V2: q [B,Hq,128]; V1: q1 [B,H,64]
@@ -47,13 +59,18 @@ struct DecodeArgs {
   long long total;          // B * Hkv * nblk
   float scale_log2;         // log2(e) / sqrt(d)
   Watch watch;
+  // paged mode
+  const int* block_table;   // [B, max_pages] page ids
+  const int* seq_lens;      // [B]
+  int* cu_out;              // [B+1] block prefix, written by CTA 0 for the combine
+  int max_pages, page_size, page_shift;
 };
 
 __host__ __device__ __forceinline__ long long dec_blk_start(long long i, long long total, int grid) {
   return i * total / grid;
 }
 
-template <int NST>
+template <int NST, bool PAGED = false>
 struct DecSmem {
   alignas(1024) uint8_t k[NST][DEC_TILE_BYTES];
   alignas(1024) uint8_t v[NST][DEC_TILE_BYTES];
@@ -63,7 +80,23 @@ struct DecSmem {
   alignas(8) uint64_t full[NST];
   uint64_t empty[NST];
   int abort_flag;
+  // paged mode: flattened block offset of each sequence (cu[B] = total) and its length
+  int cu[PAGED ? DEC_MAXB + 1 : 1];
+  int len[PAGED ? DEC_MAXB : 1];
+  int part[PAGED ? DEC_THREADS : 1];
 };
+
+// Paged mode: the sequence holding flattened block x (largest b with
+// cu[b] <= x; empty sequences have cu[b] == cu[b+1] and are skipped).
+__device__ __forceinline__ int dec_find_seq(const int* cu, int B, long long x) {
+  int lo = 0, hi = B;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= x) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
 
 // Byte offset of element (row, 16-byte chunk) inside a 128-byte-swizzled box
 // of 128-byte rows (TMA SWIZZLE_128B, box base 1024-byte aligned).
@@ -86,12 +119,12 @@ __device__ __forceinline__ bool bar_any(bool pred) {
   return r != 0;
 }
 
-template <int NST>
+template <int NST, bool PAGED = false>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
                     const __grid_constant__ CUtensorMap tmV, DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  DecSmem<NST>& S = *reinterpret_cast<DecSmem<NST>*>(
+  DecSmem<NST, PAGED>& S = *reinterpret_cast<DecSmem<NST, PAGED>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &S.abort_flag;
@@ -104,10 +137,44 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
     S.abort_flag = 0;
     mbar_fence_init();
   }
+  long long total = a.total;
+  if constexpr (PAGED) {
+    // Block prefix over the sequences: lengths clamped to [0, max_pages * page_size].
+    const int per = (a.B + DEC_THREADS - 1) / DEC_THREADS;
+    const int b0 = min(a.B, (int)threadIdx.x * per), b1 = min(a.B, b0 + per);
+    const int cap = a.max_pages * a.page_size;
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) {
+      const int n = min(max(a.seq_lens[b], 0), cap);
+      S.len[b] = n;
+      sum += ((n + DEC_KB - 1) / DEC_KB) * a.Hkv;
+    }
+    S.part[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int run = 0;
+      for (int i = 0; i < DEC_THREADS; ++i) {
+        const int v = S.part[i];
+        S.part[i] = run;
+        run += v;
+      }
+      S.cu[a.B] = run;
+    }
+    __syncthreads();
+    int run = S.part[threadIdx.x];
+    for (int b = b0; b < b1; ++b) {
+      S.cu[b] = run;
+      run += ((S.len[b] + DEC_KB - 1) / DEC_KB) * a.Hkv;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0)
+      for (int i = threadIdx.x; i <= a.B; i += DEC_THREADS) a.cu_out[i] = S.cu[i];
+    total = S.cu[a.B];
+  }
   __syncthreads();
 
-  const long long lo = dec_blk_start(blockIdx.x, a.total, a.grid);
-  const long long hi = dec_blk_start(blockIdx.x + 1, a.total, a.grid);
+  const long long lo = dec_blk_start(blockIdx.x, total, a.grid);
+  const long long hi = dec_blk_start(blockIdx.x + 1, total, a.grid);
   const bool load_k2 = a.v1 ? (a.maps & 2) != 0 : true;
   const bool load_k1 = a.v1 ? (a.maps & 1) != 0 : true;
 
@@ -128,14 +195,45 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
           ok = false;
           break;
         }
+        const uint32_t fb = smem_u32(&S.full[st]);
+        const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
+        if constexpr (PAGED) {
+          const int b = dec_find_seq(S.cu, a.B, x);
+          const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
+          const int within = (int)(x - S.cu[b]);
+          const int g = within / nb, key0 = (within % nb) * DEC_KB;
+          const int* row = a.block_table + (size_t)b * a.max_pages;
+          if (a.page_size >= DEC_KB) {
+            const int page = row[key0 >> a.page_shift], y = key0 & (a.page_size - 1);
+            mbar_expect_tx(fb, 2 * DEC_TILE_BYTES);
+            tma_load_4d(kd, &tmK1, fb, 0, g, y, page);
+            tma_load_4d(kd + DEC_TILE_BYTES / 2, &tmK1, fb, 64, g, y, page);
+            tma_load_4d(vd, &tmV, fb, 0, g, y, page);
+            tma_load_4d(vd + DEC_TILE_BYTES / 2, &tmV, fb, 64, g, y, page);
+          } else {
+            // several pages per block; parts wholly past the sequence are not
+            // loaded (their rows are masked and their V rows zeroed)
+            const int len = S.len[b], ps = a.page_size;
+            const int parts = min(DEC_KB, len - key0 + ps - 1) / ps;   // >= 1: the block holds a key
+            mbar_expect_tx(fb, (uint32_t)(parts * ps * 128 * 4));
+            for (int i = 0; i < parts; ++i) {
+              const int page = row[(key0 >> a.page_shift) + i];
+              const uint32_t off = (uint32_t)(i * ps * 128);
+              tma_load_4d(kd + off, &tmK1, fb, 0, g, 0, page);
+              tma_load_4d(kd + DEC_TILE_BYTES / 2 + off, &tmK1, fb, 64, g, 0, page);
+              tma_load_4d(vd + off, &tmV, fb, 0, g, 0, page);
+              tma_load_4d(vd + DEC_TILE_BYTES / 2 + off, &tmV, fb, 64, g, 0, page);
+            }
+          }
+          issued_last[st] = use;
+          continue;
+        }
         const long long bg = x / a.nblk;
         const int key0 = (int)((x % a.nblk) * DEC_KB);
-        const uint32_t fb = smem_u32(&S.full[st]);
         uint32_t bytes = DEC_TILE_BYTES;  // V
         if (a.v1) bytes += (load_k1 ? DEC_TILE_BYTES / 2 : 0) + (load_k2 ? DEC_TILE_BYTES / 2 : 0);
         else bytes += DEC_TILE_BYTES;
         mbar_expect_tx(fb, bytes);
-        const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
         if (a.v1) {
           if (load_k1) tma_load_3d(kd, &tmK1, fb, 0, key0, (int)bg);
           if (load_k2) tma_load_3d(kd + DEC_TILE_BYTES / 2, &tmK2, fb, 0, key0, (int)bg);
@@ -159,16 +257,31 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
   const int w = warp;                 // 16-key slice of each block
   const int col0 = 2 * (lane & 3);    // this thread's two query columns
   const int grp = a.v1 ? a.Hq / a.Hkv : a.Hq / a.Hkv;
-  const int seg_first_bg = (int)(lo / a.nblk);
+  const int seg_first_bg = PAGED ? 0 : (int)(lo / a.nblk);
   // V1 single-map passes load only one K half: skip the other half's k-steps.
   const int kk_lo = (a.v1 && !load_k1) ? 4 : 0;
   const int kk_hi = (a.v1 && !load_k2) ? 4 : 8;
   bool aborted = false;
   long long x = lo;
   while (x < hi) {
-    const long long bg = x / a.nblk;
-    const long long seg_end = min(hi, (bg + 1) * a.nblk);
-    const int b = (int)(bg / a.Hkv), g = (int)(bg % a.Hkv);
+    long long bg, seg_end, seg_x0;   // segment (b, g), its end in this range, its first block
+    int b, g, len;
+    if constexpr (PAGED) {
+      b = dec_find_seq(S.cu, a.B, x);
+      const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
+      g = (int)(x - S.cu[b]) / nb;
+      bg = (long long)b * a.Hkv + g;
+      seg_x0 = S.cu[b] + (long long)g * nb;
+      seg_end = min(hi, seg_x0 + nb);
+      len = S.len[b];
+    } else {
+      bg = x / a.nblk;
+      seg_x0 = bg * a.nblk;
+      seg_end = min(hi, (bg + 1) * a.nblk);
+      b = (int)(bg / a.Hkv);
+      g = (int)(bg % a.Hkv);
+      len = a.T;
+    }
 
     // query operand (B fragments) for the 8 columns: n = lane / 4
     uint32_t qb[8][2];
@@ -226,8 +339,22 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
         mma16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
       }
       // mask the ragged tail of the cache
-      const int key_lo = (int)((x % a.nblk) * DEC_KB) + r0 + (lane >> 2);
-      const bool v_lo = key_lo < a.T, v_hi = key_lo + 8 < a.T;
+      const int blk_key0 = (int)(x - seg_x0) * DEC_KB;
+      const int key_lo = blk_key0 + r0 + (lane >> 2);
+      const bool v_lo = key_lo < len, v_hi = key_lo + 8 < len;
+      // Paged mode: a block that ends past the sequence may hold anything in
+      // its tail rows (unused page rows, or rows of parts not loaded); zero this
+      // warp's V rows there so that P = 0 meets finite values.
+      const bool sanitize = PAGED && blk_key0 + DEC_KB > len;
+      if (sanitize) {
+        const int rr = r0 + (lane & 15);
+        if (blk_key0 + rr >= len) {
+          uint4* vrow = reinterpret_cast<uint4*>(S.v[st] + (lane >> 4) * (DEC_TILE_BYTES / 2) + rr * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+      }
       float xs[4];
       xs[0] = v_lo ? s[0] * a.scale_log2 : -INFINITY;
       xs[1] = v_lo ? s[1] * a.scale_log2 : -INFINITY;
@@ -271,6 +398,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
         mma16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
         mma16816(acc[mt], a0, a1, a2, a3, pr0, pr1);
       }
+      // generic-proxy writes to the stage must be ordered before the next
+      // copy into it (async proxy)
+      if (sanitize) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[st]));
     }
@@ -296,7 +426,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
     if (bar_any(aborted || *abort_flag)) break;
     {
       const int t = threadIdx.x;  // 0..127: output dv index, all 8 columns
-      float* rec = a.ws + ((size_t)blockIdx.x * a.maxseg + (size_t)(bg - seg_first_bg)) * DEC_REC;
+      float* rec = PAGED ? a.ws + ((size_t)blockIdx.x + (size_t)bg) * DEC_REC
+                         : a.ws + ((size_t)blockIdx.x * a.maxseg + (size_t)(bg - seg_first_bg)) * DEC_REC;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         float M = -INFINITY;
@@ -327,6 +458,7 @@ struct CombineArgs {
   long long nblk, total;
   int two_pass;        // V1 unfused: map 2 records live in a second workspace half
   size_t half_floats;  // offset of the second half
+  const int* cu;       // paged mode: block prefix written by the split kernel (null otherwise)
 };
 
 // One CTA (128 threads = the value width) per (batch, output head).
@@ -339,30 +471,43 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
   if (a.v1) { g = h / grp; c1 = h % grp; c2 = 4 + h % grp; }
   else { g = (2 * h) / grp; c1 = (2 * h) % grp; c2 = c1 + 1; }
   const long long bg = (long long)b * a.Hkv + g;
-  const long long x0 = bg * a.nblk, x1 = x0 + a.nblk;
+  long long x0, x1, total = a.total;
+  if (a.cu) {   // paged: this sequence's blocks per KV head from the prefix
+    const int nb = (a.cu[b + 1] - a.cu[b]) / a.Hkv;
+    x0 = a.cu[b] + (long long)g * nb;
+    x1 = x0 + nb;
+    total = a.cu[a.B];
+  } else {
+    x0 = bg * a.nblk;
+    x1 = x0 + a.nblk;
+  }
 
   // CTAs whose block range overlaps [x0, x1)
-  long long i0 = a.total > 0 ? x0 * a.grid / a.total : 0;
-  while (i0 > 0 && dec_blk_start(i0, a.total, a.grid) > x0) --i0;
-  while (i0 + 1 < a.grid && dec_blk_start(i0 + 1, a.total, a.grid) <= x0) ++i0;
+  long long i0 = total > 0 ? x0 * a.grid / total : 0;
+  while (i0 > 0 && dec_blk_start(i0, total, a.grid) > x0) --i0;
+  while (i0 + 1 < a.grid && dec_blk_start(i0 + 1, total, a.grid) <= x0) ++i0;
 
   float res[2];
   for (int mp = 0; mp < 2; ++mp) {
     const int c = mp == 0 ? c1 : c2;
     const float* base = a.ws + ((a.two_pass && mp == 1) ? a.half_floats : 0);
     float M = -INFINITY;
-    for (long long i = i0; i < a.grid && dec_blk_start(i, a.total, a.grid) < x1; ++i) {
-      const long long s = dec_blk_start(i, a.total, a.grid);
-      if (dec_blk_start(i + 1, a.total, a.grid) <= x0 || s >= x1) continue;
-      const float* rec = base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
+    for (long long i = i0; x1 > x0 && i < a.grid && dec_blk_start(i, total, a.grid) < x1; ++i) {
+      // CTAs with an empty range (paged mode: more CTAs than blocks) wrote nothing
+      const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
+      if (e <= x0 || s >= x1 || e <= s) continue;
+      const float* rec = a.cu ? base + ((size_t)i + (size_t)bg) * DEC_REC
+                              : base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
       M = fmaxf(M, rec[c]);
     }
     const float Mu = M == -INFINITY ? 0.f : M;
     float o = 0.f, l = 0.f;
-    for (long long i = i0; i < a.grid && dec_blk_start(i, a.total, a.grid) < x1; ++i) {
-      const long long s = dec_blk_start(i, a.total, a.grid);
-      if (dec_blk_start(i + 1, a.total, a.grid) <= x0 || s >= x1) continue;
-      const float* rec = base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
+    for (long long i = i0; x1 > x0 && i < a.grid && dec_blk_start(i, total, a.grid) < x1; ++i) {
+      // CTAs with an empty range (paged mode: more CTAs than blocks) wrote nothing
+      const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
+      if (e <= x0 || s >= x1 || e <= s) continue;
+      const float* rec = a.cu ? base + ((size_t)i + (size_t)bg) * DEC_REC
+                              : base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
       const float f = ex2(rec[c] - Mu);
       o += rec[16 + c * 128 + t] * f;
       l += rec[8 + c] * f;

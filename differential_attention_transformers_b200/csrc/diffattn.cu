@@ -81,6 +81,7 @@ template <int DQK>
 constexpr size_t prefill_smem() { return sizeof(PfSmem<DQK>) + 1024; }
 constexpr int kDecNst = 2;
 constexpr size_t decode_smem() { return sizeof(DecSmem<kDecNst>) + 1024; }
+constexpr size_t decode_paged_smem() { return sizeof(DecSmem<kDecNst, true>) + 1024; }
 constexpr int kDecCtasPerSm = 2;
 
 // Per-device set-up: SM count, status word address, kernel attributes,
@@ -108,6 +109,8 @@ int device_setup(DeviceInfo** out) {
                                   (int)prefill_smem<128>()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)decode_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_paged_smem()));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -135,6 +138,21 @@ int make_map(CUtensorMap* m, const void* base, int X, long long Y, long long Z, 
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DIFFATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DIFFATTN_OK;
+}
+
+// 4-D bf16 tensor map over a token-major page pool [num_pages, page_size, Hkv,
+// 128]: box {64 dims, 1 head, min(page_size, 64) tokens, 1 page}, 128-byte
+// swizzle, zero fill outside the pool (so a page id out of range reads zeros).
+int make_map_paged(CUtensorMap* m, const void* base, int Hkv, int page_size, int num_pages) {
+  cuuint64_t dims[4] = {128, (cuuint64_t)Hkv, (cuuint64_t)page_size, (cuuint64_t)num_pages};
+  cuuint64_t strides[3] = {256, (cuuint64_t)Hkv * 256, (cuuint64_t)page_size * Hkv * 256};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)std::min(page_size, DEC_KB), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DIFFATTN_ERR_CUDA, "cuTensorMapEncodeTiled (paged) failed (%d)", (int)r);
   return DIFFATTN_OK;
 }
 
@@ -232,7 +250,7 @@ int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2
     if (int e = make_map(&mk1, k1, dk, T, (long long)B * Hkv, DEC_KB)) return e;
     if (int e = make_map(&mk2, v1 ? k2 : k1, dk, T, (long long)B * Hkv, DEC_KB)) return e;
     if (int e = make_map(&mv, v, 128, T, (long long)B * Hkv, DEC_KB)) return e;
-    DecodeArgs a;
+    DecodeArgs a{};
     a.q1 = static_cast<const __nv_bfloat16*>(q1);
     a.q2 = static_cast<const __nv_bfloat16*>(v1 ? q2 : q1);
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T = T;
@@ -247,7 +265,7 @@ int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2
       CUDA_TRY(cudaGetLastError());
     }
   }
-  CombineArgs c;
+  CombineArgs c{};
   c.ws = static_cast<const float*>(ws);
   c.lambda = lambda;
   c.out = static_cast<__nv_bfloat16*>(out);
@@ -255,8 +273,58 @@ int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2
   c.grid = p.grid; c.maxseg = p.maxseg; c.nblk = p.nblk; c.total = p.total;
   c.two_pass = passes == 2 ? 1 : 0;
   c.half_floats = p.bytes_per_pass / sizeof(float);
+  c.cu = nullptr;
   const int Hout = v1 ? Hq : Hq / 2;
   decode_combine_kernel<<<(unsigned)(B * Hout), 128, 0, s>>>(c);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+// Paged decode workspace: the block prefix (B+1 ints, padded to 256 bytes),
+// then one partial record per slot CTA + b*Hkv + g, i.e. grid + B*Hkv records.
+int paged_grid(const DeviceInfo* dev) { return dev->sms * kDecCtasPerSm; }
+size_t paged_prefix_bytes(int B) { return ((size_t)(B + 1) * sizeof(int) + 255) & ~(size_t)255; }
+size_t paged_ws_bytes(const DeviceInfo* dev, int B, int Hkv) {
+  return paged_prefix_bytes(B) + ((size_t)paged_grid(dev) + (size_t)B * Hkv) * DEC_REC * sizeof(float);
+}
+
+int launch_decode_paged(const void* q, const void* kp, const void* vp, const int* table, const int* lens,
+                        const float* lambda, void* out, int B, int Hq, int Hkv, int num_pages, int page_size,
+                        int max_pages, void* ws, size_t ws_bytes, cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  const size_t need = paged_ws_bytes(dev, B, Hkv);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(DIFFATTN_ERR_WORKSPACE, "paged decode workspace %zu B < required %zu B", ws_bytes, need);
+  if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  CUtensorMap mk, mv;
+  if (int e = make_map_paged(&mk, kp, Hkv, page_size, num_pages)) return e;
+  if (int e = make_map_paged(&mv, vp, Hkv, page_size, num_pages)) return e;
+  int* cu = static_cast<int*>(ws);
+  float* rec = reinterpret_cast<float*>(static_cast<char*>(ws) + paged_prefix_bytes(B));
+  DecodeArgs a{};
+  a.q1 = a.q2 = static_cast<const __nv_bfloat16*>(q);
+  a.ws = rec;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T = 0;
+  a.v1 = 0; a.maps = 3;
+  a.grid = paged_grid(dev); a.maxseg = 0; a.nblk = 0; a.total = 0;
+  a.scale_log2 = log2e_over_sqrt(128);
+  a.watch = make_watch(dev);
+  a.block_table = table; a.seq_lens = lens; a.cu_out = cu;
+  a.max_pages = max_pages; a.page_size = page_size;
+  a.page_shift = 0;
+  while ((1 << a.page_shift) < page_size) ++a.page_shift;
+  decode_split_kernel<kDecNst, true><<<a.grid, DEC_THREADS, decode_paged_smem(), s>>>(mk, mk, mv, a);
+  CUDA_TRY(cudaGetLastError());
+  CombineArgs c{};
+  c.ws = rec;
+  c.lambda = lambda;
+  c.out = static_cast<__nv_bfloat16*>(out);
+  c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.v1 = 0;
+  c.grid = a.grid; c.maxseg = 0; c.nblk = 0; c.total = 0;
+  c.two_pass = 0; c.half_floats = 0;
+  c.cu = cu;
+  decode_combine_kernel<<<(unsigned)(B * (Hq / 2)), 128, 0, s>>>(c);
   CUDA_TRY(cudaGetLastError());
   return ok();
 }
@@ -407,6 +475,38 @@ int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const floa
                 Hkv);
   if (int e = check_bf16_ptrs({q, kc, vc, out})) return e;
   return launch_decode(q, nullptr, kc, nullptr, vc, lambda, out, B, Hq, Hkv, T, false, 1, ws, ws_bytes, s);
+}
+
+size_t diffattn_decode_paged_workspace_size(int B, int Hkv) {
+  if (B < 1 || B > DEC_MAXB || Hkv < 1) return 0;
+  DeviceInfo* dev = nullptr;
+  if (device_setup(&dev)) return 0;
+  return paged_ws_bytes(dev, B, Hkv);
+}
+
+int diffattn_decode_v2_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                             const int* seq_lens, const float* lambda, void* out, diffattn_dtype dtype, int B,
+                             int Hq, int Hkv, int num_pages, int page_size, int max_pages, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (B < 1 || B > DEC_MAXB || Hq < 2 || Hkv < 1 || num_pages < 1 || max_pages < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d num_pages=%d max_pages=%d; 1 <= B <= %d)",
+                B, Hq, Hkv, num_pages, max_pages, DEC_MAXB);
+  if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128 && page_size != 256)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "page_size %d: must be 16, 32, 64, 128 or 256", page_size);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the paged decode takes bf16 only");
+  if (Hq / Hkv > 8) return fail(DIFFATTN_ERR_UNSUPPORTED, "paged decode needs Hq/Hkv <= 8 (Hq=%d Hkv=%d)", Hq, Hkv);
+  const long long max_blocks = ((long long)max_pages * page_size + DEC_KB - 1) / DEC_KB;
+  if ((long long)B * Hkv * max_blocks >= (1LL << 31))
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "B * Hkv * max_pages * page_size / 64 must stay below 2^31");
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !lambda || !out)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (int e = check_bf16_ptrs({q, k_pages, v_pages, out})) return e;
+  if ((reinterpret_cast<uintptr_t>(block_table) | reinterpret_cast<uintptr_t>(seq_lens)) & 3u)
+    return fail(DIFFATTN_ERR_MISALIGNED, "block_table / seq_lens not 4-byte aligned");
+  return launch_decode_paged(q, k_pages, v_pages, block_table, seq_lens, lambda, out, B, Hq, Hkv, num_pages,
+                             page_size, max_pages, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int diffattn_decode_v2_noalloc(const void* q, const void* kc, const void* vc, const float* lambda, void* out,

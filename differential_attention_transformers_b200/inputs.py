@@ -163,6 +163,14 @@ def paged_cache(kc, vc, page_size: int, seed: int, spare_pages: int = 3, lens=No
     perm = torch.randperm(num_pages, generator=gen).tolist()
     kp = torch.full((num_pages, page_size, Hkv, D), float("nan"), dtype=kc.dtype, device=kc.device)
     vp = torch.full_like(kp, float("nan"))
+    if all(n == T for n in lens) and T % page_size == 0:
+        # every sequence full and page-aligned: one scatter of all pages at once
+        npg = T // page_size
+        ids = torch.tensor(perm[: B * npg], dtype=torch.long, device=kc.device)
+        for src, dst in ((kc, kp), (vc, vp)):
+            dst[ids] = src.reshape(B, Hkv, npg, page_size, D).permute(0, 2, 3, 1, 4).reshape(B * npg, page_size, Hkv, D)
+        table = torch.tensor(perm[: B * npg], dtype=torch.int32).reshape(B, npg)
+        return kp, vp, table.to(kc.device), torch.tensor(lens, dtype=torch.int32, device=kc.device)
     table = torch.full((B, max_pages), -1, dtype=torch.int32)
     nxt = 0
     for b in range(B):

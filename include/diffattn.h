@@ -182,6 +182,42 @@ DIFFATTN_API int diffattn_decode_v2_noalloc(const void* q, const void* kc, const
                                             void* out, diffattn_dtype dtype, int B, int Hq, int Hkv, int T,
                                             int D, void* stream);
 
+/* Workspace, in bytes, that diffattn_decode_v2_paged needs on the current
+ * device for B sequences over Hkv KV heads (independent of the lengths and the
+ * page size).  0 for invalid sizes. */
+DIFFATTN_API size_t diffattn_decode_paged_workspace_size(int B, int Hkv);
+
+/* Paged, variable-length single-token V2 decode (serving layout).  Same
+ * operation as diffattn_decode_v2, each sequence against its own cache.
+ * The tutorial ("差分注意力", section V1 到 V2 的 diff) names serving engines
+ * such as vLLM and SGLang as the integration target but gives no layout; the
+ * layout below is the common token-major page pool.
+ *   q           : [B, Hq, 128] bf16                  (device)
+ *   k_pages,
+ *   v_pages     : [num_pages, page_size, Hkv, 128] bf16: page p holds
+ *                 page_size consecutive tokens of one sequence, every KV head
+ *                 of a token side by side                           (device)
+ *   block_table : int32 [B, max_pages]; row b lists sequence b's page ids in
+ *                 token order                                       (device)
+ *   seq_lens    : int32 [B]; sequence b is its first seq_lens[b] tokens.
+ *                 Values are clamped to [0, max_pages * page_size]; only the
+ *                 first ceil(seq_lens[b] / page_size) entries of row b are
+ *                 read, and a page id outside [0, num_pages) reads zeros.
+ *                 A length of 0 gives a zero output.                (device)
+ *   lambda      : f32 [Hq/2];  out : [B, Hq/2, 128] bf16            (device)
+ *   ws          : device workspace of diffattn_decode_paged_workspace_size
+ *                 bytes, 16-byte aligned, owned by the caller.  The call also
+ *                 leaves the per-sequence block prefix there.
+ * Requires bf16, Hq even, Hq % Hkv == 0, Hq/Hkv even and <= 8, page_size in
+ * {16, 32, 64, 128, 256}, 1 <= B <= 2048, and B * Hkv * max_pages *
+ * page_size / 64 < 2^31.  Rows of a page past a sequence's length are never
+ * used, whatever they hold (they may be uninitialised). */
+DIFFATTN_API int diffattn_decode_v2_paged(const void* q, const void* k_pages, const void* v_pages,
+                                          const int* block_table, const int* seq_lens, const float* lambda,
+                                          void* out, diffattn_dtype dtype, int B, int Hq, int Hkv,
+                                          int num_pages, int page_size, int max_pages, void* ws,
+                                          size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,23 @@ def test_argument_errors_before_any_device_call(L):
     assert L.diffattn_decode_v2(P, P, P, P, P, da.BF16, 1, 5, 1, 64, 128, P, 1 << 20, s) == da.ERR_INVALID_ARG
     assert L.diffattn_decode_v2(P, P, P, P, P, da.BF16, 1, 32, 2, 64, 128, P, 1 << 20, s) == da.ERR_UNSUPPORTED
     assert L.diffattn_decode_v1(P, P, P, P, P, P, P, da.BF16, 1, 16, 2, 64, 64, 128, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+    # paged decode: (q, k_pages, v_pages, table, lens, lambda, out, dtype, B, Hq, Hkv, num_pages, page_size,
+    # max_pages, ws, ws_bytes, stream)
+    pg = lambda *args: L.diffattn_decode_v2_paged(*args)  # noqa: E731
+    assert pg(P, P, P, P, P, P, P, da.BF16, 0, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_INVALID_ARG     # B = 0
+    assert pg(P, P, P, P, P, P, P, da.BF16, 4096, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_INVALID_ARG  # B > 2048
+    assert pg(P, P, P, P, P, P, P, da.BF16, 2, 6, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_INVALID_ARG      # Hq/Hkv odd
+    assert pg(P, P, P, P, P, P, P, da.BF16, 2, 16, 2, 0, 16, 4, P, 1 << 20, s) == da.ERR_INVALID_ARG     # no pages
+    assert pg(P, P, P, P, P, P, P, da.BF16, 2, 16, 2, 8, 48, 4, P, 1 << 20, s) == da.ERR_UNSUPPORTED     # page size
+    assert "page_size" in da.last_error()
+    assert pg(P, P, P, P, P, P, P, da.F32, 2, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_UNSUPPORTED      # f32
+    assert pg(P, P, P, P, P, P, P, da.BF16, 2, 32, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_UNSUPPORTED     # 16 per group
+    assert pg(P, P, P, None, P, P, P, da.BF16, 2, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_INVALID_ARG  # null table
+    assert pg(Pm, P, P, P, P, P, P, da.BF16, 2, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_MISALIGNED     # q
+    Pi = ctypes.c_void_p(66)
+    assert pg(P, P, P, Pi, P, P, P, da.BF16, 2, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_MISALIGNED     # table
+    assert pg(P, P, P, P, P, P, P, da.BF16, 2048, 16, 8, 8, 256, 1 << 20, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+    assert "2^31" in da.last_error()
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch):
