@@ -191,6 +191,27 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
         const long long it = x - lo;
         const int st = (int)(it % NST);
         const long long use = it / NST;
+        // Paged mode: locate the block and read its page ids before waiting
+        // for the stage, so the table reads overlap the wait.
+        int pg = 0, pkey0 = 0, pparts = 1, pages[4] = {0, 0, 0, 0};
+        if constexpr (PAGED) {
+          const int b = dec_find_seq(S.cu, a.B, x);
+          const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
+          const int within = (int)(x - S.cu[b]);
+          pg = within / nb;
+          pkey0 = (within % nb) * DEC_KB;
+          const int* row = a.block_table + (size_t)b * a.max_pages + (pkey0 >> a.page_shift);
+          if (a.page_size >= DEC_KB) {
+            pages[0] = row[0];
+          } else {
+            // page parts of the block that hold a key of the sequence (>= 1);
+            // parts wholly past it are not loaded (masked, V rows zeroed)
+            pparts = min(DEC_KB, S.len[b] - pkey0 + a.page_size - 1) / a.page_size;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (i < pparts) pages[i] = row[i];
+          }
+        }
         if (use > 0 && !wait_bar(smem_u32(&S.empty[st]), (uint32_t)((use - 1) & 1), abort_flag, a.watch)) {
           ok = false;
           break;
@@ -198,31 +219,24 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
         const uint32_t fb = smem_u32(&S.full[st]);
         const uint32_t kd = smem_u32(S.k[st]), vd = smem_u32(S.v[st]);
         if constexpr (PAGED) {
-          const int b = dec_find_seq(S.cu, a.B, x);
-          const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
-          const int within = (int)(x - S.cu[b]);
-          const int g = within / nb, key0 = (within % nb) * DEC_KB;
-          const int* row = a.block_table + (size_t)b * a.max_pages;
           if (a.page_size >= DEC_KB) {
-            const int page = row[key0 >> a.page_shift], y = key0 & (a.page_size - 1);
+            const int y = pkey0 & (a.page_size - 1);
             mbar_expect_tx(fb, 2 * DEC_TILE_BYTES);
-            tma_load_4d(kd, &tmK1, fb, 0, g, y, page);
-            tma_load_4d(kd + DEC_TILE_BYTES / 2, &tmK1, fb, 64, g, y, page);
-            tma_load_4d(vd, &tmV, fb, 0, g, y, page);
-            tma_load_4d(vd + DEC_TILE_BYTES / 2, &tmV, fb, 64, g, y, page);
+            tma_load_4d(kd, &tmK1, fb, 0, pg, y, pages[0]);
+            tma_load_4d(kd + DEC_TILE_BYTES / 2, &tmK1, fb, 64, pg, y, pages[0]);
+            tma_load_4d(vd, &tmV, fb, 0, pg, y, pages[0]);
+            tma_load_4d(vd + DEC_TILE_BYTES / 2, &tmV, fb, 64, pg, y, pages[0]);
           } else {
-            // several pages per block; parts wholly past the sequence are not
-            // loaded (their rows are masked and their V rows zeroed)
-            const int len = S.len[b], ps = a.page_size;
-            const int parts = min(DEC_KB, len - key0 + ps - 1) / ps;   // >= 1: the block holds a key
-            mbar_expect_tx(fb, (uint32_t)(parts * ps * 128 * 4));
-            for (int i = 0; i < parts; ++i) {
-              const int page = row[(key0 >> a.page_shift) + i];
+            const int ps = a.page_size;
+            mbar_expect_tx(fb, (uint32_t)(pparts * ps * 128 * 4));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (i >= pparts) break;
               const uint32_t off = (uint32_t)(i * ps * 128);
-              tma_load_4d(kd + off, &tmK1, fb, 0, g, 0, page);
-              tma_load_4d(kd + DEC_TILE_BYTES / 2 + off, &tmK1, fb, 64, g, 0, page);
-              tma_load_4d(vd + off, &tmV, fb, 0, g, 0, page);
-              tma_load_4d(vd + DEC_TILE_BYTES / 2 + off, &tmV, fb, 64, g, 0, page);
+              tma_load_4d(kd + off, &tmK1, fb, 0, pg, 0, pages[i]);
+              tma_load_4d(kd + DEC_TILE_BYTES / 2 + off, &tmK1, fb, 64, pg, 0, pages[i]);
+              tma_load_4d(vd + off, &tmV, fb, 0, pg, 0, pages[i]);
+              tma_load_4d(vd + DEC_TILE_BYTES / 2 + off, &tmV, fb, 64, pg, 0, pages[i]);
             }
           }
           issued_last[st] = use;
