@@ -9,7 +9,10 @@ There is no CPU fallback: if the library is missing, every call raises.
 
 Inputs may be CUDA tensors (results stay on the device) or CPU tensors (they
 are copied to the current CUDA device, the kernels run there, and the result
-is copied back: the end-to-end path).
+is copied back: the end-to-end path).  For large CPU inputs the prefill
+entry points overlap the copies with the kernels: the work is cut into chunks
+of (batch, KV-head group), each uploaded, computed and downloaded on its own
+stream, so chunk c computes while chunk c+1 uploads and chunk c-1 downloads.
 """
 
 from __future__ import annotations
@@ -144,8 +147,78 @@ def compute_lambda(lq1, lk1, lq2, lk2, lam_init: float, out=None):
     return _finish(host, out)
 
 
+# ----------------------------------------------------------------------------
+# end-to-end prefill on host tensors: chunked, with copies overlapping kernels
+_PIPELINE_MIN_BYTES = 64 << 20     # smaller inputs take the plain copy-compute-copy path
+_PIPELINE_CHUNK_UNITS = 1024       # 128-row blocks per chunk kernel: several waves of CTAs
+_pipe_streams = {}
+
+
+def _pipelined(tensors, out):
+    return (out is None and all(t.device.type == "cpu" for t in tensors)
+            and sum(t.numel() * t.element_size() for t in tensors) >= _PIPELINE_MIN_BYTES)
+
+
+def _prefill_host_pipelined(v1, qs, ks, v, lam, causal, rmsnorm, eps):
+    """CPU q/k/v in, pinned CPU output back.  qs: [q] (V2) or [q1, q2] (V1);
+    ks: [k] or [k1, k2].  Chunk = one batch entry and a run of whole KV heads
+    (with their query heads and outputs), all contiguous slices."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pin = lambda t: t.contiguous() if t.is_pinned() else t.contiguous().pin_memory()  # noqa: E731
+    qs, ks, v = [pin(t) for t in qs], [pin(t) for t in ks], pin(v)
+    B, Hq, Lq, d = qs[0].shape
+    Hkv, Lk, dv = ks[0].shape[1], ks[0].shape[2], v.shape[3]
+    if Hkv < 1 or Hq % Hkv:
+        raise ValueError("query heads must be a multiple of the KV heads")
+    grp = Hq // Hkv
+    opg = grp if v1 else grp // 2                       # output heads per KV head
+    Hout = Hq if v1 else Hq // 2
+    n_rb = -(-Lq // 128)
+    gpc = max(1, min(Hkv, -(-_PIPELINE_CHUNK_UNITS // max(1, n_rb * opg))))
+    chunks = [(b, g0, min(Hkv, g0 + gpc)) for b in range(B) for g0 in range(0, Hkv, gpc)]
+
+    lam_d = lam.to(dev, non_blocking=False).contiguous()
+    qd = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in qs]
+    kd = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in ks]
+    vd = torch.empty(v.shape, dtype=v.dtype, device=dev)
+    out_d = torch.empty((B, Hout, Lq, dv), dtype=qs[0].dtype, device=dev)
+    out_h = torch.empty(out_d.shape, dtype=out_d.dtype, pin_memory=True)
+    if dev.index not in _pipe_streams:
+        _pipe_streams[dev.index] = tuple(torch.cuda.Stream(device=dev) for _ in range(3))
+    s_in, s_run, s_out = _pipe_streams[dev.index]
+    for st in (s_in, s_run, s_out):
+        st.wait_stream(torch.cuda.current_stream())
+    L, dt = load(), _dtype_code(qs[0])
+    for b, g0, g1 in chunks:
+        hq, hk, ho = slice(g0 * grp, g1 * grp), slice(g0, g1), slice(g0 * opg, g1 * opg)
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(qd, qs):
+                dst[b, hq].copy_(src[b, hq], non_blocking=True)
+            for dst, src in zip(kd, ks):
+                dst[b, hk].copy_(src[b, hk], non_blocking=True)
+            vd[b, hk].copy_(v[b, hk], non_blocking=True)
+        s_run.wait_stream(s_in)
+        with torch.cuda.stream(s_run):
+            nq, nk = (g1 - g0) * grp, g1 - g0
+            if v1:
+                _check(L.diffattn_fwd_v1(_ptr(qd[0][b, hq]), _ptr(kd[0][b, hk]), _ptr(qd[1][b, hq]),
+                                         _ptr(kd[1][b, hk]), _ptr(vd[b, hk]), _ptr(lam_d[ho]), _ptr(out_d[b, ho]),
+                                         dt, 1, nq, nk, Lq, Lk, d, dv, int(causal), int(rmsnorm), float(eps),
+                                         _stream()))
+            else:
+                _check(L.diffattn_fwd_v2(_ptr(qd[0][b, hq]), _ptr(kd[0][b, hk]), _ptr(vd[b, hk]), _ptr(lam_d[ho]),
+                                         _ptr(out_d[b, ho]), dt, 1, nq, nk, Lq, Lk, d, int(causal), _stream()))
+        s_out.wait_stream(s_run)
+        with torch.cuda.stream(s_out):
+            out_h[b, ho].copy_(out_d[b, ho], non_blocking=True)
+    s_out.synchronize()
+    return out_h
+
+
 def fwd_v1(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5, out=None):
     """V1 layout: q1,q2 [B,H,Lq,d]; k1,k2 [B,Hkv,Lk,d]; v [B,Hkv,Lk,dv]; lam f32 [H]."""
+    if _pipelined([q1, k1, q2, k2, v], out):
+        return _prefill_host_pipelined(True, [q1, q2], [k1, k2], v, lam, causal, rmsnorm, eps)
     host, (q1, k1, q2, k2, v, lam) = _prep([q1, k1, q2, k2, v, lam])
     B, H, Lq, d = q1.shape
     Hkv, Lk, dv = k1.shape[1], k1.shape[2], v.shape[3]
@@ -159,6 +232,8 @@ def fwd_v1(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5, out=Non
 
 def fwd_v2(q, k, v, lam, causal=True, out=None):
     """V2 layout: q [B,Hq,Lq,D]; k,v [B,Hkv,Lk,D]; lam f32 [Hq/2] -> [B,Hq/2,Lq,D]."""
+    if _pipelined([q, k, v], out):
+        return _prefill_host_pipelined(False, [q], [k], v, lam, causal, False, 1e-5)
     host, (q, k, v, lam) = _prep([q, k, v, lam])
     B, Hq, Lq, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]

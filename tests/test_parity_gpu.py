@@ -326,3 +326,25 @@ def test_bf16_near_unit_lambda_with_similar_maps(lam_value):
     out = da.fwd_v2(q, k, v, lam, causal=True)
     ref = orc.diffattn_v2(q, k, v, np.array([lam_value]), causal=True)
     assert rel_err(out, ref) <= BF16_TOL
+
+
+def test_host_pipelined_prefill_matches_device_path(monkeypatch):
+    """CPU inputs take the chunked path (copies overlapping kernels); forced on
+    here for small shapes with many chunks, it must give the device path's bits."""
+    monkeypatch.setattr(da, "_PIPELINE_MIN_BYTES", 0)
+    monkeypatch.setattr(da, "_PIPELINE_CHUNK_UNITS", 3)
+    g = torch.Generator(device="cpu").manual_seed(404)
+    s = 1 / math.sqrt(128)
+    mk = lambda *shape, std=s: (torch.randn(*shape, generator=g) * std).to(torch.bfloat16)  # noqa: E731
+    q, k, v = mk(2, 8, 300, 128), mk(2, 4, 300, 128), mk(2, 4, 300, 128)
+    lam = torch.rand(4, generator=g) * 0.8
+    host = da.fwd_v2(q, k, v, lam, causal=True)
+    dev = da.fwd_v2(q.to(DEV), k.to(DEV), v.to(DEV), lam.to(DEV), causal=True)
+    assert host.device.type == "cpu" and torch.equal(host, dev.cpu())
+    q1, q2 = mk(2, 6, 200, 64, std=0.125), mk(2, 6, 200, 64, std=0.125)
+    k1, k2, vv = mk(2, 3, 200, 64, std=0.125), mk(2, 3, 200, 64, std=0.125), mk(2, 3, 200, 128, std=0.125)
+    lam1 = torch.rand(6, generator=g) * 0.8
+    host = da.fwd_v1(q1, k1, q2, k2, vv, lam1, causal=True, rmsnorm=True)
+    dev = da.fwd_v1(q1.to(DEV), k1.to(DEV), q2.to(DEV), k2.to(DEV), vv.to(DEV), lam1.to(DEV), causal=True,
+                    rmsnorm=True)
+    assert torch.equal(host, dev.cpu())
