@@ -19,10 +19,13 @@ Modules:
               step, no blocking beyond a row chunk that does not change the math).
   brute    -- pure-Python per-element loops for tiny shapes; an independent twin
               used to cross-check ``diffattn``.
+  backward -- the chain rule of the forward (dQ, dK, dV, dlambda and lambda's
+              parameter gradients) in fp64, pinned by finite differences and an
+              independent autograd derivation (tests/test_oracle_backward.py).
 
 Parity status: every function is pinned by tests in ``tests/test_oracle.py``
 except the page's claimed noise-floor percentages and the SNR claim of the
 tutorial's Step 3, which are "parity unpinned" (see ``diffattn.noise_probe``).
 """
 
-from . import diffattn, brute  # noqa: F401
+from . import backward, brute, diffattn  # noqa: F401
