@@ -31,7 +31,8 @@ F32, BF16 = 0, 1
 EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffattn_fwd_v1", "diffattn_fwd_v2",
            "diffattn_decode_workspace_size", "diffattn_decode_v2", "diffattn_decode_v1", "diffattn_last_error",
            "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc",
-           "diffattn_decode_paged_workspace_size", "diffattn_decode_v2_paged"]
+           "diffattn_decode_paged_workspace_size", "diffattn_decode_v2_paged", "diffattn_fwd_v2_train",
+           "diffattn_bwd_v2_workspace_size", "diffattn_bwd_v2", "diffattn_lambda_backward"]
 
 _lib = None
 
@@ -67,6 +68,10 @@ def load():
         "diffattn_decode_v2_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, I, P]),
         "diffattn_decode_paged_workspace_size": (Z, [I, I]),
         "diffattn_decode_v2_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]),
+        "diffattn_fwd_v2_train": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]),
+        "diffattn_bwd_v2_workspace_size": (Z, [I, I, I]),
+        "diffattn_bwd_v2": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]),
+        "diffattn_lambda_backward": (I, [P, P, P, P, P, I, I, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -243,6 +248,43 @@ def fwd_v2(q, k, v, lam, causal=True, out=None):
     _check(load().diffattn_fwd_v2(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), dt, B, Hq, Hkv, Lq, Lk, D,
                                   int(causal), _stream()))
     return _finish(host, out)
+
+
+def fwd_v2_train(q, k, v, lam, causal=True):
+    """V2 forward that also returns what the backward needs: (out [B,Hq/2,Lq,D],
+    lse f32 [B,Hq/2,2,Lq] (log2 units), o_maps [B,Hq/2,2,Lq,D] = O_m / l_m).  bf16, device tensors."""
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    out = torch.empty((B, Hq // 2, Lq, D), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, Hq // 2, 2, Lq), dtype=torch.float32, device=q.device)
+    o_maps = torch.empty((B, Hq // 2, 2, Lq, D), dtype=q.dtype, device=q.device)
+    _check(load().diffattn_fwd_v2_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(lse), _ptr(o_maps),
+                                        _dtype_code(q), B, Hq, Hkv, Lq, Lk, D, int(causal), _stream()))
+    return out, lse, o_maps
+
+
+def bwd_v2(q, k, v, lam, dout, lse, o_maps, causal=True, workspace=None):
+    """Gradients of the V2 forward: (dq, dk, dv, dlam) given dout [B,Hq/2,Lq,D] and the
+    training forward's lse and o_maps.  bf16 gradients, f32 dlam.  Device tensors."""
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dlam = torch.empty(Hq // 2, dtype=torch.float32, device=q.device)
+    need = int(load().diffattn_bwd_v2_workspace_size(B, Hq, Lq))
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check(load().diffattn_bwd_v2(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(dout), _ptr(lse), _ptr(o_maps),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _dtype_code(q), B, Hq, Hkv, Lq, Lk, D,
+                                  int(causal), _ptr(ws), ws.numel() * ws.element_size(), _stream()))
+    return dq, dk, dv, dlam
+
+
+def lambda_backward(lq1, lk1, lq2, lk2, dlam):
+    """Gradients of the four lambda parameter vectors ([H, dim] f32) given dlam [H]."""
+    H, dim = lq1.shape
+    outs = [torch.empty_like(lq1) for _ in range(4)]
+    _check(load().diffattn_lambda_backward(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), _ptr(dlam), H, dim,
+                                           *[_ptr(t) for t in outs], _stream()))
+    return tuple(outs)
 
 
 def decode_workspace_size(B: int, Hkv: int, T: int, dv: int = 128) -> int:

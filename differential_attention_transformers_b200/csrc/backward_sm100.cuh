@@ -1,0 +1,587 @@
+// backward_sm100.cuh -- gradients of the V2 differential attention prefill on tcgen05.
+//
+// Forward ("差分注意力" tutorial, section 差分思路 and Step 2; V2 layout from
+// its section V1 到 V2 的 diff): per diff pair h, with maps m = 1, 2 on Q heads
+// (2h, 2h+1) and the pair's KV head g,
+//   A_m = softmax(Q_m K^T / sqrt(d)),  O = (A_1 - lambda A_2) V.
+// Chain rule, given dO (the pages print no backward):
+//   dV  = sum over the pairs of g of (A_1 - lambda A_2)^T dO
+//   dW  = dO V^T,  D_m = rowsum(dO * O_m)  with O_m = A_m V
+//   dS_1 = A_1 (dW - D_1),  dS_2 = -lambda A_2 (dW - D_2)
+//   dQ_m = dS_m K / sqrt(d),  dK = sum over the group of dS_m^T Q_m / sqrt(d)
+//   dlambda = -sum(dO * O_2)
+// A_m is recomputed from the scores and the forward's per-row log-sum-exp
+// (log2 units): A_m = 2^(S_m log2(e)/sqrt(d) - lse_m).
+//
+// Three kernels:
+//   bwd_prep_kernel  D_m per row from dO and the forward's normalised map
+//                    outputs, the log-sum-exp copied into a padded layout, and
+//                    per-block partial sums of dlambda (reduced in a fixed
+//                    order by bwd_dlambda_kernel, so the result is
+//                    deterministic).
+//   bwd_dq_kernel    query-stationary: one CTA per 128 rows of one Q head (one
+//                    map).  Per 64-key tile: S = Q K^T and dP = dO V^T into
+//                    TMEM, dS = c P (dP - D) written over S as bf16, then
+//                    dQ += dS K with dS as the TMEM operand.
+//   bwd_dkv_kernel   key-stationary: one CTA per 128 keys of one KV head.  Per
+//                    64-row step of each Q head of the group: S^T = K Q^T and
+//                    dP^T = V dO^T into TMEM, then w P^T (w = 1 or -lambda)
+//                    and dS^T written back as bf16, and dV += (w P)^T dO,
+//                    dK += dS^T Q with those as the TMEM operands.
+// Computing dQ apart from dK/dV recomputes S and dP once more but needs no
+// atomics, and each kernel fits TMEM: dQ 384 columns, dK/dV 512.
+// Both MMA kernels use the forward's pipeline: a TMA producer warp, one
+// issuing thread for the S-type products and one for the accumulating ones,
+// and four warps (thread = TMEM lane) between them.
+#pragma once
+
+#include "common.cuh"
+#include "prefill_sm100.cuh"
+
+namespace da {
+
+constexpr int BW_THREADS = 224;   // warps 0-3 elementwise, 4 producer/TMEM, 5 accumulating MMAs, 6 S-type MMAs
+constexpr int BW_NS = 3;          // pipeline stages
+constexpr int BW_RB = 64;         // rows per step of the key-stationary kernel
+
+struct BwdArgs {
+  const float* lambda;   // [Hp]
+  const float* lse_p;    // [B, Hp, 2, Lp] log-sum-exp (log2 units), +inf past Lq
+  const float* dd;       // [B, Hp, 2, Lp] D_m, 0 past Lq
+  __nv_bfloat16* dq;     // [B, Hq, Lq, 128]
+  __nv_bfloat16* dk;     // [B, Hkv, Lk, 128]
+  __nv_bfloat16* dv;     // [B, Hkv, Lk, 128]
+  int B, Hq, Hkv, Lq, Lk, Lp;
+  int causal;
+  float scale, scale_log2;
+  Watch watch;
+};
+
+// ------------------------------------------------------------------- prep --
+struct BwdPrepArgs {
+  const __nv_bfloat16* dout;    // [B, Hp, Lq, 128]
+  const __nv_bfloat16* o_maps;  // [B, Hp, 2, Lq, 128]
+  const float* lse;             // [B, Hp, 2, Lq]
+  float* lse_p;                 // [B, Hp, 2, Lp]
+  float* dd;                    // [B, Hp, 2, Lp]
+  float* part;                  // [B * Hp, Lp / 64] partial sums of -D_2
+  int B, Hp, Lq, Lp;
+};
+
+// grid (Lp / 64, B * Hp), 256 threads: warp w handles rows 8w .. 8w+7 of the block.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
+  __shared__ float wsum[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  float acc = 0.f;
+  for (int i = 0; i < 8; ++i) {
+    const int row = blockIdx.x * 64 + warp * 8 + i;
+    float d[2] = {0.f, 0.f};
+    if (row < a.Lq) {
+      const __nv_bfloat16* go = a.dout + ((size_t)bh * a.Lq + row) * 128 + lane * 4;
+      const uint2 gv = *reinterpret_cast<const uint2*>(go);
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint2 ov =
+            *reinterpret_cast<const uint2*>(a.o_maps + (((size_t)bh * 2 + m) * a.Lq + row) * 128 + lane * 4);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float2 gf = __bfloat1622float2(g2[j]), of = __bfloat1622float2(o2[j]);
+          s = fmaf(gf.x, of.x, s);
+          s = fmaf(gf.y, of.y, s);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        d[m] = s;
+      }
+    }
+    if (lane < 2) {
+      const size_t at = ((size_t)bh * 2 + lane) * a.Lp + row;
+      a.dd[at] = d[lane];
+      a.lse_p[at] = row < a.Lq ? a.lse[((size_t)bh * 2 + lane) * a.Lq + row] : INFINITY;
+    }
+    acc -= d[1];
+  }
+  if (lane == 0) wsum[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += wsum[w];
+    a.part[(size_t)bh * (a.Lp / 64) + blockIdx.x] = t;
+  }
+}
+
+// One thread per pair: dlambda[h] = sum over batch and row blocks, fixed order.
+__global__ void bwd_dlambda_kernel(const float* part, float* dlambda, int B, int Hp, int nblk) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= Hp) return;
+  double t = 0.0;
+  for (int b = 0; b < B; ++b)
+    for (int i = 0; i < nblk; ++i) t += (double)part[((size_t)b * Hp + h) * nblk + i];
+  dlambda[h] = (float)t;
+}
+
+// ------------------------------------------------------------ dQ (Q-stationary) --
+struct BwQSmem {
+  alignas(1024) uint8_t q[2 * PF_QBOX];            // Q tile of the head: 128 rows, dims 0-63 box, 64-127 box
+  alignas(1024) uint8_t o[2 * PF_QBOX];            // dO tile of the pair, same layout
+  alignas(1024) uint8_t k[BW_NS][2 * PF_KBOX];     // K tile: 64 keys, two boxes
+  alignas(1024) uint8_t v[BW_NS][2 * PF_KBOX];     // V tile
+  alignas(16) uint8_t stage[4][16 * 128];          // epilogue staging, per elementwise warp
+  alignas(8) uint64_t q_full;
+  uint64_t k_full[BW_NS], v_full[BW_NS], kv_empty[BW_NS];
+  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t fin;
+  uint64_t drain[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(BW_THREADS, 1)
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  BwQSmem& S = *reinterpret_cast<BwQSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &S.abort_flag;
+
+  // unit: rows r0..r0+127 of Q head qh of batch b, heaviest row blocks first
+  const int BQ = a.B * a.Hq;
+  const int n_rb = (a.Lq + PF_BM - 1) / PF_BM;
+  const int rb = n_rb - 1 - (int)(blockIdx.x / BQ);
+  const int b = (int)(blockIdx.x % BQ) / a.Hq, qh = (int)(blockIdx.x % BQ) % a.Hq;
+  const int Hp = a.Hq / 2, h = qh / 2, m = qh & 1, g = qh / (a.Hq / a.Hkv);
+  const int r0 = rb * PF_BM;
+  long long kend = a.causal ? (long long)min(r0 + PF_BM, a.Lq) - 1 + (a.Lk - a.Lq) + 1 : a.Lk;
+  kend = max(0LL, min(kend, (long long)a.Lk));
+  const int nT = (int)((kend + PF_BN - 1) / PF_BN);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&S.q_full), 1);
+    for (int i = 0; i < BW_NS; ++i) {
+      mbar_init(smem_u32(&S.k_full[i]), 1);
+      mbar_init(smem_u32(&S.v_full[i]), 1);
+      mbar_init(smem_u32(&S.kv_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&S.s_full[i]), 1);
+      mbar_init(smem_u32(&S.p_full[i]), 128);
+      mbar_init(smem_u32(&S.s_free[i]), 1);
+      mbar_init(smem_u32(&S.drain[i]), 1);
+    }
+    mbar_init(smem_u32(&S.fin), 1);
+    S.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(&S.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;   // S [0,128), dP [128,256), dQ [256,384)
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0 && nT > 0) {
+      const uint32_t qb = smem_u32(&S.q_full);
+      mbar_expect_tx(qb, 4 * PF_QBOX);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(smem_u32(S.q) + x * PF_QBOX, &tmQ, qb, 64 * x, r0, b * a.Hq + qh);
+        tma_load_3d(smem_u32(S.o) + x * PF_QBOX, &tmO, qb, 64 * x, r0, b * Hp + h);
+      }
+      int last_use[BW_NS];
+      for (int i = 0; i < BW_NS; ++i) last_use[i] = -1;
+      for (int j = 0; j < nT; ++j) {
+        const int st = j % BW_NS, use = j / BW_NS;
+        if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
+        const uint32_t kb = smem_u32(&S.k_full[st]), vb = smem_u32(&S.v_full[st]);
+        mbar_expect_tx(kb, 2 * PF_KBOX);
+        tma_load_3d(smem_u32(S.k[st]), &tmK, kb, 0, j * PF_BN, b * a.Hkv + g);
+        tma_load_3d(smem_u32(S.k[st]) + PF_KBOX, &tmK, kb, 64, j * PF_BN, b * a.Hkv + g);
+        mbar_expect_tx(vb, 2 * PF_KBOX);
+        tma_load_3d(smem_u32(S.v[st]), &tmV, vb, 0, j * PF_BN, b * a.Hkv + g);
+        tma_load_3d(smem_u32(S.v[st]) + PF_KBOX, &tmV, vb, 64, j * PF_BN, b * a.Hkv + g);
+        last_use[st] = use;
+      }
+      drain_bar(qb, 0, a.watch.status);
+      for (int i = 0; i < BW_NS; ++i) {
+        if (last_use[i] >= 0) {
+          drain_bar(smem_u32(&S.k_full[i]), last_use[i] & 1, a.watch.status);
+          drain_bar(smem_u32(&S.v_full[i]), last_use[i] & 1, a.watch.status);
+        }
+      }
+    }
+  } else if (warp >= 5) {
+    // --------------------------------------------------------- MMA issuers --
+    if (lane == 0 && nT > 0) {
+      constexpr uint32_t HI = umma_desc_hi(1024);
+      constexpr uint32_t KSTAGE = (2 * PF_KBOX) >> 4;
+      const int issuer = warp - 5;   // 0: dQ += dS K, 1: S = Q K^T and dP = dO V^T
+      bool ok = true;
+      if (issuer == 0) {
+        constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, true);
+        const uint32_t k_mn0 = umma_desc_lo(smem_u32(S.k[0]), PF_KBOX);   // K as the N-major B operand
+        for (int j = 0; ok && j < nT; ++j) {
+          const int bb = j & 1;
+          // this thread reads the K stage too: acquire it here
+          if (!(ok = wait_bar(smem_u32(&S.k_full[j % BW_NS]), (j / BW_NS) & 1, abort_flag, a.watch))) break;
+          if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
+          tc_fence_after();
+          const uint32_t klo = k_mn0 + (uint32_t)(j % BW_NS) * KSTAGE;
+#pragma unroll
+          for (int s = 0; s < PF_BN / 16; ++s)
+            mma_ts_w(tmem + 256, tmem + bb * 64 + s * 8, klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+                     (j > 0 || s > 0));
+          mma_commit(smem_u32(&S.s_free[bb]));
+          mma_commit(smem_u32(&S.kv_empty[j % BW_NS]));
+        }
+        if (ok) mma_commit(smem_u32(&S.fin));
+      } else {
+        constexpr uint32_t IDESC_S = idesc_bf16_f32(128, PF_BN, false);
+        const uint32_t q_lo = umma_desc_lo(smem_u32(S.q), 16), o_lo = umma_desc_lo(smem_u32(S.o), 16);
+        const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16), v_lo0 = umma_desc_lo(smem_u32(S.v[0]), 16);
+        ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
+        for (int j = 0; ok && j < nT; ++j) {
+          const int bb = j & 1, st = j % BW_NS;
+          if (!(ok = wait_bar(smem_u32(&S.k_full[st]), (j / BW_NS) & 1, abort_flag, a.watch))) break;
+          if (!(ok = wait_bar(smem_u32(&S.v_full[st]), (j / BW_NS) & 1, abort_flag, a.watch))) break;
+          if (j >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch)))
+            break;
+          tc_fence_after();
+          const uint32_t klo = k_lo0 + (uint32_t)st * KSTAGE, vlo = v_lo0 + (uint32_t)st * KSTAGE;
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+            mma_ss_w(tmem + bb * 64, q_lo + ao, HI, klo + bo, HI, IDESC_S, s > 0);
+          }
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+            mma_ss_w(tmem + 128 + bb * 64, o_lo + ao, HI, vlo + bo, HI, IDESC_S, s > 0);
+          }
+          mma_commit(smem_u32(&S.s_full[bb]));
+        }
+      }
+      mma_commit(smem_u32(&S.drain[issuer]));
+      drain_bar(smem_u32(&S.drain[issuer]), 0, a.watch.status);
+    }
+  } else {
+    // ------------------------------------------- elementwise (thread = row) --
+    const int wq = warp, r = threadIdx.x;
+    const int rg = r0 + r;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const size_t stat = (((size_t)b * Hp + h) * 2 + m) * a.Lp + rg;
+    const float lse = a.lse_p[stat], dsum = a.dd[stat];
+    const float c = a.scale * (m == 0 ? 1.f : -a.lambda[h]);
+    const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
+    bool ok = true;
+    for (int j = 0; j < nT; ++j) {
+      const int bb = j & 1;
+      if (!(ok = warp_wait(smem_u32(&S.s_full[bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t sv[32], pv[32], ds[16];
+        tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
+        tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
+        tmem_wait_ld();
+        const long long lim = lastk - (long long)j * PF_BN - ch * 32;   // columns > lim are masked
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 2 * i + e;
+            const float x = col > lim ? -INFINITY : fmaf(__uint_as_float(sv[col]), a.scale_log2, -lse);
+            dsv[e] = c * ex2(x) * (__uint_as_float(pv[col]) - dsum);
+          }
+          ds[i] = pack_bf16(dsv[0], dsv[1]);
+        }
+        tmem_st16p(tmem + lane_off + bb * 64 + ch * 16, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&S.p_full[bb]));
+    }
+    // ---- epilogue: dQ rows ----
+    bool have = nT == 0;
+    float y[64];
+    if (nT > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
+    if (have) {
+      if (nT > 0) tc_fence_after();
+      __nv_bfloat16* base = a.dq + ((size_t)b * a.Hq + qh) * a.Lq * 128;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t o[32];
+          if (nT > 0) {
+            tmem_ld32p(tmem + lane_off + 256 + hf * 64 + cc * 32, o);
+            tmem_wait_ld();
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[cc * 32 + i] = nT > 0 ? __uint_as_float(o[i]) : 0.f;
+        }
+        pf_store_rows(S.stage[warp], y, base + hf * 64, r0 + wq * 32, a.Lq, lane);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------- dK/dV (KV-stationary) --
+struct BwKSmem {
+  alignas(1024) uint8_t k[2 * PF_QBOX];             // K tile: 128 keys, dims 0-63 box, 64-127 box
+  alignas(1024) uint8_t v[2 * PF_QBOX];             // V tile, same layout
+  alignas(1024) uint8_t q[BW_NS][2 * PF_KBOX];      // Q rows: 64, two boxes
+  alignas(1024) uint8_t o[BW_NS][2 * PF_KBOX];      // dO rows
+  alignas(16) float lse[BW_NS][BW_RB];
+  alignas(16) float dd[BW_NS][BW_RB];
+  alignas(16) uint8_t stage[4][16 * 128];
+  alignas(8) uint64_t kv_full;
+  uint64_t st_full[BW_NS], st_empty[BW_NS];
+  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t fin;
+  uint64_t drain[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(BW_THREADS, 1)
+bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  BwKSmem& S = *reinterpret_cast<BwKSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &S.abort_flag;
+
+  // unit: keys k0..k0+127 of KV head g of batch b; low key tiles (most rows) first
+  const int BG = a.B * a.Hkv;
+  const int kt = (int)(blockIdx.x / BG);
+  const int b = (int)(blockIdx.x % BG) / a.Hkv, g = (int)(blockIdx.x % BG) % a.Hkv;
+  const int k0 = kt * PF_BM;
+  const int grp = a.Hq / a.Hkv, Hp = a.Hq / 2;
+  const int off = a.Lk - a.Lq;
+  // first 64-row block holding a row that sees key k0 (causal: row >= k0 - off)
+  const int rb0 = (a.causal && k0 - off > 0) ? (k0 - off) / BW_RB : 0;
+  const int n_rb = (a.Lq + BW_RB - 1) / BW_RB;
+  const int per_head = max(0, n_rb - rb0);
+  const int nS = grp * per_head;   // steps: (head of the group, row block)
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&S.kv_full), 1);
+    for (int i = 0; i < BW_NS; ++i) {
+      mbar_init(smem_u32(&S.st_full[i]), 1);
+      mbar_init(smem_u32(&S.st_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&S.s_full[i]), 1);
+      mbar_init(smem_u32(&S.p_full[i]), 128);
+      mbar_init(smem_u32(&S.s_free[i]), 1);
+      mbar_init(smem_u32(&S.drain[i]), 1);
+    }
+    mbar_init(smem_u32(&S.fin), 1);
+    S.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(&S.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;   // S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512)
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0 && nS > 0) {
+      const uint32_t kvb = smem_u32(&S.kv_full);
+      mbar_expect_tx(kvb, 4 * PF_QBOX);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(smem_u32(S.k) + x * PF_QBOX, &tmK, kvb, 64 * x, k0, b * a.Hkv + g);
+        tma_load_3d(smem_u32(S.v) + x * PF_QBOX, &tmV, kvb, 64 * x, k0, b * a.Hkv + g);
+      }
+      int last_use[BW_NS];
+      for (int i = 0; i < BW_NS; ++i) last_use[i] = -1;
+      for (int i = 0; i < nS; ++i) {
+        const int st = i % BW_NS, use = i / BW_NS;
+        if (use > 0 && !wait_bar(smem_u32(&S.st_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
+        const int qh = g * grp + i / per_head, rb = rb0 + i % per_head;
+        const int hq = qh / 2, mq = qh & 1;
+        const uint32_t fb = smem_u32(&S.st_full[st]);
+        mbar_expect_tx(fb, 4 * PF_KBOX + 2 * BW_RB * 4);
+        for (int x = 0; x < 2; ++x) {
+          tma_load_3d(smem_u32(S.q[st]) + x * PF_KBOX, &tmQ, fb, 64 * x, rb * BW_RB, b * a.Hq + qh);
+          tma_load_3d(smem_u32(S.o[st]) + x * PF_KBOX, &tmO, fb, 64 * x, rb * BW_RB, b * Hp + hq);
+        }
+        const size_t stat = (((size_t)b * Hp + hq) * 2 + mq) * a.Lp + (size_t)rb * BW_RB;
+        bulk_load(smem_u32(S.lse[st]), a.lse_p + stat, BW_RB * 4, fb);
+        bulk_load(smem_u32(S.dd[st]), a.dd + stat, BW_RB * 4, fb);
+        last_use[st] = use;
+      }
+      drain_bar(kvb, 0, a.watch.status);
+      for (int i = 0; i < BW_NS; ++i)
+        if (last_use[i] >= 0) drain_bar(smem_u32(&S.st_full[i]), last_use[i] & 1, a.watch.status);
+    }
+  } else if (warp >= 5) {
+    // --------------------------------------------------------- MMA issuers --
+    if (lane == 0 && nS > 0) {
+      constexpr uint32_t HI = umma_desc_hi(1024);
+      constexpr uint32_t QSTAGE = (2 * PF_KBOX) >> 4;
+      const int issuer = warp - 5;   // 0: dV, dK accumulation; 1: S^T and dP^T
+      bool ok = true;
+      if (issuer == 0) {
+        constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, true);
+        const uint32_t o_mn0 = umma_desc_lo(smem_u32(S.o[0]), PF_KBOX), q_mn0 = umma_desc_lo(smem_u32(S.q[0]), PF_KBOX);
+        for (int i = 0; ok && i < nS; ++i) {
+          const int bb = i & 1, st = i % BW_NS;
+          // this thread reads the stage's Q and dO too: acquire them here
+          if (!(ok = wait_bar(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
+          if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
+          tc_fence_after();
+          const uint32_t olo = o_mn0 + (uint32_t)st * QSTAGE, qlo = q_mn0 + (uint32_t)st * QSTAGE;
+#pragma unroll
+          for (int s = 0; s < BW_RB / 16; ++s)   // dV += (w P)^T dO
+            mma_ts_w(tmem + 256, tmem + bb * 64 + s * 8, olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+                     (i > 0 || s > 0));
+#pragma unroll
+          for (int s = 0; s < BW_RB / 16; ++s)   // dK += dS^T Q
+            mma_ts_w(tmem + 384, tmem + 128 + bb * 64 + s * 8, qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+                     (i > 0 || s > 0));
+          mma_commit(smem_u32(&S.s_free[bb]));
+          mma_commit(smem_u32(&S.st_empty[st]));
+        }
+        if (ok) mma_commit(smem_u32(&S.fin));
+      } else {
+        constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BW_RB, false);
+        const uint32_t k_lo = umma_desc_lo(smem_u32(S.k), 16), v_lo = umma_desc_lo(smem_u32(S.v), 16);
+        const uint32_t q_lo0 = umma_desc_lo(smem_u32(S.q[0]), 16), o_lo0 = umma_desc_lo(smem_u32(S.o[0]), 16);
+        ok = wait_bar(smem_u32(&S.kv_full), 0, abort_flag, a.watch);
+        for (int i = 0; ok && i < nS; ++i) {
+          const int bb = i & 1, st = i % BW_NS;
+          if (!(ok = wait_bar(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
+          if (i >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[bb]), ((i - 2) >> 1) & 1, abort_flag, a.watch)))
+            break;
+          tc_fence_after();
+          const uint32_t qlo = q_lo0 + (uint32_t)st * QSTAGE, olo = o_lo0 + (uint32_t)st * QSTAGE;
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+            mma_ss_w(tmem + bb * 64, k_lo + ao, HI, qlo + bo, HI, IDESC_S, s > 0);
+          }
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+            mma_ss_w(tmem + 128 + bb * 64, v_lo + ao, HI, olo + bo, HI, IDESC_S, s > 0);
+          }
+          mma_commit(smem_u32(&S.s_full[bb]));
+        }
+      }
+      mma_commit(smem_u32(&S.drain[issuer]));
+      drain_bar(smem_u32(&S.drain[issuer]), 0, a.watch.status);
+    }
+  } else {
+    // ------------------------------------------- elementwise (thread = key) --
+    const int wq = warp, kr = threadIdx.x;
+    const int kg = k0 + kr;   // this thread's key
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    bool ok = true;
+    for (int i = 0; i < nS; ++i) {
+      const int bb = i & 1, st = i % BW_NS;
+      const int qh = g * grp + i / per_head, rb = rb0 + i % per_head;
+      const int mq = qh & 1;
+      const float w = mq == 0 ? 1.f : -a.lambda[qh / 2];   // weight of this map in A_1 - lambda A_2
+      const float cd = a.scale * w;
+      // The stage's log-sum-exp and D values came by bulk copy: wait for them here too.
+      if (!(ok = warp_wait(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
+      if (!(ok = warp_wait(smem_u32(&S.s_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
+      tc_fence_after();
+      // rows r = rb*64 + col see this key iff kg < Lk and (not causal or kg <= r + off)
+      const int rfirst = a.causal ? kg - off : 0;   // first row that sees kg (causal)
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t sv[32], pv[32], pw[16], ds[16];
+        tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
+        tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = ch * 32 + 2 * j + e;
+            const int row = rb * BW_RB + col;
+            const bool vis = kg < a.Lk && row >= rfirst;
+            const float x = vis ? fmaf(__uint_as_float(sv[2 * j + e]), a.scale_log2, -S.lse[st][col]) : -INFINITY;
+            const float p = ex2(x);
+            p2[e] = w * p;
+            d2[e] = cd * p * (__uint_as_float(pv[2 * j + e]) - S.dd[st][col]);
+          }
+          pw[j] = pack_bf16(p2[0], p2[1]);
+          ds[j] = pack_bf16(d2[0], d2[1]);
+        }
+        tmem_st16p(tmem + lane_off + bb * 64 + ch * 16, pw);
+        tmem_st16p(tmem + lane_off + 128 + bb * 64 + ch * 16, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&S.p_full[bb]));
+    }
+    // ---- epilogue: dV and dK rows of this tile's keys ----
+    bool have = nS == 0;
+    float y[64];
+    if (nS > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
+    if (have) {
+      if (nS > 0) tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK
+        __nv_bfloat16* base = (which ? a.dk : a.dv) + ((size_t)b * a.Hkv + g) * a.Lk * 128;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t o[32];
+            if (nS > 0) {
+              tmem_ld32p(tmem + lane_off + 256 + which * 128 + hf * 64 + cc * 32, o);
+              tmem_wait_ld();
+            }
+#pragma unroll
+            for (int t = 0; t < 32; ++t) y[cc * 32 + t] = nS > 0 ? __uint_as_float(o[t]) : 0.f;
+          }
+          pf_store_rows(S.stage[warp], y, base + hf * 64, k0 + wq * 32, a.Lk, lane);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace da

@@ -19,6 +19,7 @@
 #include "decode.cuh"
 #include "lambda_simt.cuh"
 #include "prefill_sm100.cuh"
+#include "backward_sm100.cuh"
 
 using namespace da;
 
@@ -82,6 +83,8 @@ constexpr size_t prefill_smem() { return sizeof(PfSmem<DQK>) + 1024; }
 constexpr int kDecNst = 2;
 constexpr size_t decode_smem() { return sizeof(DecSmem<kDecNst>) + 1024; }
 constexpr size_t decode_paged_smem() { return sizeof(DecSmem<kDecNst, true>) + 1024; }
+constexpr size_t bwd_dq_smem() { return sizeof(BwQSmem) + 1024; }
+constexpr size_t bwd_dkv_smem() { return sizeof(BwKSmem) + 1024; }
 constexpr int kDecCtasPerSm = 2;
 
 // Per-device set-up: SM count, status word address, kernel attributes,
@@ -111,6 +114,8 @@ int device_setup(DeviceInfo** out) {
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_paged_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_dq_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_dkv_smem()));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -177,7 +182,8 @@ int launch_simt(const SimtArgs& a, cudaStream_t s) {
 
 int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
                    const float* lambda, void* out, int B, int Hout, int Hq, int Hkv, int Lq, int Lk, int dqk,
-                   bool v1, int causal, int rms, float eps, cudaStream_t s) {
+                   bool v1, int causal, int rms, float eps, cudaStream_t s, float* lse = nullptr,
+                   void* o_maps = nullptr) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   if (Lq == 0 || B == 0 || Hout == 0) return ok();
@@ -201,6 +207,8 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.n_rb = (Lq + PF_BM - 1) / PF_BM;
   a.resid_tau = DIFFATTN_RESID_TAU;
   a.watch = make_watch(dev);
+  a.lse = lse;
+  a.o_maps = static_cast<__nv_bfloat16*>(o_maps);
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
   if (dqk == 64)
@@ -277,6 +285,71 @@ int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2
   const int Hout = v1 ? Hq : Hq / 2;
   decode_combine_kernel<<<(unsigned)(B * Hout), 128, 0, s>>>(c);
   CUDA_TRY(cudaGetLastError());
+  return ok();
+}
+
+// Backward workspace: padded log-sum-exp and D values [B, Hp, 2, Lp] (Lp = Lq
+// rounded up to 128; +inf / 0 past Lq), then the dlambda partials [B*Hp, Lp/64].
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+int bwd_rows_padded(int Lq) { return (Lq + PF_BM - 1) / PF_BM * PF_BM; }
+size_t bwd_ws_bytes(int B, int Hq, int Lq) {
+  const size_t Hp = (size_t)Hq / 2, Lp = (size_t)bwd_rows_padded(Lq);
+  return 2 * align256((size_t)B * Hp * 2 * Lp * 4) + align256((size_t)B * Hp * (Lp / 64) * 4);
+}
+
+int launch_backward_v2(const void* q, const void* k, const void* v, const float* lambda, const void* dout,
+                       const float* lse, const void* o_maps, void* dq, void* dk, void* dv, float* dlambda, int B,
+                       int Hq, int Hkv, int Lq, int Lk, int causal, void* ws, size_t ws_bytes, cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  const size_t need = bwd_ws_bytes(B, Hq, Lq);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(DIFFATTN_ERR_WORKSPACE, "backward workspace %zu B < required %zu B", ws_bytes, need);
+  if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  const int Hp = Hq / 2, Lp = bwd_rows_padded(Lq);
+  float* lse_p = static_cast<float*>(ws);
+  float* dd = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)B * Hp * 2 * Lp * 4));
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * align256((size_t)B * Hp * 2 * Lp * 4));
+  if (Lp > 0) {
+    BwdPrepArgs pa{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o_maps), lse,
+                   lse_p, dd, part, B, Hp, Lq, Lp};
+    bwd_prep_kernel<<<dim3((unsigned)(Lp / 64), (unsigned)(B * Hp)), 256, 0, s>>>(pa);
+    CUDA_TRY(cudaGetLastError());
+  }
+  bwd_dlambda_kernel<<<(Hp + 127) / 128, 128, 0, s>>>(part, dlambda, B, Hp, Lp / 64);
+  CUDA_TRY(cudaGetLastError());
+  BwdArgs a{};
+  a.lambda = lambda; a.lse_p = lse_p; a.dd = dd;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk; a.Lp = Lp;
+  a.causal = causal ? 1 : 0;
+  a.scale = (float)(1.0 / std::sqrt(128.0));
+  a.scale_log2 = log2e_over_sqrt(128);
+  a.watch = make_watch(dev);
+  const long long Lk_map = Lk > 0 ? Lk : 1;   // a zero extent is not encodable; no key is then loaded
+  const long long Lq_map = Lq > 0 ? Lq : 1;
+  if (Lq > 0) {   // dQ: one CTA per 128 rows of each Q head
+    CUtensorMap mq, mo, mk, mv;
+    if (int e = make_map(&mq, q, 128, Lq_map, (long long)B * Hq, PF_BM)) return e;
+    if (int e = make_map(&mo, dout, 128, Lq_map, (long long)B * Hp, PF_BM)) return e;
+    if (int e = make_map(&mk, Lk > 0 ? k : q, 128, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+    if (int e = make_map(&mv, Lk > 0 ? v : q, 128, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+    const long long units = (long long)((Lq + PF_BM - 1) / PF_BM) * B * Hq;
+    bwd_dq_kernel<<<(unsigned)units, BW_THREADS, bwd_dq_smem(), s>>>(mq, mo, mk, mv, a);
+    CUDA_TRY(cudaGetLastError());
+  }
+  if (Lk > 0) {   // dK, dV: one CTA per 128 keys of each KV head
+    CUtensorMap mk, mv, mq, mo;
+    if (int e = make_map(&mk, k, 128, Lk_map, (long long)B * Hkv, PF_BM)) return e;
+    if (int e = make_map(&mv, v, 128, Lk_map, (long long)B * Hkv, PF_BM)) return e;
+    if (int e = make_map(&mq, Lq > 0 ? q : k, 128, Lq_map, (long long)B * Hq, BW_RB)) return e;
+    if (int e = make_map(&mo, Lq > 0 ? dout : k, 128, Lq_map, (long long)B * Hp, BW_RB)) return e;
+    const long long units = (long long)((Lk + PF_BM - 1) / PF_BM) * B * Hkv;
+    bwd_dkv_kernel<<<(unsigned)units, BW_THREADS, bwd_dkv_smem(), s>>>(mk, mv, mq, mo, a);
+    CUDA_TRY(cudaGetLastError());
+  }
   return ok();
 }
 
@@ -475,6 +548,62 @@ int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const floa
                 Hkv);
   if (int e = check_bf16_ptrs({q, kc, vc, out})) return e;
   return launch_decode(q, nullptr, kc, nullptr, vc, lambda, out, B, Hq, Hkv, T, false, 1, ws, ws_bytes, s);
+}
+
+int diffattn_fwd_v2_train(const void* q, const void* k, const void* v, const float* lambda, void* out, float* lse,
+                          void* o_maps, diffattn_dtype dtype, int B, int Hq, int Hkv, int Lq, int Lk, int D,
+                          int causal, void* stream) {
+  if (B < 0 || Hq < 2 || Hkv < 1 || Lq < 0 || Lk < 0 || D < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d Lq=%d Lk=%d D=%d)", B, Hq, Hkv, Lq, Lk, D);
+  if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the training forward takes bf16 only");
+  if (D != 128) return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 V2 path needs D == 128 (got %d)", D);
+  if (B == 0 || Lq == 0) return ok();
+  if (!q || !lambda || !out || !lse || !o_maps || (Lk > 0 && (!k || !v)))
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (Lk == 0) k = v = q;
+  if (int e = check_bf16_ptrs({q, k, v, out, o_maps})) return e;
+  return launch_prefill(q, q, k, k, v, lambda, out, B, Hq / 2, Hq, Hkv, Lq, Lk, 128, false, causal, 0, 0.f,
+                        static_cast<cudaStream_t>(stream), lse, o_maps);
+}
+
+size_t diffattn_bwd_v2_workspace_size(int B, int Hq, int Lq) {
+  if (B < 0 || Hq < 2 || Hq % 2 || Lq < 0) return 0;
+  return bwd_ws_bytes(B, Hq, Lq);
+}
+
+int diffattn_bwd_v2(const void* q, const void* k, const void* v, const float* lambda, const void* dout,
+                    const float* lse, const void* o_maps, void* dq, void* dk, void* dv, float* dlambda,
+                    diffattn_dtype dtype, int B, int Hq, int Hkv, int Lq, int Lk, int D, int causal, void* ws,
+                    size_t ws_bytes, void* stream) {
+  if (B < 0 || Hq < 2 || Hkv < 1 || Lq < 0 || Lk < 0 || D < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d Hq=%d Hkv=%d Lq=%d Lk=%d D=%d)", B, Hq, Hkv, Lq, Lk, D);
+  if (Hq % 2 || Hq % Hkv || (Hq / Hkv) % 2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "need Hq even and Hq/Hkv even (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the backward takes bf16 only");
+  if (D != 128) return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 V2 backward needs D == 128 (got %d)", D);
+  if (!lambda || !dlambda) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (B == 0) return ok();
+  if ((Lq > 0 && (!q || !dout || !lse || !o_maps || !dq)) || (Lk > 0 && (!k || !v || !dk || !dv)))
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  for (const void* p : std::initializer_list<const void*>{q, k, v, dout, o_maps, dq, dk, dv})
+    if (p && !aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
+  return launch_backward_v2(q, k, v, lambda, dout, lse, o_maps, dq, dk, dv, dlambda, B, Hq, Hkv, Lq, Lk, causal,
+                            ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int diffattn_lambda_backward(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                             const float* dlambda, int heads, int dim, float* dlq1, float* dlk1, float* dlq2,
+                             float* dlk2, void* stream) {
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !dlambda || !dlq1 || !dlk1 || !dlq2 || !dlk2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (heads < 1 || dim < 1) return fail(DIFFATTN_ERR_INVALID_ARG, "heads and dim must be >= 1");
+  const int threads = 128;
+  lambda_backward_kernel<<<(heads + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      lq1, lk1, lq2, lk2, dlambda, heads, dim, dlq1, dlk1, dlq2, dlk2);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
 }
 
 size_t diffattn_decode_paged_workspace_size(int B, int Hkv) {

@@ -24,6 +24,31 @@ __global__ void lambda_kernel(const float* __restrict__ lq1, const float* __rest
   out[h] = (float)__dadd_rn(__dsub_rn(exp(d1), exp(d2)), lambda_init);
 }
 
+// Gradients of the four λ parameter vectors given dlambda[h] (the chain rule
+// of the λ above): dlq1 = g e1 lk1, dlk1 = g e1 lq1, dlq2 = -g e2 lk2,
+// dlk2 = -g e2 lq2 with e_i = exp(lq_i . lk_i), in fp64, rounded once to f32.
+__global__ void lambda_backward_kernel(const float* __restrict__ lq1, const float* __restrict__ lk1,
+                                       const float* __restrict__ lq2, const float* __restrict__ lk2,
+                                       const float* __restrict__ dlambda, int heads, int dim,
+                                       float* __restrict__ dlq1, float* __restrict__ dlk1, float* __restrict__ dlq2,
+                                       float* __restrict__ dlk2) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= heads) return;
+  double d1 = 0.0, d2 = 0.0;
+  const size_t base = (size_t)h * dim;
+  for (int i = 0; i < dim; ++i) {
+    d1 = __dadd_rn(d1, __dmul_rn((double)lq1[base + i], (double)lk1[base + i]));
+    d2 = __dadd_rn(d2, __dmul_rn((double)lq2[base + i], (double)lk2[base + i]));
+  }
+  const double g = (double)dlambda[h], g1 = g * exp(d1), g2 = -g * exp(d2);
+  for (int i = 0; i < dim; ++i) {
+    dlq1[base + i] = (float)(g1 * (double)lk1[base + i]);
+    dlk1[base + i] = (float)(g1 * (double)lq1[base + i]);
+    dlq2[base + i] = (float)(g2 * (double)lk2[base + i]);
+    dlk2[base + i] = (float)(g2 * (double)lq2[base + i]);
+  }
+}
+
 // Where each operand of one (batch, output head) lives, for both layouts.
 struct SimtArgs {
   const float* q1;   // V1: q1 [B,H,Lq,d];  V2: q [B,Hq,Lq,D]

@@ -62,6 +62,12 @@ struct PrefillArgs {
   // factor would exceed ~12 and the residual restores ~2^-17.
   float resid_tau;
   Watch watch;
+  // Training outputs (null for inference): per row and map the log-sum-exp of
+  // the scaled scores in log2 units, lse[B, Hout, 2, Lq] (+inf for a row that
+  // sees no key), and the normalised map outputs O_m / l_m, o_maps[B, Hout, 2,
+  // Lq, 128] bf16.
+  float* lse;
+  __nv_bfloat16* o_maps;
 };
 
 template <int DQK>
@@ -128,6 +134,40 @@ __device__ __forceinline__ float pf_exp_store(const float (&s)[PF_BN], float2 sc
   const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
   const float2 a03 = __fadd2_rn(a01, a23);
   return a03.x + a03.y;
+}
+
+// Store 64 bf16 columns of each of a warp's 32 rows (thread i holds row
+// row_w0 + i): the warp stages 16 rows at a time in its shared buffer (16-byte
+// chunks XOR-swizzled by row, conflict-free both ways) and writes them back as
+// 4 rows x 128 contiguous bytes per instruction (a direct store of each
+// thread's own row would touch 32 lines per instruction).  base points at
+// column 0 of row 0; rows are 128 elements apart; rows >= Lq are skipped.
+__device__ __forceinline__ void pf_store_rows(uint8_t* st, const float (&y)[64], __nv_bfloat16* base, int row_w0,
+                                              int Lq, int lane) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    if ((lane >> 4) == half) {
+      const int rr = lane & 15;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v;
+        v.x = pack_bf16(y[8 * c + 0], y[8 * c + 1]);
+        v.y = pack_bf16(y[8 * c + 2], y[8 * c + 3]);
+        v.z = pack_bf16(y[8 * c + 4], y[8 * c + 5]);
+        v.w = pack_bf16(y[8 * c + 6], y[8 * c + 7]);
+        *reinterpret_cast<uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4)) = v;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rr = 4 * i + (lane >> 3), c = lane & 7;
+      const int row = row_w0 + 16 * half + rr;
+      const uint4 v = *reinterpret_cast<const uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4));
+      if (row < Lq) *reinterpret_cast<uint4*>(base + (size_t)row * PF_DV + c * 8) = v;
+    }
+    __syncwarp();
+  }
 }
 
 template <int DQK>
@@ -426,39 +466,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       for (int i = 0; i < 64; ++i) y[i] = 0.f;
       have = true;
     }
-    // Coalesced output: each thread holds 64 columns (128 bytes) of its own
-    // row, so storing them directly would touch 32 lines per warp
-    // instruction.  Instead the warp stages 16 rows at a time in its shared
-    // buffer (16-byte chunks XOR-swizzled by row, conflict-free both ways) and
-    // writes them back as 4 rows x 128 contiguous bytes per instruction.
     have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;   // warp-uniform (ok is)
-    if (have) {
-      uint8_t* st = S.stage[warp];
-      const int row_w0 = r0 + wq * 32;                    // first row of this warp
-      __nv_bfloat16* obase = a.out + (((size_t)b * a.Hout + h) * a.Lq) * PF_DV + m * 64;
+    const int row_w0 = r0 + wq * 32;                          // first row of this warp
+    if (have)
+      pf_store_rows(S.stage[warp], y, a.out + (((size_t)b * a.Hout + h) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq,
+                    lane);
+    // Training outputs: this map's log-sum-exp, and 64 columns of both
+    // normalised map outputs.
+    if (a.lse != nullptr && have) {
+      const size_t stat = ((size_t)b * a.Hout + h) * 2;
+      if (rg < a.Lq) a.lse[(stat + m) * a.Lq + rg] = l_run > 0.f ? m_run + log2f(l_run) : INFINITY;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if ((lane >> 4) == half) {
-          const int rr = lane & 15;
+      for (int mm = 0; mm < 2; ++mm) {
+        const float inv = (nT > 0 && S.l[mm][r] > 0.f) ? 1.f / S.l[mm][r] : 0.f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 v;
-            v.x = pack_bf16(y[8 * c + 0], y[8 * c + 1]);
-            v.y = pack_bf16(y[8 * c + 2], y[8 * c + 3]);
-            v.z = pack_bf16(y[8 * c + 4], y[8 * c + 5]);
-            v.w = pack_bf16(y[8 * c + 6], y[8 * c + 7]);
-            *reinterpret_cast<uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4)) = v;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t o[32];
+          if (nT > 0) {
+            tmem_ld32p(tmem + lane_off + 256 + mm * 128 + m * 64 + c * 32, o);
+            tmem_wait_ld();
           }
-        }
-        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int rr = 4 * i + (lane >> 3), c = lane & 7;
-          const int row = row_w0 + 16 * half + rr;
-          const uint4 v = *reinterpret_cast<const uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4));
-          if (row < a.Lq) *reinterpret_cast<uint4*>(obase + (size_t)row * PF_DV + c * 8) = v;
+          for (int i = 0; i < 32; ++i) y[c * 32 + i] = nT > 0 ? __uint_as_float(o[i]) * inv : 0.f;
         }
-        __syncwarp();
+        pf_store_rows(S.stage[warp], y, a.o_maps + ((stat + mm) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq, lane);
       }
     }
   }

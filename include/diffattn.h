@@ -182,6 +182,48 @@ DIFFATTN_API int diffattn_decode_v2_noalloc(const void* q, const void* kc, const
                                             void* out, diffattn_dtype dtype, int B, int Hq, int Hkv, int T,
                                             int D, void* stream);
 
+/* Training forward, V2 layout, bf16 (same operation and arguments as
+ * diffattn_fwd_v2, D == 128), that also writes what the backward needs:
+ *   lse    : f32 [B, Hq/2, 2, Lq]: per row and map, log2 of the softmax
+ *            normaliser of the scores scaled by log2(e)/sqrt(D), i.e.
+ *            A_m[i, j] = 2^(S_m[i, j] log2(e)/sqrt(D) - lse[.., m, i]);
+ *            +inf for a row that sees no key.                    (device)
+ *   o_maps : bf16 [B, Hq/2, 2, Lq, 128]: O_m = A_m V per map.    (device)
+ * The λ parameterisation (tutorial, Step 4) makes λ learnable, so the layer
+ * is trained; the pages print no backward. */
+DIFFATTN_API int diffattn_fwd_v2_train(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                                       float* lse, void* o_maps, diffattn_dtype dtype, int B, int Hq, int Hkv,
+                                       int Lq, int Lk, int D, int causal, void* stream);
+
+/* Workspace, in bytes, for diffattn_bwd_v2 (B sequences, Hq Q heads, Lq rows). */
+DIFFATTN_API size_t diffattn_bwd_v2_workspace_size(int B, int Hq, int Lq);
+
+/* Backward of the V2 forward (bf16, D == 128), the chain rule of
+ *   A_m = softmax(Q_m K^T / sqrt(D)),  O = (A_1 - λ A_2) V:
+ *   dV = Σ (A_1 - λ A_2)^T dO,  dS_1 = A_1 (dO V^T - D_1),
+ *   dS_2 = -λ A_2 (dO V^T - D_2),  D_m = rowsum(dO * O_m),
+ *   dQ_m = dS_m K / sqrt(D),  dK = Σ dS_m^T Q_m / sqrt(D),
+ *   dλ = -Σ dO * O_2.
+ *   q, k, v, lambda : the forward's inputs                        (device)
+ *   dout            : bf16 [B, Hq/2, Lq, 128]                     (device)
+ *   lse, o_maps     : from diffattn_fwd_v2_train                  (device)
+ *   dq              : bf16 [B, Hq, Lq, 128]; dk, dv : bf16 [B, Hkv, Lk, 128]
+ *   dlambda         : f32 [Hq/2], summed over batch and rows in a fixed
+ *                     order (deterministic)                      (device)
+ *   ws              : diffattn_bwd_v2_workspace_size bytes, 16-byte aligned.
+ * dK and dV sum over every Q head of a KV group and both maps. */
+DIFFATTN_API int diffattn_bwd_v2(const void* q, const void* k, const void* v, const float* lambda, const void* dout,
+                                 const float* lse, const void* o_maps, void* dq, void* dk, void* dv, float* dlambda,
+                                 diffattn_dtype dtype, int B, int Hq, int Hkv, int Lq, int Lk, int D, int causal,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Gradients of λ = exp(lq1.lk1) - exp(lq2.lk2) + λ_init with respect to its
+ * parameter vectors ([heads, dim] f32 each), given dlambda [heads]: fp64
+ * inside, f32 out.                                                 (device) */
+DIFFATTN_API int diffattn_lambda_backward(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                                          const float* dlambda, int heads, int dim, float* dlq1, float* dlk1,
+                                          float* dlq2, float* dlk2, void* stream);
+
 /* Workspace, in bytes, that diffattn_decode_v2_paged needs on the current
  * device for B sequences over Hkv KV heads (independent of the lengths and the
  * page size).  0 for invalid sizes. */

@@ -1,0 +1,117 @@
+"""Backward of the V2 forward (training forward, dQ, dK, dV, dlambda, lambda's
+parameter gradients) against the fp64 oracle.  Needs a B200.
+
+Tolerance as for the forward: max|g - g_ref| <= 2e-2 max|g_ref| per gradient
+tensor (bf16 outputs of fp32 arithmetic)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import differential_attention_transformers_b200 as da
+from differential_attention_transformers_b200 import inputs
+from oracle import backward as bwd
+from oracle import diffattn as orc
+from tests.test_parity_gpu import BF16_TOL, DEV, lam_gpu_and_ref
+
+pytestmark = pytest.mark.gpu
+
+
+def _rel(got, ref):
+    got = got.double().cpu().numpy() if hasattr(got, "cpu") else np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = float(np.max(np.abs(ref)))
+    return float(np.max(np.abs(got - ref))) / scale if scale > 0 else float(np.max(np.abs(got)))
+
+
+def _case(B, Hq, Hkv, Lq, Lk, seed, lam_lo=-0.2, lam_hi=1.0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    s = 1 / math.sqrt(128)
+    mk = lambda *shape, std=s: (torch.randn(*shape, generator=g) * std).to(torch.bfloat16).to(DEV)  # noqa: E731
+    q, k, v = mk(B, Hq, Lq, 128), mk(B, Hkv, Lk, 128), mk(B, Hkv, Lk, 128)
+    dout = mk(B, Hq // 2, Lq, 128, std=1.0)
+    lam = (torch.rand(Hq // 2, generator=g) * (lam_hi - lam_lo) + lam_lo).to(DEV)
+    return q, k, v, dout, lam
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, Lk, causal
+    (1, 4, 1, 200, 200, True),      # ragged tails, one KV head for both pairs
+    (2, 8, 2, 300, 300, False),     # non-causal, GQA groups of 4 Q heads
+    (1, 4, 2, 130, 257, True),      # Lq < Lk: bottom-right causal offset
+    (1, 8, 1, 64, 64, True),        # a single tile
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,causal", CASES)
+def test_backward_matches_oracle(B, Hq, Hkv, Lq, Lk, causal):
+    q, k, v, dout, lam = _case(B, Hq, Hkv, Lq, Lk, seed=Lq + 7 * Lk + Hq)
+    out, lse, om = da.fwd_v2_train(q, k, v, lam, causal=causal)
+    assert torch.equal(out, da.fwd_v2(q, k, v, lam, causal=causal))   # the training forward is the forward
+    dq, dk, dv, dlam = da.bwd_v2(q, k, v, lam, dout, lse, om, causal=causal)
+    torch.cuda.synchronize()
+    assert da.last_status() == da.OK
+    rq, rk, rv, rl = bwd.diffattn_v2_backward(q, k, v, lam.cpu().numpy(), dout, causal=causal)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        assert torch.isfinite(got.float()).all(), name
+        assert _rel(got, ref) <= BF16_TOL, (name, _rel(got, ref))
+    assert _rel(dlam, rl) <= BF16_TOL, ("dlambda", dlam.cpu().numpy(), rl)
+
+
+def test_training_forward_statistics():
+    q, k, v, dout, lam = _case(1, 4, 2, 190, 190, seed=31)
+    out, lse, om = da.fwd_v2_train(q, k, v, lam, causal=True)
+    qd, kd, vd = (orc._f64(t) for t in (q, k, v))
+    sl = math.log2(math.e) / math.sqrt(128)
+    for h in range(2):
+        for m in range(2):
+            qh = 2 * h + m
+            g = qh // 2
+            S = qd[0, qh] @ kd[0, g].T * sl
+            vis = np.tril(np.ones((190, 190), dtype=bool))
+            S = np.where(vis, S, -np.inf)
+            mx = S.max(axis=1, keepdims=True)
+            ref_lse = (mx + np.log2(np.sum(np.exp2(S - mx), axis=1, keepdims=True)))[:, 0]
+            assert np.max(np.abs(lse[0, h, m].cpu().numpy() - ref_lse)) <= 1e-3
+            A = np.exp2(S - ref_lse[:, None])
+            assert _rel(om[0, h, m], A @ vd[0, g]) <= BF16_TOL
+
+
+def test_lambda_parameter_gradients():
+    g = torch.Generator(device="cpu").manual_seed(5)
+    p = [(torch.randn(6, 32, generator=g) * 0.1).to(DEV) for _ in range(4)]
+    dlam = torch.randn(6, generator=g).to(DEV)
+    got = da.lambda_backward(*p, dlam)
+    ref = bwd.lambda_backward(*[t.cpu().numpy() for t in p], dlam.cpu().numpy())
+    for a, b in zip(got, ref):
+        assert np.allclose(a.cpu().numpy(), b, rtol=1e-5, atol=1e-7)
+
+
+def test_backward_full_size_sampled():
+    # the V2 prefill workload; one KV group of one batch entry against the oracle
+    w = inputs.WORKLOADS["v2_prefill"]
+    x = inputs.make(w, device=DEV)
+    lam, lref = lam_gpu_and_ref(w)
+    gen = torch.Generator(device=DEV).manual_seed(77)
+    dout = torch.randn((w.B, w.pairs, w.Lq, w.dv), generator=gen, device=DEV).to(torch.bfloat16)
+    out, lse, om = da.fwd_v2_train(x["q"], x["k"], x["v"], lam, causal=True)
+    dq, dk, dv, dlam = da.bwd_v2(x["q"], x["k"], x["v"], lam, dout, lse, om, causal=True)
+    torch.cuda.synchronize()
+    assert da.last_status() == da.OK
+    for t in (dq, dk, dv, dlam):
+        assert torch.isfinite(t.float()).all()
+    b, g = 1, 3
+    grp = w.H // w.Hkv
+    rk, rv = 0.0, 0.0
+    for h in range(g * grp // 2, (g + 1) * grp // 2):
+        h1, h2 = 2 * h, 2 * h + 1
+        a = bwd.head_backward(x["q"][b, h1], x["k"][b, g], x["q"][b, h2], x["k"][b, g], x["v"][b, g], float(lref[h]),
+                              dout[b, h], causal=True)
+        assert _rel(dq[b, h1], a[0]) <= BF16_TOL, ("dq", h1)
+        assert _rel(dq[b, h2], a[2]) <= BF16_TOL, ("dq", h2)
+        rk = rk + a[1] + a[3]
+        rv = rv + a[4]
+    assert _rel(dk[b, g], rk) <= BF16_TOL
+    assert _rel(dv[b, g], rv) <= BF16_TOL
