@@ -248,7 +248,52 @@ class PagedDecode:
                                   host["seq_lens"], lam)
 
 
+class Backward:
+    """Backward of the V2 prefill workload: the training forward runs once (untimed)
+    for its statistics, then each step is lambda + the full backward."""
+
+    def __init__(self, w, device):
+        self.w = w
+        self.x = inputs.make(w, device=device)
+        self.lp = inputs.lambda_params(w, device=device)
+        self.init = da.lambda_init(w.layer)
+        self.lam = torch.empty(w.pairs, dtype=torch.float32, device=device)
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        gen = torch.Generator(device=device).manual_seed(w.seed + 1)
+        self.dout = torch.randn((w.B, w.pairs, w.Lq, w.dv), generator=gen, device=device).to(w.dtype)
+        _, self.lse, self.om = da.fwd_v2_train(self.x["q"], self.x["k"], self.x["v"], self.lam, causal=w.causal)
+        self.ws = torch.empty(int(da.load().diffattn_bwd_v2_workspace_size(w.B, w.H, w.Lq)), dtype=torch.uint8,
+                              device=device)
+        self.launches_per_step = 6   # lambda, prep, dlambda, dQ, dK/dV, lambda's parameter gradients
+
+    def step(self, ev=None):
+        w, x = self.w, self.x
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        if ev is not None:
+            ev[0].record()
+        _, _, _, dlam = da.bwd_v2(x["q"], x["k"], x["v"], self.lam, self.dout, self.lse, self.om, causal=w.causal,
+                                  workspace=self.ws)
+        da.lambda_backward(*self.lp, dlam)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        # the five contractions per map of the chain rule: 2.5 x the forward's executed-minimum FLOP
+        return 2.5 * prefill_flops(self.w) / 1e12, "TFLOP/s"
+
+    def host_call(self, host):
+        raise NotImplementedError("the backward is timed on device tensors only")
+
+
+def base_workload(name):
+    """The workload a bench name is built on (variants share their base's shapes)."""
+    return {"v2_backward": "v2_prefill", "v2_decode_paged": "v2_decode",
+            "v1_decode_unfused": "v1_decode"}.get(name, name)
+
+
 def make_runner(name, device):
+    if name == "v2_backward":
+        return Backward(inputs.WORKLOADS["v2_prefill"], device)
     if name == "v2_decode_paged":
         return PagedDecode(inputs.WORKLOADS["v2_decode"], device)
     w = inputs.WORKLOADS[name.replace("_unfused", "")]
@@ -258,12 +303,14 @@ def make_runner(name, device):
 
 
 def describe(name):
-    w = inputs.WORKLOADS[name.replace("_unfused", "").replace("_paged", "")]
+    w = inputs.WORKLOADS[base_workload(name)]
     d = {"workload": name, "layout": w.layout, "B": w.B, "heads": w.H, "kv_heads": w.Hkv, "Lq": w.Lq, "Lk": w.Lk,
          "d": w.d, "dv": w.dv, "causal": w.causal, "layer": w.layer, "rmsnorm": w.rmsnorm,
          "l2": "inputs larger than L2 (126 MB): no flush between steps"}
     if name.endswith("_unfused"):
         d["mode"] = "two passes, V read twice (comparison)"
+    if name == "v2_backward":
+        d["mode"] = "backward: dQ, dK, dV, dlambda from the training forward's statistics; dO ~ N(0,1)"
     if name.endswith("_paged"):
         d["mode"] = f"paged: shuffled pool of {PAGE_SIZE}-token pages [num_pages, {PAGE_SIZE}, Hkv, 128], block table"
     return d
@@ -378,17 +425,24 @@ def cpu_oracle_run(name, budget_s=12.0):
         cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
     except Exception:
         cores = len(os.sched_getaffinity(0))
-    paged = name == "v2_decode_paged"
-    w = inputs.WORKLOADS[name.replace("_unfused", "").replace("_paged", "")]
+    paged, backward = name == "v2_decode_paged", name == "v2_backward"
+    w = inputs.WORKLOADS[base_workload(name)]
     x = inputs.make(w, device="cpu") if w.layout in ("v1", "v2") else None
     lam = np.full(w.pairs, 0.5)
     done_work, t_total, n = 0.0, 0.0, 0
     if w.layout in ("v1", "v2"):
-        per_slice = prefill_flops(w) / (w.B * w.pairs) / 1e12
+        per_slice = (2.5 if backward else 1.0) * prefill_flops(w) / (w.B * w.pairs) / 1e12
         units = [(b, h) for h in range(w.pairs) for b in range(w.B)]
+        if backward:
+            from oracle import backward as obwd
+            dout = torch.randn((1, w.Lq, w.dv), generator=torch.Generator().manual_seed(w.seed)).to(w.dtype)
         for b, h in units:
             t0 = time.perf_counter()
-            if w.layout == "v2":
+            if backward:
+                g = (2 * h) // (w.H // w.Hkv)
+                obwd.head_backward(x["q"][b, 2 * h], x["k"][b, g], x["q"][b, 2 * h + 1], x["k"][b, g], x["v"][b, g],
+                                   lam[h], dout[0], causal=w.causal)
+            elif w.layout == "v2":
                 g = (2 * h) // (w.H // w.Hkv)
                 orc.diffattn_v2(x["q"][b:b + 1, 2 * h:2 * h + 2], x["k"][b:b + 1, g:g + 1],
                                 x["v"][b:b + 1, g:g + 1], lam[h:h + 1], causal=w.causal)
@@ -447,7 +501,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="v2_prefill",
-                    choices=["v2_prefill", "v1_prefill", "v2_decode", "v2_decode_paged", "v1_decode",
+                    choices=["v2_prefill", "v1_prefill", "v2_backward", "v2_decode", "v2_decode_paged", "v1_decode",
                              "v1_decode_unfused"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -457,13 +511,13 @@ def main():
                     help="override the batch size of the workload (smaller profiling cases)")
     args = ap.parse_args()
     if args.batch is not None:
-        base = args.workload.replace("_unfused", "")
+        base = base_workload(args.workload)
         inputs.WORKLOADS[base] = inputs.with_shape(inputs.WORKLOADS[base], B=args.batch)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = inputs.WORKLOADS[args.workload.replace("_unfused", "")]
+    w = inputs.WORKLOADS[base_workload(args.workload)]
 
     if args.impl == "reference":
         # The reference arm is the fp64 CPU oracle, on rank 0 only.
@@ -514,7 +568,8 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        names = ["v1_prefill", "v2_decode", "v2_decode_paged", "v1_decode", "v1_decode_unfused", "v2_prefill"]
+        names = ["v1_prefill", "v2_backward", "v2_decode", "v2_decode_paged", "v1_decode", "v1_decode_unfused",
+                 "v2_prefill"]
         for name in names:
             if name == args.workload:
                 continue

@@ -32,7 +32,8 @@
 // atomics, and each kernel fits TMEM: dQ 384 columns, dK/dV 512.
 // Both MMA kernels use the forward's pipeline: a TMA producer warp, one
 // issuing thread for the S-type products and one for the accumulating ones,
-// and four warps (thread = TMEM lane) between them.
+// and eight warps (two per TMEM lane quadrant, one per 32-column chunk)
+// between them.
 #pragma once
 
 #include "common.cuh"
@@ -40,7 +41,13 @@
 
 namespace da {
 
-constexpr int BW_THREADS = 224;   // warps 0-3 elementwise, 4 producer/TMEM, 5 accumulating MMAs, 6 S-type MMAs
+// Warps 0-7 elementwise (warp w: TMEM lane quadrant w & 3, 32-column chunk
+// w >> 2 of each 64-column buffer), 8 producer and TMEM owner, 9 accumulating
+// MMAs, 10 S-type MMAs.  In every bf16 buffer a chunk keeps its values in its
+// own 32 columns -- the hi parts in the first 16, the residuals (when used) in
+// the next 16 -- so no warp overwrites scores another warp has yet to load.
+constexpr int BW_THREADS = 352;
+constexpr int BW_EW = 256;        // elementwise threads
 constexpr int BW_NS = 3;          // pipeline stages
 constexpr int BW_RB = 64;         // rows per step of the key-stationary kernel
 
@@ -54,6 +61,12 @@ struct BwdArgs {
   int B, Hq, Hkv, Lq, Lk, Lp;
   int causal;
   float scale, scale_log2;
+  // Heads with |1 - lambda| < resid_tau keep the bf16 residual of w P and of
+  // dS in the key-stationary kernel (a second MMA for dV and for dK): with
+  // alike maps, dV = sum (A_1 - lambda A_2)^T dO and dK = sum dS_m^T Q_m
+  // cancel, and the separate bf16 roundings of the two maps' operands would be
+  // amplified as in the forward.
+  float resid_tau;
   Watch watch;
 };
 
@@ -130,7 +143,7 @@ struct BwQSmem {
   alignas(1024) uint8_t o[2 * PF_QBOX];            // dO tile of the pair, same layout
   alignas(1024) uint8_t k[BW_NS][2 * PF_KBOX];     // K tile: 64 keys, two boxes
   alignas(1024) uint8_t v[BW_NS][2 * PF_KBOX];     // V tile
-  alignas(16) uint8_t stage[4][16 * 128];          // epilogue staging, per elementwise warp
+  alignas(16) uint8_t stage[8][16 * 128];          // epilogue staging, per elementwise warp
   alignas(8) uint64_t q_full;
   uint64_t k_full[BW_NS], v_full[BW_NS], kv_empty[BW_NS];
   uint64_t s_full[2], p_full[2], s_free[2];
@@ -140,7 +153,11 @@ struct BwQSmem {
   int abort_flag;
 };
 
-__global__ void __launch_bounds__(BW_THREADS, 1)
+// A_PART: TMEM column offset of the s-th 16-element K slice of a chunk-laid
+// bf16 buffer (slices 0, 1 in chunk 0; 2, 3 in chunk 1).
+__device__ __forceinline__ uint32_t bw_slice(int s) { return (uint32_t)((s >> 1) * 32 + (s & 1) * 8); }
+
+__global__ void __maxnreg__(168)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -168,7 +185,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&S.s_full[i]), 1);
-      mbar_init(smem_u32(&S.p_full[i]), 128);
+      mbar_init(smem_u32(&S.p_full[i]), BW_EW);
       mbar_init(smem_u32(&S.s_free[i]), 1);
       mbar_init(smem_u32(&S.drain[i]), 1);
     }
@@ -176,7 +193,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     S.abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(&S.tmem_base), 512);
     tmem_relinquish();
   }
@@ -185,7 +202,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;   // S [0,128), dP [128,256), dQ [256,384)
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer --
     if (lane == 0 && nT > 0) {
       const uint32_t qb = smem_u32(&S.q_full);
@@ -216,12 +233,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
-  } else if (warp >= 5) {
+  } else if (warp >= 9) {
     // --------------------------------------------------------- MMA issuers --
     if (lane == 0 && nT > 0) {
       constexpr uint32_t HI = umma_desc_hi(1024);
       constexpr uint32_t KSTAGE = (2 * PF_KBOX) >> 4;
-      const int issuer = warp - 5;   // 0: dQ += dS K, 1: S = Q K^T and dP = dO V^T
+      const int issuer = warp - 9;   // 0: dQ += dS K, 1: S = Q K^T and dP = dO V^T
       bool ok = true;
       if (issuer == 0) {
         constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, true);
@@ -235,7 +252,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           const uint32_t klo = k_mn0 + (uint32_t)(j % BW_NS) * KSTAGE;
 #pragma unroll
           for (int s = 0; s < PF_BN / 16; ++s)
-            mma_ts_w(tmem + 256, tmem + bb * 64 + s * 8, klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+            mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s), klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
                      (j > 0 || s > 0));
           mma_commit(smem_u32(&S.s_free[bb]));
           mma_commit(smem_u32(&S.kv_empty[j % BW_NS]));
@@ -274,7 +291,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
   } else {
     // ------------------------------------------- elementwise (thread = row) --
-    const int wq = warp, r = threadIdx.x;
+    const int wq = warp & 3, ch = warp >> 2, r = threadIdx.x & 127;
     const int rg = r0 + r;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const size_t stat = (((size_t)b * Hp + h) * 2 + m) * a.Lp + rg;
@@ -286,26 +303,23 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const int bb = j & 1;
       if (!(ok = warp_wait(smem_u32(&S.s_full[bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
       tc_fence_after();
+      uint32_t sv[32], pv[32], ds[16];
+      tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
+      tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
+      tmem_wait_ld();
+      const long long lim = lastk - (long long)j * PF_BN - ch * 32;   // columns > lim are masked
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t sv[32], pv[32], ds[16];
-        tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
-        tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
-        tmem_wait_ld();
-        const long long lim = lastk - (long long)j * PF_BN - ch * 32;   // columns > lim are masked
+      for (int i = 0; i < 16; ++i) {
+        float dsv[2];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float dsv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 2 * i + e;
-            const float x = col > lim ? -INFINITY : fmaf(__uint_as_float(sv[col]), a.scale_log2, -lse);
-            dsv[e] = c * ex2(x) * (__uint_as_float(pv[col]) - dsum);
-          }
-          ds[i] = pack_bf16(dsv[0], dsv[1]);
+        for (int e = 0; e < 2; ++e) {
+          const int col = 2 * i + e;
+          const float x = col > lim ? -INFINITY : fmaf(__uint_as_float(sv[col]), a.scale_log2, -lse);
+          dsv[e] = c * ex2(x) * (__uint_as_float(pv[col]) - dsum);
         }
-        tmem_st16p(tmem + lane_off + bb * 64 + ch * 16, ds);
+        ds[i] = pack_bf16(dsv[0], dsv[1]);
       }
+      tmem_st16p(tmem + lane_off + bb * 64 + ch * 32, ds);   // the chunk's own columns
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&S.p_full[bb]));
@@ -314,29 +328,26 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool have = nT == 0;
     float y[64];
     if (nT > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
-    if (have) {
+    if (have) {   // chunk ch writes dQ columns [64 ch, 64 ch + 64) of its rows
       if (nT > 0) tc_fence_after();
       __nv_bfloat16* base = a.dq + ((size_t)b * a.Hq + qh) * a.Lq * 128;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t o[32];
-          if (nT > 0) {
-            tmem_ld32p(tmem + lane_off + 256 + hf * 64 + cc * 32, o);
-            tmem_wait_ld();
-          }
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[cc * 32 + i] = nT > 0 ? __uint_as_float(o[i]) : 0.f;
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t o[32];
+        if (nT > 0) {
+          tmem_ld32p(tmem + lane_off + 256 + ch * 64 + cc * 32, o);
+          tmem_wait_ld();
         }
-        pf_store_rows(S.stage[warp], y, base + hf * 64, r0 + wq * 32, a.Lq, lane);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) y[cc * 32 + i] = nT > 0 ? __uint_as_float(o[i]) : 0.f;
       }
+      pf_store_rows(S.stage[warp], y, base + ch * 64, r0 + wq * 32, a.Lq, lane);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -350,7 +361,7 @@ struct BwKSmem {
   alignas(1024) uint8_t o[BW_NS][2 * PF_KBOX];      // dO rows
   alignas(16) float lse[BW_NS][BW_RB];
   alignas(16) float dd[BW_NS][BW_RB];
-  alignas(16) uint8_t stage[4][16 * 128];
+  alignas(16) uint8_t stage[8][16 * 128];
   alignas(8) uint64_t kv_full;
   uint64_t st_full[BW_NS], st_empty[BW_NS];
   uint64_t s_full[2], p_full[2], s_free[2];
@@ -366,7 +377,46 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
-__global__ void __launch_bounds__(BW_THREADS, 1)
+// One step of the key-stationary kernel for this thread's key and this warp's
+// 32-row chunk: from S^T and dP^T (the chunk's columns at tS, tP) write w P^T
+// and dS^T back as bf16 into the chunk's first 16 columns and, with RESID,
+// their bf16 residuals into its next 16.
+template <bool RESID>
+__device__ __forceinline__ void bw_kv_elementwise(uint32_t tS, uint32_t tP, int row0, int kg, int rfirst, int Lk,
+                                                  float w, float cd, float sl, const float* lse, const float* dd) {
+  uint32_t sv[32], pv[32], pw[16], ds[16];
+  tmem_ld32p(tS, sv);
+  tmem_ld32p(tP, pv);
+  tmem_wait_ld();
+  uint32_t rpw[RESID ? 16 : 1], rds[RESID ? 16 : 1];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    float p2[2], d2[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int col = 2 * j + e;
+      const bool vis = kg < Lk && row0 + col >= rfirst;
+      const float x = vis ? fmaf(__uint_as_float(sv[col]), sl, -lse[col]) : -INFINITY;
+      const float p = ex2(x);
+      p2[e] = w * p;
+      d2[e] = cd * p * (__uint_as_float(pv[col]) - dd[col]);
+    }
+    pw[j] = pack_bf16(p2[0], p2[1]);
+    ds[j] = pack_bf16(d2[0], d2[1]);
+    if constexpr (RESID) {   // x - bf16(x), exact in f32
+      rpw[j] = pack_bf16(p2[0] - __uint_as_float(pw[j] << 16), p2[1] - __uint_as_float(pw[j] & 0xFFFF0000u));
+      rds[j] = pack_bf16(d2[0] - __uint_as_float(ds[j] << 16), d2[1] - __uint_as_float(ds[j] & 0xFFFF0000u));
+    }
+  }
+  tmem_st16p(tS, pw);
+  tmem_st16p(tP, ds);
+  if constexpr (RESID) {
+    tmem_st16p(tS + 16, rpw);
+    tmem_st16p(tP + 16, rds);
+  }
+}
+
+__global__ void __maxnreg__(168)
 bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -395,7 +445,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&S.s_full[i]), 1);
-      mbar_init(smem_u32(&S.p_full[i]), 128);
+      mbar_init(smem_u32(&S.p_full[i]), BW_EW);
       mbar_init(smem_u32(&S.s_free[i]), 1);
       mbar_init(smem_u32(&S.drain[i]), 1);
     }
@@ -403,7 +453,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     S.abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(&S.tmem_base), 512);
     tmem_relinquish();
   }
@@ -412,7 +462,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;   // S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512)
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer --
     if (lane == 0 && nS > 0) {
       const uint32_t kvb = smem_u32(&S.kv_full);
@@ -443,12 +493,12 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       for (int i = 0; i < BW_NS; ++i)
         if (last_use[i] >= 0) drain_bar(smem_u32(&S.st_full[i]), last_use[i] & 1, a.watch.status);
     }
-  } else if (warp >= 5) {
+  } else if (warp >= 9) {
     // --------------------------------------------------------- MMA issuers --
     if (lane == 0 && nS > 0) {
       constexpr uint32_t HI = umma_desc_hi(1024);
       constexpr uint32_t QSTAGE = (2 * PF_KBOX) >> 4;
-      const int issuer = warp - 5;   // 0: dV, dK accumulation; 1: S^T and dP^T
+      const int issuer = warp - 9;   // 0: dV, dK accumulation; 1: S^T and dP^T
       bool ok = true;
       if (issuer == 0) {
         constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, true);
@@ -460,14 +510,26 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
           tc_fence_after();
           const uint32_t olo = o_mn0 + (uint32_t)st * QSTAGE, qlo = q_mn0 + (uint32_t)st * QSTAGE;
+          const int qh = g * grp + i / per_head;
+          const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
 #pragma unroll
           for (int s = 0; s < BW_RB / 16; ++s)   // dV += (w P)^T dO
-            mma_ts_w(tmem + 256, tmem + bb * 64 + s * 8, olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+            mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s), olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
                      (i > 0 || s > 0));
 #pragma unroll
           for (int s = 0; s < BW_RB / 16; ++s)   // dK += dS^T Q
-            mma_ts_w(tmem + 384, tmem + 128 + bb * 64 + s * 8, qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
-                     (i > 0 || s > 0));
+            mma_ts_w(tmem + 384, tmem + 128 + bb * 64 + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI,
+                     IDESC_ACC, (i > 0 || s > 0));
+          if (resid) {   // the bf16 residuals, 16 columns after each chunk's hi part
+#pragma unroll
+            for (int s = 0; s < BW_RB / 16; ++s)
+              mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s) + 16, olo + (uint32_t)(s * (2048 >> 4)), HI,
+                       IDESC_ACC, 1);
+#pragma unroll
+            for (int s = 0; s < BW_RB / 16; ++s)
+              mma_ts_w(tmem + 384, tmem + 128 + bb * 64 + bw_slice(s) + 16, qlo + (uint32_t)(s * (2048 >> 4)), HI,
+                       IDESC_ACC, 1);
+          }
           mma_commit(smem_u32(&S.s_free[bb]));
           mma_commit(smem_u32(&S.st_empty[st]));
         }
@@ -504,7 +566,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------- elementwise (thread = key) --
-    const int wq = warp, kr = threadIdx.x;
+    const int wq = warp & 3, ch = warp >> 2, kr = threadIdx.x & 127;
     const int kg = k0 + kr;   // this thread's key
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     bool ok = true;
@@ -520,31 +582,16 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       tc_fence_after();
       // rows r = rb*64 + col see this key iff kg < Lk and (not causal or kg <= r + off)
       const int rfirst = a.causal ? kg - off : 0;   // first row that sees kg (causal)
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t sv[32], pv[32], pw[16], ds[16];
-        tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
-        tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = ch * 32 + 2 * j + e;
-            const int row = rb * BW_RB + col;
-            const bool vis = kg < a.Lk && row >= rfirst;
-            const float x = vis ? fmaf(__uint_as_float(sv[2 * j + e]), a.scale_log2, -S.lse[st][col]) : -INFINITY;
-            const float p = ex2(x);
-            p2[e] = w * p;
-            d2[e] = cd * p * (__uint_as_float(pv[2 * j + e]) - S.dd[st][col]);
-          }
-          pw[j] = pack_bf16(p2[0], p2[1]);
-          ds[j] = pack_bf16(d2[0], d2[1]);
-        }
-        tmem_st16p(tmem + lane_off + bb * 64 + ch * 16, pw);
-        tmem_st16p(tmem + lane_off + 128 + bb * 64 + ch * 16, ds);
-      }
+      const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
+      const uint32_t tS = tmem + lane_off + bb * 64 + ch * 32, tP = tmem + lane_off + 128 + bb * 64 + ch * 32;
+      const int row0 = rb * BW_RB + ch * 32;
+      // branch once per step: each variant's loop is one straight-line block
+      if (resid)
+        bw_kv_elementwise<true>(tS, tP, row0, kg, rfirst, a.Lk, w, cd, a.scale_log2, S.lse[st] + ch * 32,
+                                S.dd[st] + ch * 32);
+      else
+        bw_kv_elementwise<false>(tS, tP, row0, kg, rfirst, a.Lk, w, cd, a.scale_log2, S.lse[st] + ch * 32,
+                                 S.dd[st] + ch * 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&S.p_full[bb]));
@@ -553,32 +600,29 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     bool have = nS == 0;
     float y[64];
     if (nS > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
-    if (have) {
+    if (have) {   // chunk 0 writes dV, chunk 1 dK
       if (nS > 0) tc_fence_after();
+      __nv_bfloat16* base = (ch ? a.dk : a.dv) + ((size_t)b * a.Hkv + g) * a.Lk * 128;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK
-        __nv_bfloat16* base = (which ? a.dk : a.dv) + ((size_t)b * a.Hkv + g) * a.Lk * 128;
+      for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint32_t o[32];
-            if (nS > 0) {
-              tmem_ld32p(tmem + lane_off + 256 + which * 128 + hf * 64 + cc * 32, o);
-              tmem_wait_ld();
-            }
-#pragma unroll
-            for (int t = 0; t < 32; ++t) y[cc * 32 + t] = nS > 0 ? __uint_as_float(o[t]) : 0.f;
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t o[32];
+          if (nS > 0) {
+            tmem_ld32p(tmem + lane_off + 256 + ch * 128 + hf * 64 + cc * 32, o);
+            tmem_wait_ld();
           }
-          pf_store_rows(S.stage[warp], y, base + hf * 64, k0 + wq * 32, a.Lk, lane);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) y[cc * 32 + t] = nS > 0 ? __uint_as_float(o[t]) : 0.f;
         }
+        pf_store_rows(S.stage[warp], y, base + hf * 64, k0 + wq * 32, a.Lk, lane);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -327,6 +327,7 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
   a.causal = causal ? 1 : 0;
   a.scale = (float)(1.0 / std::sqrt(128.0));
   a.scale_log2 = log2e_over_sqrt(128);
+  a.resid_tau = DIFFATTN_RESID_TAU;
   a.watch = make_watch(dev);
   const long long Lk_map = Lk > 0 ? Lk : 1;   // a zero extent is not encodable; no key is then loaded
   const long long Lq_map = Lq > 0 ? Lq : 1;

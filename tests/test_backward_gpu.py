@@ -115,3 +115,23 @@ def test_backward_full_size_sampled():
         rv = rv + a[4]
     assert _rel(dk[b, g], rk) <= BF16_TOL
     assert _rel(dv[b, g], rv) <= BF16_TOL
+
+
+@pytest.mark.parametrize("lam_value", [0.97, 1.0, 0.86, 1.14])
+def test_backward_near_unit_lambda_with_similar_maps(lam_value):
+    """The hardest case for bf16 P and dS: near-uniform, nearly identical maps and
+    lambda close to 1, where A_1 - lambda A_2 cancels."""
+    g = torch.Generator(device="cpu").manual_seed(int(lam_value * 1000) + 1)
+    s = 1 / math.sqrt(128)
+    q1 = torch.randn(1, 1, 512, 128, generator=g) * s
+    q2 = q1 + 0.05 * s * torch.randn(1, 1, 512, 128, generator=g)
+    q = torch.cat([q1, q2], dim=1).to(torch.bfloat16).to(DEV)
+    k = (torch.randn(1, 1, 512, 128, generator=g) * s).to(torch.bfloat16).to(DEV)
+    v = (torch.randn(1, 1, 512, 128, generator=g) * s).to(torch.bfloat16).to(DEV)
+    dout = torch.randn(1, 1, 512, 128, generator=g).to(torch.bfloat16).to(DEV)
+    lam = torch.tensor([lam_value], device=DEV)
+    _, lse, om = da.fwd_v2_train(q, k, v, lam, causal=True)
+    dq, dk, dv, dlam = da.bwd_v2(q, k, v, lam, dout, lse, om, causal=True)
+    rq, rk, rv, rl = bwd.diffattn_v2_backward(q, k, v, np.array([lam_value]), dout, causal=True)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        assert _rel(got, ref) <= BF16_TOL, (name, lam_value, _rel(got, ref))
