@@ -95,6 +95,21 @@ def test_argument_errors_before_any_device_call(L):
     assert pg(P, P, P, Pi, P, P, P, da.BF16, 2, 16, 2, 8, 16, 4, P, 1 << 20, s) == da.ERR_MISALIGNED     # table
     assert pg(P, P, P, P, P, P, P, da.BF16, 2048, 16, 8, 8, 256, 1 << 20, P, 1 << 20, s) == da.ERR_UNSUPPORTED
     assert "2^31" in da.last_error()
+    # training forward and backward: (q, k, v, lambda, out, lse, o_maps, dtype, B, Hq, Hkv, Lq, Lk, D, causal, s)
+    assert L.diffattn_fwd_v2_train(P, P, P, P, P, P, P, da.F32, 1, 4, 2, 8, 8, 128, 1, s) == da.ERR_UNSUPPORTED
+    assert L.diffattn_fwd_v2_train(P, P, P, P, P, None, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, s) == da.ERR_INVALID_ARG
+    assert L.diffattn_fwd_v2_train(P, P, P, P, P, P, P, da.BF16, 1, 6, 2, 8, 8, 128, 1, s) == da.ERR_INVALID_ARG
+    assert L.diffattn_fwd_v2_train(P, P, P, P, P, P, P, da.BF16, 1, 4, 2, 8, 8, 64, 1, s) == da.ERR_UNSUPPORTED
+    bw = lambda *args: L.diffattn_bwd_v2(*args)  # noqa: E731
+    # (q, k, v, lambda, dout, lse, o_maps, dq, dk, dv, dlambda, dtype, B, Hq, Hkv, Lq, Lk, D, causal, ws, bytes, s)
+    assert bw(P, P, P, P, P, P, P, P, P, P, P, da.F32, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+    assert bw(P, P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 4, 3, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    assert bw(P, P, P, P, P, None, P, P, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    assert bw(P, P, P, P, P, P, P, Pm, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_MISALIGNED
+    assert L.diffattn_bwd_v2_workspace_size(2, 64, 8192) > 0
+    assert L.diffattn_bwd_v2_workspace_size(2, 63, 8192) == 0
+    assert L.diffattn_lambda_backward(P, P, P, P, P, 0, 8, P, P, P, P, s) == da.ERR_INVALID_ARG
+    assert L.diffattn_lambda_backward(P, P, P, None, P, 2, 8, P, P, P, P, s) == da.ERR_INVALID_ARG
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch):
