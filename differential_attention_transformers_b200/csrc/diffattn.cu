@@ -110,6 +110,8 @@ int device_setup(DeviceInfo** out) {
                                   (int)prefill_smem<64>()));
     CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)prefill_smem<128>()));
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)prefill_smem<128>()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
@@ -211,7 +213,11 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.o_maps = static_cast<__nv_bfloat16*>(o_maps);
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
-  if (dqk == 64)
+  if (lse != nullptr && dqk == 128)   // training forward (V2)
+    prefill_kernel<128, true><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+  else if (lse != nullptr)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "the training forward needs the 128-wide QK layout");
+  else if (dqk == 64)
     prefill_kernel<64><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else
     prefill_kernel<128><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);

@@ -170,7 +170,9 @@ __device__ __forceinline__ void pf_store_rows(uint8_t* st, const float (&y)[64],
   }
 }
 
-template <int DQK>
+// TRAIN: also write the training outputs (lse, o_maps); a template flag so the
+// inference kernel carries none of that code.
+template <int DQK, bool TRAIN = false>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
@@ -473,7 +475,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
                     lane);
     // Training outputs: this map's log-sum-exp, and 64 columns of both
     // normalised map outputs.
-    if (a.lse != nullptr && have) {
+    if (TRAIN && have) {
       const size_t stat = ((size_t)b * a.Hout + h) * 2;
       if (rg < a.Lq) a.lse[(stat + m) * a.Lq + rg] = l_run > 0.f ? m_run + log2f(l_run) : INFINITY;
 #pragma unroll
