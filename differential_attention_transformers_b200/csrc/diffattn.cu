@@ -591,7 +591,10 @@ int diffattn_bwd_v2(const void* q, const void* k, const void* v, const float* la
   if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the backward takes bf16 only");
   if (D != 128) return fail(DIFFATTN_ERR_UNSUPPORTED, "bf16 V2 backward needs D == 128 (got %d)", D);
   if (!lambda || !dlambda) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
-  if (B == 0) return ok();
+  if (B == 0) {   // nothing to differentiate: dlambda is an empty sum
+    CUDA_TRY(cudaMemsetAsync(dlambda, 0, sizeof(float) * (size_t)(Hq / 2), static_cast<cudaStream_t>(stream)));
+    return ok();
+  }
   if ((Lq > 0 && (!q || !dout || !lse || !o_maps || !dq)) || (Lk > 0 && (!k || !v || !dk || !dv)))
     return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   for (const void* p : std::initializer_list<const void*>{q, k, v, dout, o_maps, dq, dk, dv})
