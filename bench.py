@@ -248,8 +248,15 @@ class PagedDecode:
                                   host["seq_lens"], lam)
 
 
+def backward_flops(w) -> float:
+    """Executed-minimum FLOP of the backward: five contractions per map and
+    visible (row, key) pair -- S (2d), dP (2dv), dV (2dv), dQ (2d), dK (2d) --
+    against the forward's two (2d + 2dv); 2.5 x the forward for V2."""
+    return prefill_flops(w) * (6 * w.d + 4 * w.dv) / (2 * w.d + 2 * w.dv)
+
+
 class Backward:
-    """Backward of the V2 prefill workload: the training forward runs once (untimed)
+    """Backward of a prefill workload: the training forward runs once (untimed)
     for its statistics, then each step is lambda + the full backward."""
 
     def __init__(self, w, device):
@@ -261,25 +268,36 @@ class Backward:
         da.compute_lambda(*self.lp, self.init, out=self.lam)
         gen = torch.Generator(device=device).manual_seed(w.seed + 1)
         self.dout = torch.randn((w.B, w.pairs, w.Lq, w.dv), generator=gen, device=device).to(w.dtype)
-        _, self.lse, self.om = da.fwd_v2_train(self.x["q"], self.x["k"], self.x["v"], self.lam, causal=w.causal)
-        self.ws = torch.empty(int(da.load().diffattn_bwd_v2_workspace_size(w.B, w.H, w.Lq)), dtype=torch.uint8,
-                              device=device)
-        self.launches_per_step = 6   # lambda, prep, dlambda, dQ, dK/dV, lambda's parameter gradients
+        x = self.x
+        if w.layout == "v2":
+            _, self.lse, self.om = da.fwd_v2_train(x["q"], x["k"], x["v"], self.lam, causal=w.causal)
+            nws = da.load().diffattn_bwd_v2_workspace_size(w.B, w.H, w.Lq)
+            self.launches_per_step = 6   # lambda, prep, dlambda, dQ, dK/dV, lambda's parameter gradients
+        else:
+            self.out, self.lse, self.om, self.rstd = da.fwd_v1_train(x["q1"], x["k1"], x["q2"], x["k2"], x["v"],
+                                                                     self.lam, causal=w.causal, rmsnorm=w.rmsnorm)
+            nws = da.load().diffattn_bwd_v1_workspace_size(w.B, w.H, w.Hkv, w.Lq, w.Lk, int(w.rmsnorm))
+            # lambda, pack, [RMSNorm gradient], prep, dlambda, dQ, dK/dV, unpack, lambda's parameter gradients
+            self.launches_per_step = 9 if w.rmsnorm else 8
+        self.ws = torch.empty(int(nws), dtype=torch.uint8, device=device)
 
     def step(self, ev=None):
         w, x = self.w, self.x
         da.compute_lambda(*self.lp, self.init, out=self.lam)
         if ev is not None:
             ev[0].record()
-        _, _, _, dlam = da.bwd_v2(x["q"], x["k"], x["v"], self.lam, self.dout, self.lse, self.om, causal=w.causal,
-                                  workspace=self.ws)
+        if w.layout == "v2":
+            dlam = da.bwd_v2(x["q"], x["k"], x["v"], self.lam, self.dout, self.lse, self.om, causal=w.causal,
+                             workspace=self.ws)[-1]
+        else:
+            dlam = da.bwd_v1(x["q1"], x["k1"], x["q2"], x["k2"], x["v"], self.lam, self.dout, self.out, self.lse,
+                             self.om, self.rstd, causal=w.causal, rmsnorm=w.rmsnorm, workspace=self.ws)[-1]
         da.lambda_backward(*self.lp, dlam)
         if ev is not None:
             ev[1].record()
 
     def work(self):
-        # the five contractions per map of the chain rule: 2.5 x the forward's executed-minimum FLOP
-        return 2.5 * prefill_flops(self.w) / 1e12, "TFLOP/s"
+        return backward_flops(self.w) / 1e12, "TFLOP/s"
 
     def host_call(self, host):
         raise NotImplementedError("the backward is timed on device tensors only")
@@ -287,13 +305,13 @@ class Backward:
 
 def base_workload(name):
     """The workload a bench name is built on (variants share their base's shapes)."""
-    return {"v2_backward": "v2_prefill", "v2_decode_paged": "v2_decode",
+    return {"v2_backward": "v2_prefill", "v1_backward": "v1_prefill", "v2_decode_paged": "v2_decode",
             "v1_decode_unfused": "v1_decode"}.get(name, name)
 
 
 def make_runner(name, device):
-    if name == "v2_backward":
-        return Backward(inputs.WORKLOADS["v2_prefill"], device)
+    if name.endswith("_backward"):
+        return Backward(inputs.WORKLOADS[base_workload(name)], device)
     if name == "v2_decode_paged":
         return PagedDecode(inputs.WORKLOADS["v2_decode"], device)
     w = inputs.WORKLOADS[name.replace("_unfused", "")]
@@ -311,6 +329,9 @@ def describe(name):
         d["mode"] = "two passes, V read twice (comparison)"
     if name == "v2_backward":
         d["mode"] = "backward: dQ, dK, dV, dlambda from the training forward's statistics; dO ~ N(0,1)"
+    if name == "v1_backward":
+        d["mode"] = ("backward: dQ1, dK1, dQ2, dK2, dV, dlambda (RMSNorm gradient first) from the training "
+                     "forward's statistics; dO ~ N(0,1)")
     if name.endswith("_paged"):
         d["mode"] = f"paged: shuffled pool of {PAGE_SIZE}-token pages [num_pages, {PAGE_SIZE}, Hkv, 128], block table"
     return d
@@ -425,20 +446,24 @@ def cpu_oracle_run(name, budget_s=12.0):
         cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
     except Exception:
         cores = len(os.sched_getaffinity(0))
-    paged, backward = name == "v2_decode_paged", name == "v2_backward"
+    paged, backward = name == "v2_decode_paged", name.endswith("_backward")
     w = inputs.WORKLOADS[base_workload(name)]
     x = inputs.make(w, device="cpu") if w.layout in ("v1", "v2") else None
     lam = np.full(w.pairs, 0.5)
     done_work, t_total, n = 0.0, 0.0, 0
     if w.layout in ("v1", "v2"):
-        per_slice = (2.5 if backward else 1.0) * prefill_flops(w) / (w.B * w.pairs) / 1e12
+        per_slice = (backward_flops(w) if backward else prefill_flops(w)) / (w.B * w.pairs) / 1e12
         units = [(b, h) for h in range(w.pairs) for b in range(w.B)]
         if backward:
             from oracle import backward as obwd
             dout = torch.randn((1, w.Lq, w.dv), generator=torch.Generator().manual_seed(w.seed)).to(w.dtype)
         for b, h in units:
             t0 = time.perf_counter()
-            if backward:
+            if backward and w.layout == "v1":
+                g = h // (w.H // w.Hkv)
+                obwd.head_backward(x["q1"][b, h], x["k1"][b, g], x["q2"][b, h], x["k2"][b, g], x["v"][b, g], lam[h],
+                                   dout[0], causal=w.causal, rms=w.rmsnorm)
+            elif backward:
                 g = (2 * h) // (w.H // w.Hkv)
                 obwd.head_backward(x["q"][b, 2 * h], x["k"][b, g], x["q"][b, 2 * h + 1], x["k"][b, g], x["v"][b, g],
                                    lam[h], dout[0], causal=w.causal)
@@ -501,8 +526,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="v2_prefill",
-                    choices=["v2_prefill", "v1_prefill", "v2_backward", "v2_decode", "v2_decode_paged", "v1_decode",
-                             "v1_decode_unfused"])
+                    choices=["v2_prefill", "v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged",
+                             "v1_decode", "v1_decode_unfused"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
@@ -568,7 +593,7 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        names = ["v1_prefill", "v2_backward", "v2_decode", "v2_decode_paged", "v1_decode", "v1_decode_unfused",
+        names = ["v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged", "v1_decode", "v1_decode_unfused",
                  "v2_prefill"]
         for name in names:
             if name == args.workload:

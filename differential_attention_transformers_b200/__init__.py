@@ -32,7 +32,8 @@ EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffa
            "diffattn_decode_workspace_size", "diffattn_decode_v2", "diffattn_decode_v1", "diffattn_last_error",
            "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc",
            "diffattn_decode_paged_workspace_size", "diffattn_decode_v2_paged", "diffattn_fwd_v2_train",
-           "diffattn_bwd_v2_workspace_size", "diffattn_bwd_v2", "diffattn_lambda_backward"]
+           "diffattn_bwd_v2_workspace_size", "diffattn_bwd_v2", "diffattn_lambda_backward",
+           "diffattn_fwd_v1_train", "diffattn_bwd_v1_workspace_size", "diffattn_bwd_v1"]
 
 _lib = None
 
@@ -72,6 +73,9 @@ def load():
         "diffattn_bwd_v2_workspace_size": (Z, [I, I, I]),
         "diffattn_bwd_v2": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]),
         "diffattn_lambda_backward": (I, [P, P, P, P, P, I, I, P, P, P, P, P]),
+        "diffattn_fwd_v1_train": (I, [P] * 10 + [I] * 10 + [F, P]),
+        "diffattn_bwd_v1_workspace_size": (Z, [I] * 6),
+        "diffattn_bwd_v1": (I, [P] * 17 + [I] * 10 + [P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -276,6 +280,39 @@ def bwd_v2(q, k, v, lam, dout, lse, o_maps, causal=True, workspace=None):
                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _dtype_code(q), B, Hq, Hkv, Lq, Lk, D,
                                   int(causal), _ptr(ws), ws.numel() * ws.element_size(), _stream()))
     return dq, dk, dv, dlam
+
+
+def fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5):
+    """V1 forward (bf16, d = 64, dv = 128) that also returns what bwd_v1 needs:
+    (out [B,H,Lq,128], lse f32 [B,H,2,Lq], o_maps [B,H,2,Lq,128], rstd f32 [B,H,Lq]
+    or None without RMSNorm).  Device tensors."""
+    B, H, Lq, d = q1.shape
+    Hkv, Lk, dv = k1.shape[1], k1.shape[2], v.shape[3]
+    out = torch.empty((B, H, Lq, dv), dtype=q1.dtype, device=q1.device)
+    lse = torch.empty((B, H, 2, Lq), dtype=torch.float32, device=q1.device)
+    o_maps = torch.empty((B, H, 2, Lq, dv), dtype=q1.dtype, device=q1.device)
+    rstd = torch.empty((B, H, Lq), dtype=torch.float32, device=q1.device) if rmsnorm else None
+    _check(load().diffattn_fwd_v1_train(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(v), _ptr(lam), _ptr(out),
+                                        _ptr(lse), _ptr(o_maps), _ptr(rstd), _dtype_code(q1), B, H, Hkv, Lq, Lk, d,
+                                        dv, int(causal), int(rmsnorm), float(eps), _stream()))
+    return out, lse, o_maps, rstd
+
+
+def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, causal=True, rmsnorm=False, workspace=None):
+    """Gradients of the V1 forward: (dq1, dk1, dq2, dk2, dv, dlam) given dout [B,H,Lq,128]
+    and fwd_v1_train's outputs.  bf16 gradients, f32 dlam.  Device tensors."""
+    B, H, Lq, d = q1.shape
+    Hkv, Lk, dvw = k1.shape[1], k1.shape[2], v.shape[3]
+    dq1, dq2 = torch.empty_like(q1), torch.empty_like(q2)
+    dk1, dk2, dv = torch.empty_like(k1), torch.empty_like(k2), torch.empty_like(v)
+    dlam = torch.empty(H, dtype=torch.float32, device=q1.device)
+    need = int(load().diffattn_bwd_v1_workspace_size(B, H, Hkv, Lq, Lk, int(rmsnorm)))
+    ws = workspace if workspace is not None else _workspace(need, q1.device)
+    _check(load().diffattn_bwd_v1(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(v), _ptr(lam), _ptr(dout),
+                                  _ptr(out), _ptr(lse), _ptr(o_maps), _ptr(rstd), _ptr(dq1), _ptr(dk1), _ptr(dq2),
+                                  _ptr(dk2), _ptr(dv), _ptr(dlam), _dtype_code(q1), B, H, Hkv, Lq, Lk, d, dvw,
+                                  int(causal), int(rmsnorm), _ptr(ws), ws.numel() * ws.element_size(), _stream()))
+    return dq1, dk1, dq2, dk2, dv, dlam
 
 
 def lambda_backward(lq1, lk1, lq2, lk2, dlam):

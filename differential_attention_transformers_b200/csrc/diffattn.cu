@@ -20,6 +20,7 @@
 #include "lambda_simt.cuh"
 #include "prefill_sm100.cuh"
 #include "backward_sm100.cuh"
+#include "v1_adapter.cuh"
 
 using namespace da;
 
@@ -112,6 +113,8 @@ int device_setup(DeviceInfo** out) {
                                   (int)prefill_smem<128>()));
     CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)prefill_smem<128>()));
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)prefill_smem<64>()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
@@ -185,7 +188,7 @@ int launch_simt(const SimtArgs& a, cudaStream_t s) {
 int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
                    const float* lambda, void* out, int B, int Hout, int Hq, int Hkv, int Lq, int Lk, int dqk,
                    bool v1, int causal, int rms, float eps, cudaStream_t s, float* lse = nullptr,
-                   void* o_maps = nullptr) {
+                   void* o_maps = nullptr, float* rstd = nullptr) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   if (Lq == 0 || B == 0 || Hout == 0) return ok();
@@ -211,12 +214,13 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.watch = make_watch(dev);
   a.lse = lse;
   a.o_maps = static_cast<__nv_bfloat16*>(o_maps);
+  a.rstd = rstd;
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
   if (lse != nullptr && dqk == 128)   // training forward (V2)
     prefill_kernel<128, true><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
-  else if (lse != nullptr)
-    return fail(DIFFATTN_ERR_UNSUPPORTED, "the training forward needs the 128-wide QK layout");
+  else if (lse != nullptr)            // training forward (V1, d = 64)
+    prefill_kernel<64, true><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (dqk == 64)
     prefill_kernel<64><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else
@@ -303,9 +307,12 @@ size_t bwd_ws_bytes(int B, int Hq, int Lq) {
   return 2 * align256((size_t)B * Hp * 2 * Lp * 4) + align256((size_t)B * Hp * (Lp / 64) * 4);
 }
 
+// dqk: the width that sets the score scale 1/sqrt(dqk) -- 128 for V2, 64 for
+// the packed V1 layout (whose zero halves leave the scores unchanged).
 int launch_backward_v2(const void* q, const void* k, const void* v, const float* lambda, const void* dout,
                        const float* lse, const void* o_maps, void* dq, void* dk, void* dv, float* dlambda, int B,
-                       int Hq, int Hkv, int Lq, int Lk, int causal, void* ws, size_t ws_bytes, cudaStream_t s) {
+                       int Hq, int Hkv, int Lq, int Lk, int causal, void* ws, size_t ws_bytes, cudaStream_t s,
+                       int dqk = 128) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   const size_t need = bwd_ws_bytes(B, Hq, Lq);
@@ -331,8 +338,8 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk; a.Lp = Lp;
   a.causal = causal ? 1 : 0;
-  a.scale = (float)(1.0 / std::sqrt(128.0));
-  a.scale_log2 = log2e_over_sqrt(128);
+  a.scale = (float)(1.0 / std::sqrt((double)dqk));
+  a.scale_log2 = log2e_over_sqrt(dqk);
   a.resid_tau = DIFFATTN_RESID_TAU;
   a.watch = make_watch(dev);
   const long long Lk_map = Lk > 0 ? Lk : 1;   // a zero extent is not encodable; no key is then loaded
@@ -355,6 +362,73 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
     if (int e = make_map(&mo, Lq > 0 ? dout : k, 128, Lq_map, (long long)B * Hp, BW_RB)) return e;
     const long long units = (long long)((Lk + PF_BM - 1) / PF_BM) * B * Hkv;
     bwd_dkv_kernel<<<(unsigned)units, BW_THREADS, bwd_dkv_smem(), s>>>(mk, mv, mq, mo, a);
+    CUDA_TRY(cudaGetLastError());
+  }
+  return ok();
+}
+
+// V1 backward workspace: the packed [Q1|0], [0|Q2] rows and their gradient
+// (B*2H*Lq rows of 128), the packed [K1|K2] rows and their gradient
+// (B*Hkv*Lk rows of 128), the RMSNorm input gradient dX (B*H*Lq rows of 128,
+// with RMSNorm only), then the V2 backward's own workspace.
+struct V1BwdLayout {
+  size_t qp, dqp, kp, dkp, dx, bw, total;
+};
+V1BwdLayout v1_bwd_layout(int B, int H, int Hkv, int Lq, int Lk, int rms) {
+  const size_t nq = (size_t)B * H * Lq, nk = (size_t)B * Hkv * Lk;
+  V1BwdLayout l;
+  l.qp = 0;
+  l.dqp = l.qp + align256(nq * 512);
+  l.kp = l.dqp + align256(nq * 512);
+  l.dkp = l.kp + align256(nk * 256);
+  l.dx = l.dkp + align256(nk * 256);
+  l.bw = l.dx + (rms ? align256(nq * 256) : 0);
+  l.total = l.bw + bwd_ws_bytes(B, 2 * H, Lq);
+  return l;
+}
+
+unsigned stream_grid(const DeviceInfo* dev, long long items, int per_block) {
+  long long g = (items + per_block - 1) / per_block;
+  const long long cap = (long long)dev->sms * 8;
+  return (unsigned)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+int launch_backward_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                       const float* lambda, const void* dout, const void* out, const float* lse, const void* o_maps,
+                       const float* rstd, void* dq1, void* dk1, void* dq2, void* dk2, void* dv, float* dlambda,
+                       int B, int H, int Hkv, int Lq, int Lk, int causal, int rms, void* ws, size_t ws_bytes,
+                       cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  const V1BwdLayout L = v1_bwd_layout(B, H, Hkv, Lq, Lk, rms);
+  if (ws == nullptr || ws_bytes < L.total)
+    return fail(DIFFATTN_ERR_WORKSPACE, "V1 backward workspace %zu B < required %zu B", ws_bytes, L.total);
+  if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  char* w = static_cast<char*>(ws);
+  auto at = [w](size_t off) { return reinterpret_cast<__nv_bfloat16*>(w + off); };
+  const long long nq = (long long)B * H * Lq, nk = (long long)B * Hkv * Lk;
+  if (nq + nk > 0) {
+    V1PackArgs pa{static_cast<const __nv_bfloat16*>(q1), static_cast<const __nv_bfloat16*>(q2),
+                  static_cast<const __nv_bfloat16*>(k1), static_cast<const __nv_bfloat16*>(k2), at(L.qp), at(L.kp),
+                  nq, nk, Lq};
+    v1_pack_kernel<<<stream_grid(dev, (nq + nk) * 8, V1A_THREADS), V1A_THREADS, 0, s>>>(pa);
+    CUDA_TRY(cudaGetLastError());
+  }
+  const void* g = dout;
+  if (rms && nq > 0) {
+    V1RmsArgs ra{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), rstd, at(L.dx),
+                 nq};
+    v1_rms_backward_kernel<<<stream_grid(dev, nq, V1A_THREADS / 32), V1A_THREADS, 0, s>>>(ra);
+    CUDA_TRY(cudaGetLastError());
+    g = at(L.dx);
+  }
+  if (int e = launch_backward_v2(at(L.qp), at(L.kp), v, lambda, g, lse, o_maps, at(L.dqp), at(L.dkp), dv, dlambda,
+                                 B, 2 * H, Hkv, Lq, Lk, causal, w + L.bw, ws_bytes - L.bw, s, 64))
+    return e;
+  if (nq + nk > 0) {
+    V1UnpackArgs ua{at(L.dqp), at(L.dkp), static_cast<__nv_bfloat16*>(dq1), static_cast<__nv_bfloat16*>(dq2),
+                    static_cast<__nv_bfloat16*>(dk1), static_cast<__nv_bfloat16*>(dk2), nq, nk, Lq};
+    v1_unpack_kernel<<<stream_grid(dev, (nq + nk) * 8, V1A_THREADS), V1A_THREADS, 0, s>>>(ua);
     CUDA_TRY(cudaGetLastError());
   }
   return ok();
@@ -601,6 +675,61 @@ int diffattn_bwd_v2(const void* q, const void* k, const void* v, const float* la
     if (p && !aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
   return launch_backward_v2(q, k, v, lambda, dout, lse, o_maps, dq, dk, dv, dlambda, B, Hq, Hkv, Lq, Lk, causal,
                             ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                          const float* lambda, void* out, float* lse, void* o_maps, float* rstd,
+                          diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk, int d, int dv, int causal,
+                          int rmsnorm, float eps, void* stream) {
+  if (B < 0 || H < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || d < 1 || dv < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d Lq=%d Lk=%d d=%d dv=%d)", B, H, Hkv, Lq,
+                Lk, d, dv);
+  if (H % Hkv) return fail(DIFFATTN_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+  if (rmsnorm && !(eps >= 0.f)) return fail(DIFFATTN_ERR_INVALID_ARG, "eps must be >= 0");
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the training forward takes bf16 only");
+  if (d != 64 || dv != 128)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "V1 training path needs d == 64 and dv == 128 (got d=%d dv=%d)", d, dv);
+  if (B == 0 || Lq == 0) return ok();
+  if (!q1 || !q2 || !lambda || !out || !lse || !o_maps || (rmsnorm && !rstd) ||
+      (Lk > 0 && (!k1 || !k2 || !v)))
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (Lk == 0) k1 = k2 = v = q1;
+  if (int e = check_bf16_ptrs({q1, k1, q2, k2, v, out, o_maps})) return e;
+  return launch_prefill(q1, q2, k1, k2, v, lambda, out, B, H, H, Hkv, Lq, Lk, 64, true, causal, rmsnorm, eps,
+                        static_cast<cudaStream_t>(stream), lse, o_maps, rstd);
+}
+
+size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int rmsnorm) {
+  if (B < 0 || H < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || H % Hkv) return 0;
+  return v1_bwd_layout(B, H, Hkv, Lq, Lk, rmsnorm ? 1 : 0).total;
+}
+
+int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                    const float* lambda, const void* dout, const void* out, const float* lse, const void* o_maps,
+                    const float* rstd, void* dq1, void* dk1, void* dq2, void* dk2, void* dv, float* dlambda,
+                    diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk, int d, int dv_width, int causal,
+                    int rmsnorm, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 0 || H < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || d < 1 || dv_width < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d Lq=%d Lk=%d d=%d dv=%d)", B, H, Hkv, Lq,
+                Lk, d, dv_width);
+  if (H % Hkv) return fail(DIFFATTN_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the backward takes bf16 only");
+  if (d != 64 || dv_width != 128)
+    return fail(DIFFATTN_ERR_UNSUPPORTED, "V1 backward needs d == 64 and dv == 128 (got d=%d dv=%d)", d, dv_width);
+  if (!lambda || !dlambda) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  const int rms = rmsnorm ? 1 : 0;
+  if (B == 0) {   // nothing to differentiate: dlambda is an empty sum
+    CUDA_TRY(cudaMemsetAsync(dlambda, 0, sizeof(float) * (size_t)H, static_cast<cudaStream_t>(stream)));
+    return ok();
+  }
+  if ((Lq > 0 && (!q1 || !q2 || !dout || !lse || !o_maps || !dq1 || !dq2 || (rms && (!out || !rstd)))) ||
+      (Lk > 0 && (!k1 || !k2 || !v || !dk1 || !dk2 || !dv)))
+    return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  for (const void* p : std::initializer_list<const void*>{q1, k1, q2, k2, v, dout, out, o_maps, dq1, dk1, dq2, dk2,
+                                                          dv})
+    if (p && !aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
+  return launch_backward_v1(q1, k1, q2, k2, v, lambda, dout, out, lse, o_maps, rstd, dq1, dk1, dq2, dk2, dv, dlambda,
+                            B, H, Hkv, Lq, Lk, causal, rms, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int diffattn_lambda_backward(const float* lq1, const float* lk1, const float* lq2, const float* lk2,

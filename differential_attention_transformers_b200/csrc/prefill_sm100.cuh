@@ -65,9 +65,11 @@ struct PrefillArgs {
   // Training outputs (null for inference): per row and map the log-sum-exp of
   // the scaled scores in log2 units, lse[B, Hout, 2, Lq] (+inf for a row that
   // sees no key), and the normalised map outputs O_m / l_m, o_maps[B, Hout, 2,
-  // Lq, 128] bf16.
+  // Lq, 128] bf16; with RMSNorm also the row's 1/rms, rstd[B, Hout, Lq] (0 for
+  // a row that sees no key).
   float* lse;
   __nv_bfloat16* o_maps;
+  float* rstd;
 };
 
 template <int DQK>
@@ -141,9 +143,10 @@ __device__ __forceinline__ float pf_exp_store(const float (&s)[PF_BN], float2 sc
 // chunks XOR-swizzled by row, conflict-free both ways) and writes them back as
 // 4 rows x 128 contiguous bytes per instruction (a direct store of each
 // thread's own row would touch 32 lines per instruction).  base points at
-// column 0 of row 0; rows are 128 elements apart; rows >= Lq are skipped.
+// column 0 of row 0; rows are `stride` elements apart (128 by default); rows
+// >= Lq are skipped.
 __device__ __forceinline__ void pf_store_rows(uint8_t* st, const float (&y)[64], __nv_bfloat16* base, int row_w0,
-                                              int Lq, int lane) {
+                                              int Lq, int lane, int stride = PF_DV) {
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     if ((lane >> 4) == half) {
@@ -164,7 +167,7 @@ __device__ __forceinline__ void pf_store_rows(uint8_t* st, const float (&y)[64],
       const int rr = 4 * i + (lane >> 3), c = lane & 7;
       const int row = row_w0 + 16 * half + rr;
       const uint4 v = *reinterpret_cast<const uint4*>(st + rr * 128 + ((c ^ (rr & 7)) << 4));
-      if (row < Lq) *reinterpret_cast<uint4*>(base + (size_t)row * PF_DV + c * 8) = v;
+      if (row < Lq) *reinterpret_cast<uint4*>(base + (size_t)row * stride + c * 8) = v;
     }
     __syncwarp();
   }
@@ -460,6 +463,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
             const float rs = rsqrtf((S.ss[0][r] + S.ss[1][r]) / (float)PF_DV + a.eps);
 #pragma unroll
             for (int i = 0; i < 64; ++i) y[i] *= rs;
+            if (TRAIN && m == 0 && rg < a.Lq)
+              a.rstd[((size_t)b * a.Hout + h) * a.Lq + rg] = l_run > 0.f ? rs : 0.f;
           }
         }
       }
@@ -467,6 +472,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 #pragma unroll
       for (int i = 0; i < 64; ++i) y[i] = 0.f;
       have = true;
+      if (TRAIN && a.rms && m == 0 && rg < a.Lq) a.rstd[((size_t)b * a.Hout + h) * a.Lq + rg] = 0.f;
     }
     have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;   // warp-uniform (ok is)
     const int row_w0 = r0 + wq * 32;                          // first row of this warp

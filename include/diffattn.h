@@ -217,6 +217,47 @@ DIFFATTN_API int diffattn_bwd_v2(const void* q, const void* k, const void* v, co
                                  diffattn_dtype dtype, int B, int Hq, int Hkv, int Lq, int Lk, int D, int causal,
                                  void* ws, size_t ws_bytes, void* stream);
 
+/* Training forward, V1 layout, bf16 (same operation and arguments as
+ * diffattn_fwd_v1, with d == 64 and dv == 128), that also writes what
+ * diffattn_bwd_v1 needs:
+ *   lse    : f32 [B, H, 2, Lq], as for diffattn_fwd_v2_train, with the scores
+ *            of map m = Q_m K_m^T scaled by log2(e)/sqrt(d)       (device)
+ *   o_maps : bf16 [B, H, 2, Lq, 128]: O_m = A_m V per map         (device)
+ *   rstd   : f32 [B, H, Lq]: with rmsnorm != 0, the row's
+ *            1/sqrt(mean(x^2) + eps) of the difference output x (0 for a row
+ *            that sees no key); not touched, and may be NULL, without. (device)
+ * The per-head RMSNorm is the tutorial's (section V1 到 V2 的 diff). */
+DIFFATTN_API int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const void* k2,
+                                       const void* v, const float* lambda, void* out, float* lse, void* o_maps,
+                                       float* rstd, diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk,
+                                       int d, int dv, int causal, int rmsnorm, float eps, void* stream);
+
+/* Workspace, in bytes, for diffattn_bwd_v1.  0 for invalid sizes. */
+DIFFATTN_API size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int rmsnorm);
+
+/* Backward of the V1 forward (bf16, d == 64, dv == 128), with the RMSNorm
+ * gradient dX = r (dY - y <y, dY> / dv) first when rmsnorm != 0:
+ *   q1, k1, q2, k2, v, lambda : the forward's inputs               (device)
+ *   dout            : bf16 [B, H, Lq, 128], the gradient of out    (device)
+ *   out, lse,
+ *   o_maps, rstd    : from diffattn_fwd_v1_train (out and rstd are read
+ *                     only with rmsnorm != 0 and may be NULL without) (device)
+ *   dq1, dq2        : bf16 [B, H, Lq, 64]; dk1, dk2 : bf16 [B, Hkv, Lk, 64];
+ *   dv              : bf16 [B, Hkv, Lk, 128]; dlambda : f32 [H]    (device)
+ *   ws              : diffattn_bwd_v1_workspace_size bytes, 16-byte aligned.
+ * The maps are those of diffattn_bwd_v2 with Q_1 K_1^T and Q_2 K_2^T as the
+ * scores.  The call packs [Q1 | 0], [0 | Q2] and [K1 | K2] into 128-wide
+ * tensors in the workspace, runs the V2 backward on them at scale 1/sqrt(64)
+ * (the zero halves leave every score unchanged) and takes dQ1, dQ2, dK1 and
+ * dK2 back out of the fixed halves of the packed gradients.  dK1, dK2 and dV
+ * sum over the heads of a KV group. */
+DIFFATTN_API int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
+                                 const float* lambda, const void* dout, const void* out, const float* lse,
+                                 const void* o_maps, const float* rstd, void* dq1, void* dk1, void* dq2, void* dk2,
+                                 void* dv, float* dlambda, diffattn_dtype dtype, int B, int H, int Hkv, int Lq,
+                                 int Lk, int d, int dv_width, int causal, int rmsnorm, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /* Gradients of λ = exp(lq1.lk1) - exp(lq2.lk2) + λ_init with respect to its
  * parameter vectors ([heads, dim] f32 each), given dlambda [heads]: fp64
  * inside, f32 out.                                                 (device) */

@@ -80,6 +80,25 @@ def head_backward(q1, k1, q2, k2, v, lam: float, dout, causal: bool, rms: bool =
     return dq1, dk1, dq2, dk2, dv, dlam
 
 
+def dlambda_terms(q1, k1, q2, k2, v, lam: float, dout, causal: bool, rms: bool = False, eps: float = 1e-5):
+    """The products dX * O_2 whose sum, negated, is one head's dlambda ([Lq, dv] fp64).
+
+    Used to state the error a bf16 implementation can reach: dlambda sums
+    Lq * dv products of two stored bf16 operands, so its rounding scales with
+    the terms' size, not with the sum's.  With RMSNorm, dX is orthogonal to X
+    (up to eps), and when the two maps are alike O_2 is nearly parallel to X,
+    so the sum is a small remainder of large terms."""
+    q1, k1, q2, k2, v, dout = (_f64(t) for t in (q1, k1, q2, k2, v, dout))
+    A1, A2 = maps(q1, k1, q2, k2, causal, 0, q1.shape[0])
+    O1, O2 = A1 @ v, A2 @ v
+    dx = dout
+    if rms:
+        x = O1 - float(lam) * O2
+        r = 1.0 / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + eps)
+        dx = r * dx - (r ** 3 / x.shape[1]) * x * np.sum(x * dx, axis=1, keepdims=True)
+    return dx * O2
+
+
 def diffattn_v2_backward(q, k, v, lam, dout, causal=True):
     """V2 layout.  q [B,Hq,Lq,D]; k,v [B,Hkv,Lk,D]; lam [Hq/2]; dout [B,Hq/2,Lq,D].
 

@@ -26,6 +26,23 @@ def _rel(got, ref):
     return float(np.max(np.abs(got - ref))) / scale if scale > 0 else float(np.max(np.abs(got)))
 
 
+# dlambda sums Lq * dv products of two stored bf16 operands (dX, or dO, and the
+# forward's O_2), each rounded to 2^-9 relative, and further rounding enters
+# through P and the RMSNorm gradient.  Its error therefore scales with the
+# terms, not with their sum, which is small against them when the maps are
+# alike and RMSNorm makes dX orthogonal to X.  Bound: the output tolerance plus
+# ten unit roundings of the terms' 2-norm (a dropped term or a sign error
+# misses it by far more).
+DLAM_ROUND = 10 * 2.0 ** -9
+
+
+def _dlam_ok(got, ref, term_norms):
+    got = got.double().cpu().numpy()
+    ref = np.asarray(ref, dtype=np.float64)
+    bound = BF16_TOL * np.max(np.abs(ref)) + DLAM_ROUND * np.asarray(term_norms)
+    return bool(np.all(np.abs(got - ref) <= bound)), np.abs(got - ref), bound
+
+
 def _case(B, Hq, Hkv, Lq, Lk, seed, lam_lo=-0.2, lam_hi=1.0):
     g = torch.Generator(device="cpu").manual_seed(seed)
     s = 1 / math.sqrt(128)
@@ -135,3 +152,67 @@ def test_backward_near_unit_lambda_with_similar_maps(lam_value):
     rq, rk, rv, rl = bwd.diffattn_v2_backward(q, k, v, np.array([lam_value]), dout, causal=True)
     for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
         assert _rel(got, ref) <= BF16_TOL, (name, lam_value, _rel(got, ref))
+
+
+# ----------------------------------------------------------------- V1 layout --
+def _case_v1(B, H, Hkv, Lq, Lk, seed, lam_lo=-0.2, lam_hi=1.0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    s = 1 / math.sqrt(64)
+    mk = lambda *shape, std=s: (torch.randn(*shape, generator=g) * std).to(torch.bfloat16).to(DEV)  # noqa: E731
+    q1, q2 = mk(B, H, Lq, 64), mk(B, H, Lq, 64)
+    k1, k2 = mk(B, Hkv, Lk, 64), mk(B, Hkv, Lk, 64)
+    v = mk(B, Hkv, Lk, 128)
+    dout = mk(B, H, Lq, 128, std=1.0)
+    lam = (torch.rand(H, generator=g) * (lam_hi - lam_lo) + lam_lo).to(DEV)
+    return q1, k1, q2, k2, v, dout, lam
+
+
+CASES_V1 = [
+    # B, H, Hkv, Lq, Lk, causal, rmsnorm
+    (1, 2, 1, 200, 200, True, False),    # ragged tails, two heads share a KV head
+    (2, 4, 2, 300, 300, False, True),    # non-causal, RMSNorm
+    (1, 2, 2, 130, 257, True, True),     # Lq < Lk: bottom-right causal offset
+    (1, 2, 1, 257, 130, True, True),     # Lq > Lk: the first rows see no key
+    (1, 4, 4, 64, 64, True, False),      # a single tile
+]
+
+
+@pytest.mark.parametrize("B,H,Hkv,Lq,Lk,causal,rms", CASES_V1)
+def test_v1_backward_matches_oracle(B, H, Hkv, Lq, Lk, causal, rms):
+    q1, k1, q2, k2, v, dout, lam = _case_v1(B, H, Hkv, Lq, Lk, seed=3 * Lq + Lk + H)
+    out, lse, om, rstd = da.fwd_v1_train(q1, k1, q2, k2, v, lam, causal=causal, rmsnorm=rms)
+    assert torch.equal(out, da.fwd_v1(q1, k1, q2, k2, v, lam, causal=causal, rmsnorm=rms))
+    grads = da.bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, om, rstd, causal=causal, rmsnorm=rms)
+    torch.cuda.synchronize()
+    assert da.last_status() == da.OK
+    lr = lam.cpu().numpy()
+    ref = bwd.diffattn_v1_backward(q1, k1, q2, k2, v, lr, dout, causal=causal, rms=rms, eps=1e-5)
+    for name, got, r in zip(("dq1", "dk1", "dq2", "dk2", "dv"), grads, ref):
+        assert torch.isfinite(got.float()).all(), name
+        assert _rel(got, r) <= BF16_TOL, (name, _rel(got, r))
+    grp = H // Hkv
+    norms = [np.sqrt(sum(np.sum(bwd.dlambda_terms(q1[b, h], k1[b, h // grp], q2[b, h], k2[b, h // grp],
+                                                  v[b, h // grp], lr[h], dout[b, h], causal, rms=rms) ** 2)
+                         for b in range(B))) for h in range(H)]
+    ok, err, bound = _dlam_ok(grads[5], ref[5], norms)
+    assert ok, ("dlambda", err, bound)
+
+
+def test_v1_training_forward_statistics():
+    q1, k1, q2, k2, v, dout, lam = _case_v1(1, 2, 1, 190, 190, seed=41)
+    out, lse, om, rstd = da.fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=True)
+    sl = math.log2(math.e) / 8.0
+    vis = np.tril(np.ones((190, 190), dtype=bool))
+    vd = orc._f64(v[0, 0])
+    for h in range(2):
+        A = []
+        for m, (q, k) in enumerate(((q1, k1), (q2, k2))):
+            S = np.where(vis, orc._f64(q[0, h]) @ orc._f64(k[0, 0]).T * sl, -np.inf)
+            mx = S.max(axis=1, keepdims=True)
+            ref_lse = (mx + np.log2(np.sum(np.exp2(S - mx), axis=1, keepdims=True)))[:, 0]
+            assert np.max(np.abs(lse[0, h, m].cpu().numpy() - ref_lse)) <= 1e-3
+            A.append(np.exp2(S - ref_lse[:, None]))
+            assert _rel(om[0, h, m], A[m] @ vd) <= BF16_TOL
+        x = (A[0] - float(lam[h]) * A[1]) @ vd
+        r = 1.0 / np.sqrt(np.mean(x * x, axis=1) + 1e-5)
+        assert np.max(np.abs(rstd[0, h].cpu().numpy() - r) / r) <= 1e-2

@@ -127,3 +127,42 @@ def test_zero_upstream_gives_zero_gradients_and_linearity():
     c = bwd.diffattn_v2_backward(q, k, v, lam, 2 * d1 - d2)
     for x, y, z in zip(a, b, c):
         assert np.allclose(z, 2 * x - y, rtol=1e-12, atol=1e-12)
+
+
+def test_v1_gradients_are_v2_gradients_of_the_packed_layout():
+    """The library's V1 backward runs the V2 backward on [Q1|0], [0|Q2] and
+    [K1|K2].  Check that identity on the oracle: with d = 64 and the V2 scale
+    1/sqrt(128), Q' is multiplied by sqrt(2) so that the scores are Q_m K_m^T / 8;
+    the V1 gradients are then fixed halves of the packed ones."""
+    rng = np.random.default_rng(29)
+    B, H, Hkv, Lq, Lk, d = 1, 4, 2, 7, 9, 64
+    q1, q2 = _rand((B, H, Lq, d), rng, 0.3), _rand((B, H, Lq, d), rng, 0.3)
+    k1, k2 = _rand((B, Hkv, Lk, d), rng, 0.3), _rand((B, Hkv, Lk, d), rng, 0.3)
+    v = _rand((B, Hkv, Lk, 2 * d), rng)
+    lam = np.array([0.3, 0.9, -0.1, 1.2])
+    dout = _rand((B, H, Lq, 2 * d), rng)
+    want = bwd.diffattn_v1_backward(q1, k1, q2, k2, v, lam, dout, causal=True)
+
+    c = math.sqrt(2.0)
+    qp = np.zeros((B, 2 * H, Lq, 2 * d))
+    qp[:, 0::2, :, :d] = c * q1
+    qp[:, 1::2, :, d:] = c * q2
+    kp = np.concatenate([k1, k2], axis=-1)
+    dqp, dkp, dv, dlam = bwd.diffattn_v2_backward(qp, kp, v, lam, dout, causal=True)
+    got = (c * dqp[:, 0::2, :, :d], dkp[:, :, :, :d], c * dqp[:, 1::2, :, d:], dkp[:, :, :, d:], dv, dlam)
+    for a, b in zip(got, want):
+        assert np.allclose(a, b, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("rms", [False, True])
+def test_dlambda_terms_sum_to_dlambda(rms):
+    """dlambda_terms (the error scale of dlambda in the GPU tests) sums to the
+    finite-difference-pinned dlambda; without RMSNorm its terms are dO * O_2."""
+    rng = np.random.default_rng(31 + rms)
+    q1, q2, k1, k2 = (_rand((6, 3), rng) for _ in range(4))
+    v, dout = _rand((6, 5), rng), _rand((6, 5), rng)
+    t = bwd.dlambda_terms(q1, k1, q2, k2, v, 0.6, dout, True, rms=rms)
+    assert np.isclose(-t.sum(), bwd.head_backward(q1, k1, q2, k2, v, 0.6, dout, True, rms=rms)[5], rtol=1e-12)
+    if not rms:
+        _, A2 = orc.maps(q1, k1, q2, k2, True)
+        assert np.allclose(t, dout * (A2 @ v), rtol=1e-13, atol=0)
