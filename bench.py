@@ -5,7 +5,8 @@ One step = the whole hot path for one batch of the primary workload: the
 per-head lambda kernel, then the prefill kernel (default workload: V2 causal
 prefill, B2 Hq64 Hkv8 N8192 D128 bf16, layer 24).  The other hot-path
 workloads (V1 prefill with RMSNorm, V2 64k decode, V1-layout 64k decode fused
-and unfused) are timed the same way and reported under "secondary".
+and unfused) are timed the same way and reported under "secondary".  The
+SNR-vs-context-length sweep (``--workload snr_sweep``) runs on request only.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl reference] [--no-cpu-baseline] [--no-secondary]
@@ -20,6 +21,7 @@ time over ranks.
 from __future__ import annotations
 
 import argparse
+import functools
 import json
 import math
 import os
@@ -35,6 +37,7 @@ sys.path.insert(0, ROOT)
 
 import differential_attention_transformers_b200 as da  # noqa: E402
 from differential_attention_transformers_b200 import inputs  # noqa: E402
+from differential_attention_transformers_b200 import noise  # noqa: E402
 
 METRIC = "diff-attn fwd prefill TFLOP/s & decode KV GB/s on 1 B200 (% of roofline)"
 L2_BYTES = 126 * 1024 * 1024
@@ -303,6 +306,61 @@ class Backward:
         raise NotImplementedError("the backward is timed on device tensors only")
 
 
+def sweep_bytes(n=inputs.SWEEP_INSTANCES, lengths=inputs.SWEEP_LENGTHS) -> int:
+    """Algorithmic bytes of one sweep step: every context length decoded twice
+    (plain and difference), each reading K1, K2 (64 wide) and V (128 wide) once."""
+    return sum(2 * n * N * (64 + 64 + 128) * 2 for N in lengths)
+
+
+class SnrSweep:
+    """The SNR-vs-context-length sweep (tutorial exercise 1): one step decodes
+    the noise construction at every length from 1k to 256k keys, with lambda = 0
+    (plain softmax) and lambda = 0.5 (the difference), on the V1 decode kernel."""
+
+    def __init__(self, device, n=inputs.SWEEP_INSTANCES, lengths=inputs.SWEEP_LENGTHS):
+        self.n, self.lengths = n, tuple(lengths)
+        base = inputs.noise_sweep(n, max(self.lengths), device=device)
+        self.parts = [inputs.sweep_prefix(base, N) for N in self.lengths]
+        del base
+        self.lams = (torch.zeros(1, dtype=torch.float32, device=device),
+                     torch.full((1,), 0.5, dtype=torch.float32, device=device))
+        self.outs = [[torch.empty((n, 1, 128), dtype=torch.bfloat16, device=device) for _ in self.lams]
+                     for _ in self.lengths]
+        self.ws = torch.empty(da.decode_workspace_size(n, 1, max(self.lengths)), dtype=torch.uint8, device=device)
+        self.launches_per_step = 2 * len(self.lengths) * 2   # split-KV kernel + combine, per decode
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        for p, outs in zip(self.parts, self.outs):
+            for lam, out in zip(self.lams, outs):
+                da.decode_v1(p["q1"], p["k1"], p["q2"], p["k2"], p["v"], lam, out=out, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        return sweep_bytes(self.n, self.lengths) / 1e9, "GB/s"
+
+    def summary(self):
+        return [noise.summarize(N, o[0][:, 0, 0].float(), o[0][:, 0, 1].float(), o[1][:, 0, 0].float(),
+                                o[1][:, 0, 1].float()) for N, o in zip(self.lengths, self.outs)]
+
+    def host_call(self, host):
+        raise NotImplementedError("the sweep is timed on device tensors only")
+
+
+def workload_work(name):
+    """(algorithmic work of one step, unit) of a bench workload."""
+    if name == "snr_sweep":
+        return sweep_bytes() / 1e9, "GB/s"
+    w = inputs.WORKLOADS[base_workload(name)]
+    if name.endswith("_backward"):
+        return backward_flops(w) / 1e12, "TFLOP/s"
+    if w.layout in ("v1", "v2"):
+        return prefill_flops(w) / 1e12, "TFLOP/s"
+    return decode_bytes(w) / 1e9 * (1.5 if name.endswith("_unfused") else 1.0), "GB/s"
+
+
 def base_workload(name):
     """The workload a bench name is built on (variants share their base's shapes)."""
     return {"v2_backward": "v2_prefill", "v1_backward": "v1_prefill", "v2_decode_paged": "v2_decode",
@@ -310,6 +368,8 @@ def base_workload(name):
 
 
 def make_runner(name, device):
+    if name == "snr_sweep":
+        return SnrSweep(device)
     if name.endswith("_backward"):
         return Backward(inputs.WORKLOADS[base_workload(name)], device)
     if name == "v2_decode_paged":
@@ -321,6 +381,12 @@ def make_runner(name, device):
 
 
 def describe(name):
+    if name == "snr_sweep":
+        return {"workload": name, "layout": "v1_decode", "instances": inputs.SWEEP_INSTANCES,
+                "Lk": list(inputs.SWEEP_LENGTHS), "d": 64, "dv": 128, "lambda": [0.0, 0.5],
+                "mode": "noise construction (key 0 = 5q among N(0,1) keys), plain and difference rows; "
+                        "V = two indicator columns",
+                "l2": "inputs larger than L2 (126 MB) at the long lengths; no flush between steps"}
     w = inputs.WORKLOADS[base_workload(name)]
     d = {"workload": name, "layout": w.layout, "B": w.B, "heads": w.H, "kv_heads": w.Hkv, "Lq": w.Lq, "Lk": w.Lk,
          "d": w.d, "dv": w.dv, "causal": w.causal, "layer": w.layer, "rmsnorm": w.rmsnorm,
@@ -433,6 +499,33 @@ def roofline(r, kern_ms, peaks, power_capped=False):
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
+@functools.lru_cache(maxsize=1)
+def _sweep_host_inputs():
+    """The sweep's inputs on the host, drawn once per process (about 12 s)."""
+    return inputs.noise_sweep(inputs.SWEEP_INSTANCES, inputs.SWEEP_LENGTHS[-1])
+
+
+def cpu_oracle_sweep(cores, budget_s):
+    """The oracle's noise probe on instances of the sweep, longest context
+    first, both rows (plain and difference) per probe; bytes counted as on the
+    GPU (K1, K2 and V of the instance, per row)."""
+    from oracle import diffattn as orc
+    N = inputs.SWEEP_LENGTHS[-1]
+    x = _sweep_host_inputs()
+    done, t_total, n = 0.0, 0.0, 0
+    for i in range(inputs.SWEEP_INSTANCES):
+        t0 = time.perf_counter()
+        orc.noise_probe(x["q1"][i:i + 1, 0], x["k1"][i:i + 1, 0], x["q2"][i:i + 1, 0], x["k2"][i:i + 1, 0], 0.5)
+        t_total += time.perf_counter() - t0
+        done += 2 * N * (64 + 64 + 128) * 2 / 1e9
+        n += 1
+        if t_total >= budget_s:
+            break
+    return {"value": done / t_total, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {inputs.SWEEP_INSTANCES} instances at {N} keys, plain and difference rows, fp64 NumPy",
+            "seconds": t_total}
+
+
 def cpu_oracle_run(name, budget_s=12.0):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload.
 
@@ -446,6 +539,8 @@ def cpu_oracle_run(name, budget_s=12.0):
         cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
     except Exception:
         cores = len(os.sched_getaffinity(0))
+    if name == "snr_sweep":
+        return cpu_oracle_sweep(cores, budget_s)
     paged, backward = name == "v2_decode_paged", name.endswith("_backward")
     w = inputs.WORKLOADS[base_workload(name)]
     x = inputs.make(w, device="cpu") if w.layout in ("v1", "v2") else None
@@ -527,7 +622,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="v2_prefill",
                     choices=["v2_prefill", "v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged",
-                             "v1_decode", "v1_decode_unfused"])
+                             "v1_decode", "v1_decode_unfused", "snr_sweep"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
@@ -535,14 +630,13 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size of the workload (smaller profiling cases)")
     args = ap.parse_args()
-    if args.batch is not None:
+    if args.batch is not None and args.workload != "snr_sweep":
         base = base_workload(args.workload)
         inputs.WORKLOADS[base] = inputs.with_shape(inputs.WORKLOADS[base], B=args.batch)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = inputs.WORKLOADS[base_workload(args.workload)]
 
     if args.impl == "reference":
         # The reference arm is the fp64 CPU oracle, on rank 0 only.
@@ -556,7 +650,7 @@ def main():
         cb = dict(res[-1])
         cb["value"] = v
         unit = cb["unit"]
-        work_unit = prefill_flops(w) / 1e12 if unit == "TFLOP/s" else decode_bytes(w) / 1e9
+        work_unit = workload_work(args.workload)[0]
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
                 "steps": steps, "warmup": args.warmup, "ms_per_step": work_unit / v * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -609,8 +703,11 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_measure(r, max(2, min(args.steps, 5)))
-        e2e["value"] *= world
+        try:
+            e2e = e2e_measure(r, max(2, min(args.steps, 5)))
+            e2e["value"] *= world
+        except NotImplementedError as exc:   # workloads timed on device tensors only
+            e2e = {"unavailable": str(exc)}
 
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -620,6 +717,8 @@ def main():
             "clocks": clocks}
     if secondary:
         line["secondary"] = secondary
+    if isinstance(r, SnrSweep):
+        line["snr"] = r.summary()
     if rank == 0 and not args.no_cpu_baseline and not dist_on:
         line["cpu_baseline"] = cpu_oracle_run(args.workload)
     if rank == 0:

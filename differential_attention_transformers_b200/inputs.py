@@ -21,6 +21,14 @@ Workloads (shapes, value distributions):
                N(0,1)/sqrt(128), layer 24.
   v1_decode    the same decode shape in the V1 layout: 32 heads over 8 KV
                heads, Q1/Q2/K1/K2 width 64, V width 128.
+  noise sweep  (noise_sweep / sweep_prefix) the noise_probe construction at
+               context lengths 1k..256k keys (tutorial exercise 1), in bf16 for
+               the V1 decode layout: 64 instances, each a query q ~ N(0,1) in
+               d=64 with key 0 = 5q among N(0,1) keys and an independent second
+               map; shorter contexts are prefixes of the longest one.  V has
+               width 128: column 0 is 1 at key 0, column 1 is 1 at keys 1..N-1,
+               the rest 0, so the output holds the row's weight on the signal
+               key and its total weight on the noise keys.
 
 bf16 tensors are drawn in fp32 and rounded to bf16 (round-to-nearest-even);
 the oracle receives those rounded values.  lq/lk are fp32 N(0,1)*0.1 with the
@@ -183,3 +191,34 @@ def paged_cache(kc, vc, page_size: int, seed: int, spare_pages: int = 3, lens=No
             vp[pid, : t1 - t0] = vc[b, :, t0:t1].transpose(0, 1)
     return kp, vp, table.to(kc.device), torch.tensor(lens, dtype=torch.int32, device=kc.device)
 
+
+
+SWEEP_LENGTHS = tuple(1024 << i for i in range(9))    # 1k, 2k, ..., 256k keys
+SWEEP_INSTANCES = 64
+
+
+def noise_sweep(n: int = SWEEP_INSTANCES, N: int = SWEEP_LENGTHS[-1], seed: int = 1010, device="cpu"):
+    """The noise-floor construction over N keys for n instances, bf16, V1
+    decode layout: q1, q2 [n, 1, 64]; k1, k2 [n, 1, N, 64]; v [n, 1, N, 128]
+    (indicator columns, see the module notes).  Key 0 of k1 is 5 q1, formed in
+    fp32 before the rounding to bf16."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    d = 64
+    q1 = _randn(gen, (n, 1, d), 1.0, torch.float32, device)
+    k1 = _randn(gen, (n, 1, N, d), 1.0, torch.float32, device)
+    k1[:, 0, 0, :] = 5.0 * q1[:, 0, :]
+    q2 = _randn(gen, (n, 1, d), 1.0, torch.float32, device)
+    k2 = _randn(gen, (n, 1, N, d), 1.0, torch.float32, device)
+    v = torch.zeros((n, 1, N, 128), dtype=torch.bfloat16, device=device)
+    v[:, 0, 0, 0] = 1.0
+    v[:, 0, 1:, 1] = 1.0
+    bf = torch.bfloat16
+    return {"q1": q1.to(bf), "k1": k1.to(bf), "q2": q2.to(bf), "k2": k2.to(bf), "v": v}
+
+
+def sweep_prefix(x, N: int):
+    """The same instances over their first N keys (contiguous copies)."""
+    out = {"q1": x["q1"], "q2": x["q2"]}
+    for name in ("k1", "k2", "v"):
+        out[name] = x[name][:, :, :N].contiguous()
+    return out
