@@ -22,10 +22,13 @@ Modules:
   backward -- the chain rule of the forward (dQ, dK, dV, dlambda and lambda's
               parameter gradients) in fp64, pinned by finite differences and an
               independent autograd derivation (tests/test_oracle_backward.py).
+  lowrank  -- the fixed low-rank substitute for A2 (paper note, sections
+              基于分析的改进建议 and 亮点与洞察), under the reading in its
+              header, pinned in tests/test_oracle_lowrank.py.
 
 Parity status: every function is pinned by tests in ``tests/test_oracle.py``
 except the page's claimed noise-floor percentages and the SNR claim of the
 tutorial's Step 3, which are "parity unpinned" (see ``diffattn.noise_probe``).
 """
 
-from . import backward, brute, diffattn  # noqa: F401
+from . import backward, brute, diffattn, lowrank  # noqa: F401
