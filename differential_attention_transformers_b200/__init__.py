@@ -109,12 +109,49 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
 
 
+def _expect(*specs):
+    """Shape and dtype checks, made before anything reaches the library: the C
+    ABI takes plain pointers and sizes, so a tensor smaller than the sizes say
+    would be read or written out of bounds.  specs: (name, tensor, shape, dtype
+    or None)."""
+    for name, t, shape, dt in specs:
+        if t is None:
+            raise ValueError(f"{name} is required")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if dt is not None and t.dtype != dt:
+            raise ValueError(f"{name} must be {dt}, got {t.dtype}")
+
+
+def _dims(name, t, n):
+    if t is None or t.dim() != n:
+        raise ValueError(f"{name} must be a {n}-d tensor")
+    return tuple(t.shape)
+
+
+def _device_only(named):
+    """Entry points that take device tensors: contiguous, on the current CUDA device."""
+    for name, t in named:
+        if t is None:
+            continue
+        if t.device.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    dev = torch.cuda.current_device()
+    for name, t in named:
+        if t is not None and t.device.index != dev:
+            raise ValueError(f"{name} is on cuda:{t.device.index}, the current device is cuda:{dev}")
+
+
 def _prep(tensors):
     """Move CPU inputs to the current CUDA device; report whether we did."""
     host = any(t.device.type == "cpu" for t in tensors)
     dev = torch.device("cuda", torch.cuda.current_device())
     out = []
     for t in tensors:
+        if t.device.type == "cuda" and t.device.index != dev.index:
+            raise ValueError(f"a tensor is on cuda:{t.device.index}, the current device is cuda:{dev.index}")
         if t.device.type == "cpu":
             t = t.pin_memory().to(dev, non_blocking=True) if not t.is_pinned() else t.to(dev, non_blocking=True)
         if not t.is_contiguous():
@@ -226,6 +263,14 @@ def _prefill_host_pipelined(v1, qs, ks, v, lam, causal, rmsnorm, eps):
 
 def fwd_v1(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5, out=None):
     """V1 layout: q1,q2 [B,H,Lq,d]; k1,k2 [B,Hkv,Lk,d]; v [B,Hkv,Lk,dv]; lam f32 [H]."""
+    B, H, Lq, d = _dims("q1", q1, 4)
+    _, Hkv, Lk, _ = _dims("k1", k1, 4)
+    dv = _dims("v", v, 4)[3]
+    _expect(("q2", q2, (B, H, Lq, d), q1.dtype), ("k1", k1, (B, Hkv, Lk, d), q1.dtype),
+            ("k2", k2, (B, Hkv, Lk, d), q1.dtype), ("v", v, (B, Hkv, Lk, dv), q1.dtype),
+            ("lam", lam, (H,), torch.float32))
+    if out is not None:
+        _expect(("out", out, (B, H, Lq, dv), q1.dtype))
     if _pipelined([q1, k1, q2, k2, v], out):
         return _prefill_host_pipelined(True, [q1, q2], [k1, k2], v, lam, causal, rmsnorm, eps)
     host, (q1, k1, q2, k2, v, lam) = _prep([q1, k1, q2, k2, v, lam])
@@ -241,6 +286,12 @@ def fwd_v1(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5, out=Non
 
 def fwd_v2(q, k, v, lam, causal=True, out=None):
     """V2 layout: q [B,Hq,Lq,D]; k,v [B,Hkv,Lk,D]; lam f32 [Hq/2] -> [B,Hq/2,Lq,D]."""
+    B, Hq, Lq, D = _dims("q", q, 4)
+    _, Hkv, Lk, _ = _dims("k", k, 4)
+    _expect(("k", k, (B, Hkv, Lk, D), q.dtype), ("v", v, (B, Hkv, Lk, D), q.dtype),
+            ("lam", lam, (Hq // 2,), torch.float32))
+    if out is not None:
+        _expect(("out", out, (B, Hq // 2, Lq, D), q.dtype))
     if _pipelined([q, k, v], out):
         return _prefill_host_pipelined(False, [q], [k], v, lam, causal, False, 1e-5)
     host, (q, k, v, lam) = _prep([q, k, v, lam])
@@ -257,8 +308,11 @@ def fwd_v2(q, k, v, lam, causal=True, out=None):
 def fwd_v2_train(q, k, v, lam, causal=True):
     """V2 forward that also returns what the backward needs: (out [B,Hq/2,Lq,D],
     lse f32 [B,Hq/2,2,Lq] (log2 units), o_maps [B,Hq/2,2,Lq,D] = O_m / l_m).  bf16, device tensors."""
-    B, Hq, Lq, D = q.shape
-    Hkv, Lk = k.shape[1], k.shape[2]
+    B, Hq, Lq, D = _dims("q", q, 4)
+    _, Hkv, Lk, _ = _dims("k", k, 4)
+    _expect(("q", q, (B, Hq, Lq, D), torch.bfloat16), ("k", k, (B, Hkv, Lk, D), torch.bfloat16),
+            ("v", v, (B, Hkv, Lk, D), torch.bfloat16), ("lam", lam, (Hq // 2,), torch.float32))
+    _device_only([("q", q), ("k", k), ("v", v), ("lam", lam)])
     out = torch.empty((B, Hq // 2, Lq, D), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, Hq // 2, 2, Lq), dtype=torch.float32, device=q.device)
     o_maps = torch.empty((B, Hq // 2, 2, Lq, D), dtype=q.dtype, device=q.device)
@@ -270,8 +324,14 @@ def fwd_v2_train(q, k, v, lam, causal=True):
 def bwd_v2(q, k, v, lam, dout, lse, o_maps, causal=True, workspace=None):
     """Gradients of the V2 forward: (dq, dk, dv, dlam) given dout [B,Hq/2,Lq,D] and the
     training forward's lse and o_maps.  bf16 gradients, f32 dlam.  Device tensors."""
-    B, Hq, Lq, D = q.shape
-    Hkv, Lk = k.shape[1], k.shape[2]
+    B, Hq, Lq, D = _dims("q", q, 4)
+    _, Hkv, Lk, _ = _dims("k", k, 4)
+    bf, f32, Hp = torch.bfloat16, torch.float32, Hq // 2
+    _expect(("q", q, (B, Hq, Lq, D), bf), ("k", k, (B, Hkv, Lk, D), bf), ("v", v, (B, Hkv, Lk, D), bf),
+            ("lam", lam, (Hp,), f32), ("dout", dout, (B, Hp, Lq, D), bf), ("lse", lse, (B, Hp, 2, Lq), f32),
+            ("o_maps", o_maps, (B, Hp, 2, Lq, D), bf))
+    _device_only([("q", q), ("k", k), ("v", v), ("lam", lam), ("dout", dout), ("lse", lse), ("o_maps", o_maps),
+                  ("workspace", workspace)])
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dlam = torch.empty(Hq // 2, dtype=torch.float32, device=q.device)
     need = int(load().diffattn_bwd_v2_workspace_size(B, Hq, Lq))
@@ -286,8 +346,13 @@ def fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5):
     """V1 forward (bf16, d = 64, dv = 128) that also returns what bwd_v1 needs:
     (out [B,H,Lq,128], lse f32 [B,H,2,Lq], o_maps [B,H,2,Lq,128], rstd f32 [B,H,Lq]
     or None without RMSNorm).  Device tensors."""
-    B, H, Lq, d = q1.shape
-    Hkv, Lk, dv = k1.shape[1], k1.shape[2], v.shape[3]
+    B, H, Lq, d = _dims("q1", q1, 4)
+    _, Hkv, Lk, _ = _dims("k1", k1, 4)
+    dv = _dims("v", v, 4)[3]
+    bf = torch.bfloat16
+    _expect(("q1", q1, (B, H, Lq, d), bf), ("q2", q2, (B, H, Lq, d), bf), ("k1", k1, (B, Hkv, Lk, d), bf),
+            ("k2", k2, (B, Hkv, Lk, d), bf), ("v", v, (B, Hkv, Lk, dv), bf), ("lam", lam, (H,), torch.float32))
+    _device_only([("q1", q1), ("k1", k1), ("q2", q2), ("k2", k2), ("v", v), ("lam", lam)])
     out = torch.empty((B, H, Lq, dv), dtype=q1.dtype, device=q1.device)
     lse = torch.empty((B, H, 2, Lq), dtype=torch.float32, device=q1.device)
     o_maps = torch.empty((B, H, 2, Lq, dv), dtype=q1.dtype, device=q1.device)
@@ -301,8 +366,18 @@ def fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5):
 def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, causal=True, rmsnorm=False, workspace=None):
     """Gradients of the V1 forward: (dq1, dk1, dq2, dk2, dv, dlam) given dout [B,H,Lq,128]
     and fwd_v1_train's outputs.  bf16 gradients, f32 dlam.  Device tensors."""
-    B, H, Lq, d = q1.shape
-    Hkv, Lk, dvw = k1.shape[1], k1.shape[2], v.shape[3]
+    B, H, Lq, d = _dims("q1", q1, 4)
+    _, Hkv, Lk, _ = _dims("k1", k1, 4)
+    dvw = _dims("v", v, 4)[3]
+    bf, f32 = torch.bfloat16, torch.float32
+    _expect(("q1", q1, (B, H, Lq, d), bf), ("q2", q2, (B, H, Lq, d), bf), ("k1", k1, (B, Hkv, Lk, d), bf),
+            ("k2", k2, (B, Hkv, Lk, d), bf), ("v", v, (B, Hkv, Lk, dvw), bf), ("lam", lam, (H,), f32),
+            ("dout", dout, (B, H, Lq, dvw), bf), ("lse", lse, (B, H, 2, Lq), f32),
+            ("o_maps", o_maps, (B, H, 2, Lq, dvw), bf))
+    if rmsnorm:
+        _expect(("out", out, (B, H, Lq, dvw), bf), ("rstd", rstd, (B, H, Lq), f32))
+    _device_only([("q1", q1), ("k1", k1), ("q2", q2), ("k2", k2), ("v", v), ("lam", lam), ("dout", dout),
+                  ("out", out), ("lse", lse), ("o_maps", o_maps), ("rstd", rstd), ("workspace", workspace)])
     dq1, dq2 = torch.empty_like(q1), torch.empty_like(q2)
     dk1, dk2, dv = torch.empty_like(k1), torch.empty_like(k2), torch.empty_like(v)
     dlam = torch.empty(H, dtype=torch.float32, device=q1.device)
@@ -317,7 +392,11 @@ def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, causal=Tru
 
 def lambda_backward(lq1, lk1, lq2, lk2, dlam):
     """Gradients of the four lambda parameter vectors ([H, dim] f32) given dlam [H]."""
-    H, dim = lq1.shape
+    H, dim = _dims("lq1", lq1, 2)
+    f32 = torch.float32
+    _expect(("lq1", lq1, (H, dim), f32), ("lk1", lk1, (H, dim), f32), ("lq2", lq2, (H, dim), f32),
+            ("lk2", lk2, (H, dim), f32), ("dlam", dlam, (H,), f32))
+    _device_only([("lq1", lq1), ("lk1", lk1), ("lq2", lq2), ("lk2", lk2), ("dlam", dlam)])
     outs = [torch.empty_like(lq1) for _ in range(4)]
     _check(load().diffattn_lambda_backward(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), _ptr(dlam), H, dim,
                                            *[_ptr(t) for t in outs], _stream()))
@@ -342,6 +421,12 @@ def _workspace(nbytes, device):
 
 def decode_v2(q, kc, vc, lam, out=None, workspace=None):
     """Single-token V2 decode: q [B,Hq,D]; kc,vc [B,Hkv,T,D]; lam [Hq/2] -> [B,Hq/2,D]."""
+    B, Hq, D = _dims("q", q, 3)
+    _, Hkv, T, _ = _dims("kc", kc, 4)
+    _expect(("kc", kc, (B, Hkv, T, D), q.dtype), ("vc", vc, (B, Hkv, T, D), q.dtype),
+            ("lam", lam, (Hq // 2,), torch.float32))
+    if out is not None:
+        _expect(("out", out, (B, Hq // 2, D), q.dtype))
     host, (q, kc, vc, lam) = _prep([q, kc, vc, lam])
     B, Hq, D = q.shape
     Hkv, T = kc.shape[1], kc.shape[2]
@@ -362,6 +447,14 @@ def decode_paged_workspace_size(B: int, Hkv: int) -> int:
 def decode_v2_paged(q, k_pages, v_pages, block_table, seq_lens, lam, out=None, workspace=None):
     """Paged, variable-length V2 decode: q [B,Hq,128]; k_pages, v_pages [num_pages, page_size, Hkv, 128];
     block_table int32 [B, max_pages]; seq_lens int32 [B]; lam [Hq/2] -> [B, Hq/2, 128]."""
+    B, Hq, D = _dims("q", q, 3)
+    P, ps, Hkv, _ = _dims("k_pages", k_pages, 4)
+    M = _dims("block_table", block_table, 2)[1]
+    _expect(("k_pages", k_pages, (P, ps, Hkv, D), q.dtype), ("v_pages", v_pages, (P, ps, Hkv, D), q.dtype),
+            ("block_table", block_table, (B, M), torch.int32), ("seq_lens", seq_lens, (B,), torch.int32),
+            ("lam", lam, (Hq // 2,), torch.float32))
+    if out is not None:
+        _expect(("out", out, (B, Hq // 2, D), q.dtype))
     host, (q, k_pages, v_pages, block_table, seq_lens, lam) = _prep([q, k_pages, v_pages, block_table, seq_lens,
                                                                       lam])
     B, Hq, D = q.shape
@@ -382,6 +475,14 @@ def decode_v2_paged(q, k_pages, v_pages, block_table, seq_lens, lam, out=None, w
 
 def decode_v1(q1, k1, q2, k2, v, lam, fused=True, out=None, workspace=None):
     """Single-token V1-layout decode: q1,q2 [B,H,d]; k1,k2 [B,Hkv,T,d]; v [B,Hkv,T,dv] -> [B,H,dv]."""
+    B, H, d = _dims("q1", q1, 3)
+    _, Hkv, T, _ = _dims("k1", k1, 4)
+    dv = _dims("v", v, 4)[3]
+    _expect(("q2", q2, (B, H, d), q1.dtype), ("k1", k1, (B, Hkv, T, d), q1.dtype),
+            ("k2", k2, (B, Hkv, T, d), q1.dtype), ("v", v, (B, Hkv, T, dv), q1.dtype),
+            ("lam", lam, (H,), torch.float32))
+    if out is not None:
+        _expect(("out", out, (B, H, dv), q1.dtype))
     host, (q1, k1, q2, k2, v, lam) = _prep([q1, k1, q2, k2, v, lam])
     B, H, d = q1.shape
     Hkv, T, dv = k1.shape[1], k1.shape[2], v.shape[3]
