@@ -411,7 +411,10 @@ _ws_cache = {}
 
 
 def _workspace(nbytes, device):
-    key = (device.index, )
+    """Scratch of at least nbytes for a call on the current stream of ``device``:
+    one buffer per (device, stream).  Calls on one stream run in order and can
+    share it; calls on two streams may overlap, so each stream has its own."""
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
