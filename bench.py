@@ -135,6 +135,23 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workloads
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of the current kernel on a smaller batch of the same workload;
+# traffic grows with the batch (independent (batch, head) units), so a full
+# launch is scaled by B / captured B.  None where no capture of the current
+# kernel exists.
+MEASURED_TRAFFIC = {
+    "v2_prefill": (168.1e6 + 44.1e6, 1),       # prefill_kernel<128, false>, B1
+    "v2_decode": (537.0e6 + 4.1e6, 2),         # decode_split_kernel<2, false>, B2
+    "v2_decode_paged": (537.0e6 + 4.2e6, 2),   # decode_split_kernel<2, true>, B2, 16-token pages
+}
+
+
+def measured_traffic(name, B):
+    t = MEASURED_TRAFFIC.get(name)
+    return None if t is None else t[0] * B / t[1]
+
+
 class Prefill:
     def __init__(self, w, device):
         self.w = w
@@ -476,25 +493,29 @@ def e2e_measure(r, steps):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
-def roofline(r, kern_ms, peaks, power_capped=False):
+def roofline(r, kern_ms, peaks, power_capped=False, name=None):
     """Achieved work rate of the step's dominant kernel against the measured peak.
 
     A tensor-bound kernel is compared with the cuBLAS bf16 figure measured in the
     same regime: the sustained (power-capped) one when the clock record of the
     timed region shows sw_power_cap, else the burst one; the fraction of the
-    burst figure is reported beside it either way."""
+    burst figure is reported beside it either way.  traffic: the DRAM bytes of
+    one launch from the kernel's ncu capture, scaled to this batch (None
+    without a capture of the current kernel)."""
     work, unit = r.work()
+    w = getattr(r, "w", None)
+    traffic = measured_traffic(name, w.B) if (name is not None and w is not None) else None
     if unit == "TFLOP/s":
         ach = work / (kern_ms / 1e3)
         sustained = power_capped and peaks.get("bf16_tflops_sustained")
         peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
         kind = "sustained (power-capped)" if sustained else "burst"
         return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                "traffic": None, "peak_kind": f"{peaks['source']} {kind} cuBLAS bf16",
+                "traffic": traffic, "peak_kind": f"{peaks['source']} {kind} cuBLAS bf16",
                 "frac_of_burst": ach / peaks["bf16_tflops"], "kernel_ms": kern_ms}
     ach = work / (kern_ms / 1e3)
     peak = peaks["hbm_gbs"]
-    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": None,
+    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
             "peak_kind": f"{peaks['source']} HBM copy", "kernel_ms": kern_ms}
 
 
@@ -683,7 +704,7 @@ def main():
     value = aggregate(work, world, ms)
     clocks = clk.summary()
     capped = "sw_power_cap" in clocks["reasons"]
-    rf = roofline(r, kern_ms, peaks, capped)
+    rf = roofline(r, kern_ms, peaks, capped, args.workload)
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
@@ -696,7 +717,7 @@ def main():
             t2, k2 = time_runner(r2, max(3, args.steps // 2), args.warmup, False)
             wk, un = r2.work()
             secondary[name] = {"value": wk / (t2 / max(3, args.steps // 2) / 1e3), "unit": un,
-                               "ms_per_step": t2 / max(3, args.steps // 2), "roofline": roofline(r2, k2, peaks, capped),
+                               "ms_per_step": t2 / max(3, args.steps // 2), "roofline": roofline(r2, k2, peaks, capped, name),
                                "config": describe(name)}
             del r2
             torch.cuda.empty_cache()
