@@ -366,10 +366,55 @@ class SnrSweep:
         raise NotImplementedError("the sweep is timed on device tensors only")
 
 
+def lowrank_flops(B, H, L, **_) -> float:
+    """Executed-min FLOP of the low-rank forward's attention: one QK^T and one
+    PV product per head over the causal pairs (the scan of N V adds about
+    6 r dv FLOP per row and key-step, under 1 % here, and is not counted)."""
+    nc = causal_pairs(L, L, True)
+    return nc * (2 * 128 + 2 * 128) * H * B
+
+
+class LowRank:
+    """The fixed low-rank substitute for A2: one step is lambda, then
+    out = A1 V - lambda N V (single-map prefill, then the N V scan)."""
+
+    def __init__(self, device, shape=None):
+        self.shape = dict(inputs.LOWRANK_SHAPE if shape is None else shape)
+        sh = self.shape
+        self.x = inputs.lowrank_inputs(**sh, device=device)
+        gen = torch.Generator(device=device).manual_seed(1012)
+        self.lp = tuple(torch.randn(sh["H"], 128, generator=gen, device=device) * 0.1 for _ in range(4))
+        self.init = da.lambda_init(24)
+        self.lam = torch.empty(sh["H"], dtype=torch.float32, device=device)
+        self.out = torch.empty((sh["B"], sh["H"], sh["L"], 128), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(int(da.load().diffattn_fwd_lowrank_workspace_size(sh["B"], sh["H"], sh["L"], sh["L"],
+                                                                                sh["r"], 1)),
+                              dtype=torch.uint8, device=device)
+        self.launches_per_step = 5   # lambda, single-map prefill, chunk sums, prefix, emit
+
+    def step(self, ev=None):
+        x = self.x
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        if ev is not None:
+            ev[0].record()
+        da.fwd_lowrank(x["q"], x["k"], x["v"], x["F"], x["G"], self.lam, causal=True, out=self.out,
+                       workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        return lowrank_flops(**self.shape) / 1e12, "TFLOP/s"
+
+    def host_call(self, host):
+        raise NotImplementedError("the low-rank forward is timed on device tensors only")
+
+
 def workload_work(name):
     """(algorithmic work of one step, unit) of a bench workload."""
     if name == "snr_sweep":
         return sweep_bytes() / 1e9, "GB/s"
+    if name == "lowrank_prefill":
+        return lowrank_flops(**inputs.LOWRANK_SHAPE) / 1e12, "TFLOP/s"
     w = inputs.WORKLOADS[base_workload(name)]
     if name.endswith("_backward"):
         return backward_flops(w) / 1e12, "TFLOP/s"
@@ -387,6 +432,8 @@ def base_workload(name):
 def make_runner(name, device):
     if name == "snr_sweep":
         return SnrSweep(device)
+    if name == "lowrank_prefill":
+        return LowRank(device)
     if name.endswith("_backward"):
         return Backward(inputs.WORKLOADS[base_workload(name)], device)
     if name == "v2_decode_paged":
@@ -398,6 +445,13 @@ def make_runner(name, device):
 
 
 def describe(name):
+    if name == "lowrank_prefill":
+        sh = inputs.LOWRANK_SHAPE
+        return {"workload": name, "layout": "one Q head per output head", "B": sh["B"], "heads": sh["H"],
+                "kv_heads": sh["Hkv"], "Lq": sh["L"], "Lk": sh["L"], "d": 128, "dv": 128, "causal": True,
+                "rank": sh["r"], "layer": 24,
+                "mode": "A1 V - lambda N V, N fixed from positional factors F, G ~ U(0,1)",
+                "l2": "inputs larger than L2 (126 MB): no flush between steps"}
     if name == "snr_sweep":
         return {"workload": name, "layout": "v1_decode", "instances": inputs.SWEEP_INSTANCES,
                 "Lk": list(inputs.SWEEP_LENGTHS), "d": 64, "dv": 128, "lambda": [0.0, 0.5],
@@ -520,6 +574,36 @@ def roofline(r, kern_ms, peaks, power_capped=False, name=None):
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
+def cpu_oracle_lowrank(cores, budget_s):
+    """The oracle's low-rank head on whole (batch, head) slices of the workload."""
+    from oracle import lowrank as olr
+    sh = inputs.LOWRANK_SHAPE
+    x = _lowrank_host_inputs()
+    grp = sh["H"] // sh["Hkv"]
+    per_slice = lowrank_flops(**sh) / (sh["B"] * sh["H"]) / 1e12
+    done, t_total, n = 0.0, 0.0, 0
+    for h in range(sh["H"]):
+        for b in range(sh["B"]):
+            t0 = time.perf_counter()
+            olr.lowrank_head(x["q"][b, h], x["k"][b, h // grp], x["v"][b, h // grp], x["F"][h].numpy(),
+                             x["G"][h].numpy(), 0.5, True)
+            t_total += time.perf_counter() - t0
+            done += per_slice
+            n += 1
+            if t_total >= budget_s:
+                break
+        if t_total >= budget_s:
+            break
+    return {"value": done / t_total, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {sh['B'] * sh['H']} (batch, head) slices, all {sh['L']} rows, fp64 NumPy",
+            "seconds": t_total}
+
+
+@functools.lru_cache(maxsize=1)
+def _lowrank_host_inputs():
+    return inputs.lowrank_inputs(**inputs.LOWRANK_SHAPE)
+
+
 @functools.lru_cache(maxsize=1)
 def _sweep_host_inputs():
     """The sweep's inputs on the host, drawn once per process (about 12 s)."""
@@ -562,6 +646,8 @@ def cpu_oracle_run(name, budget_s=12.0):
         cores = len(os.sched_getaffinity(0))
     if name == "snr_sweep":
         return cpu_oracle_sweep(cores, budget_s)
+    if name == "lowrank_prefill":
+        return cpu_oracle_lowrank(cores, budget_s)
     paged, backward = name == "v2_decode_paged", name.endswith("_backward")
     w = inputs.WORKLOADS[base_workload(name)]
     x = inputs.make(w, device="cpu") if w.layout in ("v1", "v2") else None
@@ -643,7 +729,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="v2_prefill",
                     choices=["v2_prefill", "v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged",
-                             "v1_decode", "v1_decode_unfused", "snr_sweep"])
+                             "v1_decode", "v1_decode_unfused", "snr_sweep", "lowrank_prefill"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
@@ -651,7 +737,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size of the workload (smaller profiling cases)")
     args = ap.parse_args()
-    if args.batch is not None and args.workload != "snr_sweep":
+    if args.batch is not None and args.workload not in ("snr_sweep", "lowrank_prefill"):
         base = base_workload(args.workload)
         inputs.WORKLOADS[base] = inputs.with_shape(inputs.WORKLOADS[base], B=args.batch)
 

@@ -33,7 +33,8 @@ EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffa
            "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc",
            "diffattn_decode_paged_workspace_size", "diffattn_decode_v2_paged", "diffattn_fwd_v2_train",
            "diffattn_bwd_v2_workspace_size", "diffattn_bwd_v2", "diffattn_lambda_backward",
-           "diffattn_fwd_v1_train", "diffattn_bwd_v1_workspace_size", "diffattn_bwd_v1"]
+           "diffattn_fwd_v1_train", "diffattn_bwd_v1_workspace_size", "diffattn_bwd_v1",
+           "diffattn_fwd_lowrank_workspace_size", "diffattn_fwd_lowrank"]
 
 _lib = None
 
@@ -76,6 +77,8 @@ def load():
         "diffattn_fwd_v1_train": (I, [P] * 10 + [I] * 10 + [F, P]),
         "diffattn_bwd_v1_workspace_size": (Z, [I] * 6),
         "diffattn_bwd_v1": (I, [P] * 17 + [I] * 10 + [P, Z, P]),
+        "diffattn_fwd_lowrank_workspace_size": (Z, [I] * 6),
+        "diffattn_fwd_lowrank": (I, [P] * 7 + [I] * 9 + [P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -388,6 +391,31 @@ def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, causal=Tru
                                   _ptr(dk2), _ptr(dv), _ptr(dlam), _dtype_code(q1), B, H, Hkv, Lq, Lk, d, dvw,
                                   int(causal), int(rmsnorm), _ptr(ws), ws.numel() * ws.element_size(), _stream()))
     return dq1, dk1, dq2, dk2, dv, dlam
+
+
+def fwd_lowrank(q, k, v, F, G, lam, causal=True, out=None, workspace=None):
+    """Differential attention with a fixed low-rank map in place of A2:
+    out = softmax(Q K^T / sqrt(128)) V - lam N V, N[i, j] = f_i.g_j / sum over
+    visible j' of f_i.g_j'.  q [B,H,Lq,128], k, v [B,Hkv,Lk,128] bf16; F [H,Lq,r],
+    G [H,Lk,r] f32 >= 0; lam f32 [H] -> [B,H,Lq,128].  Device tensors."""
+    B, H, Lq, D = _dims("q", q, 4)
+    _, Hkv, Lk, _ = _dims("k", k, 4)
+    r = _dims("F", F, 3)[2]
+    bf, f32 = torch.bfloat16, torch.float32
+    _expect(("q", q, (B, H, Lq, D), bf), ("k", k, (B, Hkv, Lk, D), bf), ("v", v, (B, Hkv, Lk, D), bf),
+            ("F", F, (H, Lq, r), f32), ("G", G, (H, Lk, r), f32), ("lam", lam, (H,), f32))
+    if out is not None:
+        _expect(("out", out, (B, H, Lq, D), bf))
+    _device_only([("q", q), ("k", k), ("v", v), ("F", F), ("G", G), ("lam", lam), ("out", out),
+                  ("workspace", workspace)])
+    if out is None:
+        out = torch.empty((B, H, Lq, D), dtype=bf, device=q.device)
+    need = int(load().diffattn_fwd_lowrank_workspace_size(B, H, Lq, Lk, r, int(causal)))
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    _check(load().diffattn_fwd_lowrank(_ptr(q), _ptr(k), _ptr(v), _ptr(F), _ptr(G), _ptr(lam), _ptr(out), BF16,
+                                       B, H, Hkv, Lq, Lk, D, r, int(causal), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream()))
+    return out
 
 
 def lambda_backward(lq1, lk1, lq2, lk2, dlam):

@@ -21,6 +21,7 @@
 #include "prefill_sm100.cuh"
 #include "backward_sm100.cuh"
 #include "v1_adapter.cuh"
+#include "lowrank.cuh"
 
 using namespace da;
 
@@ -434,6 +435,29 @@ int launch_backward_v1(const void* q1, const void* k1, const void* q2, const voi
   return ok();
 }
 
+// Low-rank forward workspace: the zero lambda of the single-map prefill
+// [H/2], its by-product output [B, H/2, Lq, 128] bf16 and log-sum-exp
+// [B, H/2, 2, Lq], the per-head single-map outputs A1 V [B, H, Lq, 128] bf16,
+// and the chunk sums [B*H, nc+1, r, 128] and [B*H, nc+1, r] f32.
+struct LowrankLayout {
+  size_t lam, pre, lse, a1v, tot, ztot, total;
+  int nc;
+};
+LowrankLayout lowrank_layout(int B, int H, int Lq, int Lk, int r, int causal) {
+  LowrankLayout l;
+  const long long rows = causal ? Lq : Lk;
+  l.nc = (int)((rows + LR_C - 1) / LR_C);
+  const size_t BH = (size_t)B * H, Hp = (size_t)H / 2;
+  l.lam = 0;
+  l.pre = align256(Hp * 4);
+  l.lse = l.pre + align256((size_t)B * Hp * Lq * 256);
+  l.a1v = l.lse + align256((size_t)B * Hp * 2 * Lq * 4);
+  l.tot = l.a1v + align256(BH * Lq * 256);
+  l.ztot = l.tot + align256(BH * (l.nc + 1) * r * LR_DV * 4);
+  l.total = l.ztot + align256(BH * (l.nc + 1) * r * 4);
+  return l;
+}
+
 // Paged decode workspace: the block prefix (B+1 ints, padded to 256 bytes),
 // then one partial record per slot CTA + b*Hkv + g, i.e. grid + B*Hkv records.
 int paged_grid(const DeviceInfo* dev) { return dev->sms * kDecCtasPerSm; }
@@ -730,6 +754,66 @@ int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* 
     if (p && !aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
   return launch_backward_v1(q1, k1, q2, k2, v, lambda, dout, out, lse, o_maps, rstd, dq1, dk1, dq2, dk2, dv, dlambda,
                             B, H, Hkv, Lq, Lk, causal, rms, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t diffattn_fwd_lowrank_workspace_size(int B, int H, int Lq, int Lk, int r, int causal) {
+  if (B < 0 || H < 2 || H % 2 || Lq < 0 || Lk < 0 || r < 1 || r > LR_RMAX) return 0;
+  return lowrank_layout(B, H, Lq, Lk, r, causal ? 1 : 0).total;
+}
+
+int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const float* F, const float* G,
+                         const float* lambda, void* out, diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk,
+                         int D, int r, int causal, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 0 || H < 2 || Hkv < 1 || Lq < 0 || Lk < 0 || D < 1 || r < 1)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d Lq=%d Lk=%d D=%d r=%d)", B, H, Hkv, Lq, Lk, D,
+                r);
+  if (H % Hkv || (H / Hkv) % 2)
+    return fail(DIFFATTN_ERR_INVALID_ARG, "need H/Hkv even: heads run in pairs over a KV head (H=%d Hkv=%d)", H, Hkv);
+  if (dtype != DIFFATTN_BF16) return fail(DIFFATTN_ERR_UNSUPPORTED, "the low-rank forward takes bf16 only");
+  if (D != 128) return fail(DIFFATTN_ERR_UNSUPPORTED, "the low-rank forward needs D == 128 (got %d)", D);
+  if (r > LR_RMAX) return fail(DIFFATTN_ERR_UNSUPPORTED, "rank r=%d above %d", r, LR_RMAX);
+  if ((long long)B * H > 65535) return fail(DIFFATTN_ERR_UNSUPPORTED, "B*H=%lld above 65535", (long long)B * H);
+  if (B == 0 || Lq == 0) return ok();
+  if (!q || !F || !lambda || !out || (Lk > 0 && (!k || !v || !G))) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
+  if (Lk == 0) k = v = q;   // never read: no key is visible
+  if (int e = check_bf16_ptrs({q, k, v, out})) return e;
+  const LowrankLayout L = lowrank_layout(B, H, Lq, Lk, r, causal ? 1 : 0);
+  if (ws == nullptr || ws_bytes < L.total)
+    return fail(DIFFATTN_ERR_WORKSPACE, "low-rank workspace %zu B < required %zu B", ws_bytes, L.total);
+  if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  DeviceInfo* dev = nullptr;
+  if (int e = device_setup(&dev)) return e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* zero_lam = reinterpret_cast<float*>(w + L.lam);
+  CUDA_TRY(cudaMemsetAsync(zero_lam, 0, sizeof(float) * (size_t)(H / 2), s));
+  // A1 V for every head: the training prefill with heads (2j, 2j+1) as a pair
+  // writes both maps' normalised outputs, [B, H/2, 2, Lq, 128] = [B, H, Lq, 128].
+  if (int e = launch_prefill(q, q, k, k, v, zero_lam, w + L.pre, B, H / 2, H, Hkv, Lq, Lk, 128, false, causal, 0,
+                             0.f, s, reinterpret_cast<float*>(w + L.lse), w + L.a1v))
+    return e;
+  LowrankArgs a{};
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.F = F; a.G = G; a.lambda = lambda;
+  a.a1v = reinterpret_cast<const __nv_bfloat16*>(w + L.a1v);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.tot = reinterpret_cast<float*>(w + L.tot);
+  a.ztot = reinterpret_cast<float*>(w + L.ztot);
+  a.B = B; a.H = H; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk; a.r = r; a.causal = causal ? 1 : 0;
+  a.nc = L.nc;
+  const unsigned BH = (unsigned)(B * H);
+  if (L.nc > 0 && Lk > 0) {
+    lr_totals_kernel<<<dim3((unsigned)L.nc, BH), LR_DV, 0, s>>>(a);
+    CUDA_TRY(cudaGetLastError());
+  } else if (L.nc > 0) {   // no key: every chunk sum is zero
+    CUDA_TRY(cudaMemsetAsync(a.tot, 0, sizeof(float) * (size_t)BH * (L.nc + 1) * r * LR_DV, s));
+    CUDA_TRY(cudaMemsetAsync(a.ztot, 0, sizeof(float) * (size_t)BH * (L.nc + 1) * r, s));
+  }
+  lr_prefix_kernel<<<BH, LR_DV, 0, s>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  lr_emit_kernel<<<dim3((unsigned)((Lq + LR_C - 1) / LR_C), BH), LR_DV, 0, s>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return ok();
 }
 
 int diffattn_lambda_backward(const float* lq1, const float* lk1, const float* lq2, const float* lk2,

@@ -21,6 +21,10 @@ Workloads (shapes, value distributions):
                N(0,1)/sqrt(128), layer 24.
   v1_decode    the same decode shape in the V1 layout: 32 heads over 8 KV
                heads, Q1/Q2/K1/K2 width 64, V width 128.
+  lowrank      (lowrank_inputs) the fixed low-rank substitute for A2 on the
+               V2 prefill's attention shape with one Q head per output head:
+               B2 H32 Hkv8 N8192 D128 causal, N(0,1)/sqrt(128); positional
+               factors F [H, N, r], G [H, N, r] ~ U(0, 1), r = 16.
   noise sweep  (noise_sweep / sweep_prefix) the noise_probe construction at
                context lengths 1k..256k keys (tutorial exercise 1), in bf16 for
                the V1 decode layout: 64 instances, each a query q ~ N(0,1) in
@@ -222,3 +226,19 @@ def sweep_prefix(x, N: int):
     for name in ("k1", "k2", "v"):
         out[name] = x[name][:, :, :N].contiguous()
     return out
+
+
+LOWRANK_SHAPE = dict(B=2, H=32, Hkv=8, L=8192, r=16)
+
+
+def lowrank_inputs(B=2, H=32, Hkv=8, L=8192, r=16, seed=1011, device="cpu"):
+    """q [B, H, L, 128], k, v [B, Hkv, L, 128] bf16 ~ N(0,1)/sqrt(128); F, G
+    [H, L, r] fp32 ~ U(0, 1)."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    s = 1.0 / math.sqrt(128)
+    q = _randn(gen, (B, H, L, 128), s, torch.bfloat16, device)
+    k = _randn(gen, (B, Hkv, L, 128), s, torch.bfloat16, device)
+    v = _randn(gen, (B, Hkv, L, 128), s, torch.bfloat16, device)
+    F = torch.rand((H, L, r), generator=gen, device=device, dtype=torch.float32)
+    G = torch.rand((H, L, r), generator=gen, device=device, dtype=torch.float32)
+    return {"q": q, "k": k, "v": v, "F": F, "G": G}

@@ -258,6 +258,31 @@ DIFFATTN_API int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2,
                                  int Lk, int d, int dv_width, int causal, int rmsnorm, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* Workspace, in bytes, for diffattn_fwd_lowrank.  0 for invalid sizes. */
+DIFFATTN_API size_t diffattn_fwd_lowrank_workspace_size(int B, int H, int Lq, int Lk, int r, int causal);
+
+/* Differential attention with a fixed low-rank map N in place of A2 (paper
+ * note "Understanding Differential Transformer Unchains Pretrained
+ * Self-Attentions", sections 基于分析的改进建议 and 亮点与洞察; the note gives
+ * the idea, the form below is this library's reading):
+ *   N[i, j] = f_i.g_j / Σ_{j' visible from i} f_i.g_j'  on visible keys, 0 elsewhere
+ *             (a row with zero mass is 0)
+ *   out     = softmax(Q K^T / sqrt(D)) V - λ N V        per head
+ *   q      : bf16 [B, H, Lq, 128]       k, v : bf16 [B, Hkv, Lk, 128]  (device)
+ *   F      : f32 [H, Lq, r], G : f32 [H, Lk, r], non-negative          (device)
+ *   lambda : f32 [H];  out : bf16 [B, H, Lq, 128]                      (device)
+ *   ws     : diffattn_fwd_lowrank_workspace_size bytes, 16-byte aligned,
+ *            owned by the caller.
+ * Head h reads KV head h / (H / Hkv); H / Hkv must be even (heads are
+ * computed in pairs that share a KV head).  Requires bf16, D == 128,
+ * 1 <= r <= 16 and B * H <= 65535.  The causal mask is the library's
+ * bottom-right one.  Negative factors are not checked; they give a result
+ * that is not a map. */
+DIFFATTN_API int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const float* F, const float* G,
+                                      const float* lambda, void* out, diffattn_dtype dtype, int B, int H, int Hkv,
+                                      int Lq, int Lk, int D, int r, int causal, void* ws, size_t ws_bytes,
+                                      void* stream);
+
 /* Gradients of λ = exp(lq1.lk1) - exp(lq2.lk2) + λ_init with respect to its
  * parameter vectors ([heads, dim] f32 each), given dlambda [heads]: fp64
  * inside, f32 out.                                                 (device) */

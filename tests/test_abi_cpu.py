@@ -133,6 +133,21 @@ def test_argument_errors_before_any_device_call(L):
     assert L.diffattn_bwd_v1_workspace_size(1, 3, 2, 8, 8, 0) == 0
     assert L.diffattn_lambda_backward(P, P, P, P, P, 0, 8, P, P, P, P, s) == da.ERR_INVALID_ARG
     assert L.diffattn_lambda_backward(P, P, P, None, P, 2, 8, P, P, P, P, s) == da.ERR_INVALID_ARG
+    # low-rank forward: (q, k, v, F, G, lambda, out, dtype, B, H, Hkv, Lq, Lk, D, r, causal, ws, bytes, s)
+    lrf = lambda *args: L.diffattn_fwd_lowrank(*args)  # noqa: E731
+    p7 = [P] * 7
+    assert lrf(*p7, da.BF16, 1, 6, 2, 8, 8, 128, 4, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG    # H/Hkv odd
+    assert lrf(*p7, da.F32, 1, 4, 2, 8, 8, 128, 4, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+    assert lrf(*p7, da.BF16, 1, 4, 2, 8, 8, 64, 4, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED
+    assert lrf(*p7, da.BF16, 1, 4, 2, 8, 8, 128, 17, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED   # r > 16
+    assert lrf(*p7, da.BF16, 1, 4, 2, 8, 8, 128, 0, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    no_f = [P, P, P, None, P, P, P]
+    assert lrf(*no_f, da.BF16, 1, 4, 2, 8, 8, 128, 4, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    bad_out = [P] * 6 + [Pm]
+    assert lrf(*bad_out, da.BF16, 1, 4, 2, 8, 8, 128, 4, 1, P, 1 << 20, s) == da.ERR_MISALIGNED
+    assert lrf(*p7, da.BF16, 1, 4, 2, 8, 8, 128, 4, 1, P, 16, s) == da.ERR_WORKSPACE
+    w1 = L.diffattn_fwd_lowrank_workspace_size(2, 32, 8192, 8192, 16, 1)
+    assert w1 > 2 * 32 * 8192 * 256 and L.diffattn_fwd_lowrank_workspace_size(2, 32, 8192, 8192, 17, 1) == 0
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch):

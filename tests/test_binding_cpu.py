@@ -89,3 +89,18 @@ def test_training_shapes_and_device():
         da.lambda_backward(*p, z(4, dtype=f32))
     with pytest.raises(ValueError, match="lk2 has shape"):
         da.lambda_backward(p[0], p[1], p[2], z(3, 7, dtype=f32), z(3, dtype=f32))
+
+
+def test_lowrank_shapes_and_device():
+    q, k, lam = z(1, 4, 16, 128), z(1, 2, 20, 128), z(4, dtype=f32)
+    F, G = z(4, 16, 3, dtype=f32), z(4, 20, 3, dtype=f32)
+    with pytest.raises(ValueError, match="G has shape"):
+        da.fwd_lowrank(q, k, k, F, z(4, 19, 3, dtype=f32), lam)
+    with pytest.raises(ValueError, match="F has shape"):
+        da.fwd_lowrank(q, k, k, z(4, 15, 3, dtype=f32), G, lam)
+    with pytest.raises(ValueError, match="lam has shape"):
+        da.fwd_lowrank(q, k, k, F, G, z(2, dtype=f32))
+    with pytest.raises(ValueError, match="v must be"):
+        da.fwd_lowrank(q, k, k.float(), F, G, lam)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        da.fwd_lowrank(q, k, k, F, G, lam)
