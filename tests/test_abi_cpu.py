@@ -26,6 +26,20 @@ def declared_symbols():
     return sorted(set(re.findall(r"\b(diffattn_\w+)\s*\(", text)))
 
 
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])
+def test_header_is_plain_c(lang, std):
+    """The boundary header needs no CUDA, torch or C++ types: it compiles alone
+    as C99 and as C++11, warnings as errors."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    res = subprocess.run([cc, "-fsyntax-only", "-x", lang, f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                          HEADER], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+
+
 def test_header_declares_the_binding_exports():
     assert declared_symbols() == sorted(da.EXPORTS)
 
