@@ -170,3 +170,22 @@ def test_binding_has_no_cpu_fallback(monkeypatch):
     monkeypatch.setattr(da, "LIB_PATH", "/nonexistent/libdiffattn.so")
     with pytest.raises(RuntimeError, match="missing"):
         da.load()
+
+
+def test_plain_c_client_links_and_runs(L, tmp_path):
+    """A C program built against the header and linked to the library (no
+    Python) gets the version, lambda_init, argument errors and workspace sizes."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    exe = str(tmp_path / "abi_c_client")
+    libdir = os.path.dirname(da.LIB_PATH)
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", os.path.join(ROOT, "tests", "host", "abi_c_client.c"),
+                          "-I", os.path.join(ROOT, "include"), "-L", libdir, "-ldiffattn", "-lm", "-o", exe],
+                         capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    env = dict(os.environ, LD_LIBRARY_PATH=libdir + os.pathsep + os.environ.get("LD_LIBRARY_PATH", ""))
+    run = subprocess.run([exe], capture_output=True, text=True, env=env)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stderr)
