@@ -30,7 +30,7 @@ from oracle import backward as bwd
 from oracle import diffattn as orc
 from oracle import lowrank as lr
 
-SETTINGS = settings(max_examples=25, deadline=None)
+SETTINGS = settings(max_examples=25, deadline=None, derandomize=True)   # reproducible runs
 
 
 @st.composite
