@@ -18,7 +18,9 @@ sign error, a crossed map or a broken GQA index breaks at least one of them.
   * with eps = 0 the RMSNorm output does not depend on the scale of V;
   * the key gradient of each map sums to zero over the keys (softmax rows
     are shift invariant), so dK sums to zero in the V2 layout;
-  * the low-rank map is unchanged by positive scalings of its factors' rows."""
+  * the low-rank map is unchanged by positive scalings of F's rows (each
+    row of N is normalised), by one positive scale of G, and by permuting
+    the rank index of both factors together."""
 
 import math
 
