@@ -12,15 +12,14 @@ import numpy as np
 import pytest
 
 from oracle import diffattn as orc
-from oracle import lowrank as lr
+from oracle import lowrank
 
 
 def _rng(seed):
     return np.random.default_rng(seed)
 
 
-@pytest.mark.parametrize("Lq,Lk", [(7, 7), (4, 9)])
-def test_uniform_case_is_the_prefix_mean(Lq, Lk):
+def pin_uniform_case_is_the_prefix_mean(lr, Lq, Lk):
     rng = _rng(Lq + Lk)
     v = rng.standard_normal((Lk, 5))
     N = lr.noise_map(np.ones((Lq, 1)), np.ones((Lk, 1)), Lq, Lk, causal=True)
@@ -33,7 +32,7 @@ def test_uniform_case_is_the_prefix_mean(Lq, Lk):
     assert np.allclose(Nn @ v, np.broadcast_to(v.mean(axis=0), (Lq, 5)), rtol=1e-13, atol=1e-14)
 
 
-def test_softmax_map_tends_to_the_uniform_substitute():
+def pin_softmax_map_tends_to_the_uniform_substitute(lr):
     """As Q2 K2^T -> 0, A2 -> the r = 1, F = G = 1 map, at rate O(eps)."""
     rng = _rng(3)
     L, d = 12, 8
@@ -47,8 +46,7 @@ def test_softmax_map_tends_to_the_uniform_substitute():
     assert errs[1] / errs[0] == pytest.approx(0.1, rel=0.05) and errs[2] / errs[1] == pytest.approx(0.1, rel=0.05)
 
 
-@pytest.mark.parametrize("r", [1, 3])
-def test_unmasked_map_has_rank_r_and_unit_rows(r):
+def pin_unmasked_map_has_rank_r_and_unit_rows(lr, r):
     rng = _rng(10 + r)
     F, G = rng.random((20, r)) + 0.1, rng.random((30, r)) + 0.1
     N = lr.noise_map(F, G, 20, 30, causal=False)
@@ -58,7 +56,7 @@ def test_unmasked_map_has_rank_r_and_unit_rows(r):
     assert np.all(N >= 0)
 
 
-def test_prefix_sum_evaluation_matches_the_map():
+def pin_prefix_sum_evaluation_matches_the_map(lr):
     """(N V)_i = f_i^T S_i / f_i^T z_i with S_i = sum_{j<=i} g_j v_j^T, z_i = sum_{j<=i} g_j:
     the linear-time evaluation of the causal map."""
     rng = _rng(21)
@@ -70,7 +68,7 @@ def test_prefix_sum_evaluation_matches_the_map():
     assert np.allclose(lr.noise_map(F, G, L, L, causal=True) @ v, scan, rtol=1e-12, atol=1e-13)
 
 
-def test_loop_twin_and_rows():
+def pin_loop_twin_and_rows(lr):
     rng = _rng(5)
     Lq, Lk, d, dv, r, lam = 3, 5, 4, 2, 2, 0.7
     q, k, v = rng.standard_normal((Lq, d)), rng.standard_normal((Lk, d)), rng.standard_normal((Lk, dv))
@@ -92,7 +90,7 @@ def test_loop_twin_and_rows():
     assert np.allclose(ones, 1 - lam, rtol=0, atol=1e-14)
 
 
-def test_zero_mass_rows_and_bad_factors():
+def pin_zero_mass_rows_and_bad_factors(lr):
     F = np.array([[0.0], [1.0]])
     N = lr.noise_map(F, np.ones((2, 1)), 2, 2, causal=True)
     assert np.all(N[0] == 0) and np.allclose(N[1], [0.5, 0.5])
@@ -100,7 +98,7 @@ def test_zero_mass_rows_and_bad_factors():
         lr.noise_map(-F, np.ones((2, 1)), 2, 2, causal=True)
 
 
-def test_batched_layout_matches_heads():
+def pin_batched_layout_matches_heads(lr):
     rng = _rng(8)
     B, H, Hkv, L, d, dv, r = 2, 4, 2, 6, 4, 3, 2
     q, k, v = rng.standard_normal((B, H, L, d)), rng.standard_normal((B, Hkv, L, d)), rng.standard_normal((B, Hkv, L, dv))
@@ -110,3 +108,23 @@ def test_batched_layout_matches_heads():
     for b in range(B):
         for h in range(H):
             assert np.array_equal(out[b, h], lr.lowrank_head(q[b, h], k[b, h // 2], v[b, h // 2], F[h], G[h], lam[h], True))
+
+
+# Every pin with its arguments; test_oracle_lowrank_mutations.py runs the same
+# list against planted mistakes.
+PINS = [
+    (pin_uniform_case_is_the_prefix_mean, (7, 7)),
+    (pin_uniform_case_is_the_prefix_mean, (4, 9)),
+    (pin_softmax_map_tends_to_the_uniform_substitute, ()),
+    (pin_unmasked_map_has_rank_r_and_unit_rows, (1,)),
+    (pin_unmasked_map_has_rank_r_and_unit_rows, (3,)),
+    (pin_prefix_sum_evaluation_matches_the_map, ()),
+    (pin_loop_twin_and_rows, ()),
+    (pin_zero_mass_rows_and_bad_factors, ()),
+    (pin_batched_layout_matches_heads, ()),
+]
+
+
+@pytest.mark.parametrize("pin,args", PINS, ids=lambda x: getattr(x, "__name__", str(x)))
+def test_pin(pin, args):
+    pin(lowrank, *args)
