@@ -37,8 +37,7 @@ def _fd(f, x, eps=1e-6):
     return g
 
 
-@pytest.mark.parametrize("causal,Lq,Lk", [(True, 5, 5), (False, 4, 6), (True, 3, 6)])
-def test_v2_gradients_match_finite_differences(causal, Lq, Lk):
+def pin_v2_finite_differences(b, causal, Lq, Lk):
     rng = np.random.default_rng(11 + Lq + Lk)
     q = _rand((1, 4, Lq, 3), rng)
     k = _rand((1, 1, Lk, 3), rng)
@@ -46,14 +45,13 @@ def test_v2_gradients_match_finite_differences(causal, Lq, Lk):
     lam = np.array([0.7, -0.2])
     dout = _rand((1, 2, Lq, 3), rng)
     loss = lambda: float(np.sum(dout * orc.diffattn_v2(q, k, v, lam, causal=causal)))  # noqa: E731
-    dq, dk, dv, dlam = bwd.diffattn_v2_backward(q, k, v, lam, dout, causal=causal)
+    dq, dk, dv, dlam = b.diffattn_v2_backward(q, k, v, lam, dout, causal=causal)
     for got, x in ((dq, q), (dk, k), (dv, v), (dlam, lam)):
         want = _fd(loss, x)
         assert np.allclose(got, want, rtol=1e-6, atol=1e-8)
 
 
-@pytest.mark.parametrize("rms", [False, True])
-def test_v1_gradients_match_finite_differences(rms):
+def pin_v1_finite_differences(b, rms):
     rng = np.random.default_rng(23 + rms)
     q1, q2 = _rand((2, 2, 4, 3), rng), _rand((2, 2, 4, 3), rng)
     k1, k2 = _rand((2, 1, 4, 3), rng), _rand((2, 1, 4, 3), rng)
@@ -62,12 +60,12 @@ def test_v1_gradients_match_finite_differences(rms):
     dout = _rand((2, 2, 4, 5), rng)
     loss = lambda: float(np.sum(dout * orc.diffattn_v1(q1, k1, q2, k2, v, lam, causal=True,  # noqa: E731
                                                          rms=rms, eps=1e-5)))
-    grads = bwd.diffattn_v1_backward(q1, k1, q2, k2, v, lam, dout, causal=True, rms=rms, eps=1e-5)
+    grads = b.diffattn_v1_backward(q1, k1, q2, k2, v, lam, dout, causal=True, rms=rms, eps=1e-5)
     for got, x in zip(grads, (q1, k1, q2, k2, v, lam)):
         assert np.allclose(got, _fd(loss, x), rtol=1e-6, atol=1e-8)
 
 
-def test_lambda_parameter_gradients_match_finite_differences():
+def pin_lambda_parameters(b):
     rng = np.random.default_rng(5)
     p = [_rand((3, 4), rng, 0.3) for _ in range(4)]
     dlam = np.array([0.5, -1.5, 2.0])
@@ -78,7 +76,7 @@ def test_lambda_parameter_gradients_match_finite_differences():
         return a - b + 0.2
 
     loss = lambda: float(np.sum(dlam * lam64()))  # noqa: E731
-    for got, x in zip(bwd.lambda_backward(*p, dlam), p):
+    for got, x in zip(b.lambda_backward(*p, dlam), p):
         assert np.allclose(got, _fd(loss, x), rtol=1e-7, atol=1e-10)
 
 
@@ -102,7 +100,7 @@ def _torch_forward_v2(q, k, v, lam, causal):
     return torch.stack(outs, dim=1)
 
 
-def test_v2_gradients_match_autograd_with_gqa():
+def pin_autograd_with_gqa(b):
     g = torch.Generator().manual_seed(3)
     q = torch.randn(2, 8, 33, 16, generator=g, dtype=torch.float64, requires_grad=True)
     k = torch.randn(2, 2, 33, 16, generator=g, dtype=torch.float64, requires_grad=True)
@@ -110,9 +108,27 @@ def test_v2_gradients_match_autograd_with_gqa():
     lam = torch.tensor([0.3, 0.9, -0.1, 0.6], dtype=torch.float64, requires_grad=True)
     dout = torch.randn(2, 4, 33, 16, generator=g, dtype=torch.float64)
     _torch_forward_v2(q, k, v, lam, True).backward(dout)
-    dq, dk, dv, dlam = bwd.diffattn_v2_backward(q.detach(), k.detach(), v.detach(), lam.detach(), dout)
+    dq, dk, dv, dlam = b.diffattn_v2_backward(q.detach(), k.detach(), v.detach(), lam.detach(), dout)
     for got, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad), (dlam, lam.grad)):
         assert np.allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# The pins above with their arguments; test_oracle_backward_mutations.py runs
+# the same list against planted mistakes.
+PINS = [
+    (pin_v2_finite_differences, (True, 5, 5)),
+    (pin_v2_finite_differences, (False, 4, 6)),
+    (pin_v2_finite_differences, (True, 3, 6)),
+    (pin_v1_finite_differences, (False,)),
+    (pin_v1_finite_differences, (True,)),
+    (pin_lambda_parameters, ()),
+    (pin_autograd_with_gqa, ()),
+]
+
+
+@pytest.mark.parametrize("pin,args", PINS, ids=lambda x: getattr(x, "__name__", str(x)))
+def test_pin(pin, args):
+    pin(bwd, *args)
 
 
 def test_zero_upstream_gives_zero_gradients_and_linearity():
