@@ -319,8 +319,7 @@ class Backward:
     def work(self):
         return backward_flops(self.w) / 1e12, "TFLOP/s"
 
-    def host_call(self, host):
-        raise NotImplementedError("the backward is timed on device tensors only")
+    host_path = "the backward is timed on device tensors only"
 
 
 def sweep_bytes(n=inputs.SWEEP_INSTANCES, lengths=inputs.SWEEP_LENGTHS) -> int:
@@ -362,8 +361,7 @@ class SnrSweep:
         return [noise.summarize(N, o[0][:, 0, 0].float(), o[0][:, 0, 1].float(), o[1][:, 0, 0].float(),
                                 o[1][:, 0, 1].float()) for N, o in zip(self.lengths, self.outs)]
 
-    def host_call(self, host):
-        raise NotImplementedError("the sweep is timed on device tensors only")
+    host_path = "the sweep is timed on device tensors only"
 
 
 def lowrank_flops(B, H, L, **_) -> float:
@@ -405,8 +403,7 @@ class LowRank:
     def work(self):
         return lowrank_flops(**self.shape) / 1e12, "TFLOP/s"
 
-    def host_call(self, host):
-        raise NotImplementedError("the low-rank forward is timed on device tensors only")
+    host_path = "the low-rank forward is timed on device tensors only"
 
 
 def workload_work(name):
@@ -523,7 +520,10 @@ def aggregate(work_per_rank, world, ms_per_step):
 def e2e_measure(r, steps):
     """Same metric through the public API with pinned HOST buffers: the
     host->device copies of the step's inputs and the device->host copy of its
-    output are inside the timed region."""
+    output are inside the timed region.  A runner without a host path names
+    why in its ``host_path`` string."""
+    if isinstance(getattr(r, "host_path", None), str):
+        raise NotImplementedError(r.host_path)
     host = {k: v.cpu().pin_memory() for k, v in r.x.items()}
     host["lp"] = [t.cpu().pin_memory() for t in r.lp]
     h2d = sum(v.numel() * v.element_size() for k, v in host.items() if k != "lp")
