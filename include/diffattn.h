@@ -1,6 +1,7 @@
 /*
- * diffattn.h -- C ABI of libdiffattn.so, the B200 (sm_100a) differential
- * attention forward.
+ * diffattn.h -- C ABI of libdiffattn.so, B200 (sm_100a) differential
+ * attention: prefill and decode forward, the training forward and backward,
+ * and the low-rank substitute for the second map.
  *
  * The operation (sources cited by page title and section):
  *
