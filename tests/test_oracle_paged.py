@@ -9,11 +9,12 @@ length, rows read past the sequence) would break."""
 import math
 
 import numpy as np
+import pytest
 import torch
 
 from differential_attention_transformers_b200 import inputs
 from oracle import brute
-from oracle import diffattn as orc
+from oracle import diffattn
 
 
 def _case(B=3, Hq=8, Hkv=2, T=150, D=16, seed=0):
@@ -26,7 +27,7 @@ def _case(B=3, Hq=8, Hkv=2, T=150, D=16, seed=0):
     return q, kc, vc, lam
 
 
-def test_identity_reading_full_lengths_equals_contiguous_decode():
+def pin_identity_reading_full_lengths_equals_contiguous_decode(orc):
     q, kc, vc, lam = _case()
     for ps in (16, 64):
         kp, vp, bt, sl = inputs.paged_cache(kc, vc, ps, seed=ps)
@@ -35,7 +36,7 @@ def test_identity_reading_full_lengths_equals_contiguous_decode():
         assert np.allclose(got, ref, rtol=0, atol=1e-13)
 
 
-def test_variable_lengths_equal_truncated_contiguous_decode():
+def pin_variable_lengths_equal_truncated_contiguous_decode(orc):
     q, kc, vc, lam = _case(T=200)
     lens = [200, 1, 77]
     kp, vp, bt, sl = inputs.paged_cache(kc, vc, 32, seed=5, lens=lens)
@@ -46,14 +47,14 @@ def test_variable_lengths_equal_truncated_contiguous_decode():
         assert np.all(np.isfinite(got[b]))     # NaN rows past the length never read
 
 
-def test_page_permutation_invariance():
+def pin_page_permutation_invariance(orc):
     q, kc, vc, lam = _case(T=96)
     a = orc.decode_v2_paged(q, *inputs.paged_cache(kc, vc, 16, seed=1), lam)
     b = orc.decode_v2_paged(q, *inputs.paged_cache(kc, vc, 16, seed=2), lam)
     assert np.array_equal(a, b)
 
 
-def test_zero_length_sequence_gives_zeros():
+def pin_zero_length_sequence_gives_zeros(orc):
     q, kc, vc, lam = _case(T=40)
     kp, vp, bt, sl = inputs.paged_cache(kc, vc, 16, seed=3, lens=[40, 0, 17])
     got = orc.decode_v2_paged(q, kp, vp, bt, sl, lam)
@@ -61,7 +62,7 @@ def test_zero_length_sequence_gives_zeros():
     assert np.all(np.isfinite(got))
 
 
-def test_single_token_sequence_is_one_minus_lambda_times_value():
+def pin_single_token_sequence_is_one_minus_lambda_times_value(orc):
     # one visible key: both maps put weight 1 on it, O = (1 - lambda) v
     q, kc, vc, lam = _case(B=1, T=5)
     kp, vp, bt, sl = inputs.paged_cache(kc, vc, 16, seed=4, lens=[1])
@@ -72,7 +73,7 @@ def test_single_token_sequence_is_one_minus_lambda_times_value():
         assert np.allclose(got[0, h], (1 - lam[h]) * vc[0, g, 0].numpy(), rtol=0, atol=1e-14)
 
 
-def test_brute_force_twin_on_a_tiny_paged_case():
+def pin_brute_force_twin_on_a_tiny_paged_case(orc):
     q, kc, vc, lam = _case(B=2, Hq=4, Hkv=1, T=21, D=4)
     lens = [21, 9]
     kp, vp, bt, sl = inputs.paged_cache(kc, vc, 16, seed=6, lens=lens)
@@ -83,3 +84,13 @@ def test_brute_force_twin_on_a_tiny_paged_case():
         vv = [[vc[b, 0, :n].tolist()]]
         ref = np.array(brute.v2(qq, kk, vv, list(lam), causal=True))[0, :, 0]
         assert np.allclose(got[b], ref, rtol=0, atol=1e-12)
+
+
+# The pins above; test_oracle_paged_mutations.py runs them against planted
+# gather mistakes.
+PINS = [pin_identity_reading_full_lengths_equals_contiguous_decode, pin_variable_lengths_equal_truncated_contiguous_decode, pin_page_permutation_invariance, pin_zero_length_sequence_gives_zeros, pin_single_token_sequence_is_one_minus_lambda_times_value, pin_brute_force_twin_on_a_tiny_paged_case]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin(diffattn)
