@@ -441,12 +441,11 @@ int launch_backward_v1(const void* q1, const void* k1, const void* q2, const voi
 // and the chunk sums [B*H, nc+1, r, 128] and [B*H, nc+1, r] f32.
 struct LowrankLayout {
   size_t lam, pre, lse, a1v, tot, ztot, total;
-  int nc;
+  int n_lead, nc;
 };
 LowrankLayout lowrank_layout(int B, int H, int Lq, int Lk, int r, int causal) {
   LowrankLayout l;
-  const long long rows = causal ? Lq : Lk;
-  l.nc = (int)((rows + LR_C - 1) / LR_C);
+  lr_slots(Lq, Lk, causal, l.n_lead, l.nc);
   const size_t BH = (size_t)B * H, Hp = (size_t)H / 2;
   l.lam = 0;
   l.pre = align256(Hp * 4);
@@ -800,6 +799,7 @@ int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const floa
   a.tot = reinterpret_cast<float*>(w + L.tot);
   a.ztot = reinterpret_cast<float*>(w + L.ztot);
   a.B = B; a.H = H; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk; a.r = r; a.causal = causal ? 1 : 0;
+  a.n_lead = L.n_lead;
   a.nc = L.nc;
   const unsigned BH = (unsigned)(B * H);
   if (L.nc > 0 && Lk > 0) {

@@ -14,17 +14,19 @@
 //     out_i   = (A1 V)_i - lambda (N V)_i          (0 for N's row when f_i^T z_i = 0)
 //
 // Under the causal mask the keys row i sees are a prefix, j <= i + (Lk - Lq),
-// so S_i and z_i are prefix sums over keys.  Query rows are cut into chunks of
-// LR_C; chunk c starts from the keys before P_c = clamp(c LR_C + Lk - Lq, 0, Lk)
-// and each of its rows adds one key.  Three HBM-bound passes:
+// so S_i and z_i are prefix sums over keys.  The keys are cut into slots: first
+// n_lead slots of LR_C keys covering the leading keys [0, P_0) that every row
+// sees, then one slot per chunk of LR_C query rows, row chunk c holding the
+// keys [P_c, P_{c+1}) with P_c = clamp(c LR_C + Lk - Lq, 0, Lk), one per row.
+// Three HBM-bound passes:
 //
-//   lr_totals_kernel  per chunk, the sums of g_j v_j^T and g_j over the keys it
-//                     adds: [0, P_1) for chunk 0, [P_c, P_{c+1}) after
-//                     (unmasked: key chunks [c LR_C, (c+1) LR_C))
-//   lr_prefix_kernel  exclusive prefix of those sums over the chunks, plus the
+//   lr_totals_kernel  per slot, the sums of g_j v_j^T and g_j over its keys
+//                     (unmasked: plain key chunks [c LR_C, (c+1) LR_C))
+//   lr_prefix_kernel  exclusive prefix of those sums over the slots, plus the
 //                     grand total in slot nc (used by every row when unmasked)
-//   lr_emit_kernel    chunk 0 first adds the keys [0, P_0); then each row adds
-//                     its key i + Lk - Lq and writes out_i
+//   lr_emit_kernel    row chunk c starts from the prefix at its slot, i.e. the
+//                     keys [0, P_c); each row adds its key i + Lk - Lq and
+//                     writes out_i
 //
 // A1 V comes from the prefill's training variant, which already writes each
 // map's normalised output O_m / l_m: pairing heads (2j, 2j+1) of one KV group
@@ -55,17 +57,37 @@ struct LowrankArgs {
   float* tot;                 // [B*H, nc + 1, r, 128] chunk sums of g v^T, then their prefix; slot nc = total
   float* ztot;                // [B*H, nc + 1, r] the same for g
   int B, H, Hkv, Lq, Lk, r, causal;
-  int nc;                     // key chunks: ceil(Lq / LR_C) causal, ceil(Lk / LR_C) unmasked
+  int n_lead;                 // causal: slots of leading keys, ceil(clamp(Lk - Lq, 0, Lk) / LR_C); else 0
+  int nc;                     // slots: n_lead + ceil(Lq / LR_C) causal, ceil(Lk / LR_C) unmasked
 };
+
+// Slot counts for the sizes in a (host and device use the same rule).
+__host__ __device__ inline void lr_slots(int Lq, int Lk, int causal, int& n_lead, int& nc) {
+  if (causal) {
+    const long long off = (long long)Lk - Lq;
+    const long long lead = off < 0 ? 0 : (off > Lk ? Lk : off);
+    n_lead = (int)((lead + LR_C - 1) / LR_C);
+    nc = n_lead + (int)(((long long)Lq + LR_C - 1) / LR_C);
+  } else {
+    n_lead = 0;
+    nc = (int)(((long long)Lk + LR_C - 1) / LR_C);
+  }
+}
 
 __host__ __device__ inline long long lr_clamp(long long x, long long hi) { return x < 0 ? 0 : (x > hi ? hi : x); }
 
-// Keys whose sums chunk c contributes (see the header).
+// Keys whose sums slot c contributes (see the header).
 __host__ __device__ inline void lr_key_range(const LowrankArgs& a, int c, long long& ks, long long& ke) {
   if (a.causal) {
-    const long long off = (long long)a.Lk - a.Lq;
-    ks = c == 0 ? 0 : lr_clamp((long long)c * LR_C + off, a.Lk);
-    ke = lr_clamp((long long)(c + 1) * LR_C + off, a.Lk);
+    const long long off = (long long)a.Lk - a.Lq, lead = lr_clamp(off, a.Lk);
+    if (c < a.n_lead) {            // leading keys, seen by every row
+      ks = (long long)c * LR_C;
+      ke = ks + LR_C < lead ? ks + LR_C : lead;
+    } else {                       // the keys the rows of chunk c - n_lead add
+      const long long rc = c - a.n_lead;
+      ks = rc == 0 ? lead : lr_clamp(rc * LR_C + off, a.Lk);
+      ke = lr_clamp((rc + 1) * LR_C + off, a.Lk);
+    }
   } else {
     ks = (long long)c * LR_C;
     ke = lr_clamp((long long)(c + 1) * LR_C, a.Lk);
@@ -128,7 +150,7 @@ __host__ __device__ inline void lr_prefix_body(const LowrankArgs& a, int bh, int
 // Row chunk c (rows [c LR_C, min(Lq, (c+1) LR_C))) of head bh, value column col.
 __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh, int col) {
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
-  const size_t slot = (size_t)bh * (a.nc + 1) + (a.causal ? c : a.nc);
+  const size_t slot = (size_t)bh * (a.nc + 1) + (a.causal ? a.n_lead + c : a.nc);
   float S[LR_RMAX], z[LR_RMAX];
 #pragma unroll
   for (int t = 0; t < LR_RMAX; ++t) {
@@ -138,8 +160,6 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
   const long long off = (long long)a.Lk - a.Lq;
   const __nv_bfloat16* vcol = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lk * LR_DV + col;
   const float* gh = a.G + (size_t)h * a.Lk * a.r;
-  if (a.causal && c == 0)
-    for (long long j = 0; j < lr_clamp(off, a.Lk); ++j) lr_add_key(a, vcol, gh, j, S, z);
   const long long r0 = (long long)c * LR_C;
   const long long r1 = r0 + LR_C < a.Lq ? r0 + LR_C : a.Lq;
   const float lam = a.lambda[h];

@@ -42,8 +42,7 @@ int main(int argc, char** argv) {
 
   LowrankArgs a{};
   a.B = B; a.H = H; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk; a.r = r; a.causal = causal;
-  const long long rows = causal ? Lq : Lk;
-  a.nc = (int)((rows + da::LR_C - 1) / da::LR_C);
+  da::lr_slots(Lq, Lk, causal, a.n_lead, a.nc);
   std::vector<float> tot(BH * (a.nc + 1) * r * da::LR_DV, 0.f), ztot(BH * (a.nc + 1) * r, 0.f);
   std::vector<uint16_t> out(BH * Lq * da::LR_DV, 0);
   a.v = reinterpret_cast<const __nv_bfloat16*>(v.data());

@@ -59,6 +59,7 @@ CASES = [
     (2, 4, 1, 300, 700, 3, True),     # Lq < Lk: bottom-right causal offset
     (1, 2, 1, 700, 300, 1, True),     # Lq > Lk: the first rows see no key
     (1, 4, 2, 300, 600, 16, False),   # unmasked, largest rank
+    (1, 2, 1, 40, 1000, 4, True),     # decode-like: 960 leading keys every row sees
     (1, 2, 1, 64, 0, 2, True),        # no keys: zero output
 ]
 

@@ -66,6 +66,7 @@ CASES = [
     (1, 2, 1, 300, 700, 3, True),     # Lq < Lk: offset 400, beyond one chunk
     (1, 2, 2, 700, 300, 1, True),     # Lq > Lk: the first 400 rows see no key
     (1, 2, 1, 300, 600, 16, False),   # unmasked, largest rank
+    (1, 2, 1, 40, 1000, 4, True),     # decode-like: 960 leading keys, four slots, the last partial
     (1, 2, 1, 70, 0, 2, True),        # no keys
     (1, 2, 1, 70, 0, 2, False),
 ]
