@@ -70,6 +70,13 @@ __host__ __device__ __forceinline__ long long dec_blk_start(long long i, long lo
   return i * total / grid;
 }
 
+// The CTA whose range [dec_blk_start(i), dec_blk_start(i + 1)) holds block x,
+// 0 <= x < total: the largest i with i * total / grid <= x, i.e. with
+// i * total < (x + 1) * grid.  Its range is never empty.
+__host__ __device__ __forceinline__ long long dec_owner(long long x, long long total, int grid) {
+  return ((x + 1) * grid - 1) / total;
+}
+
 template <int NST, bool PAGED = false>
 struct DecSmem {
   alignas(1024) uint8_t k[NST][DEC_TILE_BYTES];
@@ -496,38 +503,42 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
     x1 = x0 + a.nblk;
   }
 
-  // CTAs whose block range overlaps [x0, x1)
-  long long i0 = total > 0 ? x0 * a.grid / total : 0;
-  while (i0 > 0 && dec_blk_start(i0, total, a.grid) > x0) --i0;
-  while (i0 + 1 < a.grid && dec_blk_start(i0 + 1, total, a.grid) <= x0) ++i0;
-
-  float res[2];
-  for (int mp = 0; mp < 2; ++mp) {
-    const int c = mp == 0 ? c1 : c2;
+  // The CTAs whose ranges overlap [x0, x1), in ascending order: start at the
+  // owner of x0, then jump to the owner of the block after each range.  Only
+  // CTAs that wrote a record for this segment are visited (with short caches
+  // most CTAs of the grid have an empty range and none of them is touched).
+  // Two walks: the maxima of both maps first, then the scaled sums, so every
+  // record is scaled by its exact distance to the global maximum.
+  auto record = [&](long long i, long long s, int mp) -> const float* {
     const float* base = a.ws + ((a.two_pass && mp == 1) ? a.half_floats : 0);
-    float M = -INFINITY;
-    for (long long i = i0; x1 > x0 && i < a.grid && dec_blk_start(i, total, a.grid) < x1; ++i) {
-      // CTAs with an empty range (paged mode: more CTAs than blocks) wrote nothing
-      const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
-      if (e <= x0 || s >= x1 || e <= s) continue;
-      const float* rec = a.cu ? base + ((size_t)i + (size_t)bg) * DEC_REC
-                              : base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
-      M = fmaxf(M, rec[c]);
-    }
-    const float Mu = M == -INFINITY ? 0.f : M;
-    float o = 0.f, l = 0.f;
-    for (long long i = i0; x1 > x0 && i < a.grid && dec_blk_start(i, total, a.grid) < x1; ++i) {
-      // CTAs with an empty range (paged mode: more CTAs than blocks) wrote nothing
-      const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
-      if (e <= x0 || s >= x1 || e <= s) continue;
-      const float* rec = a.cu ? base + ((size_t)i + (size_t)bg) * DEC_REC
-                              : base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
-      const float f = ex2(rec[c] - Mu);
-      o += rec[16 + c * 128 + t] * f;
-      l += rec[8 + c] * f;
-    }
-    res[mp] = l > 0.f ? o / l : 0.f;
+    return a.cu ? base + ((size_t)i + (size_t)bg) * DEC_REC
+                : base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
+  };
+  const int cc[2] = {c1, c2};
+  float M[2] = {-INFINITY, -INFINITY};
+  for (long long x = x0; x < x1;) {
+    const long long i = dec_owner(x, total, a.grid);
+    const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
+#pragma unroll
+    for (int mp = 0; mp < 2; ++mp) M[mp] = fmaxf(M[mp], record(i, s, mp)[cc[mp]]);
+    x = e;
   }
+  float o[2] = {0.f, 0.f}, l[2] = {0.f, 0.f};
+  for (long long x = x0; x < x1;) {
+    const long long i = dec_owner(x, total, a.grid);
+    const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
+#pragma unroll
+    for (int mp = 0; mp < 2; ++mp) {
+      const float* rec = record(i, s, mp);
+      const float f = ex2(rec[cc[mp]] - (M[mp] == -INFINITY ? 0.f : M[mp]));
+      o[mp] += rec[16 + cc[mp] * 128 + t] * f;
+      l[mp] += rec[8 + cc[mp]] * f;
+    }
+    x = e;
+  }
+  float res[2];
+#pragma unroll
+  for (int mp = 0; mp < 2; ++mp) res[mp] = l[mp] > 0.f ? o[mp] / l[mp] : 0.f;
   const float lam = a.lambda[h];
   a.out[((size_t)b * Hout + h) * 128 + t] = __float2bfloat16_rn(__fsub_rn(res[0], __fmul_rn(lam, res[1])));
 }

@@ -112,10 +112,12 @@ int device_setup(DeviceInfo** out) {
                                   (int)prefill_smem<64>()));
     CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)prefill_smem<128>()));
-    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128, PF_TRAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)prefill_smem<128>()));
-    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<64, PF_TRAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)prefill_smem<64>()));
+    CUDA_TRY(cudaFuncSetAttribute(prefill_kernel<128, PF_SINGLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)prefill_smem<128>()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
@@ -189,7 +191,7 @@ int launch_simt(const SimtArgs& a, cudaStream_t s) {
 int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
                    const float* lambda, void* out, int B, int Hout, int Hq, int Hkv, int Lq, int Lk, int dqk,
                    bool v1, int causal, int rms, float eps, cudaStream_t s, float* lse = nullptr,
-                   void* o_maps = nullptr, float* rstd = nullptr) {
+                   void* o_maps = nullptr, float* rstd = nullptr, float* o_f32 = nullptr) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   if (Lq == 0 || B == 0 || Hout == 0) return ok();
@@ -216,12 +218,16 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.lse = lse;
   a.o_maps = static_cast<__nv_bfloat16*>(o_maps);
   a.rstd = rstd;
+  a.o_f32 = o_f32;
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
-  if (lse != nullptr && dqk == 128)   // training forward (V2)
-    prefill_kernel<128, true><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+  if (o_f32 != nullptr)               // single-map outputs (V2 layout)
+    prefill_kernel<128, PF_SINGLE><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv,
+                                                                                           a);
+  else if (lse != nullptr && dqk == 128)   // training forward (V2)
+    prefill_kernel<128, PF_TRAIN><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (lse != nullptr)            // training forward (V1, d = 64)
-    prefill_kernel<64, true><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<64, PF_TRAIN><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (dqk == 64)
     prefill_kernel<64><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else
@@ -435,23 +441,19 @@ int launch_backward_v1(const void* q1, const void* k1, const void* q2, const voi
   return ok();
 }
 
-// Low-rank forward workspace: the zero lambda of the single-map prefill
-// [H/2], its by-product output [B, H/2, Lq, 128] bf16 and log-sum-exp
-// [B, H/2, 2, Lq], the per-head single-map outputs A1 V [B, H, Lq, 128] bf16,
-// and the chunk sums [B*H, nc+1, r, 128] and [B*H, nc+1, r] f32.
+// Low-rank forward workspace: the per-head single-map outputs A1 V
+// [B, H, Lq, 128] f32, then the chunk sums [B*H, nc+1, r, 128] and
+// [B*H, nc+1, r] f32.
 struct LowrankLayout {
-  size_t lam, pre, lse, a1v, tot, ztot, total;
+  size_t a1v, tot, ztot, total;
   int n_lead, nc;
 };
 LowrankLayout lowrank_layout(int B, int H, int Lq, int Lk, int r, int causal) {
   LowrankLayout l;
   lr_slots(Lq, Lk, causal, l.n_lead, l.nc);
-  const size_t BH = (size_t)B * H, Hp = (size_t)H / 2;
-  l.lam = 0;
-  l.pre = align256(Hp * 4);
-  l.lse = l.pre + align256((size_t)B * Hp * Lq * 256);
-  l.a1v = l.lse + align256((size_t)B * Hp * 2 * Lq * 4);
-  l.tot = l.a1v + align256(BH * Lq * 256);
+  const size_t BH = (size_t)B * H;
+  l.a1v = 0;
+  l.tot = l.a1v + align256(BH * Lq * LR_DV * 4);
   l.ztot = l.tot + align256(BH * (l.nc + 1) * r * LR_DV * 4);
   l.total = l.ztot + align256(BH * (l.nc + 1) * r * 4);
   return l;
@@ -564,8 +566,7 @@ int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const 
                     double lambda_init, float* lambda_out, void* stream) {
   if (!lq1 || !lk1 || !lq2 || !lk2 || !lambda_out) return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   if (heads < 1 || dim < 1) return fail(DIFFATTN_ERR_INVALID_ARG, "heads and dim must be >= 1");
-  const int threads = 128;
-  lambda_kernel<<<(heads + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  lambda_kernel<<<(heads + LAM_WARPS - 1) / LAM_WARPS, 32 * LAM_WARPS, 0, static_cast<cudaStream_t>(stream)>>>(
       lq1, lk1, lq2, lk2, heads, dim, lambda_init, lambda_out);
   CUDA_TRY(cudaGetLastError());
   return ok();
@@ -784,17 +785,17 @@ int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const floa
   if (int e = device_setup(&dev)) return e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  float* zero_lam = reinterpret_cast<float*>(w + L.lam);
-  CUDA_TRY(cudaMemsetAsync(zero_lam, 0, sizeof(float) * (size_t)(H / 2), s));
-  // A1 V for every head: the training prefill with heads (2j, 2j+1) as a pair
-  // writes both maps' normalised outputs, [B, H/2, 2, Lq, 128] = [B, H, Lq, 128].
-  if (int e = launch_prefill(q, q, k, k, v, zero_lam, w + L.pre, B, H / 2, H, Hkv, Lq, Lk, 128, false, causal, 0,
-                             0.f, s, reinterpret_cast<float*>(w + L.lse), w + L.a1v))
+  // A1 V for every head in f32: the single-map prefill runs heads (2j, 2j+1)
+  // of one KV group as the two maps of a CTA and writes each one's O / l,
+  // [B, H/2, 2, Lq, 128] = [B, H, Lq, 128]; lambda only sets each head's
+  // residual choice there.
+  if (int e = launch_prefill(q, q, k, k, v, lambda, nullptr, B, H / 2, H, Hkv, Lq, Lk, 128, false, causal, 0, 0.f,
+                             s, nullptr, nullptr, nullptr, reinterpret_cast<float*>(w + L.a1v)))
     return e;
   LowrankArgs a{};
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.F = F; a.G = G; a.lambda = lambda;
-  a.a1v = reinterpret_cast<const __nv_bfloat16*>(w + L.a1v);
+  a.a1v = reinterpret_cast<const float*>(w + L.a1v);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.tot = reinterpret_cast<float*>(w + L.tot);
   a.ztot = reinterpret_cast<float*>(w + L.ztot);
@@ -822,8 +823,8 @@ int diffattn_lambda_backward(const float* lq1, const float* lk1, const float* lq
   if (!lq1 || !lk1 || !lq2 || !lk2 || !dlambda || !dlq1 || !dlk1 || !dlq2 || !dlk2)
     return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   if (heads < 1 || dim < 1) return fail(DIFFATTN_ERR_INVALID_ARG, "heads and dim must be >= 1");
-  const int threads = 128;
-  lambda_backward_kernel<<<(heads + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  lambda_backward_kernel<<<(heads + LAM_WARPS - 1) / LAM_WARPS, 32 * LAM_WARPS, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
       lq1, lk1, lq2, lk2, dlambda, heads, dim, dlq1, dlk1, dlq2, dlk2);
   CUDA_TRY(cudaGetLastError());
   return ok();

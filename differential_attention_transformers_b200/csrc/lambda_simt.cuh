@@ -10,38 +10,77 @@ namespace da {
 // ("差分注意力" tutorial, Step 4 λ 参数化).  fp64 throughout: the products of
 // two fp32 values are exact in fp64, the dot products are summed in index
 // order, and the result is rounded once to fp32.
-__global__ void lambda_kernel(const float* __restrict__ lq1, const float* __restrict__ lk1,
-                              const float* __restrict__ lq2, const float* __restrict__ lk2, int heads,
-                              int dim, double lambda_init, float* __restrict__ out) {
-  const int h = blockIdx.x * blockDim.x + threadIdx.x;
-  if (h >= heads) return;
-  double d1 = 0.0, d2 = 0.0;
-  const size_t base = (size_t)h * dim;
-  for (int i = 0; i < dim; ++i) {
-    d1 = __dadd_rn(d1, __dmul_rn((double)lq1[base + i], (double)lk1[base + i]));
-    d2 = __dadd_rn(d2, __dmul_rn((double)lq2[base + i], (double)lk2[base + i]));
+//
+// One warp per head.  The warp stages a chunk of each of the four parameter
+// rows in shared memory with coalesced loads; lane 0 then runs the sequential
+// sums out of shared memory, so the order of the additions (and with it every
+// bit of the result) is that of a plain loop over the index.
+constexpr int LAM_WARPS = 4;      // heads per block
+constexpr int LAM_CHUNK = 128;    // elements of each row staged at a time
+
+__device__ __forceinline__ void lambda_dots(const float* __restrict__ lq1, const float* __restrict__ lk1,
+                                            const float* __restrict__ lq2, const float* __restrict__ lk2,
+                                            size_t base, int dim, float (*st)[LAM_CHUNK], int lane, double& d1,
+                                            double& d2) {
+  d1 = 0.0;
+  d2 = 0.0;
+  for (int c0 = 0; c0 < dim; c0 += LAM_CHUNK) {
+    const int n = min(LAM_CHUNK, dim - c0);
+    for (int i = lane; i < n; i += 32) {
+      st[0][i] = lq1[base + c0 + i];
+      st[1][i] = lk1[base + c0 + i];
+      st[2][i] = lq2[base + c0 + i];
+      st[3][i] = lk2[base + c0 + i];
+    }
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll 8
+      for (int i = 0; i < n; ++i) {
+        d1 = __dadd_rn(d1, __dmul_rn((double)st[0][i], (double)st[1][i]));
+        d2 = __dadd_rn(d2, __dmul_rn((double)st[2][i], (double)st[3][i]));
+      }
+    }
+    __syncwarp();
   }
-  out[h] = (float)__dadd_rn(__dsub_rn(exp(d1), exp(d2)), lambda_init);
+}
+
+__global__ void __launch_bounds__(32 * LAM_WARPS)
+lambda_kernel(const float* __restrict__ lq1, const float* __restrict__ lk1, const float* __restrict__ lq2,
+              const float* __restrict__ lk2, int heads, int dim, double lambda_init, float* __restrict__ out) {
+  __shared__ float st[LAM_WARPS][4][LAM_CHUNK];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x * LAM_WARPS + w;
+  if (h >= heads) return;   // warp-uniform
+  double d1, d2;
+  lambda_dots(lq1, lk1, lq2, lk2, (size_t)h * dim, dim, st[w], lane, d1, d2);
+  if (lane == 0) out[h] = (float)__dadd_rn(__dsub_rn(exp(d1), exp(d2)), lambda_init);
 }
 
 // Gradients of the four λ parameter vectors given dlambda[h] (the chain rule
 // of the λ above): dlq1 = g e1 lk1, dlk1 = g e1 lq1, dlq2 = -g e2 lk2,
 // dlk2 = -g e2 lq2 with e_i = exp(lq_i . lk_i), in fp64, rounded once to f32.
-__global__ void lambda_backward_kernel(const float* __restrict__ lq1, const float* __restrict__ lk1,
-                                       const float* __restrict__ lq2, const float* __restrict__ lk2,
-                                       const float* __restrict__ dlambda, int heads, int dim,
-                                       float* __restrict__ dlq1, float* __restrict__ dlk1, float* __restrict__ dlq2,
-                                       float* __restrict__ dlk2) {
-  const int h = blockIdx.x * blockDim.x + threadIdx.x;
-  if (h >= heads) return;
-  double d1 = 0.0, d2 = 0.0;
+// One warp per head: the dot products as in lambda_kernel, then every lane
+// writes its share of the four gradient rows (coalesced).
+__global__ void __launch_bounds__(32 * LAM_WARPS)
+lambda_backward_kernel(const float* __restrict__ lq1, const float* __restrict__ lk1, const float* __restrict__ lq2,
+                       const float* __restrict__ lk2, const float* __restrict__ dlambda, int heads, int dim,
+                       float* __restrict__ dlq1, float* __restrict__ dlk1, float* __restrict__ dlq2,
+                       float* __restrict__ dlk2) {
+  __shared__ float st[LAM_WARPS][4][LAM_CHUNK];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x * LAM_WARPS + w;
+  if (h >= heads) return;   // warp-uniform
   const size_t base = (size_t)h * dim;
-  for (int i = 0; i < dim; ++i) {
-    d1 = __dadd_rn(d1, __dmul_rn((double)lq1[base + i], (double)lk1[base + i]));
-    d2 = __dadd_rn(d2, __dmul_rn((double)lq2[base + i], (double)lk2[base + i]));
+  double d1, d2, g1 = 0.0, g2 = 0.0;
+  lambda_dots(lq1, lk1, lq2, lk2, base, dim, st[w], lane, d1, d2);
+  if (lane == 0) {
+    const double g = (double)dlambda[h];
+    g1 = g * exp(d1);
+    g2 = -g * exp(d2);
   }
-  const double g = (double)dlambda[h], g1 = g * exp(d1), g2 = -g * exp(d2);
-  for (int i = 0; i < dim; ++i) {
+  g1 = __shfl_sync(0xffffffffu, g1, 0);
+  g2 = __shfl_sync(0xffffffffu, g2, 0);
+  for (int i = lane; i < dim; i += 32) {
     dlq1[base + i] = (float)(g1 * (double)lk1[base + i]);
     dlk1[base + i] = (float)(g1 * (double)lq1[base + i]);
     dlq2[base + i] = (float)(g2 * (double)lk2[base + i]);

@@ -28,9 +28,14 @@
 //                     keys [0, P_c); each row adds its key i + Lk - Lq and
 //                     writes out_i
 //
-// A1 V comes from the prefill's training variant, which already writes each
-// map's normalised output O_m / l_m: pairing heads (2j, 2j+1) of one KV group
-// gives every head's single-map attention without extra products.
+// A1 V comes from the prefill's single-map mode: pairing heads (2j, 2j+1) of
+// one KV group as a CTA's two maps gives every head's single-map attention
+// without extra products.  It is written in f32, O_m / l_m straight from the
+// accumulator, and P keeps its bf16 residual for heads with |1 - lambda| below
+// the forward's threshold: when N is close to A1 and lambda close to 1 the
+// output is a small difference of two near-equal terms, and a bf16 A1 V (or a
+// bf16-only P) would leave an error of A1 V's own rounding scale in it.  The
+// subtraction here is then the only rounding to bf16.
 //
 // One thread owns one of the 128 value columns and r <= LR_RMAX accumulators;
 // there is no shared memory and no wait.  Each kernel body is a host-device
@@ -52,7 +57,7 @@ struct LowrankArgs {
   const float* F;             // [H, Lq, r], >= 0
   const float* G;             // [H, Lk, r], >= 0
   const float* lambda;        // [H]
-  const __nv_bfloat16* a1v;   // [B, H, Lq, 128]: A1 V per head
+  const float* a1v;           // [B, H, Lq, 128]: A1 V per head, f32
   __nv_bfloat16* out;         // [B, H, Lq, 128]
   float* tot;                 // [B*H, nc + 1, r, 128] chunk sums of g v^T, then their prefix; slot nc = total
   float* ztot;                // [B*H, nc + 1, r] the same for g
@@ -164,7 +169,7 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
   const long long r1 = r0 + LR_C < a.Lq ? r0 + LR_C : a.Lq;
   const float lam = a.lambda[h];
   const float* fh = a.F + (size_t)h * a.Lq * a.r;
-  const __nv_bfloat16* arow = a.a1v + (size_t)bh * a.Lq * LR_DV + col;
+  const float* arow = a.a1v + (size_t)bh * a.Lq * LR_DV + col;
   __nv_bfloat16* orow = a.out + (size_t)bh * a.Lq * LR_DV + col;
   for (long long i = r0; i < r1; ++i) {
     if (a.causal) {
@@ -180,7 +185,7 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
         den = fmaf(f, z[t], den);
       }
     const float nv = den > 0.f ? num / den : 0.f;
-    orow[i * LR_DV] = __float2bfloat16_rn(__bfloat162float(arow[i * LR_DV]) - lam * nv);
+    orow[i * LR_DV] = __float2bfloat16_rn(arow[i * LR_DV] - lam * nv);
   }
 }
 

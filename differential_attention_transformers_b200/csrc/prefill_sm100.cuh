@@ -70,7 +70,18 @@ struct PrefillArgs {
   float* lse;
   __nv_bfloat16* o_maps;
   float* rstd;
+  // Single-map mode (PF_SINGLE): output heads are pairs of independent
+  // heads (2h, 2h+1) over one KV head, each with its own lambda[2h + m] (which
+  // sets only its residual choice); the kernel writes each head's normalised
+  // map output O_m / l_m in f32, o_f32[B, Hout, 2, Lq, 128] = [B, 2 Hout, Lq,
+  // 128], and nothing else.
+  float* o_f32;
 };
+
+// What a launch writes (template argument of prefill_kernel).
+constexpr int PF_INFER = 0;    // out
+constexpr int PF_TRAIN = 1;    // out, lse, o_maps [, rstd]
+constexpr int PF_SINGLE = 2;   // o_f32 only
 
 template <int DQK>
 struct PfSmem {
@@ -173,14 +184,40 @@ __device__ __forceinline__ void pf_store_rows(uint8_t* st, const float (&y)[64],
   }
 }
 
-// TRAIN: also write the training outputs (lse, o_maps); a template flag so the
-// inference kernel carries none of that code.
-template <int DQK, bool TRAIN = false>
+// f32 variant of pf_store_rows: the warp stages all 32 rows (256 bytes each,
+// 16-byte chunks XOR-swizzled by row, conflict-free both ways) in 8 KB and
+// writes them back as 2 rows x 256 contiguous bytes per instruction.
+constexpr int PF_STAGE_F32 = 32 * 64 * 4;
+__device__ __forceinline__ void pf_store_rows_f32(uint8_t* st, const float (&y)[64], float* base, int row_w0,
+                                                  int Lq, int lane) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    *reinterpret_cast<float4*>(st + lane * 256 + ((c ^ (lane & 15)) << 4)) =
+        make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int rr = 2 * i + (lane >> 4), c = lane & 15;
+    const float4 v = *reinterpret_cast<const float4*>(st + rr * 256 + ((c ^ (rr & 15)) << 4));
+    const int row = row_w0 + rr;
+    if (row < Lq) *reinterpret_cast<float4*>(base + (size_t)row * PF_DV + c * 4) = v;
+  }
+  __syncwarp();
+}
+
+// MODE: PF_INFER, PF_TRAIN (also the training outputs lse, o_maps) or
+// PF_SINGLE (single-map outputs in f32); a template argument so the inference
+// kernel carries none of the other modes' code.
+template <int DQK, int MODE = PF_INFER>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
                const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
   static_assert(DQK == 64 || DQK == 128, "QK width 64 or 128");
+  static_assert(sizeof(PfSmem<DQK>::k) + sizeof(PfSmem<DQK>::v) >= 8 * PF_STAGE_F32 &&
+                    offsetof(PfSmem<DQK>, v) == offsetof(PfSmem<DQK>, k) + sizeof(PfSmem<DQK>::k),
+                "the single-map epilogue stages 8 warps' rows in the contiguous K/V stages");
+  constexpr bool TRAIN = MODE == PF_TRAIN, SINGLE = MODE == PF_SINGLE;
   constexpr int QBOXES = DQK / 64;
   extern __shared__ uint8_t smem_raw[];
   PfSmem<DQK>& S = *reinterpret_cast<PfSmem<DQK>*>(
@@ -202,7 +239,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
   long long kend = a.causal ? (long long)min(r0 + PF_BM, a.Lq) - 1 + (a.Lk - a.Lq) + 1 : a.Lk;
   kend = max(0LL, min(kend, (long long)a.Lk));
   const int nT = (int)((kend + PF_BN - 1) / PF_BN);
-  const bool resid = fabsf(1.f - a.lambda[h]) < a.resid_tau;
+  // Residual choice per map: one lambda per output head, or in single-map
+  // mode each head's own.
+  const bool resid1 = fabsf(1.f - a.lambda[SINGLE ? 2 * h : h]) < a.resid_tau;
+  const bool resid2 = SINGLE ? fabsf(1.f - a.lambda[2 * h + 1]) < a.resid_tau : resid1;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&S.q_full), 1);
@@ -298,7 +338,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 #pragma unroll
             for (int s = 0; s < PF_BN / 16; ++s)
               mma_ts_w(o, p + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, (j > 0 || s > 0));
-            if (resid) {
+            if (m ? resid2 : resid1) {
 #pragma unroll
               for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
                 mma_ts_w(o, p + 32 + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, 1);
@@ -400,7 +440,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       // The residual choice is per head: branch once per tile, so each
       // variant's exp loop is one straight-line block the scheduler can
       // interleave across key pairs.
-      const float rowsum = resid ? pf_exp_store<true>(s, sc2, nm2, tS) : pf_exp_store<false>(s, sc2, nm2, tS);
+      const float rowsum =
+          (m ? resid2 : resid1) ? pf_exp_store<true>(s, sc2, nm2, tS) : pf_exp_store<false>(s, sc2, nm2, tS);
       l_run = l_run * alpha + rowsum;
       // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs
       // it (rows whose alpha is 1 multiply by 1).  O_m must be complete first:
@@ -427,7 +468,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 
     // --------------------------------------------------------- epilogue --
     // Rows that saw no key (l == 0) output zeros.
-    const float lam = a.lambda[h];
+    const float lam = SINGLE ? 0.f : a.lambda[h];
     float y[64];
     bool have = false;
     if (ok && nT > 0) {
@@ -435,7 +476,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       mbar_arrive(smem_u32(&S.xl));
       ok = warp_wait(smem_u32(&S.xl), 0, abort_flag, a.watch) &&
            warp_wait(smem_u32(&S.o_final), 0, abort_flag, a.watch);
-      if (ok) {
+      if (ok && SINGLE) {
+        tc_fence_after();
+        have = true;
+      } else if (ok) {
         tc_fence_after();
         const float l1 = S.l[0][r], l2 = S.l[1][r];
         const float c1 = l1 > 0.f ? 1.f / l1 : 0.f;
@@ -476,7 +520,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     }
     have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;   // warp-uniform (ok is)
     const int row_w0 = r0 + wq * 32;                          // first row of this warp
-    if (have)
+    if (have && !SINGLE)
       pf_store_rows(S.stage[warp], y, a.out + (((size_t)b * a.Hout + h) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq,
                     lane);
     // Training outputs: this map's log-sum-exp, and 64 columns of both
@@ -498,6 +542,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           for (int i = 0; i < 32; ++i) y[c * 32 + i] = nT > 0 ? __uint_as_float(o[i]) * inv : 0.f;
         }
         pf_store_rows(S.stage[warp], y, a.o_maps + ((stat + mm) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq, lane);
+      }
+    }
+    // Single-map outputs: 64 columns of each head's O_m / l_m in f32.  Every
+    // MMA has completed (o_final) and every K/V copy has been consumed, so the
+    // K/V stages are free: each warp stages its rows in 8 KB of them.
+    if (SINGLE && have) {
+      const size_t stat = ((size_t)b * a.Hout + h) * 2;
+      uint8_t* st = &S.k[0][0] + (size_t)warp * PF_STAGE_F32;
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm) {
+        const float inv = (nT > 0 && S.l[mm][r] > 0.f) ? 1.f / S.l[mm][r] : 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t o[32];
+          if (nT > 0) {
+            tmem_ld32p(tmem + lane_off + 256 + mm * 128 + m * 64 + c * 32, o);
+            tmem_wait_ld();
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[c * 32 + i] = nT > 0 ? __uint_as_float(o[i]) * inv : 0.f;
+        }
+        pf_store_rows_f32(st, y, a.o_f32 + ((stat + mm) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq, lane);
       }
     }
   }

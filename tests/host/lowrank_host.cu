@@ -6,7 +6,7 @@
 //
 // Input (little-endian): int32 B, H, Hkv, Lq, Lk, r, causal; then v bf16 bits
 // [B, Hkv, Lk, 128]; F f32 [H, Lq, r]; G f32 [H, Lk, r]; lambda f32 [H];
-// a1v bf16 bits [B, H, Lq, 128].  Output: out bf16 bits [B, H, Lq, 128].
+// a1v f32 [B, H, Lq, 128].  Output: out bf16 bits [B, H, Lq, 128].
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -32,8 +32,8 @@ int main(int argc, char** argv) {
   int32_t hdr[7];
   if (fread(hdr, sizeof(int32_t), 7, f) != 7) return 4;
   const int B = hdr[0], H = hdr[1], Hkv = hdr[2], Lq = hdr[3], Lk = hdr[4], r = hdr[5], causal = hdr[6];
-  std::vector<uint16_t> v, a1v;
-  std::vector<float> F, G, lam;
+  std::vector<uint16_t> v;
+  std::vector<float> F, G, lam, a1v;
   const size_t BH = (size_t)B * H;
   if (!read_n(f, v, (size_t)B * Hkv * Lk * da::LR_DV) || !read_n(f, F, (size_t)H * Lq * r) ||
       !read_n(f, G, (size_t)H * Lk * r) || !read_n(f, lam, (size_t)H) || !read_n(f, a1v, BH * Lq * da::LR_DV))
@@ -49,7 +49,7 @@ int main(int argc, char** argv) {
   a.F = F.data();
   a.G = G.data();
   a.lambda = lam.data();
-  a.a1v = reinterpret_cast<const __nv_bfloat16*>(a1v.data());
+  a.a1v = a1v.data();
   a.out = reinterpret_cast<__nv_bfloat16*>(out.data());
   a.tot = tot.data();
   a.ztot = ztot.data();

@@ -1,19 +1,14 @@
 """The low-rank substitute for A2 (out = A1 V - lambda N V, N fixed from
 positional factors) on the GPU against the fp64 oracle.  Needs a B200.
 
-A1 V runs on the prefill's training variant (heads in pairs over a KV head),
-which rounds P to bf16 and stores A1 V in bf16; N V runs on the scan kernels
-(their host runs are checked in tests/test_lowrank_host.py) in f32.
-
-Error bound.  The output is A1 V - lambda N V, and A1 V carries two bf16
-roundings (P and the stored value), each up to 2^-9 of A1 V's own scale.
-When N is close to A1 and lambda close to 1, the difference is small against
-A1 V and those roundings dominate it.  The bound is therefore the bf16 output
-bound, 2e-2 max|O_ref|, plus four roundings of A1 V, 2^-7 max|A1 V|; an error
-in the pairing, lambda, the head mapping or the workspace misses it by far.
-N V itself is checked tightly: two calls that differ only in lambda (0 and 1)
-share the same bf16 A1 V, so their difference is N V up to the rounding of the
-lambda = 1 output."""
+A1 V runs on the prefill's single-map mode (heads in pairs over a KV head),
+which writes each head's O / l in f32 and keeps the bf16 residual of P for
+heads with |1 - lambda| below the forward's threshold; N V runs on the scan
+kernels (their host runs are checked in tests/test_lowrank_host.py) in f32,
+and the subtraction is the only rounding to bf16.  Every comparison with the
+oracle uses the bf16 output bound alone, 2e-2 max|O_ref| per (batch, head)
+slice, including N close to A1 with lambda near 1, where the output is a
+small difference of two near-equal terms."""
 
 import math
 
@@ -39,18 +34,15 @@ def _case(B, H, Hkv, Lq, Lk, r, seed):
     return q, k, v, F, G, lam
 
 
-def _ratio(got, ref, a1v):
-    """Error over the bound 2e-2 max|O_ref| + 2^-7 max|A1 V| (<= 1 passes)."""
+def _ratio(got, ref):
+    """Error over the bound 2e-2 max|O_ref| (<= 1 passes)."""
     got = got.double().cpu().numpy()
-    bound = BF16_TOL * float(np.max(np.abs(ref))) + 2.0 ** -7 * float(np.max(np.abs(a1v)))
+    bound = BF16_TOL * float(np.max(np.abs(ref)))
     return float(np.max(np.abs(got - ref))) / bound if bound > 0 else float(np.max(np.abs(got)))
 
 
 def _oracle(q, k, v, F, G, lam, causal):
-    args = (q, k, v, F.cpu().numpy(), G.cpu().numpy())
-    ref = lr.diffattn_lowrank(*args, lam.cpu().numpy(), causal=causal)
-    a1v = lr.diffattn_lowrank(*args, np.zeros(lam.shape[0]), causal=causal)
-    return ref, a1v
+    return lr.diffattn_lowrank(q, k, v, F.cpu().numpy(), G.cpu().numpy(), lam.cpu().numpy(), causal=causal)
 
 
 CASES = [
@@ -70,51 +62,76 @@ def test_lowrank_matches_oracle(B, H, Hkv, Lq, Lk, r, causal):
     out = da.fwd_lowrank(q, k, v, F, G, lam, causal=causal)
     torch.cuda.synchronize()
     assert da.last_status() == da.OK
-    ref, a1v = _oracle(q, k, v, F, G, lam, causal)
+    ref = _oracle(q, k, v, F, G, lam, causal)
     assert torch.isfinite(out.float()).all()
     if Lk == 0:
         assert torch.all(out == 0)
         return
     for b in range(B):
         for h in range(H):
-            assert _ratio(out[b, h], ref[b, h], a1v[b, h]) <= 1.0, (b, h, _ratio(out[b, h], ref[b, h], a1v[b, h]))
+            assert _ratio(out[b, h], ref[b, h]) <= 1.0, (b, h, _ratio(out[b, h], ref[b, h]))
     again = da.fwd_lowrank(q, k, v, F, G, lam, causal=causal)
     assert torch.equal(out, again)                 # no atomics: bitwise repeatable
 
 
 @pytest.mark.parametrize("B,H,Hkv,Lq,Lk,r,causal", [c for c in CASES if c[4] > 0])
 def test_lowrank_nv_part_is_exact_to_the_output_rounding(B, H, Hkv, Lq, Lk, r, causal):
-    """out(lambda=0) - out(lambda=1) = N V: the bf16 A1 V is the same in both
-    calls, so the only rounding left is that of the lambda = 1 output (2^-9 of
-    its value), plus the fp32 sums over keys (2^-14 of N |V|).  One key too
-    many or too few in N V misses this bound."""
+    """(out(lambda=0) - out(lambda=64)) / 64 = N V: lambda = 0 and 64 make the
+    same residual choice (neither is near 1), so both calls share one f32
+    A1 V, and the only roundings left are the two bf16 outputs' (2^-9 of
+    each, divided by 64 here) and the fp32 sums over keys (2^-14 of N |V|).
+    One key too many or too few in N V misses this bound."""
     q, k, v, F, G, _ = _case(B, H, Hkv, Lq, Lk, r, seed=Lq + 3 * Lk + r + 1)
     out0 = da.fwd_lowrank(q, k, v, F, G, torch.zeros(H, device=DEV), causal=causal).double().cpu().numpy()
-    out1 = da.fwd_lowrank(q, k, v, F, G, torch.ones(H, device=DEV), causal=causal).double().cpu().numpy()
+    out64 = da.fwd_lowrank(q, k, v, F, G, torch.full((H,), 64.0, device=DEV), causal=causal).double().cpu().numpy()
     grp = H // Hkv
     vd = v.double().cpu().numpy()
     for b in range(B):
         for h in range(H):
             N = lr.noise_map(F[h].double().cpu().numpy(), G[h].double().cpu().numpy(), Lq, Lk, causal)
             nv, na = N @ vd[b, h // grp], N @ np.abs(vd[b, h // grp])
-            err = np.abs((out0[b, h] - out1[b, h]) - nv)
-            assert np.all(err <= 2.0 ** -8 * np.abs(out1[b, h]) + 2.0 ** -14 * na), (b, h, float(np.max(err)))
+            err = np.abs((out0[b, h] - out64[b, h]) / 64 - nv)
+            bound = 2.0 ** -8 * (np.abs(out0[b, h]) + np.abs(out64[b, h])) / 64 + 2.0 ** -14 * na
+            assert np.all(err <= bound), (b, h, float(np.max(err - bound)))
+
+
+def _uniform_case(H, Hkv, L, seed):
+    """r = 1, F = G = 1 (N = the uniform causal map) with small scores, so A1 is
+    close to N: (A1 - lambda N) V is a small difference of near-equal terms
+    when lambda is near 1."""
+    q, k, v, F, G, _ = _case(1, H, Hkv, L, L, 1, seed=seed)
+    return q, k, v, torch.ones_like(F), torch.ones_like(G)
 
 
 def test_lowrank_uniform_factors_reduce_to_the_prefix_mean():
     """r = 1, F = G = 1: N is the uniform causal map, so out = A1 V - lambda *
     (prefix mean of V); with lambda = 0 the output is plain attention."""
-    q, k, v, F, G, lam = _case(1, 2, 1, 333, 333, 1, seed=5)
-    ones_f, ones_g = torch.ones_like(F), torch.ones_like(G)
+    q, k, v, F, G = _uniform_case(2, 1, 333, seed=5)
     lam = torch.tensor([0.0, 1.0], device=DEV)
-    out = da.fwd_lowrank(q, k, v, ones_f, ones_g, lam, causal=True).double().cpu().numpy()
+    out = da.fwd_lowrank(q, k, v, F, G, lam, causal=True).double().cpu().numpy()
     vd = v[0, 0].double().cpu().numpy()
     prefix_mean = np.cumsum(vd, axis=0) / np.arange(1, 334)[:, None]
-    a1v = lr.diffattn_lowrank(q, k, v, ones_f.cpu().numpy(), ones_g.cpu().numpy(), np.zeros(2), causal=True)[0]
+    a1v = lr.diffattn_lowrank(q, k, v, F.cpu().numpy(), G.cpu().numpy(), np.zeros(2), causal=True)[0]
     assert np.max(np.abs(out[0, 0] - a1v[0])) <= BF16_TOL * np.max(np.abs(a1v[0]))
-    # lambda = 1 cancels the mean part: the bound is relative to A1 V (see the module notes)
     want = a1v[1] - prefix_mean
-    assert np.max(np.abs(out[0, 1] - want)) <= BF16_TOL * np.max(np.abs(want)) + 2.0 ** -7 * np.max(np.abs(a1v[1]))
+    assert np.max(np.abs(want)) < 0.05 * np.max(np.abs(a1v[1]))    # the case is a near-cancellation
+    assert np.max(np.abs(out[0, 1] - want)) <= BF16_TOL * np.max(np.abs(want))
+
+
+@pytest.mark.parametrize("L", [777, 4096])
+def test_lowrank_near_unit_lambda_with_n_close_to_a1(L):
+    """N close to A1 and lambda in {0.97, 1, 1.03}: every head within the bf16
+    output bound of the oracle, relative to its own (small) output."""
+    q, k, v, F, G = _uniform_case(4, 2, L, seed=L)
+    lam = torch.tensor([0.97, 1.0, 1.03, 1.0], device=DEV)
+    out = da.fwd_lowrank(q, k, v, F, G, lam, causal=True)
+    torch.cuda.synchronize()
+    assert da.last_status() == da.OK
+    ref = _oracle(q, k, v, F, G, lam, True)
+    a1v = _oracle(q, k, v, F, G, torch.zeros(4, device=DEV), True)
+    for h in range(4):
+        assert np.max(np.abs(ref[0, h])) < 0.1 * np.max(np.abs(a1v[0, h]))   # a near-cancellation
+        assert _ratio(out[0, h], ref[0, h]) <= 1.0, (h, _ratio(out[0, h], ref[0, h]))
 
 
 def test_lowrank_full_size_sampled():
@@ -125,9 +142,7 @@ def test_lowrank_full_size_sampled():
     torch.cuda.synchronize()
     assert da.last_status() == da.OK
     assert torch.isfinite(out.float()).all()
-    b, h = 1, 13
-    g = h // (H // Hkv)
-    args = (q[b, h], k[b, g], v[b, g], F[h].cpu().numpy(), G[h].cpu().numpy())
-    ref = lr.lowrank_head(*args, float(lam[h]), True)
-    a1v = lr.lowrank_head(*args, 0.0, True)
-    assert _ratio(out[b, h], ref, a1v) <= 1.0
+    for b, h in ((1, 13), (0, 31)):
+        g = h // (H // Hkv)
+        ref = lr.lowrank_head(q[b, h], k[b, g], v[b, g], F[h].cpu().numpy(), G[h].cpu().numpy(), float(lam[h]), True)
+        assert _ratio(out[b, h], ref) <= 1.0, (b, h)

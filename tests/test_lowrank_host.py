@@ -2,8 +2,8 @@
 (tests/host/lowrank_host.cu includes the library's lowrank.cuh), against the
 fp64 oracle of the fixed low-rank substitute for A2.  No GPU.
 
-The harness takes A1 V as an input and returns out = A1 V - lambda N V in
-bf16.  The checks are per element: with A1 V = 0 and lambda = 1, N V is
+The harness takes A1 V as an f32 input (the prefill writes it in f32) and
+returns out = A1 V - lambda N V in bf16, its only rounding to bf16.  The checks are per element: with A1 V = 0 and lambda = 1, N V is
 within two bf16 roundings of its own value plus the fp32 summation bound
 (one key too many or too few shows), and so is the combination.
 That covers the chunk boundaries, the causal offset on both sides (Lq < Lk,
@@ -53,7 +53,7 @@ def _run(exe, tmp_path, B, H, Hkv, Lq, Lk, r, causal, v, F, G, lam, a1v):
         f.write(np.ascontiguousarray(F, dtype=np.float32).tobytes())
         f.write(np.ascontiguousarray(G, dtype=np.float32).tobytes())
         f.write(np.ascontiguousarray(lam, dtype=np.float32).tobytes())
-        f.write(_bf16_bits(a1v).tobytes())
+        f.write(np.ascontiguousarray(a1v, dtype=np.float32).tobytes())
     res = subprocess.run([exe, str(fin), str(fout)], capture_output=True, text=True)
     assert res.returncode == 0, (res.returncode, res.stderr)
     bits = np.fromfile(fout, dtype=np.int16).reshape(B, H, Lq, 128)
@@ -94,7 +94,7 @@ def test_scan_matches_oracle(harness, tmp_path, B, H, Hkv, Lq, Lk, r, causal):
     assert np.all(err <= 2.0 ** -8 * np.abs(NV) + 2.0 ** -14 * NA), float(np.max(err - 2.0 ** -8 * np.abs(NV)))
     # the combination with A1 V and lambda
     lam = np.linspace(-0.3, 1.2, H).astype(np.float32)
-    a1v = _bf16_values(rng.standard_normal((B, H, Lq, 128)) * 0.2)   # stands in for A1 V
+    a1v = (rng.standard_normal((B, H, Lq, 128)) * 0.2).astype(np.float32).astype(np.float64)   # stands in for A1 V
     got = _run(harness, tmp_path, B, H, Hkv, Lq, Lk, r, causal, v, F, G, lam, a1v)
     lam64 = lam[None, :, None, None].astype(np.float64)
     want = a1v - lam64 * NV
@@ -102,8 +102,8 @@ def test_scan_matches_oracle(harness, tmp_path, B, H, Hkv, Lq, Lk, r, causal):
     if Lk == 0 or (causal and Lq > Lk):
         # rows without a visible key keep A1 V unchanged
         first = Lq if Lk == 0 else Lq - Lk
-        assert np.array_equal(got[:, :, :first], a1v[:, :, :first])
-    assert np.array_equal(got[:, 0, min(5, Lq - 1)], a1v[:, 0, min(5, Lq - 1)])
+        assert np.array_equal(got[:, :, :first], _bf16_values(a1v[:, :, :first]))
+    assert np.array_equal(got[:, 0, min(5, Lq - 1)], _bf16_values(a1v[:, 0, min(5, Lq - 1)]))
 
 
 def test_whole_substitute_against_oracle(harness, tmp_path):
@@ -120,3 +120,25 @@ def test_whole_substitute_against_oracle(harness, tmp_path):
     got = _run(harness, tmp_path, B, H, Hkv, L, L, r, True, v, F, G, lam, a1v)
     ref = lr.diffattn_lowrank(q, k, v, F, G, lam, causal=True)
     assert np.max(np.abs(got - ref)) <= 2e-2 * np.max(np.abs(ref))
+
+
+def test_near_cancellation_keeps_f32_precision(harness, tmp_path):
+    """A1 V close to N V and lambda = 1: the output is a small difference of two
+    near-equal terms.  With A1 V in f32 its error is the fp32 sums' (about
+    Lk 2^-24 of N |V|) plus the one bf16 rounding of the output, far inside
+    2e-2 of the output's own scale; a bf16 A1 V (2^-9 of its value) would not
+    be."""
+    rng = np.random.default_rng(7)
+    B, H, Hkv, L, r = 1, 2, 1, 600, 1
+    v = _bf16_values(rng.standard_normal((B, Hkv, L, 128)) / np.sqrt(128))
+    F, G = np.ones((H, L, r), np.float32), np.ones((H, L, r), np.float32)   # N = the causal mean
+    N = lr.noise_map(F[0].astype(np.float64), G[0].astype(np.float64), L, L, True)
+    nv = N @ v[0, 0]
+    small = rng.standard_normal((B, H, L, 128)) * 1e-3 * np.abs(nv).max()
+    a1v = (nv[None, None] + small).astype(np.float32).astype(np.float64)
+    got = _run(harness, tmp_path, B, H, Hkv, L, L, r, True, v, F, G, np.ones(H, np.float32), a1v)
+    want = a1v - nv[None, None]
+    assert np.max(np.abs(got - want)) <= 2e-2 * np.max(np.abs(want))
+    # the same output through a bf16 A1 V misses that bound
+    coarse = _bf16_values(a1v) - nv[None, None]
+    assert np.max(np.abs(coarse - want)) > 2e-2 * np.max(np.abs(want))
