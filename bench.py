@@ -3,10 +3,11 @@
 
 One step = the whole hot path for one batch of the primary workload: the
 per-head lambda kernel, then the prefill kernel (default workload: V2 causal
-prefill, B2 Hq64 Hkv8 N8192 D128 bf16, layer 24).  The other hot-path
-workloads (V1 prefill with RMSNorm, V2 64k decode, V1-layout 64k decode fused
-and unfused) are timed the same way and reported under "secondary".  The
-SNR-vs-context-length sweep (``--workload snr_sweep``) runs on request only.
+prefill, B2 Hq64 Hkv8 N8192 D128 bf16, layer 24).  The other workloads (V1
+prefill with RMSNorm, both backwards, V2 64k decode contiguous and paged, a
+serving-shaped paged decode, V1-layout 64k decode fused and unfused, the
+low-rank forward and the SNR-vs-context-length sweep) are timed the same way
+and reported, one compact row each, under "secondary" at the end of the line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl reference] [--no-cpu-baseline] [--no-secondary]
@@ -86,52 +87,66 @@ def measured_peaks():
 
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, read through NVML every few
+    milliseconds on a background thread (reads only; no setting is touched).
+    ``summary(t0, t1)`` summarises the samples taken between two host
+    perf_counter() times, so a timed region of a few tens of milliseconds has
+    a clock record of its own."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.dev, self.period = device_index, period_s
+        self.samples, self.max_mhz, self.nv, self._stop = [], None, None, None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+                h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = nv.nvmlDeviceGetHandleByIndex(self.dev)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+        except Exception:
+            return self
+        self.nv, self._stop = nv, threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.perf_counter(), mhz, [n for n, bit in bits if r & bit]))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join()
             try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+    def summary(self, t0=None, t1=None):
+        sel = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
+        return {"sm_mhz": statistics.median(x[1] for x in sel), "sm_min_mhz": min(x[1] for x in sel),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted({n for x in sel for n in x[2]}), "samples": len(sel),
+                "source": "nvml"}
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -268,6 +283,40 @@ class PagedDecode:
                                   host["seq_lens"], lam)
 
 
+class ServingDecode:
+    """A serving-shaped paged V2 decode: 256 sequences of mixed lengths
+    (16..4096 tokens) in a shared pool of 16-token pages, one query token each."""
+
+    def __init__(self, device, shape=None):
+        self.shape = dict(inputs.SERVING_SHAPE if shape is None else shape)
+        sh = self.shape
+        self.x = inputs.serving_cache(**sh, device=device)
+        self.tokens = int(self.x["seq_lens"].sum())
+        gen = torch.Generator(device=device).manual_seed(1014)
+        self.lp = tuple(torch.randn(sh["Hq"] // 2, 128, generator=gen, device=device) * 0.1 for _ in range(4))
+        self.init = da.lambda_init(24)
+        self.lam = torch.empty(sh["Hq"] // 2, dtype=torch.float32, device=device)
+        self.out = torch.empty((sh["B"], sh["Hq"] // 2, 128), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(da.decode_paged_workspace_size(sh["B"], sh["Hkv"]), dtype=torch.uint8, device=device)
+        self.launches_per_step = 3
+
+    def step(self, ev=None):
+        x = self.x
+        da.compute_lambda(*self.lp, self.init, out=self.lam)
+        if ev is not None:
+            ev[0].record()
+        da.decode_v2_paged(x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"], self.lam,
+                           out=self.out, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def work(self):
+        """Bytes of the K and V tokens the sequences hold, each read once."""
+        return self.tokens * self.shape["Hkv"] * (128 + 128) * 2 / 1e9, "GB/s"
+
+    host_path = "the serving-shaped decode is timed on device tensors only"
+
+
 def backward_flops(w) -> float:
     """Executed-minimum FLOP of the backward: five contractions per map and
     visible (row, key) pair -- S (2d), dP (2dv), dV (2dv), dQ (2d), dK (2d) --
@@ -361,6 +410,11 @@ class SnrSweep:
         return [noise.summarize(N, o[0][:, 0, 0].float(), o[0][:, 0, 1].float(), o[1][:, 0, 0].float(),
                                 o[1][:, 0, 1].float()) for N, o in zip(self.lengths, self.outs)]
 
+    def compact_summary(self):
+        """Medians per context length: [N, SNR plain, SNR difference, plain noise fraction]."""
+        return [[r["N"], float(f"{r['snr_plain'][1]:.4g}"), float(f"{r['snr_diff'][1]:.4g}"),
+                 float(f"{r['noise_fraction_plain'][1]:.4g}")] for r in self.summary()]
+
     host_path = "the sweep is timed on device tensors only"
 
 
@@ -408,6 +462,8 @@ class LowRank:
 
 def workload_work(name):
     """(algorithmic work of one step, unit) of a bench workload."""
+    if name == "v2_decode_serving":
+        return None, "GB/s"     # set by the drawn lengths (ServingDecode.work)
     if name == "snr_sweep":
         return sweep_bytes() / 1e9, "GB/s"
     if name == "lowrank_prefill":
@@ -427,6 +483,8 @@ def base_workload(name):
 
 
 def make_runner(name, device):
+    if name == "v2_decode_serving":
+        return ServingDecode(device)
     if name == "snr_sweep":
         return SnrSweep(device)
     if name == "lowrank_prefill":
@@ -442,6 +500,12 @@ def make_runner(name, device):
 
 
 def describe(name):
+    if name == "v2_decode_serving":
+        sh = inputs.SERVING_SHAPE
+        return {"workload": name, "layout": "v2_decode", "B": sh["B"], "heads": sh["Hq"], "kv_heads": sh["Hkv"],
+                "Lq": 1, "Lk": f"uniform {sh['min_len']}..{sh['max_len']}", "d": 128, "dv": 128, "layer": 24,
+                "mode": f"paged: shuffled pool of {sh['page_size']}-token pages, mixed lengths",
+                "l2": "caches larger than L2 (126 MB): no flush between steps"}
     if name == "lowrank_prefill":
         sh = inputs.LOWRANK_SHAPE
         return {"workload": name, "layout": "one Q head per output head", "B": sh["B"], "heads": sh["H"],
@@ -472,7 +536,11 @@ def describe(name):
 
 
 # ----------------------------------------------------------------------------- timing
-def time_runner(r, steps, warmup, dist_on):
+def time_runner(r, steps, warmup, dist_on, window=None):
+    """W untimed steps, then K steps bracketed by a barrier and a synchronize
+    on both sides; CUDA events on the launching stream give the whole region
+    and each step's dominant launch.  ``window``, a list, receives the host
+    perf_counter() times around the timed region (for the clock record)."""
     for _ in range(warmup):
         r.step()
     torch.cuda.synchronize()
@@ -481,13 +549,17 @@ def time_runner(r, steps, warmup, dist_on):
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    t0 = time.perf_counter()
     start.record()
     for i in range(steps):
         r.step(kev[i])
     end.record()
     torch.cuda.synchronize()
+    t1 = time.perf_counter()
     if dist_on:
         torch.distributed.barrier()
+    if window is not None:
+        window[:] = [t0, t1]
     total_ms = start.elapsed_time(end)
     kern_ms = sum(a.elapsed_time(b) for a, b in kev) / steps
     return total_ms, kern_ms
@@ -547,30 +619,52 @@ def e2e_measure(r, steps):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+SPEC_HBM_GBS = 8000.0   # the HBM3e figure the decode target is stated against (~8 TB/s)
+
+
 def roofline(r, kern_ms, peaks, power_capped=False, name=None):
     """Achieved work rate of the step's dominant kernel against the measured peak.
 
-    A tensor-bound kernel is compared with the cuBLAS bf16 figure measured in the
-    same regime: the sustained (power-capped) one when the clock record of the
-    timed region shows sw_power_cap, else the burst one; the fraction of the
-    burst figure is reported beside it either way.  traffic: the DRAM bytes of
-    one launch from the kernel's ncu capture, scaled to this batch (None
-    without a capture of the current kernel)."""
+    A tensor-bound kernel is compared with the measured burst cuBLAS bf16
+    figure: each prefill launch lasts a few milliseconds and is timed on its
+    own, which is the burst regime (a power cap seen on the clocks is a note,
+    not another roofline).  The fraction of the sustained figure is kept as a
+    side field.  An HBM-bound kernel is compared with the measured copy
+    bandwidth; a read-only stream can run above a read+write copy, so the
+    fraction of the ~8 TB/s HBM3e figure is given beside it.  traffic: the
+    DRAM bytes of one launch from the kernel's ncu capture, scaled to this
+    batch (None without a capture of the current kernel)."""
     work, unit = r.work()
     w = getattr(r, "w", None)
     traffic = measured_traffic(name, w.B) if (name is not None and w is not None) else None
-    if unit == "TFLOP/s":
-        ach = work / (kern_ms / 1e3)
-        sustained = power_capped and peaks.get("bf16_tflops_sustained")
-        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-        kind = "sustained (power-capped)" if sustained else "burst"
-        return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                "traffic": traffic, "peak_kind": f"{peaks['source']} {kind} cuBLAS bf16",
-                "frac_of_burst": ach / peaks["bf16_tflops"], "kernel_ms": kern_ms}
     ach = work / (kern_ms / 1e3)
+    if unit == "TFLOP/s":
+        peak = peaks["bf16_tflops"]
+        out = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+               "traffic": traffic, "peak_kind": f"{peaks['source']} burst cuBLAS bf16", "kernel_ms": kern_ms}
+        if peaks.get("bf16_tflops_sustained"):
+            out["frac_of_sustained"] = ach / peaks["bf16_tflops_sustained"]
+        if power_capped:
+            out["note"] = "sw_power_cap seen during the timed region"
+        return out
     peak = peaks["hbm_gbs"]
-    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
-            "peak_kind": f"{peaks['source']} HBM copy", "kernel_ms": kern_ms}
+    out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
+           "peak_kind": f"{peaks['source']} HBM copy (read+write)", "frac_of_8tbs": ach / SPEC_HBM_GBS,
+           "kernel_ms": kern_ms}
+    if ach > peak:
+        out["note"] = "read-only stream above the read+write copy figure"
+    return out
+
+
+def compact(name, r, total_ms, kern_ms, steps, rf):
+    """One secondary row: [value, unit, ms_per_step, kernel_ms, frac, frac_of_8tbs or None]."""
+    work, unit = r.work()
+    ms = total_ms / steps
+    return [round(work / (ms / 1e3), 2), unit, round(ms, 4), round(kern_ms, 4), round(rf["frac"], 4),
+            round(rf["frac_of_8tbs"], 4) if "frac_of_8tbs" in rf else None]
+
+
+SECONDARY_COLS = ["value", "unit", "ms_per_step", "kernel_ms", "frac", "frac_of_8tbs"]
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
@@ -631,6 +725,33 @@ def cpu_oracle_sweep(cores, budget_s):
             "seconds": t_total}
 
 
+@functools.lru_cache(maxsize=1)
+def _serving_host_inputs():
+    return inputs.serving_cache(**inputs.SERVING_SHAPE)
+
+
+def cpu_oracle_serving(cores, budget_s):
+    """The oracle's paged decode on whole sequences of the serving batch, in
+    order; bytes counted as on the GPU (the sequence's K and V tokens)."""
+    import numpy as np
+    from oracle import diffattn as orc
+    x = _serving_host_inputs()
+    sh = inputs.SERVING_SHAPE
+    lam = np.full(sh["Hq"] // 2, 0.5)
+    done, t_total, n = 0.0, 0.0, 0
+    for b in range(sh["B"]):
+        t0 = time.perf_counter()
+        orc.decode_v2_paged(x["q"][b:b + 1], x["k_pages"], x["v_pages"], x["block_table"][b:b + 1],
+                            x["seq_lens"][b:b + 1], lam)
+        t_total += time.perf_counter() - t0
+        done += int(x["seq_lens"][b]) * sh["Hkv"] * 256 * 2 / 1e9
+        n += 1
+        if t_total >= budget_s:
+            break
+    return {"value": done / t_total, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {sh['B']} sequences in order, fp64 NumPy", "seconds": t_total}
+
+
 def cpu_oracle_run(name, budget_s=12.0):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload.
 
@@ -646,6 +767,8 @@ def cpu_oracle_run(name, budget_s=12.0):
         cores = len(os.sched_getaffinity(0))
     if name == "snr_sweep":
         return cpu_oracle_sweep(cores, budget_s)
+    if name == "v2_decode_serving":
+        return cpu_oracle_serving(cores, budget_s)
     if name == "lowrank_prefill":
         return cpu_oracle_lowrank(cores, budget_s)
     paged, backward = name == "v2_decode_paged", name.endswith("_backward")
@@ -729,7 +852,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="v2_prefill",
                     choices=["v2_prefill", "v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged",
-                             "v1_decode", "v1_decode_unfused", "snr_sweep", "lowrank_prefill"])
+                             "v2_decode_serving", "v1_decode", "v1_decode_unfused", "snr_sweep", "lowrank_prefill"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
@@ -737,7 +860,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size of the workload (smaller profiling cases)")
     args = ap.parse_args()
-    if args.batch is not None and args.workload not in ("snr_sweep", "lowrank_prefill"):
+    if args.batch is not None and args.workload not in ("snr_sweep", "lowrank_prefill", "v2_decode_serving"):
         base = base_workload(args.workload)
         inputs.WORKLOADS[base] = inputs.with_shape(inputs.WORKLOADS[base], B=args.batch)
 
@@ -757,12 +880,20 @@ def main():
         cb = dict(res[-1])
         cb["value"] = v
         unit = cb["unit"]
+        # One step is one bounded sample of the workload: ms_per_step is its
+        # measured duration; the time the whole workload would take at this
+        # rate is extrapolated and labelled so.
+        ms_step = statistics.mean(r["seconds"] for r in res) * 1e3
         work_unit = workload_work(args.workload)[0]
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
-                "steps": steps, "warmup": args.warmup, "ms_per_step": work_unit / v * 1e3,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": describe(args.workload), "cpu_baseline": cb,
-                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                "data": "synthetic", "config": dict(describe(args.workload), parallelism="single GPU"),
+                "cpu_baseline": cb,
+                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                "step": "one bounded sample of the workload per step (see cpu_baseline.sample)"}
+        if work_unit:
+            line["full_workload_ms_extrapolated"] = work_unit / v * 1e3
         print(json.dumps(line))
         return 0
 
@@ -778,33 +909,45 @@ def main():
     peaks = measured_peaks()
 
     r = make_runner(args.workload, device)
-    with ClockSampler(local) as clk:
-        # untimed steps before and after keep the GPU under load long enough
-        # (>= ~0.4 s each side) for the 200 ms clock samples to cover the timed steps
-        keep_busy(r, 0.4)
-        total_ms, kern_ms = time_runner(r, args.steps, args.warmup, dist_on)
-        keep_busy(r, 0.4)
+    win, win_s = [], []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        # The headline region starts from the warm-up alone: a few tens of
+        # milliseconds, the regime of a launch timed on its own (burst).
+        total_ms, kern_ms = time_runner(r, args.steps, args.warmup, dist_on, win)
+        # Then the same steps after a second of continuous load, where a
+        # power cap may hold the clock lower (sustained), reported beside it.
+        keep_busy(r, 1.0)
+        sus_total, sus_kern = time_runner(r, args.steps, 0, dist_on, win_s)
     total_ms = max_over_ranks(total_ms, dist_on)
+    sus_total = max_over_ranks(sus_total, dist_on)
     ms = total_ms / args.steps
     work, unit = r.work()
     value = aggregate(work, world, ms)
-    clocks = clk.summary()
+    clocks = clk.summary(*win) if win else clk.summary()
+    clocks_s = clk.summary(*win_s) if win_s else clk.summary()
     capped = "sw_power_cap" in clocks["reasons"]
     rf = roofline(r, kern_ms, peaks, capped, args.workload)
+    rf_s = roofline(r, sus_kern, peaks, "sw_power_cap" in clocks_s["reasons"], args.workload)
+    sustained = {"value": aggregate(work, world, sus_total / args.steps), "ms_per_step": sus_total / args.steps,
+                 "kernel_ms": sus_kern, "frac": rf_s.get("frac_of_sustained", rf_s["frac"]),
+                 "peak_kind": "sustained cuBLAS bf16" if unit == "TFLOP/s" else rf_s["peak_kind"],
+                 "sm_mhz": clocks_s["sm_mhz"], "reasons": clocks_s["reasons"]}
 
-    secondary = {}
+    secondary, snr = {}, None
+    if isinstance(r, SnrSweep):
+        snr = r.compact_summary()
     if not args.no_secondary and rank == 0 and not dist_on:
-        names = ["v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged", "v1_decode", "v1_decode_unfused",
-                 "v2_prefill"]
+        names = ["v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged", "v2_decode_serving",
+                 "v1_decode", "v1_decode_unfused", "lowrank_prefill", "snr_sweep", "v2_prefill"]
+        n2 = max(3, args.steps // 2)
         for name in names:
             if name == args.workload:
                 continue
             r2 = make_runner(name, device)
-            t2, k2 = time_runner(r2, max(3, args.steps // 2), args.warmup, False)
-            wk, un = r2.work()
-            secondary[name] = {"value": wk / (t2 / max(3, args.steps // 2) / 1e3), "unit": un,
-                               "ms_per_step": t2 / max(3, args.steps // 2), "roofline": roofline(r2, k2, peaks, capped, name),
-                               "config": describe(name)}
+            t2, k2 = time_runner(r2, n2, args.warmup, False)
+            secondary[name] = compact(name, r2, t2, k2, n2, roofline(r2, k2, peaks, capped, name))
+            if isinstance(r2, SnrSweep):
+                snr = r2.compact_summary()
             del r2
             torch.cuda.empty_cache()
 
@@ -821,13 +964,15 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(d) inputs on device)",
             "config": dict(describe(args.workload), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "roofline": rf, "e2e": e2e, "gpu_launches": r.launches_per_step * args.steps,
-            "clocks": clocks}
-    if secondary:
-        line["secondary"] = secondary
-    if isinstance(r, SnrSweep):
-        line["snr"] = r.summary()
+            "clocks": clocks, "sustained": sustained}
     if rank == 0 and not args.no_cpu_baseline and not dist_on:
         line["cpu_baseline"] = cpu_oracle_run(args.workload)
+    if snr is not None:
+        line["snr_cols"] = ["N", "snr_plain_median", "snr_diff_median", "noise_fraction_plain_median"]
+        line["snr"] = snr
+    if secondary:   # last, so that a reader keeping only the end of the line keeps every row
+        line["secondary_cols"] = SECONDARY_COLS
+        line["secondary"] = secondary
     if rank == 0:
         print(json.dumps(line))
     if dist_on:

@@ -29,7 +29,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR
 F32, BF16 = 0, 1
 
 EXPORTS = ["diffattn_version", "diffattn_lambda_init", "diffattn_lambda", "diffattn_fwd_v1", "diffattn_fwd_v2",
-           "diffattn_decode_workspace_size", "diffattn_decode_v2", "diffattn_decode_v1", "diffattn_last_error",
+           "diffattn_decode_workspace_size", "diffattn_decode_v2_workspace_size", "diffattn_decode_v2",
+           "diffattn_decode_v1", "diffattn_last_error",
            "diffattn_last_status", "diffattn_set_wait_limit_ns", "diffattn_decode_v2_noalloc",
            "diffattn_decode_paged_workspace_size", "diffattn_decode_v2_paged", "diffattn_fwd_v2_train",
            "diffattn_bwd_v2_workspace_size", "diffattn_bwd_v2", "diffattn_lambda_backward",
@@ -62,6 +63,7 @@ def load():
         "diffattn_fwd_v1": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P]),
         "diffattn_fwd_v2": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, P]),
         "diffattn_decode_workspace_size": (Z, [I, I, I, I]),
+        "diffattn_decode_v2_workspace_size": (Z, [I, I, I, I]),
         "diffattn_decode_v2": (I, [P, P, P, P, P, I, I, I, I, I, I, P, Z, P]),
         "diffattn_decode_v1": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]),
         "diffattn_last_error": (ctypes.c_char_p, []),

@@ -435,7 +435,15 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   const int rb0 = (a.causal && k0 - off > 0) ? (k0 - off) / BW_RB : 0;
   const int n_rb = (a.Lq + BW_RB - 1) / BW_RB;
   const int per_head = max(0, n_rb - rb0);
-  const int nS = grp * per_head;   // steps: (head of the group, row block)
+  const int nS = grp * per_head;
+  // Steps: (row block, head of the group), heads innermost.  The CTAs of one
+  // group start at different row blocks (the first row that sees their keys)
+  // and then advance one row block per grp steps, so they stay a fixed
+  // distance apart and each Q / dO tile is read from DRAM about once and
+  // from L2 by the others; with the heads outermost they drift onto different
+  // heads and each re-reads its tiles.
+  auto step_head = [&](int i) { return g * grp + i % grp; };
+  auto step_rb = [&](int i) { return rb0 + i / grp; };
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&S.kv_full), 1);
@@ -476,7 +484,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       for (int i = 0; i < nS; ++i) {
         const int st = i % BW_NS, use = i / BW_NS;
         if (use > 0 && !wait_bar(smem_u32(&S.st_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
-        const int qh = g * grp + i / per_head, rb = rb0 + i % per_head;
+        const int qh = step_head(i), rb = step_rb(i);
         const int hq = qh / 2, mq = qh & 1;
         const uint32_t fb = smem_u32(&S.st_full[st]);
         mbar_expect_tx(fb, 4 * PF_KBOX + 2 * BW_RB * 4);
@@ -510,7 +518,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
           tc_fence_after();
           const uint32_t olo = o_mn0 + (uint32_t)st * QSTAGE, qlo = q_mn0 + (uint32_t)st * QSTAGE;
-          const int qh = g * grp + i / per_head;
+          const int qh = step_head(i);
           const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
 #pragma unroll
           for (int s = 0; s < BW_RB / 16; ++s)   // dV += (w P)^T dO
@@ -572,7 +580,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     bool ok = true;
     for (int i = 0; i < nS; ++i) {
       const int bb = i & 1, st = i % BW_NS;
-      const int qh = g * grp + i / per_head, rb = rb0 + i % per_head;
+      const int qh = step_head(i), rb = step_rb(i);
       const int mq = qh & 1;
       const float w = mq == 0 ? 1.f : -a.lambda[qh / 2];   // weight of this map in A_1 - lambda A_2
       const float cd = a.scale * w;

@@ -6,10 +6,12 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -188,6 +190,21 @@ int launch_simt(const SimtArgs& a, cudaStream_t s) {
   return ok();
 }
 
+// Launch order of the prefill's row blocks (see PrefillArgs::rb_group).  When
+// every output head has K/V of its own (V1 without GQA: 2 MB of K1, K2 and V
+// per head at N = 4096, 256 MB over the workload's 128 heads), row blocks of
+// one head launched BH CTAs apart find its K/V evicted from L2; grouping 4 row
+// blocks of a head keeps them co-resident.  With GQA the output heads of a KV
+// group are already adjacent.  DIFFATTN_PREFILL_RB_GROUP overrides the choice.
+int prefill_rb_group(bool v1, int Hq, int Hkv, int n_rb) {
+  int r = (v1 && Hq == Hkv) ? 4 : 1;
+  if (const char* e = std::getenv("DIFFATTN_PREFILL_RB_GROUP")) {
+    const int x = std::atoi(e);
+    if (x >= 1) r = x;
+  }
+  return std::max(1, std::min(r, std::max(1, n_rb)));
+}
+
 int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
                    const float* lambda, void* out, int B, int Hout, int Hq, int Hkv, int Lq, int Lk, int dqk,
                    bool v1, int causal, int rms, float eps, cudaStream_t s, float* lse = nullptr,
@@ -213,6 +230,7 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.eps = eps;
   a.scale_log2 = log2e_over_sqrt(dqk);
   a.n_rb = (Lq + PF_BM - 1) / PF_BM;
+  a.rb_group = prefill_rb_group(v1, Hq, Hkv, a.n_rb);
   a.resid_tau = DIFFATTN_RESID_TAU;
   a.watch = make_watch(dev);
   a.lse = lse;
@@ -510,7 +528,7 @@ int launch_decode_paged(const void* q, const void* kp, const void* vp, const int
 
 // Scratch for diffattn_decode_v2_noalloc: split-KV partial records of the
 // decode, for callers that cannot allocate device memory.  One copy per
-// device, reserved when the library is loaded and kept until exit.  Host code
+// device, reserved when the module is first loaded on it and kept until exit.  Host code
 // must not pass `g_noalloc_scratch` itself to a kernel (on the host it names a
 // stand-in, not device memory): it uses the address looked up below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DIFFATTN_NOALLOC_SCRATCH_BYTES];
@@ -632,6 +650,17 @@ size_t diffattn_decode_workspace_size(int B, int Hkv, int T, int dv) {
   DeviceInfo* dev = nullptr;
   if (device_setup(&dev)) return 0;
   return plan_decode(dev->sms, B, Hkv, T).bytes_per_pass * 2;  // room for the two-pass V1 comparison
+}
+
+size_t diffattn_decode_v2_workspace_size(int B, int Hq, int T, int D) {
+  if (B < 0 || Hq < 2 || Hq % 2 || T < 0 || D < 1) return 0;
+  size_t best = 0;
+  for (int Hkv = 1; Hkv <= Hq / 2; ++Hkv)
+    if (Hq % Hkv == 0 && (Hq / Hkv) % 2 == 0 && Hq / Hkv <= 8) {
+      const size_t n = diffattn_decode_workspace_size(B, Hkv, T, D);
+      if (n > best) best = n;
+    }
+  return best;
 }
 
 int diffattn_decode_v2(const void* q, const void* kc, const void* vc, const float* lambda, void* out,

@@ -55,6 +55,7 @@ struct PrefillArgs {
   int causal, rms;
   float eps, scale_log2;
   int n_rb;             // row blocks per head
+  int rb_group;         // launch order: groups of rb_group row blocks of one head are adjacent (>= 1)
   // Precision policy: P is stored as bf16 P_hi plus a bf16 residual P_lo (a
   // second PV MMA) for heads with |1 - lambda| < resid_tau.  The difference
   // O1/l1 - lambda*O2/l2 amplifies P's bf16 rounding (2^-9) by about
@@ -225,10 +226,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &S.abort_flag;
 
-  // ---- work unit: heaviest row blocks first (causal) ----
+  // ---- work unit: heaviest row blocks first (causal), in groups of
+  // rb_group row blocks of one head that are adjacent in the launch order, so
+  // that co-resident CTAs of a head read its K/V tiles together from L2 ----
   const int BH = a.B * a.Hout;
-  const int rb = a.n_rb - 1 - (int)(blockIdx.x / BH);
-  const int bh = (int)(blockIdx.x % BH);
+  int rb, bh;
+  {
+    const int R = a.rb_group, n_full = a.n_rb / R;
+    const long long idx = blockIdx.x, in_full = (long long)n_full * R * BH;
+    if (idx < in_full) {
+      const int rg = (int)(idx / ((long long)R * BH)), rem = (int)(idx % ((long long)R * BH));
+      bh = rem / R;
+      rb = a.n_rb - 1 - (rg * R + rem % R);
+    } else {                                   // the last n_rb % R row blocks
+      const int rr = a.n_rb - n_full * R, rem = (int)(idx - in_full);
+      bh = rem / rr;
+      rb = a.n_rb - 1 - (n_full * R + rem % rr);
+    }
+  }
   const int b = bh / a.Hout, h = bh % a.Hout;
   const int r0 = rb * PF_BM;
   int qh1, qh2, g;

@@ -25,6 +25,10 @@ Workloads (shapes, value distributions):
                V2 prefill's attention shape with one Q head per output head:
                B2 H32 Hkv8 N8192 D128 causal, N(0,1)/sqrt(128); positional
                factors F [H, N, r], G [H, N, r] ~ U(0, 1), r = 16.
+  serving      (serving_cache) a serving-shaped paged V2 decode: 256
+               sequences with lengths drawn uniformly from 16..4096 tokens,
+               one query token each (Hq64 Hkv8 D128), their K/V in a shared,
+               shuffled pool of 16-token pages; N(0,1)/sqrt(128), layer 24.
   noise sweep  (noise_sweep / sweep_prefix) the noise_probe construction at
                context lengths 1k..256k keys (tutorial exercise 1), in bf16 for
                the V1 decode layout: 64 instances, each a query q ~ N(0,1) in
@@ -242,3 +246,46 @@ def lowrank_inputs(B=2, H=32, Hkv=8, L=8192, r=16, seed=1011, device="cpu"):
     F = torch.rand((H, L, r), generator=gen, device=device, dtype=torch.float32)
     G = torch.rand((H, L, r), generator=gen, device=device, dtype=torch.float32)
     return {"q": q, "k": k, "v": v, "F": F, "G": G}
+
+
+SERVING_SHAPE = dict(B=256, Hq=64, Hkv=8, min_len=16, max_len=4096, page_size=16)
+
+
+def serving_cache(B=256, Hq=64, Hkv=8, min_len=16, max_len=4096, page_size=16, seed=1013, device="cpu"):
+    """A serving-shaped paged decode batch: B sequences with lengths drawn
+    uniformly from [min_len, max_len], each holding ceil(len / page_size)
+    pages drawn at random from one pool [num_pages, page_size, Hkv, 128]
+    (three spare pages).  Values ~ N(0,1)/sqrt(128) bf16; the rows of a
+    sequence's last page past its length and the spare pages hold NaN, so a
+    reader that touches them shows it.  Returns q [B, Hq, 128], k_pages,
+    v_pages, block_table [B, ceil(max_len / page_size)] int32 (-1 past a
+    sequence's pages) and seq_lens [B] int32, on ``device``."""
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    lens = torch.randint(min_len, max_len + 1, (B,), generator=gen)
+    need = (lens + page_size - 1) // page_size
+    num_pages = int(need.sum()) + 3
+    perm = torch.randperm(num_pages, generator=gen)
+    max_pages = -(-max_len // page_size)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    off = 0
+    for b in range(B):
+        n = int(need[b])
+        table[b, :n] = perm[off:off + n].to(torch.int32)
+        off += n
+    dgen = torch.Generator(device=device).manual_seed(seed + 1)
+    s = 1.0 / math.sqrt(128)
+    q = _randn(dgen, (B, Hq, 128), s, torch.bfloat16, device)
+    kp = _randn(dgen, (num_pages, page_size, Hkv, 128), s, torch.bfloat16, device)
+    vp = _randn(dgen, (num_pages, page_size, Hkv, 128), s, torch.bfloat16, device)
+    for b in range(B):
+        n = int(need[b])
+        used = int(lens[b]) - (n - 1) * page_size
+        if used < page_size:
+            last = int(table[b, n - 1])
+            kp[last, used:] = float("nan")
+            vp[last, used:] = float("nan")
+    spare = perm[off:].to(device)
+    kp[spare] = float("nan")
+    vp[spare] = float("nan")
+    return {"q": q, "k_pages": kp, "v_pages": vp, "block_table": table.to(device),
+            "seq_lens": lens.to(torch.int32).to(device)}

@@ -117,6 +117,14 @@ DIFFATTN_API int diffattn_fwd_v2(const void* q, const void* k, const void* v, co
  * the current device.  The caller allocates it (any alignment >= 16 B). */
 DIFFATTN_API size_t diffattn_decode_workspace_size(int B, int Hkv, int T, int dv);
 
+/* The same size in terms of the V2 decode's query shape, for a caller that
+ * sizes the workspace before it knows the KV-head count: bytes that suffice
+ * for diffattn_decode_v2 with B sequences, Hq Q heads, cache length T, head
+ * width D and ANY valid Hkv (Hq % Hkv == 0, (Hq/Hkv) even, Hq/Hkv <= 8), i.e.
+ * the largest diffattn_decode_workspace_size(B, Hkv, T, D) over those Hkv.
+ * 0 for invalid sizes (Hq odd or < 2, B < 0, T < 0, D < 1). */
+DIFFATTN_API size_t diffattn_decode_v2_workspace_size(int B, int Hq, int T, int D);
+
 /* Single-token V2 decode over a KV cache (tutorial section V1 到 V2 的 diff:
  * doubled Q heads, K/V read once per KV group for both maps).
  *   q      : [B, Hq, D]           kc, vc : [B, Hkv, T, D]  (bf16)
@@ -164,9 +172,14 @@ DIFFATTN_API void diffattn_set_wait_limit_ns(unsigned long long ns);
  * allocator hook that must not re-enter the allocator, or a runtime that owns
  * all device memory and hands this library only its tensors.
  * Arguments, layouts and results are those of diffattn_decode_v2 without
- * `ws` / `ws_bytes`: the split-KV partial records live instead in a scratch
- * array of DIFFATTN_NOALLOC_SCRATCH_BYTES (4 MiB) that the library reserves in
- * device memory on every GPU that loads it, until the process exits.
+ * `ws` / `ws_bytes`: the split-KV partial records live instead in a static
+ * device array of DIFFATTN_NOALLOC_SCRATCH_BYTES (4 MiB) in the library's
+ * module.  It is reserved on a device when the module is first loaded there
+ * (with CUDA's lazy module loading, at the library's first use on that
+ * device) and kept until the process exits.  Its address is looked up once
+ * per device and cached; after cudaDeviceReset of a device the cached
+ * addresses (this one and the library's status word) are stale, so the
+ * library must not be called on that device again in the same process.
  *   - Sizes whose partial records need more than that (see
  *     diffattn_decode_workspace_size; about 2.5 MB for 16 sequences x 8 KV
  *     heads x 65536 tokens) return DIFFATTN_ERR_UNSUPPORTED before any launch.

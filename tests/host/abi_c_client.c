@@ -35,6 +35,8 @@ int main(void) {
   CHECK(rc == DIFFATTN_ERR_UNSUPPORTED);
 
   /* Workspace sizes are pure functions of the sizes. */
+  CHECK(diffattn_decode_v2_workspace_size(2, 63, 8192, 128) == 0);   /* odd Hq: invalid, no device needed */
+  CHECK(diffattn_decode_v2_workspace_size(2, 64, -1, 128) == 0);
   CHECK(diffattn_bwd_v2_workspace_size(2, 64, 8192) > 0);
   CHECK(diffattn_bwd_v2_workspace_size(2, 63, 8192) == 0);
   CHECK(diffattn_bwd_v1_workspace_size(8, 16, 16, 4096, 4096, 1) > diffattn_bwd_v1_workspace_size(8, 16, 16, 4096,

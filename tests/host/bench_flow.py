@@ -75,6 +75,7 @@ def main(argv):
                      ("v2_decode", dict(Lk=2048, B=2)), ("v1_decode", dict(Lk=2048, B=2))):
         inputs.WORKLOADS[name] = inputs.with_shape(inputs.WORKLOADS[name], **kw)
     inputs.LOWRANK_SHAPE.update(B=1, H=4, Hkv=2, L=256, r=3)
+    inputs.SERVING_SHAPE.update(B=4, min_len=16, max_len=200)
     import bench
     bench.torch = host_torch
     bench.SnrSweep.__init__.__defaults__ = (4, (1024, 2048))

@@ -25,6 +25,8 @@ What pins what (page title, section):
     query sees the whole cache.
   * RMSNorm: ||y||^2 / dv = ms / (ms + eps).
   * the pure-Python loop twin on tiny ragged GQA shapes.
+  * the noise probe's SNR and noise fraction ("差分注意力" Step 1 and Step 3):
+    closed forms on constructions where every noise key gets the same score.
 """
 
 from __future__ import annotations
@@ -250,6 +252,49 @@ def pin_brute(orc):
     assert np.all(np.abs(got.astype(np.float64) - ref.astype(np.float64)) <= 1e-7)
 
 
+def pin_noise_probe_closed_form(orc):
+    """Step 3's SNR (weight at the signal key over the mean weight at the noise
+    keys) and Step 1's noise fraction on constructions with a closed form: the
+    query meets the signal key with score s0 and every noise key with one
+    score sn (the noise keys differ only in directions orthogonal to the
+    query), so with Z = e^s0 + (N-1) e^sn the plain row is e^s0/Z at the
+    signal key and e^sn/Z at each noise key: SNR_plain = e^(s0-sn) for every
+    N, the noise fraction is (N-1) e^sn/Z, and the difference's SNR is
+    (A1[0] - lam A2[0]) / (A1[j] - lam A2[j]).  Evaluated with mpmath at 40
+    digits.  A sum in place of the mean, the signal key counted as noise, or
+    a missing 1/sqrt(d) each miss it."""
+    import mpmath as mp
+    mp.mp.dps = 40
+    d, lam = 4, 0.5
+    cases = ((5, (1.5, 2.0, 0.25), (0.5, 0.75, -1.0)), (12, (2.0, 3.0, -0.5), (1.0, -0.5, 0.125)),
+             (1000, (2.5, 4.0, 0.0), (1.0, 1.0, 1.0)))
+    for N, p1, p2 in cases:
+        rng = _rng(N)
+
+        def keys(a, b, c):
+            q = np.array([a, 0.0, 0.0, 0.0])
+            k = np.zeros((N, d))
+            k[0, 0], k[1:, 0] = b, c
+            k[1:, 1:] = rng.normal(size=(N - 1, d - 1))
+            return q, k
+
+        def row(a, b, c):
+            s0, sn = mp.mpf(a) * b / mp.sqrt(d), mp.mpf(a) * c / mp.sqrt(d)
+            Z = mp.e ** s0 + (N - 1) * mp.e ** sn
+            return mp.e ** s0 / Z, mp.e ** sn / Z
+
+        (q1, k1), (q2, k2) = keys(*p1), keys(*p2)
+        r = orc.noise_probe(q1[None], k1[None], q2[None], k2[None], lam)
+        a0, an = row(*p1)
+        b0, bn = row(*p2)
+        want = {"snr_plain": a0 / an, "snr_diff": (a0 - lam * b0) / (an - lam * bn),
+                "noise_fraction_plain": (N - 1) * an}
+        assert abs(want["snr_plain"] - mp.e ** ((mp.mpf(p1[0]) * p1[1] - mp.mpf(p1[0]) * p1[2]) / 2)) < 1e-30
+        for key, w in want.items():
+            got = float(r[key][0])
+            assert abs(got - float(w)) <= 1e-12 * abs(float(w)), (N, key, got, float(w))
+
+
 ALL_PINS = [pin_lambda_init, pin_lambda, pin_standard_attention, pin_exact_zero, pin_row_sums,
             pin_masks_and_positivity, pin_suffix_consistency, pin_uniform_keys, pin_scale,
-            pin_rmsnorm, pin_brute]
+            pin_rmsnorm, pin_brute, pin_noise_probe_closed_form]

@@ -31,17 +31,26 @@ def test_default_line_has_every_key_and_secondary():
     assert line["config"]["workload"] == "v2_prefill" and line["roofline"]["traffic"] is not None
     assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
     assert set(line["secondary"]) == {"v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged",
-                                      "v1_decode", "v1_decode_unfused"}
-    for name, sec in line["secondary"].items():
-        assert [k for k in ROOF if k not in sec["roofline"]] == [], name
+                                      "v2_decode_serving", "v1_decode", "v1_decode_unfused", "lowrank_prefill",
+                                      "snr_sweep"}
+    assert line["secondary_cols"] == ["value", "unit", "ms_per_step", "kernel_ms", "frac", "frac_of_8tbs"]
+    for name, row in line["secondary"].items():
+        assert len(row) == 6 and row[1] in ("TFLOP/s", "GB/s"), name
+        assert (row[5] is None) == (row[1] == "TFLOP/s"), name
+    assert [r[0] for r in line["snr"]] == [1024, 2048]
+    # the rows come last and the whole line stays short, so the end of the
+    # output a reader keeps (about 3 KB) holds every row
+    assert list(line)[-1] == "secondary"
+    assert len(json.dumps(line)) < 2800, len(json.dumps(line))
 
 
-@pytest.mark.parametrize("workload", ["snr_sweep", "lowrank_prefill", "v2_backward", "v2_decode_paged"])
+@pytest.mark.parametrize("workload", ["snr_sweep", "lowrank_prefill", "v2_backward", "v2_decode_paged",
+                                      "v2_decode_serving"])
 def test_other_workloads(workload):
     line = _run("--workload", workload, "--no-secondary")
     assert [k for k in KEYS if k not in line] == []
     assert line["config"]["workload"] == workload
-    if workload in ("snr_sweep", "lowrank_prefill", "v2_backward"):
+    if workload in ("snr_sweep", "lowrank_prefill", "v2_backward", "v2_decode_serving"):
         assert "unavailable" in line["e2e"]
     if workload == "snr_sweep":
-        assert [r["N"] for r in line["snr"]] == [1024, 2048]
+        assert [r[0] for r in line["snr"]] == [1024, 2048]

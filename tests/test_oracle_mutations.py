@@ -96,6 +96,31 @@ MUTATIONS = [_mut_drop_scale, _mut_scale_by_d, _mut_top_left_causal, _mut_strict
              _mut_lambda_init_no_shift, _mut_lambda_sign, _mut_rms_no_eps, _mut_softmax_no_max]
 
 
+def _mut_snr_sum_not_mean(m):
+    orig = m.noise_probe
+
+    def probe(q1, k1, q2, k2, lam):
+        r = orig(q1, k1, q2, k2, lam)
+        r["snr_plain"] = r["plain"][:, 0] / r["plain"][:, 1:].sum(axis=1)
+        r["snr_diff"] = r["diff"][:, 0] / r["diff"][:, 1:].sum(axis=1)
+        return r
+    m.noise_probe = probe
+
+
+def _mut_signal_counted_as_noise(m):
+    orig = m.noise_probe
+
+    def probe(q1, k1, q2, k2, lam):
+        r = orig(q1, k1, q2, k2, lam)
+        r["snr_plain"] = r["plain"][:, 0] / r["plain"].mean(axis=1)
+        r["noise_fraction_plain"] = r["plain"].sum(axis=1)
+        return r
+    m.noise_probe = probe
+
+
+MUTATIONS += [_mut_snr_sum_not_mean, _mut_signal_counted_as_noise]
+
+
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__)
 def test_mutation_is_caught(mutate):
     m = _fresh_oracle()

@@ -103,3 +103,24 @@ def test_paged_full_size_workload():
         for i, h in enumerate(pairs):
             err = float(np.max(np.abs(got[b, h] - ref[0, i])))
             assert err <= BF16_TOL * float(np.max(np.abs(ref[0, i]))), (b, h, err)
+
+
+def test_paged_serving_shaped_batch():
+    """The bench's serving-shaped batch in its launch configuration: 256
+    sequences of lengths 16..4096 in one pool of 16-token pages.  A seeded
+    sample of 24 sequences (the shortest and longest among them) against the
+    oracle, and the whole batch bitwise repeatable."""
+    x = inputs.serving_cache(**inputs.SERVING_SHAPE, device=DEV)
+    Hq = inputs.SERVING_SHAPE["Hq"]
+    lam = (torch.rand(Hq // 2, generator=torch.Generator().manual_seed(77)) * 1.2 - 0.2).to(DEV)
+    args = (x["q"], x["k_pages"], x["v_pages"], x["block_table"], x["seq_lens"], lam)
+    out = da.decode_v2_paged(*args)
+    torch.cuda.synchronize()
+    assert da.last_status() == da.OK
+    assert torch.equal(out, da.decode_v2_paged(*args))
+    lens = x["seq_lens"].cpu()
+    pick = torch.randperm(lens.numel(), generator=torch.Generator().manual_seed(5))[:22].tolist()
+    pick += [int(lens.argmin()), int(lens.argmax())]
+    idx = torch.tensor(sorted(set(pick)), device=DEV)
+    _check_against_oracle(out[idx], x["q"][idx], x["k_pages"], x["v_pages"], x["block_table"][idx],
+                          x["seq_lens"][idx], lam, "serving batch")

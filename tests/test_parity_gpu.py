@@ -289,6 +289,25 @@ def test_decode_v2_small(case):
     assert rel_err(out, ref) <= BF16_TOL
 
 
+@pytest.mark.parametrize("B,Hq,T", [(16, 64, 65536), (3, 16, 4097), (1, 4, 1), (2, 12, 0)])
+def test_decode_v2_workspace_size_covers_every_kv_head_count(B, Hq, T):
+    """diffattn_decode_v2_workspace_size(B, Hq, T, D) is at least the exact
+    size for every valid Hkv, and a decode given exactly that many bytes runs
+    (the Hkv the caller ends up with is one of them)."""
+    L = da.load()
+    n = L.diffattn_decode_v2_workspace_size(B, Hq, T, 128)
+    valid = [h for h in range(1, Hq // 2 + 1) if Hq % h == 0 and (Hq // h) % 2 == 0 and Hq // h <= 8]
+    assert valid and n == max(L.diffattn_decode_workspace_size(B, h, T, 128) for h in valid)
+    Hkv = valid[0]
+    g = torch.Generator(device="cpu").manual_seed(B * 1000 + Hq + T)
+    s = 1 / math.sqrt(128)
+    q, kc, vc = bf16(B, Hq, 128, g=g, std=s), bf16(B, Hkv, T, 128, g=g, std=s), bf16(B, Hkv, T, 128, g=g, std=s)
+    lam = rand_lam(Hq // 2, 7)
+    ws = torch.empty(max(int(n), 16), dtype=torch.uint8, device=DEV)
+    out = da.decode_v2(q, kc, vc, lam, workspace=ws)
+    assert torch.equal(out, da.decode_v2(q, kc, vc, lam))
+
+
 @pytest.mark.parametrize("fused", [1, 0])
 @pytest.mark.parametrize("case", [(2, 8, 2, 1000), (1, 4, 4, 130), (3, 16, 4, 4097)],
                          ids=lambda c: "B%d_H%d_Hkv%d_T%d" % c)

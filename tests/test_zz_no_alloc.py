@@ -12,7 +12,11 @@ file): the entry point keeps state in the library's shared scratch, so it is
 checked both after everything else has run and, when run alone, in a fresh
 process.  It calls the new entry point through the C ABI (ctypes) and compares
 it with the existing workspace-taking entry point, on two calls in a row with
-different inputs, within the bf16 tolerance used by the other parity tests.
+different inputs.  Both run the same kernels with the same split of the keys,
+so the outputs must agree bit for bit; one case is also checked against the
+fp64 oracle within the bf16 tolerance of the other parity tests.  A call made
+after the first must leave the device's free memory (cudaMemGetInfo) and
+torch's allocated bytes unchanged.
 """
 
 import ctypes
@@ -22,6 +26,7 @@ import pytest
 import torch
 
 import differential_attention_transformers_b200 as da
+from oracle import diffattn as orc
 
 pytestmark = pytest.mark.gpu
 
@@ -37,22 +42,18 @@ def _inputs(seed, B, Hq, Hkv, T):
     return mk(B, Hq, 128), mk(B, Hkv, T, 128), mk(B, Hkv, T, 128), lam
 
 
-def _noalloc(q, kc, vc, lam):
+def _noalloc(q, kc, vc, lam, out=None):
     L = da.load()
     B, Hq, D = q.shape
     Hkv, T = kc.shape[1], kc.shape[2]
-    out = torch.empty((B, Hq // 2, D), dtype=torch.bfloat16, device=DEV)
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=torch.bfloat16, device=DEV)
     st = L.diffattn_decode_v2_noalloc(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(kc.data_ptr()),
                                       ctypes.c_void_p(vc.data_ptr()), ctypes.c_void_p(lam.data_ptr()),
                                       ctypes.c_void_p(out.data_ptr()), da.BF16, B, Hq, Hkv, T, D,
                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == da.OK, da.last_error()
     return out
-
-
-def _rel(a, b):
-    a, b = a.float(), b.float()
-    return (torch.max(torch.abs(a - b)) / torch.max(torch.abs(b))).item()
 
 
 def test_noalloc_decode_matches_workspace_decode_twice():
@@ -66,7 +67,31 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     for ((q, kc, vc, lam), what), got in zip(cases, outs):
         ref = da.decode_v2(q, kc, vc, lam)
         assert torch.isfinite(got.float()).all(), what
-        assert _rel(got, ref) <= BF16_TOL, what
+        assert torch.equal(got, ref), what            # same kernels, same split: bit for bit
+    # the second case against the fp64 oracle, every head
+    (q, kc, vc, lam), _ = cases[1]
+    want = orc.decode_v2(q, kc, vc, lam.double().cpu().numpy())
+    got = outs[1].double().cpu().numpy()
+    for b in range(want.shape[0]):
+        for h in range(want.shape[1]):
+            err = abs(got[b, h] - want[b, h]).max()
+            assert err <= BF16_TOL * abs(want[b, h]).max(), (b, h, err)
+
+
+def test_noalloc_call_allocates_nothing():
+    """After a first call (the one-time set-up), a call changes neither the
+    device's free memory nor torch's allocated bytes."""
+    q, kc, vc, lam = _inputs(303, 4, 64, 8, 9000)
+    out = torch.empty((4, 32, 128), dtype=torch.bfloat16, device=DEV)
+    _noalloc(q, kc, vc, lam, out)
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    _noalloc(q, kc, vc, lam, out)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert da.last_status() == da.OK
+    assert torch.equal(out, da.decode_v2(q, kc, vc, lam))
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
