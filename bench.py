@@ -343,7 +343,7 @@ class Backward:
             nws = da.load().diffattn_bwd_v2_workspace_size(w.B, w.H, w.Lq)
             self.launches_per_step = 6   # lambda, prep, dlambda, dQ, dK/dV, lambda's parameter gradients
         else:
-            self.out, self.lse, self.om, self.rstd = da.fwd_v1_train(x["q1"], x["k1"], x["q2"], x["k2"], x["v"],
+            self.out, self.lse, self.om, self.rstd, self.o2c = da.fwd_v1_train(x["q1"], x["k1"], x["q2"], x["k2"], x["v"],
                                                                      self.lam, causal=w.causal, rmsnorm=w.rmsnorm)
             nws = da.load().diffattn_bwd_v1_workspace_size(w.B, w.H, w.Hkv, w.Lq, w.Lk, int(w.rmsnorm))
             # lambda, pack, [RMSNorm gradient], prep, dlambda, dQ, dK/dV, unpack, lambda's parameter gradients
@@ -360,7 +360,8 @@ class Backward:
                              workspace=self.ws)[-1]
         else:
             dlam = da.bwd_v1(x["q1"], x["k1"], x["q2"], x["k2"], x["v"], self.lam, self.dout, self.out, self.lse,
-                             self.om, self.rstd, causal=w.causal, rmsnorm=w.rmsnorm, workspace=self.ws)[-1]
+                             self.om, self.rstd, self.o2c, causal=w.causal, rmsnorm=w.rmsnorm,
+                             workspace=self.ws)[-1]
         da.lambda_backward(*self.lp, dlam)
         if ev is not None:
             ev[1].record()

@@ -76,9 +76,9 @@ def load():
         "diffattn_bwd_v2_workspace_size": (Z, [I, I, I]),
         "diffattn_bwd_v2": (I, [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]),
         "diffattn_lambda_backward": (I, [P, P, P, P, P, I, I, P, P, P, P, P]),
-        "diffattn_fwd_v1_train": (I, [P] * 10 + [I] * 10 + [F, P]),
+        "diffattn_fwd_v1_train": (I, [P] * 11 + [I] * 10 + [F, P]),
         "diffattn_bwd_v1_workspace_size": (Z, [I] * 6),
-        "diffattn_bwd_v1": (I, [P] * 17 + [I] * 10 + [P, Z, P]),
+        "diffattn_bwd_v1": (I, [P] * 18 + [I] * 10 + [P, Z, P]),
         "diffattn_fwd_lowrank_workspace_size": (Z, [I] * 6),
         "diffattn_fwd_lowrank": (I, [P] * 7 + [I] * 9 + [P, Z, P]),
     }
@@ -349,8 +349,10 @@ def bwd_v2(q, k, v, lam, dout, lse, o_maps, causal=True, workspace=None):
 
 def fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5):
     """V1 forward (bf16, d = 64, dv = 128) that also returns what bwd_v1 needs:
-    (out [B,H,Lq,128], lse f32 [B,H,2,Lq], o_maps [B,H,2,Lq,128], rstd f32 [B,H,Lq]
-    or None without RMSNorm).  Device tensors."""
+    (out [B,H,Lq,128], lse f32 [B,H,2,Lq], o_maps [B,H,2,Lq,128], rstd f32 [B,H,Lq],
+    o2c f32 [B,H,Lq]); rstd and o2c are None without RMSNorm, and with it
+    o_maps[:, :, 1] holds map 2's part orthogonal to the difference output
+    (see diffattn_fwd_v1_train).  Device tensors."""
     B, H, Lq, d = _dims("q1", q1, 4)
     _, Hkv, Lk, _ = _dims("k1", k1, 4)
     dv = _dims("v", v, 4)[3]
@@ -362,13 +364,15 @@ def fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=False, eps=1e-5):
     lse = torch.empty((B, H, 2, Lq), dtype=torch.float32, device=q1.device)
     o_maps = torch.empty((B, H, 2, Lq, dv), dtype=q1.dtype, device=q1.device)
     rstd = torch.empty((B, H, Lq), dtype=torch.float32, device=q1.device) if rmsnorm else None
+    o2c = torch.empty((B, H, Lq), dtype=torch.float32, device=q1.device) if rmsnorm else None
     _check(load().diffattn_fwd_v1_train(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(v), _ptr(lam), _ptr(out),
-                                        _ptr(lse), _ptr(o_maps), _ptr(rstd), _dtype_code(q1), B, H, Hkv, Lq, Lk, d,
-                                        dv, int(causal), int(rmsnorm), float(eps), _stream()))
-    return out, lse, o_maps, rstd
+                                        _ptr(lse), _ptr(o_maps), _ptr(rstd), _ptr(o2c), _dtype_code(q1), B, H, Hkv,
+                                        Lq, Lk, d, dv, int(causal), int(rmsnorm), float(eps), _stream()))
+    return out, lse, o_maps, rstd, o2c
 
 
-def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, causal=True, rmsnorm=False, workspace=None):
+def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, o2c=None, causal=True, rmsnorm=False,
+           workspace=None):
     """Gradients of the V1 forward: (dq1, dk1, dq2, dk2, dv, dlam) given dout [B,H,Lq,128]
     and fwd_v1_train's outputs.  bf16 gradients, f32 dlam.  Device tensors."""
     B, H, Lq, d = _dims("q1", q1, 4)
@@ -380,16 +384,18 @@ def bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, o_maps, rstd=None, causal=Tru
             ("dout", dout, (B, H, Lq, dvw), bf), ("lse", lse, (B, H, 2, Lq), f32),
             ("o_maps", o_maps, (B, H, 2, Lq, dvw), bf))
     if rmsnorm:
-        _expect(("out", out, (B, H, Lq, dvw), bf), ("rstd", rstd, (B, H, Lq), f32))
+        _expect(("out", out, (B, H, Lq, dvw), bf), ("rstd", rstd, (B, H, Lq), f32), ("o2c", o2c, (B, H, Lq), f32))
     _device_only([("q1", q1), ("k1", k1), ("q2", q2), ("k2", k2), ("v", v), ("lam", lam), ("dout", dout),
-                  ("out", out), ("lse", lse), ("o_maps", o_maps), ("rstd", rstd), ("workspace", workspace)])
+                  ("out", out), ("lse", lse), ("o_maps", o_maps), ("rstd", rstd), ("o2c", o2c),
+                  ("workspace", workspace)])
     dq1, dq2 = torch.empty_like(q1), torch.empty_like(q2)
     dk1, dk2, dv = torch.empty_like(k1), torch.empty_like(k2), torch.empty_like(v)
     dlam = torch.empty(H, dtype=torch.float32, device=q1.device)
     need = int(load().diffattn_bwd_v1_workspace_size(B, H, Hkv, Lq, Lk, int(rmsnorm)))
     ws = workspace if workspace is not None else _workspace(need, q1.device)
     _check(load().diffattn_bwd_v1(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(v), _ptr(lam), _ptr(dout),
-                                  _ptr(out), _ptr(lse), _ptr(o_maps), _ptr(rstd), _ptr(dq1), _ptr(dk1), _ptr(dq2),
+                                  _ptr(out), _ptr(lse), _ptr(o_maps), _ptr(rstd), _ptr(o2c), _ptr(dq1), _ptr(dk1),
+                                  _ptr(dq2),
                                   _ptr(dk2), _ptr(dv), _ptr(dlam), _dtype_code(q1), B, H, Hkv, Lq, Lk, d, dvw,
                                   int(causal), int(rmsnorm), _ptr(ws), ws.numel() * ws.element_size(), _stream()))
     return dq1, dk1, dq2, dk2, dv, dlam

@@ -79,6 +79,7 @@ struct BwdPrepArgs {
   float* dd;                    // [B, Hp, 2, Lp]
   float* part;                  // [B * Hp, Lp / 64] partial sums of -D_2
   int B, Hp, Lq, Lp;
+  const float* d_in;            // [B, Hp, 2, Lq] D_m formed upstream (V1 with RMSNorm), or null
 };
 
 // grid (Lp / 64, B * Hp), 256 threads: warp w handles rows 8w .. 8w+7 of the block.
@@ -90,7 +91,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
   for (int i = 0; i < 8; ++i) {
     const int row = blockIdx.x * 64 + warp * 8 + i;
     float d[2] = {0.f, 0.f};
-    if (row < a.Lq) {
+    if (row < a.Lq && a.d_in != nullptr) {
+      d[0] = a.d_in[((size_t)bh * 2) * a.Lq + row];
+      d[1] = a.d_in[((size_t)bh * 2 + 1) * a.Lq + row];
+    } else if (row < a.Lq) {
       const __nv_bfloat16* go = a.dout + ((size_t)bh * a.Lq + row) * 128 + lane * 4;
       const uint2 gv = *reinterpret_cast<const uint2*>(go);
 #pragma unroll

@@ -208,7 +208,7 @@ int prefill_rb_group(bool v1, int Hq, int Hkv, int n_rb) {
 int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k2, const void* v,
                    const float* lambda, void* out, int B, int Hout, int Hq, int Hkv, int Lq, int Lk, int dqk,
                    bool v1, int causal, int rms, float eps, cudaStream_t s, float* lse = nullptr,
-                   void* o_maps = nullptr, float* rstd = nullptr, float* o_f32 = nullptr) {
+                   void* o_maps = nullptr, float* rstd = nullptr, float* o_f32 = nullptr, float* o2c = nullptr) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   if (Lq == 0 || B == 0 || Hout == 0) return ok();
@@ -236,6 +236,7 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   a.lse = lse;
   a.o_maps = static_cast<__nv_bfloat16*>(o_maps);
   a.rstd = rstd;
+  a.o2c = o2c;
   a.o_f32 = o_f32;
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
@@ -337,7 +338,7 @@ size_t bwd_ws_bytes(int B, int Hq, int Lq) {
 int launch_backward_v2(const void* q, const void* k, const void* v, const float* lambda, const void* dout,
                        const float* lse, const void* o_maps, void* dq, void* dk, void* dv, float* dlambda, int B,
                        int Hq, int Hkv, int Lq, int Lk, int causal, void* ws, size_t ws_bytes, cudaStream_t s,
-                       int dqk = 128) {
+                       int dqk = 128, const float* d_in = nullptr) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   const size_t need = bwd_ws_bytes(B, Hq, Lq);
@@ -350,7 +351,7 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
   float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * align256((size_t)B * Hp * 2 * Lp * 4));
   if (Lp > 0) {
     BwdPrepArgs pa{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o_maps), lse,
-                   lse_p, dd, part, B, Hp, Lq, Lp};
+                   lse_p, dd, part, B, Hp, Lq, Lp, d_in};
     bwd_prep_kernel<<<dim3((unsigned)(Lp / 64), (unsigned)(B * Hp)), 256, 0, s>>>(pa);
     CUDA_TRY(cudaGetLastError());
   }
@@ -394,10 +395,11 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
 
 // V1 backward workspace: the packed [Q1|0], [0|Q2] rows and their gradient
 // (B*2H*Lq rows of 128), the packed [K1|K2] rows and their gradient
-// (B*Hkv*Lk rows of 128), the RMSNorm input gradient dX (B*H*Lq rows of 128,
-// with RMSNorm only), then the V2 backward's own workspace.
+// (B*Hkv*Lk rows of 128), with RMSNorm only the input gradient dX (B*H*Lq
+// rows of 128) and the row terms D_m [B*H, 2, Lq] f32, then the V2
+// backward's own workspace.
 struct V1BwdLayout {
-  size_t qp, dqp, kp, dkp, dx, bw, total;
+  size_t qp, dqp, kp, dkp, dx, dd, bw, total;
 };
 V1BwdLayout v1_bwd_layout(int B, int H, int Hkv, int Lq, int Lk, int rms) {
   const size_t nq = (size_t)B * H * Lq, nk = (size_t)B * Hkv * Lk;
@@ -407,7 +409,8 @@ V1BwdLayout v1_bwd_layout(int B, int H, int Hkv, int Lq, int Lk, int rms) {
   l.kp = l.dqp + align256(nq * 512);
   l.dkp = l.kp + align256(nk * 256);
   l.dx = l.dkp + align256(nk * 256);
-  l.bw = l.dx + (rms ? align256(nq * 256) : 0);
+  l.dd = l.dx + (rms ? align256(nq * 256) : 0);
+  l.bw = l.dd + (rms ? align256(nq * 2 * 4) : 0);
   l.total = l.bw + bwd_ws_bytes(B, 2 * H, Lq);
   return l;
 }
@@ -420,9 +423,9 @@ unsigned stream_grid(const DeviceInfo* dev, long long items, int per_block) {
 
 int launch_backward_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
                        const float* lambda, const void* dout, const void* out, const float* lse, const void* o_maps,
-                       const float* rstd, void* dq1, void* dk1, void* dq2, void* dk2, void* dv, float* dlambda,
-                       int B, int H, int Hkv, int Lq, int Lk, int causal, int rms, void* ws, size_t ws_bytes,
-                       cudaStream_t s) {
+                       const float* rstd, const float* o2c, void* dq1, void* dk1, void* dq2, void* dk2, void* dv,
+                       float* dlambda, int B, int H, int Hkv, int Lq, int Lk, int causal, int rms, void* ws,
+                       size_t ws_bytes, cudaStream_t s) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   const V1BwdLayout L = v1_bwd_layout(B, H, Hkv, Lq, Lk, rms);
@@ -440,15 +443,18 @@ int launch_backward_v1(const void* q1, const void* k1, const void* q2, const voi
     CUDA_TRY(cudaGetLastError());
   }
   const void* g = dout;
+  const float* d_in = nullptr;
   if (rms && nq > 0) {
+    float* dd = reinterpret_cast<float*>(w + L.dd);
     V1RmsArgs ra{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), rstd, at(L.dx),
-                 nq};
+                 nq, static_cast<const __nv_bfloat16*>(o_maps), o2c, dd, Lq};
     v1_rms_backward_kernel<<<stream_grid(dev, nq, V1A_THREADS / 32), V1A_THREADS, 0, s>>>(ra);
     CUDA_TRY(cudaGetLastError());
     g = at(L.dx);
+    d_in = dd;
   }
   if (int e = launch_backward_v2(at(L.qp), at(L.kp), v, lambda, g, lse, o_maps, at(L.dqp), at(L.dkp), dv, dlambda,
-                                 B, 2 * H, Hkv, Lq, Lk, causal, w + L.bw, ws_bytes - L.bw, s, 64))
+                                 B, 2 * H, Hkv, Lq, Lk, causal, w + L.bw, ws_bytes - L.bw, s, 64, d_in))
     return e;
   if (nq + nk > 0) {
     V1UnpackArgs ua{at(L.dqp), at(L.dkp), static_cast<__nv_bfloat16*>(dq1), static_cast<__nv_bfloat16*>(dq2),
@@ -731,7 +737,7 @@ int diffattn_bwd_v2(const void* q, const void* k, const void* v, const float* la
 }
 
 int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
-                          const float* lambda, void* out, float* lse, void* o_maps, float* rstd,
+                          const float* lambda, void* out, float* lse, void* o_maps, float* rstd, float* o2_coef,
                           diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk, int d, int dv, int causal,
                           int rmsnorm, float eps, void* stream) {
   if (B < 0 || H < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || d < 1 || dv < 1)
@@ -743,13 +749,13 @@ int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const 
   if (d != 64 || dv != 128)
     return fail(DIFFATTN_ERR_UNSUPPORTED, "V1 training path needs d == 64 and dv == 128 (got d=%d dv=%d)", d, dv);
   if (B == 0 || Lq == 0) return ok();
-  if (!q1 || !q2 || !lambda || !out || !lse || !o_maps || (rmsnorm && !rstd) ||
+  if (!q1 || !q2 || !lambda || !out || !lse || !o_maps || (rmsnorm && (!rstd || !o2_coef)) ||
       (Lk > 0 && (!k1 || !k2 || !v)))
     return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   if (Lk == 0) k1 = k2 = v = q1;
   if (int e = check_bf16_ptrs({q1, k1, q2, k2, v, out, o_maps})) return e;
   return launch_prefill(q1, q2, k1, k2, v, lambda, out, B, H, H, Hkv, Lq, Lk, 64, true, causal, rmsnorm, eps,
-                        static_cast<cudaStream_t>(stream), lse, o_maps, rstd);
+                        static_cast<cudaStream_t>(stream), lse, o_maps, rstd, nullptr, o2_coef);
 }
 
 size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int rmsnorm) {
@@ -759,7 +765,7 @@ size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int
 
 int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
                     const float* lambda, const void* dout, const void* out, const float* lse, const void* o_maps,
-                    const float* rstd, void* dq1, void* dk1, void* dq2, void* dk2, void* dv, float* dlambda,
+                    const float* rstd, const float* o2_coef, void* dq1, void* dk1, void* dq2, void* dk2, void* dv, float* dlambda,
                     diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk, int d, int dv_width, int causal,
                     int rmsnorm, void* ws, size_t ws_bytes, void* stream) {
   if (B < 0 || H < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || d < 1 || dv_width < 1)
@@ -775,14 +781,14 @@ int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* 
     CUDA_TRY(cudaMemsetAsync(dlambda, 0, sizeof(float) * (size_t)H, static_cast<cudaStream_t>(stream)));
     return ok();
   }
-  if ((Lq > 0 && (!q1 || !q2 || !dout || !lse || !o_maps || !dq1 || !dq2 || (rms && (!out || !rstd)))) ||
+  if ((Lq > 0 && (!q1 || !q2 || !dout || !lse || !o_maps || !dq1 || !dq2 || (rms && (!out || !rstd || !o2_coef)))) ||
       (Lk > 0 && (!k1 || !k2 || !v || !dk1 || !dk2 || !dv)))
     return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   for (const void* p : std::initializer_list<const void*>{q1, k1, q2, k2, v, dout, out, o_maps, dq1, dk1, dq2, dk2,
                                                           dv})
     if (p && !aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
-  return launch_backward_v1(q1, k1, q2, k2, v, lambda, dout, out, lse, o_maps, rstd, dq1, dk1, dq2, dk2, dv, dlambda,
-                            B, H, Hkv, Lq, Lk, causal, rms, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+  return launch_backward_v1(q1, k1, q2, k2, v, lambda, dout, out, lse, o_maps, rstd, o2_coef, dq1, dk1, dq2, dk2, dv,
+                            dlambda, B, H, Hkv, Lq, Lk, causal, rms, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 size_t diffattn_fwd_lowrank_workspace_size(int B, int H, int Lq, int Lk, int r, int causal) {

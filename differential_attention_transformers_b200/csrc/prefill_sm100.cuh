@@ -71,6 +71,16 @@ struct PrefillArgs {
   float* lse;
   __nv_bfloat16* o_maps;
   float* rstd;
+  // With RMSNorm the backward's dlambda = -sum dX . O_2 is a small remainder
+  // of large terms: dX is orthogonal to the difference output X, and O_2 is
+  // nearly parallel to X when the maps are alike.  The training forward
+  // therefore stores map 2's normalised output as its component orthogonal to
+  // X, O_2 - c X with c = <O_2, X> / <X, X> formed in f32 (o_maps[.., 1, ..]),
+  // and per row o2c[B, Hout, Lq] = c eps r^2 (0 for a row that sees no key).
+  // Then dX . O_2 = dX . (O_2 - c X) + c dX . X with dX . X = <y, dY> eps r^2,
+  // so D_2 = dX . (O_2 - c X) + o2c <y, dY>, and the bf16 rounding of the
+  // stored operand scales with the orthogonal part only.
+  float* o2c;
   // Single-map mode (PF_SINGLE): output heads are pairs of independent
   // heads (2h, 2h+1) over one KV head, each with its own lambda[2h + m] (which
   // sets only its residual choice); the kernel writes each head's normalised
@@ -93,6 +103,7 @@ struct PfSmem {
   alignas(16) uint8_t stage[8][16 * 128];          // per softmax warp: 16 output rows of 64 bf16 (epilogue)
   float l[2][PF_BM];
   float ss[2][PF_BM];
+  float sp[2][PF_BM];     // epilogue exchange of <O_2, X> partial sums (training, RMSNorm)
   alignas(8) uint64_t q_full;
   uint64_t k_full[PF_NS];
   uint64_t v_full[PF_NS];
@@ -486,6 +497,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     const float lam = SINGLE ? 0.f : a.lambda[h];
     float y[64];
     bool have = false;
+    float kx = 0.f;   // training with RMSNorm: c / rs, so that c X = kx y once y holds rs X
     if (ok && nT > 0) {
       S.l[m][r] = l_run;
       mbar_arrive(smem_u32(&S.xl));
@@ -499,6 +511,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         const float l1 = S.l[0][r], l2 = S.l[1][r];
         const float c1 = l1 > 0.f ? 1.f / l1 : 0.f;
         const float c2 = l2 > 0.f ? lam / l2 : 0.f;
+        const float i2 = l2 > 0.f ? 1.f / l2 : 0.f;
+        float sp = 0.f;   // <O_2 / l_2, X> over this thread's 64 columns (training, RMSNorm)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t o1[32], o2[32];
@@ -506,8 +520,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           tmem_ld32p(tmem + lane_off + 384 + m * 64 + c * 32, o2);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
+          for (int i = 0; i < 32; ++i) {
             y[c * 32 + i] = __fsub_rn(__fmul_rn(__uint_as_float(o1[i]), c1), __fmul_rn(__uint_as_float(o2[i]), c2));
+            if (TRAIN) sp = fmaf(__uint_as_float(o2[i]) * i2, y[c * 32 + i], sp);
+          }
         }
         have = true;
         if (a.rms) {
@@ -515,15 +531,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 64; ++i) ss = fmaf(y[i], y[i], ss);
           S.ss[m][r] = ss;
+          if (TRAIN) S.sp[m][r] = sp;
           mbar_arrive(smem_u32(&S.xs));
           ok = warp_wait(smem_u32(&S.xs), 0, abort_flag, a.watch);
           have = ok;
           if (ok) {
-            const float rs = rsqrtf((S.ss[0][r] + S.ss[1][r]) / (float)PF_DV + a.eps);
+            const float xx = S.ss[0][r] + S.ss[1][r];
+            const float rs = rsqrtf(xx / (float)PF_DV + a.eps);
 #pragma unroll
             for (int i = 0; i < 64; ++i) y[i] *= rs;
-            if (TRAIN && m == 0 && rg < a.Lq)
-              a.rstd[((size_t)b * a.Hout + h) * a.Lq + rg] = l_run > 0.f ? rs : 0.f;
+            if (TRAIN) {
+              const float cq = (l_run > 0.f && xx > 0.f) ? (S.sp[0][r] + S.sp[1][r]) / xx : 0.f;
+              kx = cq / rs;
+              if (m == 0 && rg < a.Lq) {
+                a.rstd[((size_t)b * a.Hout + h) * a.Lq + rg] = l_run > 0.f ? rs : 0.f;
+                a.o2c[((size_t)b * a.Hout + h) * a.Lq + rg] = cq * a.eps * rs * rs;
+              }
+            }
           }
         }
       }
@@ -531,7 +555,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
 #pragma unroll
       for (int i = 0; i < 64; ++i) y[i] = 0.f;
       have = true;
-      if (TRAIN && a.rms && m == 0 && rg < a.Lq) a.rstd[((size_t)b * a.Hout + h) * a.Lq + rg] = 0.f;
+      if (TRAIN && a.rms && m == 0 && rg < a.Lq) {
+        a.rstd[((size_t)b * a.Hout + h) * a.Lq + rg] = 0.f;
+        a.o2c[((size_t)b * a.Hout + h) * a.Lq + rg] = 0.f;
+      }
     }
     have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;   // warp-uniform (ok is)
     const int row_w0 = r0 + wq * 32;                          // first row of this warp
@@ -539,12 +566,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       pf_store_rows(S.stage[warp], y, a.out + (((size_t)b * a.Hout + h) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq,
                     lane);
     // Training outputs: this map's log-sum-exp, and 64 columns of both
-    // normalised map outputs.
+    // normalised map outputs; with RMSNorm map 2's is stored as O_2 - c X.
+    // Map 2 goes first: its correction reads y (rs X, just stored) before map
+    // 1's values overwrite it.
     if (TRAIN && have) {
       const size_t stat = ((size_t)b * a.Hout + h) * 2;
       if (rg < a.Lq) a.lse[(stat + m) * a.Lq + rg] = l_run > 0.f ? m_run + log2f(l_run) : INFINITY;
 #pragma unroll
-      for (int mm = 0; mm < 2; ++mm) {
+      for (int t = 0; t < 2; ++t) {
+        const int mm = 1 - t;
         const float inv = (nT > 0 && S.l[mm][r] > 0.f) ? 1.f / S.l[mm][r] : 0.f;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -554,7 +584,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
             tmem_wait_ld();
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) y[c * 32 + i] = nT > 0 ? __uint_as_float(o[i]) * inv : 0.f;
+          for (int i = 0; i < 32; ++i) {
+            const float on = nT > 0 ? __uint_as_float(o[i]) * inv : 0.f;
+            y[c * 32 + i] = (mm == 1 && kx != 0.f) ? __fsub_rn(on, __fmul_rn(kx, y[c * 32 + i])) : on;
+          }
         }
         pf_store_rows(S.stage[warp], y, a.o_maps + ((stat + mm) * a.Lq) * PF_DV + m * 64, row_w0, a.Lq, lane);
       }

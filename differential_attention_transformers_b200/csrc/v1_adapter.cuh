@@ -97,11 +97,24 @@ __global__ void __launch_bounds__(V1A_THREADS) v1_unpack_kernel(V1UnpackArgs a) 
 // dX = r (dY - y <y, dY> / 128) per 128-wide row, one warp per row, 4 elements
 // a lane.  y is the normalised forward output, r its saved 1/rms (0 for a row
 // that saw no key, whose output and gradient are zero).
+//
+// The same pass forms the backward's row terms D_m = dX . O_m from the f32 dX
+// (before its rounding to bf16), with the training forward's stored map
+// outputs: O_1 / l_1 and, for map 2, its part orthogonal to the difference
+// output X, O_2' = O_2 / l_2 - c X, and per row e = c eps r^2.  Since
+//   dX . X = r (X . dY - r |X|^2 <y, dY> / n) = <y, dY> (1 - r^2 ms) = <y, dY> eps r^2
+// (r^2 = 1 / (ms + eps)), D_2 = dX . O_2' + e <y, dY>: a sum whose terms are
+// of the size of O_2', so its rounding no longer scales with the part of O_2
+// along X that the sum cancels.  D [rows of (b, h), 2, Lq] f32.
 struct V1RmsArgs {
   const __nv_bfloat16 *dy, *y;
   const float* rstd;
   __nv_bfloat16* dx;
   long long rows;
+  const __nv_bfloat16* o_maps;   // [B*H, 2, Lq, 128]: O_1 / l_1, O_2 / l_2 - c X
+  const float* o2c;              // [B*H, Lq]: e = c eps r^2
+  float* dd;                     // [B*H, 2, Lq]: D_1, D_2
+  int Lq;
 };
 
 __global__ void __launch_bounds__(V1A_THREADS) v1_rms_backward_kernel(V1RmsArgs a) {
@@ -123,11 +136,31 @@ __global__ void __launch_bounds__(V1A_THREADS) v1_rms_backward_kernel(V1RmsArgs 
     for (int j = 0; j < 4; ++j) dot = fmaf(g[j], y[j], dot);
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     const float r = a.rstd[row], c = dot * (1.f / 128.f);
+    float dxf[4];
+    for (int j = 0; j < 4; ++j) dxf[j] = r * fmaf(-y[j], c, g[j]);
     uint2 out;
     __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&out);
-    for (int j = 0; j < 2; ++j)
-      o2[j] = __floats2bfloat162_rn(r * fmaf(-y[2 * j], c, g[2 * j]), r * fmaf(-y[2 * j + 1], c, g[2 * j + 1]));
+    for (int j = 0; j < 2; ++j) o2[j] = __floats2bfloat162_rn(dxf[2 * j], dxf[2 * j + 1]);
     reinterpret_cast<uint2*>(a.dx + row * 128)[lane] = out;
+    // D_1, D_2 from the f32 dX
+    const long long bh = row / a.Lq, l = row - bh * a.Lq;
+    float d[2];
+    for (int m = 0; m < 2; ++m) {
+      const uint2 ov = reinterpret_cast<const uint2*>(a.o_maps + ((bh * 2 + m) * a.Lq + l) * 128)[lane];
+      const __nv_bfloat162* om = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      float s = 0.f;
+      for (int j = 0; j < 2; ++j) {
+        const float2 of = __bfloat1622float2(om[j]);
+        s = fmaf(dxf[2 * j], of.x, s);
+        s = fmaf(dxf[2 * j + 1], of.y, s);
+      }
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      d[m] = s;
+    }
+    if (lane == 0) {
+      a.dd[(bh * 2) * a.Lq + l] = d[0];
+      a.dd[(bh * 2 + 1) * a.Lq + l] = fmaf(a.o2c[row], dot, d[1]);
+    }
   }
 }
 

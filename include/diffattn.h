@@ -236,15 +236,26 @@ DIFFATTN_API int diffattn_bwd_v2(const void* q, const void* k, const void* v, co
  * diffattn_bwd_v1 needs:
  *   lse    : f32 [B, H, 2, Lq], as for diffattn_fwd_v2_train, with the scores
  *            of map m = Q_m K_m^T scaled by log2(e)/sqrt(d)       (device)
- *   o_maps : bf16 [B, H, 2, Lq, 128]: O_m = A_m V per map         (device)
- *   rstd   : f32 [B, H, Lq]: with rmsnorm != 0, the row's
+ *   o_maps : bf16 [B, H, 2, Lq, 128]: O_m = A_m V per map; with rmsnorm != 0
+ *            map 2's entry is instead O_2 - c X, its part orthogonal to the
+ *            difference output X = O_1 - λ O_2, c = <O_2, X> / <X, X> per row
+ *            (formed in f32)                                       (device)
+ *   rstd   : f32 [B, H, Lq]: with rmsnorm != 0, the row's r =
  *            1/sqrt(mean(x^2) + eps) of the difference output x (0 for a row
  *            that sees no key); not touched, and may be NULL, without. (device)
- * The per-head RMSNorm is the tutorial's (section V1 到 V2 的 diff). */
+ *   o2_coef: f32 [B, H, Lq]: with rmsnorm != 0, c eps r^2 per row (0 for a
+ *            row that sees no key); not touched, and may be NULL, without.
+ * The per-head RMSNorm is the tutorial's (section V1 到 V2 的 diff).  Why map
+ * 2 is stored that way: dλ = -Σ dX·O_2, and the RMSNorm gradient dX is
+ * orthogonal to X, to which O_2 is nearly parallel when the two maps are
+ * alike; the sum is then a small remainder of large terms, and a bf16 O_2
+ * would leave an error of the terms' size.  With X·dX = <y, dY> eps r^2,
+ * dX·O_2 = dX·(O_2 - c X) + o2_coef <y, dY> needs only the small part. */
 DIFFATTN_API int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const void* k2,
                                        const void* v, const float* lambda, void* out, float* lse, void* o_maps,
-                                       float* rstd, diffattn_dtype dtype, int B, int H, int Hkv, int Lq, int Lk,
-                                       int d, int dv, int causal, int rmsnorm, float eps, void* stream);
+                                       float* rstd, float* o2_coef, diffattn_dtype dtype, int B, int H, int Hkv,
+                                       int Lq, int Lk, int d, int dv, int causal, int rmsnorm, float eps,
+                                       void* stream);
 
 /* Workspace, in bytes, for diffattn_bwd_v1.  0 for invalid sizes. */
 DIFFATTN_API size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int rmsnorm);
@@ -253,9 +264,10 @@ DIFFATTN_API size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq
  * gradient dX = r (dY - y <y, dY> / dv) first when rmsnorm != 0:
  *   q1, k1, q2, k2, v, lambda : the forward's inputs               (device)
  *   dout            : bf16 [B, H, Lq, 128], the gradient of out    (device)
- *   out, lse,
- *   o_maps, rstd    : from diffattn_fwd_v1_train (out and rstd are read
- *                     only with rmsnorm != 0 and may be NULL without) (device)
+ *   out, lse, o_maps,
+ *   rstd, o2_coef   : from diffattn_fwd_v1_train (out, rstd and o2_coef are
+ *                     read only with rmsnorm != 0 and may be NULL without)
+ *                                                                   (device)
  *   dq1, dq2        : bf16 [B, H, Lq, 64]; dk1, dk2 : bf16 [B, Hkv, Lk, 64];
  *   dv              : bf16 [B, Hkv, Lk, 128]; dlambda : f32 [H]    (device)
  *   ws              : diffattn_bwd_v1_workspace_size bytes, 16-byte aligned.
@@ -264,12 +276,15 @@ DIFFATTN_API size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq
  * tensors in the workspace, runs the V2 backward on them at scale 1/sqrt(64)
  * (the zero halves leave every score unchanged) and takes dQ1, dQ2, dK1 and
  * dK2 back out of the fixed halves of the packed gradients.  dK1, dK2 and dV
- * sum over the heads of a KV group. */
+ * sum over the heads of a KV group.  With rmsnorm != 0 the RMSNorm pass also
+ * forms the row terms D_m = dX·O_m from its f32 dX, D_2 as
+ * dX·o_maps[.., 1, ..] + o2_coef <y, dY> (see diffattn_fwd_v1_train). */
 DIFFATTN_API int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,
                                  const float* lambda, const void* dout, const void* out, const float* lse,
-                                 const void* o_maps, const float* rstd, void* dq1, void* dk1, void* dq2, void* dk2,
-                                 void* dv, float* dlambda, diffattn_dtype dtype, int B, int H, int Hkv, int Lq,
-                                 int Lk, int d, int dv_width, int causal, int rmsnorm, void* ws, size_t ws_bytes,
+                                 const void* o_maps, const float* rstd, const float* o2_coef, void* dq1, void* dk1,
+                                 void* dq2, void* dk2, void* dv, float* dlambda, diffattn_dtype dtype, int B, int H,
+                                 int Hkv, int Lq, int Lk, int d, int dv_width, int causal, int rmsnorm, void* ws,
+                                 size_t ws_bytes,
                                  void* stream);
 
 /* Workspace, in bytes, for diffattn_fwd_lowrank.  0 for invalid sizes. */

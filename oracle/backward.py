@@ -80,14 +80,21 @@ def head_backward(q1, k1, q2, k2, v, lam: float, dout, causal: bool, rms: bool =
     return dq1, dk1, dq2, dk2, dv, dlam
 
 
-def dlambda_terms(q1, k1, q2, k2, v, lam: float, dout, causal: bool, rms: bool = False, eps: float = 1e-5):
+def dlambda_terms(q1, k1, q2, k2, v, lam: float, dout, causal: bool, rms: bool = False, eps: float = 1e-5,
+                  orthogonal: bool = False):
     """The products dX * O_2 whose sum, negated, is one head's dlambda ([Lq, dv] fp64).
 
     Used to state the error a bf16 implementation can reach: dlambda sums
     Lq * dv products of two stored bf16 operands, so its rounding scales with
     the terms' size, not with the sum's.  With RMSNorm, dX is orthogonal to X
     (up to eps), and when the two maps are alike O_2 is nearly parallel to X,
-    so the sum is a small remainder of large terms."""
+    so the sum is a small remainder of large terms.
+
+    orthogonal=True (with rms): the products dX * (O_2 - c X), c = <O_2, X> /
+    <X, X> per row, i.e. with map 2's output reduced to its part orthogonal
+    to X.  Their sum differs from that of dX * O_2 only by c dX . X, which
+    is of order eps; an implementation that stores that part instead of O_2
+    has rounding of these terms' size."""
     q1, k1, q2, k2, v, dout = (_f64(t) for t in (q1, k1, q2, k2, v, dout))
     A1, A2 = maps(q1, k1, q2, k2, causal, 0, q1.shape[0])
     O1, O2 = A1 @ v, A2 @ v
@@ -96,6 +103,10 @@ def dlambda_terms(q1, k1, q2, k2, v, lam: float, dout, causal: bool, rms: bool =
         x = O1 - float(lam) * O2
         r = 1.0 / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + eps)
         dx = r * dx - (r ** 3 / x.shape[1]) * x * np.sum(x * dx, axis=1, keepdims=True)
+        if orthogonal:
+            xx = np.sum(x * x, axis=1, keepdims=True)
+            c = np.divide(np.sum(O2 * x, axis=1, keepdims=True), xx, out=np.zeros_like(xx), where=xx > 0)
+            return dx * (O2 - c * x)
     return dx * O2
 
 

@@ -122,28 +122,31 @@ def test_argument_errors_before_any_device_call(L):
     assert bw(P, P, P, P, P, P, P, Pm, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_MISALIGNED
     assert L.diffattn_bwd_v2_workspace_size(2, 64, 8192) > 0
     assert L.diffattn_bwd_v2_workspace_size(2, 63, 8192) == 0
-    # V1 training forward: (q1, k1, q2, k2, v, lambda, out, lse, o_maps, rstd, dtype, B, H, Hkv, Lq, Lk, d, dv,
-    # causal, rmsnorm, eps, s)
+    # V1 training forward: (q1, k1, q2, k2, v, lambda, out, lse, o_maps, rstd, o2_coef, dtype, B, H, Hkv, Lq, Lk,
+    # d, dv, causal, rmsnorm, eps, s)
     f1 = lambda *args: L.diffattn_fwd_v1_train(*args)  # noqa: E731
-    assert f1(P, P, P, P, P, P, P, P, P, P, da.F32, 1, 2, 1, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_UNSUPPORTED
-    assert f1(P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 2, 1, 8, 8, 128, 128, 1, 0, 1e-5, s) == da.ERR_UNSUPPORTED
-    assert f1(P, P, P, P, P, P, P, P, P, None, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 1, 1e-5, s) == da.ERR_INVALID_ARG
-    assert f1(P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 3, 2, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_INVALID_ARG
-    assert f1(P, P, P, P, P, P, P, P, Pm, P, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_MISALIGNED
-    # V1 backward: (q1, k1, q2, k2, v, lambda, dout, out, lse, o_maps, rstd, dq1, dk1, dq2, dk2, dv, dlambda,
-    # dtype, B, H, Hkv, Lq, Lk, d, dv, causal, rmsnorm, ws, bytes, s)
+    assert f1(P, P, P, P, P, P, P, P, P, P, P, da.F32, 1, 2, 1, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_UNSUPPORTED
+    assert f1(P, P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 2, 1, 8, 8, 128, 128, 1, 0, 1e-5, s) == da.ERR_UNSUPPORTED
+    assert f1(P, P, P, P, P, P, P, P, P, None, P, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 1, 1e-5, s) == da.ERR_INVALID_ARG
+    assert f1(P, P, P, P, P, P, P, P, P, P, None, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 1, 1e-5, s) == da.ERR_INVALID_ARG
+    assert f1(P, P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 3, 2, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_INVALID_ARG
+    assert f1(P, P, P, P, P, P, P, P, Pm, P, P, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 0, 1e-5, s) == da.ERR_MISALIGNED
+    # V1 backward: (q1, k1, q2, k2, v, lambda, dout, out, lse, o_maps, rstd, o2_coef, dq1, dk1, dq2, dk2, dv,
+    # dlambda, dtype, B, H, Hkv, Lq, Lk, d, dv, causal, rmsnorm, ws, bytes, s)
     b1 = lambda *args: L.diffattn_bwd_v1(*args)  # noqa: E731
-    ptrs = [P] * 17
+    ptrs = [P] * 18
     assert b1(*ptrs, da.F32, 1, 2, 1, 8, 8, 64, 128, 1, 0, P, 1 << 20, s) == da.ERR_UNSUPPORTED
     assert b1(*ptrs, da.BF16, 1, 2, 1, 8, 8, 128, 128, 1, 0, P, 1 << 20, s) == da.ERR_UNSUPPORTED
     assert b1(*ptrs, da.BF16, 1, 4, 3, 8, 8, 64, 128, 1, 0, P, 1 << 20, s) == da.ERR_INVALID_ARG
     no_out = ptrs[:7] + [None] + ptrs[8:]        # RMSNorm needs the forward output
     assert b1(*no_out, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
-    bad_dq = ptrs[:11] + [Pm] + ptrs[12:]
+    no_coef = ptrs[:11] + [None] + ptrs[12:]     # ... and the stored coefficient
+    assert b1(*no_coef, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    bad_dq = ptrs[:12] + [Pm] + ptrs[13:]
     assert b1(*bad_dq, da.BF16, 1, 2, 1, 8, 8, 64, 128, 1, 0, P, 1 << 20, s) == da.ERR_MISALIGNED
     w_rms = L.diffattn_bwd_v1_workspace_size(8, 16, 16, 4096, 4096, 1)
     w_plain = L.diffattn_bwd_v1_workspace_size(8, 16, 16, 4096, 4096, 0)
-    assert w_rms == w_plain + 8 * 16 * 4096 * 256 and w_plain > L.diffattn_bwd_v2_workspace_size(8, 32, 4096)
+    assert w_rms == w_plain + 8 * 16 * 4096 * (256 + 8) and w_plain > L.diffattn_bwd_v2_workspace_size(8, 32, 4096)
     assert L.diffattn_bwd_v1_workspace_size(1, 3, 2, 8, 8, 0) == 0
     assert L.diffattn_lambda_backward(P, P, P, P, P, 0, 8, P, P, P, P, s) == da.ERR_INVALID_ARG
     assert L.diffattn_lambda_backward(P, P, P, None, P, 2, 8, P, P, P, P, s) == da.ERR_INVALID_ARG

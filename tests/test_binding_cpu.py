@@ -81,7 +81,10 @@ def test_training_shapes_and_device():
     with pytest.raises(ValueError, match="rstd is required"):
         da.bwd_v1(q1, k1, q1, k1, v, lam1, d1, d1, lse1, om1, None, rmsnorm=True)
     with pytest.raises(ValueError, match="out has shape"):
-        da.bwd_v1(q1, k1, q1, k1, v, lam1, d1, z(1, 2, 15, 128), lse1, om1, z(1, 2, 16, dtype=f32), rmsnorm=True)
+        da.bwd_v1(q1, k1, q1, k1, v, lam1, d1, z(1, 2, 15, 128), lse1, om1, z(1, 2, 16, dtype=f32),
+                  z(1, 2, 16, dtype=f32), rmsnorm=True)
+    with pytest.raises(ValueError, match="o2c is required"):
+        da.bwd_v1(q1, k1, q1, k1, v, lam1, d1, d1, lse1, om1, z(1, 2, 16, dtype=f32), None, rmsnorm=True)
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
         da.bwd_v1(q1, k1, q1, k1, v, lam1, d1, None, lse1, om1, None, rmsnorm=False)
     p = [z(3, 8, dtype=f32) for _ in range(4)]
