@@ -55,9 +55,11 @@ struct BwdArgs {
   const float* lambda;   // [Hp]
   const float* lse_p;    // [B, Hp, 2, Lp] log-sum-exp (log2 units), +inf past Lq
   const float* dd;       // [B, Hp, 2, Lp] D_m, 0 past Lq
-  __nv_bfloat16* dq;     // [B, Hq, Lq, 128]
-  __nv_bfloat16* dk;     // [B, Hkv, Lk, 128]
+  __nv_bfloat16* dq;     // [B, Hq, Lq, 128]; V1: dQ1 [B, Hq/2, Lq, 64]
+  __nv_bfloat16* dk;     // [B, Hkv, Lk, 128]; V1: dK1 [B, Hkv, Lk, 64]
   __nv_bfloat16* dv;     // [B, Hkv, Lk, 128]
+  __nv_bfloat16* dq2;    // V1 only: dQ2 [B, Hq/2, Lq, 64]
+  __nv_bfloat16* dk2;    // V1 only: dK2 [B, Hkv, Lk, 64]
   int B, Hq, Hkv, Lq, Lk, Lp;
   int causal;
   float scale, scale_log2;
@@ -161,9 +163,17 @@ struct BwQSmem {
 // bf16 buffer (slices 0, 1 in chunk 0; 2, 3 in chunk 1).
 __device__ __forceinline__ uint32_t bw_slice(int s) { return (uint32_t)((s >> 1) * 32 + (s & 1) * 8); }
 
+// V1: the V1 layout ("差分注意力" tutorial, section V1 到 V2 的 diff): Q head
+// qh of the Hq = 2H heads is map qh & 1 of V1 head qh / 2, read from its own
+// 64-wide tensor (tmQ for map 1, tmQ2 for map 2; tmK, tmK2 likewise), and dQ
+// of map 2 goes to dq2.  The scores then contract over 64 dimensions and dQ
+// is 64 wide; dO, V and everything else are as in V2.
+template <bool V1>
 __global__ void __maxnreg__(168)
-bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdArgs a) {
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ2,
+              const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmK2, const __grid_constant__ CUtensorMap tmV, BwdArgs a) {
+  constexpr int QB = V1 ? 1 : 2;   // 64-wide boxes per Q / K row (the QK width / 64)
   extern __shared__ uint8_t smem_raw[];
   BwQSmem& S = *reinterpret_cast<BwQSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -210,20 +220,20 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // ------------------------------------------------------------ producer --
     if (lane == 0 && nT > 0) {
       const uint32_t qb = smem_u32(&S.q_full);
-      mbar_expect_tx(qb, 4 * PF_QBOX);
-      for (int x = 0; x < 2; ++x) {
-        tma_load_3d(smem_u32(S.q) + x * PF_QBOX, &tmQ, qb, 64 * x, r0, b * a.Hq + qh);
-        tma_load_3d(smem_u32(S.o) + x * PF_QBOX, &tmO, qb, 64 * x, r0, b * Hp + h);
-      }
+      const CUtensorMap* tq = (V1 && m) ? &tmQ2 : &tmQ;
+      const CUtensorMap* tk = (V1 && m) ? &tmK2 : &tmK;
+      mbar_expect_tx(qb, (QB + 2) * PF_QBOX);
+      for (int x = 0; x < QB; ++x) tma_load_3d(smem_u32(S.q) + x * PF_QBOX, tq, qb, 64 * x, r0, V1 ? b * Hp + h : b * a.Hq + qh);
+      for (int x = 0; x < 2; ++x) tma_load_3d(smem_u32(S.o) + x * PF_QBOX, &tmO, qb, 64 * x, r0, b * Hp + h);
       int last_use[BW_NS];
       for (int i = 0; i < BW_NS; ++i) last_use[i] = -1;
       for (int j = 0; j < nT; ++j) {
         const int st = j % BW_NS, use = j / BW_NS;
         if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
         const uint32_t kb = smem_u32(&S.k_full[st]), vb = smem_u32(&S.v_full[st]);
-        mbar_expect_tx(kb, 2 * PF_KBOX);
-        tma_load_3d(smem_u32(S.k[st]), &tmK, kb, 0, j * PF_BN, b * a.Hkv + g);
-        tma_load_3d(smem_u32(S.k[st]) + PF_KBOX, &tmK, kb, 64, j * PF_BN, b * a.Hkv + g);
+        mbar_expect_tx(kb, QB * PF_KBOX);
+        for (int x = 0; x < QB; ++x)
+          tma_load_3d(smem_u32(S.k[st]) + x * PF_KBOX, tk, kb, 64 * x, j * PF_BN, b * a.Hkv + g);
         mbar_expect_tx(vb, 2 * PF_KBOX);
         tma_load_3d(smem_u32(S.v[st]), &tmV, vb, 0, j * PF_BN, b * a.Hkv + g);
         tma_load_3d(smem_u32(S.v[st]) + PF_KBOX, &tmV, vb, 64, j * PF_BN, b * a.Hkv + g);
@@ -245,7 +255,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const int issuer = warp - 9;   // 0: dQ += dS K, 1: S = Q K^T and dP = dO V^T
       bool ok = true;
       if (issuer == 0) {
-        constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, true);
+        constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 64 * QB, true);
         const uint32_t k_mn0 = umma_desc_lo(smem_u32(S.k[0]), PF_KBOX);   // K as the N-major B operand
         for (int j = 0; ok && j < nT; ++j) {
           const int bb = j & 1;
@@ -276,13 +286,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           tc_fence_after();
           const uint32_t klo = k_lo0 + (uint32_t)st * KSTAGE, vlo = v_lo0 + (uint32_t)st * KSTAGE;
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
+          for (int s = 0; s < 4 * QB; ++s) {   // S = Q K^T over the QK width
             const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
             const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
             mma_ss_w(tmem + bb * 64, q_lo + ao, HI, klo + bo, HI, IDESC_S, s > 0);
           }
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
+          for (int s = 0; s < 8; ++s) {        // dP = dO V^T over the value width
             const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
             const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
             mma_ss_w(tmem + 128 + bb * 64, o_lo + ao, HI, vlo + bo, HI, IDESC_S, s > 0);
@@ -332,9 +342,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool have = nT == 0;
     float y[64];
     if (nT > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
-    if (have) {   // chunk ch writes dQ columns [64 ch, 64 ch + 64) of its rows
+    if (have && ch < QB) {   // chunk ch writes dQ columns [64 ch, 64 ch + 64) of its rows
       if (nT > 0) tc_fence_after();
-      __nv_bfloat16* base = a.dq + ((size_t)b * a.Hq + qh) * a.Lq * 128;
+      __nv_bfloat16* base = V1 ? (m ? a.dq2 : a.dq) + ((size_t)b * Hp + h) * a.Lq * 64
+                               : a.dq + ((size_t)b * a.Hq + qh) * a.Lq * 128;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
@@ -345,7 +356,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
         for (int i = 0; i < 32; ++i) y[cc * 32 + i] = nT > 0 ? __uint_as_float(o[i]) : 0.f;
       }
-      pf_store_rows(S.stage[warp], y, base + ch * 64, r0 + wq * 32, a.Lq, lane);
+      pf_store_rows(S.stage[warp], y, base + ch * 64, r0 + wq * 32, a.Lq, lane, 64 * QB);
     }
   }
 
@@ -420,9 +431,16 @@ __device__ __forceinline__ void bw_kv_elementwise(uint32_t tS, uint32_t tP, int 
   }
 }
 
+// V1: as for bwd_dq_kernel.  The CTA holds K1 and K2 side by side in its
+// 128-wide K tile; a step with map m scores against K_m's half and
+// accumulates dK_m into its own 64 columns of the dK accumulator (dK1 in the
+// first, dK2 in the second), which the epilogue writes to dk and dk2.
+template <bool V1>
 __global__ void __maxnreg__(168)
-bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, BwdArgs a) {
+bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK2,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
+               const __grid_constant__ CUtensorMap tmQ2, const __grid_constant__ CUtensorMap tmO, BwdArgs a) {
+  constexpr int QB = V1 ? 1 : 2;   // 64-wide boxes per Q row (the QK width / 64)
   extern __shared__ uint8_t smem_raw[];
   BwKSmem& S = *reinterpret_cast<BwKSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -479,8 +497,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     if (lane == 0 && nS > 0) {
       const uint32_t kvb = smem_u32(&S.kv_full);
       mbar_expect_tx(kvb, 4 * PF_QBOX);
-      for (int x = 0; x < 2; ++x) {
-        tma_load_3d(smem_u32(S.k) + x * PF_QBOX, &tmK, kvb, 64 * x, k0, b * a.Hkv + g);
+      for (int x = 0; x < 2; ++x) {   // V1: box x is K_{x+1}
+        tma_load_3d(smem_u32(S.k) + x * PF_QBOX, (V1 && x) ? &tmK2 : &tmK, kvb, V1 ? 0 : 64 * x, k0, b * a.Hkv + g);
         tma_load_3d(smem_u32(S.v) + x * PF_QBOX, &tmV, kvb, 64 * x, k0, b * a.Hkv + g);
       }
       int last_use[BW_NS];
@@ -491,11 +509,12 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         const int qh = step_head(i), rb = step_rb(i);
         const int hq = qh / 2, mq = qh & 1;
         const uint32_t fb = smem_u32(&S.st_full[st]);
-        mbar_expect_tx(fb, 4 * PF_KBOX + 2 * BW_RB * 4);
-        for (int x = 0; x < 2; ++x) {
-          tma_load_3d(smem_u32(S.q[st]) + x * PF_KBOX, &tmQ, fb, 64 * x, rb * BW_RB, b * a.Hq + qh);
+        mbar_expect_tx(fb, (QB + 2) * PF_KBOX + 2 * BW_RB * 4);
+        for (int x = 0; x < QB; ++x)
+          tma_load_3d(smem_u32(S.q[st]) + x * PF_KBOX, (V1 && mq) ? &tmQ2 : &tmQ, fb, 64 * x, rb * BW_RB,
+                      V1 ? b * Hp + hq : b * a.Hq + qh);
+        for (int x = 0; x < 2; ++x)
           tma_load_3d(smem_u32(S.o[st]) + x * PF_KBOX, &tmO, fb, 64 * x, rb * BW_RB, b * Hp + hq);
-        }
         const size_t stat = (((size_t)b * Hp + hq) * 2 + mq) * a.Lp + (size_t)rb * BW_RB;
         bulk_load(smem_u32(S.lse[st]), a.lse_p + stat, BW_RB * 4, fb);
         bulk_load(smem_u32(S.dd[st]), a.dd + stat, BW_RB * 4, fb);
@@ -514,6 +533,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       bool ok = true;
       if (issuer == 0) {
         constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, true);
+        constexpr uint32_t IDESC_DK = idesc_bf16_f32(128, 64 * QB, true);
         const uint32_t o_mn0 = umma_desc_lo(smem_u32(S.o[0]), PF_KBOX), q_mn0 = umma_desc_lo(smem_u32(S.q[0]), PF_KBOX);
         for (int i = 0; ok && i < nS; ++i) {
           const int bb = i & 1, st = i % BW_NS;
@@ -524,14 +544,19 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           const uint32_t olo = o_mn0 + (uint32_t)st * QSTAGE, qlo = q_mn0 + (uint32_t)st * QSTAGE;
           const int qh = step_head(i);
           const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
+          // V1: map m's dK lives in its own 64 columns and first receives a
+          // value at step m (steps 0 and 1 are the two maps of the group's
+          // first head); V2: one dK for both maps
+          const uint32_t dk_t = tmem + 384 + (V1 ? (uint32_t)((qh & 1) * 64) : 0u);
+          const bool dk_acc = V1 ? i > 1 : i > 0;
 #pragma unroll
           for (int s = 0; s < BW_RB / 16; ++s)   // dV += (w P)^T dO
             mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s), olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
                      (i > 0 || s > 0));
 #pragma unroll
           for (int s = 0; s < BW_RB / 16; ++s)   // dK += dS^T Q
-            mma_ts_w(tmem + 384, tmem + 128 + bb * 64 + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI,
-                     IDESC_ACC, (i > 0 || s > 0));
+            mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_DK,
+                     (dk_acc || s > 0));
           if (resid) {   // the bf16 residuals, 16 columns after each chunk's hi part
 #pragma unroll
             for (int s = 0; s < BW_RB / 16; ++s)
@@ -539,8 +564,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                        IDESC_ACC, 1);
 #pragma unroll
             for (int s = 0; s < BW_RB / 16; ++s)
-              mma_ts_w(tmem + 384, tmem + 128 + bb * 64 + bw_slice(s) + 16, qlo + (uint32_t)(s * (2048 >> 4)), HI,
-                       IDESC_ACC, 1);
+              mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s) + 16, qlo + (uint32_t)(s * (2048 >> 4)), HI,
+                       IDESC_DK, 1);
           }
           mma_commit(smem_u32(&S.s_free[bb]));
           mma_commit(smem_u32(&S.st_empty[st]));
@@ -558,11 +583,13 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             break;
           tc_fence_after();
           const uint32_t qlo = q_lo0 + (uint32_t)st * QSTAGE, olo = o_lo0 + (uint32_t)st * QSTAGE;
+          // V1: the step's map m scores against K_m, box m of the K tile
+          const uint32_t kmo = V1 ? (uint32_t)((step_head(i) & 1) * (PF_QBOX >> 4)) : 0u;
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
+          for (int s = 0; s < 4 * QB; ++s) {   // S^T = K Q^T over the QK width
             const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
             const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
-            mma_ss_w(tmem + bb * 64, k_lo + ao, HI, qlo + bo, HI, IDESC_S, s > 0);
+            mma_ss_w(tmem + bb * 64, k_lo + kmo + ao, HI, qlo + bo, HI, IDESC_S, s > 0);
           }
 #pragma unroll
           for (int s = 0; s < 8; ++s) {
@@ -612,11 +639,14 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     bool have = nS == 0;
     float y[64];
     if (nS > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
-    if (have) {   // chunk 0 writes dV, chunk 1 dK
+    if (have) {   // chunk 0 writes dV, chunk 1 dK (V1: dK1 then dK2, 64 columns each)
       if (nS > 0) tc_fence_after();
-      __nv_bfloat16* base = (ch ? a.dk : a.dv) + ((size_t)b * a.Hkv + g) * a.Lk * 128;
+      const size_t kv_row0 = ((size_t)b * a.Hkv + g) * a.Lk;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
+        __nv_bfloat16* base = !ch ? a.dv + kv_row0 * 128 + hf * 64
+                                  : (V1 ? (hf ? a.dk2 : a.dk) + kv_row0 * 64 : a.dk + kv_row0 * 128 + hf * 64);
+        const int stride = (V1 && ch) ? 64 : 128;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
@@ -627,7 +657,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
           for (int t = 0; t < 32; ++t) y[cc * 32 + t] = nS > 0 ? __uint_as_float(o[t]) : 0.f;
         }
-        pf_store_rows(S.stage[warp], y, base + hf * 64, k0 + wq * 32, a.Lk, lane);
+        pf_store_rows(S.stage[warp], y, base, k0 + wq * 32, a.Lk, lane, stride);
       }
     }
   }

@@ -124,8 +124,14 @@ int device_setup(DeviceInfo** out) {
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_paged_smem()));
-    CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_dq_smem()));
-    CUDA_TRY(cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_dkv_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)bwd_dq_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)bwd_dq_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(bwd_dkv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)bwd_dkv_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(bwd_dkv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)bwd_dkv_smem()));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -333,12 +339,16 @@ size_t bwd_ws_bytes(int B, int Hq, int Lq) {
   return 2 * align256((size_t)B * Hp * 2 * Lp * 4) + align256((size_t)B * Hp * (Lp / 64) * 4);
 }
 
-// dqk: the width that sets the score scale 1/sqrt(dqk) -- 128 for V2, 64 for
-// the packed V1 layout (whose zero halves leave the scores unchanged).
-int launch_backward_v2(const void* q, const void* k, const void* v, const float* lambda, const void* dout,
-                       const float* lse, const void* o_maps, void* dq, void* dk, void* dv, float* dlambda, int B,
-                       int Hq, int Hkv, int Lq, int Lk, int causal, void* ws, size_t ws_bytes, cudaStream_t s,
-                       int dqk = 128, const float* d_in = nullptr) {
+// Both layouts.  V2 (v1 = false): q [B, Hq, Lq, 128], k, v [B, Hkv, Lk, 128];
+// q2, k2, dq2 and dk2 are unused.  V1 (v1 = true): Q head qh of Hq = 2H is map
+// qh & 1 of V1 head qh / 2, so q, q2 are Q1, Q2 [B, H, Lq, 64], k, k2 are K1,
+// K2 [B, Hkv, Lk, 64], and dq, dq2, dk, dk2 their gradients; the score scale
+// is then 1/sqrt(64).  dout is [B, Hq/2, Lq, 128] in both.  d_in: the row
+// terms D_m formed upstream (V1 with RMSNorm), else null.
+int launch_backward(const void* q, const void* q2, const void* k, const void* k2, const void* v,
+                    const float* lambda, const void* dout, const float* lse, const void* o_maps, void* dq, void* dq2,
+                    void* dk, void* dk2, void* dv, float* dlambda, int B, int Hq, int Hkv, int Lq, int Lk, int causal,
+                    void* ws, size_t ws_bytes, cudaStream_t s, bool v1, const float* d_in = nullptr) {
   DeviceInfo* dev = nullptr;
   if (int e = device_setup(&dev)) return e;
   const size_t need = bwd_ws_bytes(B, Hq, Lq);
@@ -346,6 +356,7 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
     return fail(DIFFATTN_ERR_WORKSPACE, "backward workspace %zu B < required %zu B", ws_bytes, need);
   if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
   const int Hp = Hq / 2, Lp = bwd_rows_padded(Lq);
+  const int w = v1 ? 64 : 128;   // QK width
   float* lse_p = static_cast<float*>(ws);
   float* dd = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)B * Hp * 2 * Lp * 4));
   float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * align256((size_t)B * Hp * 2 * Lp * 4));
@@ -362,53 +373,63 @@ int launch_backward_v2(const void* q, const void* k, const void* v, const float*
   a.dq = static_cast<__nv_bfloat16*>(dq);
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dq2 = static_cast<__nv_bfloat16*>(dq2);
+  a.dk2 = static_cast<__nv_bfloat16*>(dk2);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.Lk = Lk; a.Lp = Lp;
   a.causal = causal ? 1 : 0;
-  a.scale = (float)(1.0 / std::sqrt((double)dqk));
-  a.scale_log2 = log2e_over_sqrt(dqk);
+  a.scale = (float)(1.0 / std::sqrt((double)w));
+  a.scale_log2 = log2e_over_sqrt(w);
   a.resid_tau = DIFFATTN_RESID_TAU;
   a.watch = make_watch(dev);
+  if (!v1) { q2 = q; k2 = k; }
   const long long Lk_map = Lk > 0 ? Lk : 1;   // a zero extent is not encodable; no key is then loaded
   const long long Lq_map = Lq > 0 ? Lq : 1;
+  const long long zq = v1 ? (long long)B * Hp : (long long)B * Hq;   // Q rows' third coordinate extent
   if (Lq > 0) {   // dQ: one CTA per 128 rows of each Q head
-    CUtensorMap mq, mo, mk, mv;
-    if (int e = make_map(&mq, q, 128, Lq_map, (long long)B * Hq, PF_BM)) return e;
+    CUtensorMap mq, mq2, mo, mk, mk2, mv;
+    if (int e = make_map(&mq, q, w, Lq_map, zq, PF_BM)) return e;
+    if (int e = make_map(&mq2, q2, w, Lq_map, zq, PF_BM)) return e;
     if (int e = make_map(&mo, dout, 128, Lq_map, (long long)B * Hp, PF_BM)) return e;
-    if (int e = make_map(&mk, Lk > 0 ? k : q, 128, Lk_map, (long long)B * Hkv, PF_BN)) return e;
-    if (int e = make_map(&mv, Lk > 0 ? v : q, 128, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+    if (int e = make_map(&mk, Lk > 0 ? k : q, w, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+    if (int e = make_map(&mk2, Lk > 0 ? k2 : q, w, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+    if (int e = make_map(&mv, Lk > 0 ? v : dout, 128, Lk_map, (long long)B * Hkv, PF_BN)) return e;
     const long long units = (long long)((Lq + PF_BM - 1) / PF_BM) * B * Hq;
-    bwd_dq_kernel<<<(unsigned)units, BW_THREADS, bwd_dq_smem(), s>>>(mq, mo, mk, mv, a);
+    if (v1)
+      bwd_dq_kernel<true><<<(unsigned)units, BW_THREADS, bwd_dq_smem(), s>>>(mq, mq2, mo, mk, mk2, mv, a);
+    else
+      bwd_dq_kernel<false><<<(unsigned)units, BW_THREADS, bwd_dq_smem(), s>>>(mq, mq2, mo, mk, mk2, mv, a);
     CUDA_TRY(cudaGetLastError());
   }
   if (Lk > 0) {   // dK, dV: one CTA per 128 keys of each KV head
-    CUtensorMap mk, mv, mq, mo;
-    if (int e = make_map(&mk, k, 128, Lk_map, (long long)B * Hkv, PF_BM)) return e;
+    CUtensorMap mk, mk2, mv, mq, mq2, mo;
+    if (int e = make_map(&mk, k, w, Lk_map, (long long)B * Hkv, PF_BM)) return e;
+    if (int e = make_map(&mk2, k2, w, Lk_map, (long long)B * Hkv, PF_BM)) return e;
     if (int e = make_map(&mv, v, 128, Lk_map, (long long)B * Hkv, PF_BM)) return e;
-    if (int e = make_map(&mq, Lq > 0 ? q : k, 128, Lq_map, (long long)B * Hq, BW_RB)) return e;
-    if (int e = make_map(&mo, Lq > 0 ? dout : k, 128, Lq_map, (long long)B * Hp, BW_RB)) return e;
+    if (int e = make_map(&mq, Lq > 0 ? q : k, w, Lq_map, zq, BW_RB)) return e;
+    if (int e = make_map(&mq2, Lq > 0 ? q2 : k, w, Lq_map, zq, BW_RB)) return e;
+    if (int e = make_map(&mo, Lq > 0 ? dout : v, 128, Lq_map, (long long)B * Hp, BW_RB)) return e;
     const long long units = (long long)((Lk + PF_BM - 1) / PF_BM) * B * Hkv;
-    bwd_dkv_kernel<<<(unsigned)units, BW_THREADS, bwd_dkv_smem(), s>>>(mk, mv, mq, mo, a);
+    if (v1)
+      bwd_dkv_kernel<true><<<(unsigned)units, BW_THREADS, bwd_dkv_smem(), s>>>(mk, mk2, mv, mq, mq2, mo, a);
+    else
+      bwd_dkv_kernel<false><<<(unsigned)units, BW_THREADS, bwd_dkv_smem(), s>>>(mk, mk2, mv, mq, mq2, mo, a);
     CUDA_TRY(cudaGetLastError());
   }
   return ok();
 }
 
-// V1 backward workspace: the packed [Q1|0], [0|Q2] rows and their gradient
-// (B*2H*Lq rows of 128), the packed [K1|K2] rows and their gradient
-// (B*Hkv*Lk rows of 128), with RMSNorm only the input gradient dX (B*H*Lq
-// rows of 128) and the row terms D_m [B*H, 2, Lq] f32, then the V2
-// backward's own workspace.
+// V1 backward workspace: with RMSNorm only, the input gradient dX (B*H*Lq
+// rows of 128) and the row terms D_m [B*H, 2, Lq] f32; then the backward's
+// own workspace.
 struct V1BwdLayout {
-  size_t qp, dqp, kp, dkp, dx, dd, bw, total;
+  size_t dx, dd, bw, total;
 };
 V1BwdLayout v1_bwd_layout(int B, int H, int Hkv, int Lq, int Lk, int rms) {
-  const size_t nq = (size_t)B * H * Lq, nk = (size_t)B * Hkv * Lk;
+  (void)Hkv;
+  (void)Lk;
+  const size_t nq = (size_t)B * H * Lq;
   V1BwdLayout l;
-  l.qp = 0;
-  l.dqp = l.qp + align256(nq * 512);
-  l.kp = l.dqp + align256(nq * 512);
-  l.dkp = l.kp + align256(nk * 256);
-  l.dx = l.dkp + align256(nk * 256);
+  l.dx = 0;
   l.dd = l.dx + (rms ? align256(nq * 256) : 0);
   l.bw = l.dd + (rms ? align256(nq * 2 * 4) : 0);
   l.total = l.bw + bwd_ws_bytes(B, 2 * H, Lq);
@@ -433,36 +454,21 @@ int launch_backward_v1(const void* q1, const void* k1, const void* q2, const voi
     return fail(DIFFATTN_ERR_WORKSPACE, "V1 backward workspace %zu B < required %zu B", ws_bytes, L.total);
   if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
   char* w = static_cast<char*>(ws);
-  auto at = [w](size_t off) { return reinterpret_cast<__nv_bfloat16*>(w + off); };
-  const long long nq = (long long)B * H * Lq, nk = (long long)B * Hkv * Lk;
-  if (nq + nk > 0) {
-    V1PackArgs pa{static_cast<const __nv_bfloat16*>(q1), static_cast<const __nv_bfloat16*>(q2),
-                  static_cast<const __nv_bfloat16*>(k1), static_cast<const __nv_bfloat16*>(k2), at(L.qp), at(L.kp),
-                  nq, nk, Lq};
-    v1_pack_kernel<<<stream_grid(dev, (nq + nk) * 8, V1A_THREADS), V1A_THREADS, 0, s>>>(pa);
-    CUDA_TRY(cudaGetLastError());
-  }
+  const long long nq = (long long)B * H * Lq;
   const void* g = dout;
   const float* d_in = nullptr;
   if (rms && nq > 0) {
     float* dd = reinterpret_cast<float*>(w + L.dd);
-    V1RmsArgs ra{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), rstd, at(L.dx),
-                 nq, static_cast<const __nv_bfloat16*>(o_maps), o2c, dd, Lq};
+    V1RmsArgs ra{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), rstd,
+                 reinterpret_cast<__nv_bfloat16*>(w + L.dx), nq, static_cast<const __nv_bfloat16*>(o_maps), o2c, dd,
+                 Lq};
     v1_rms_backward_kernel<<<stream_grid(dev, nq, V1A_THREADS / 32), V1A_THREADS, 0, s>>>(ra);
     CUDA_TRY(cudaGetLastError());
-    g = at(L.dx);
+    g = w + L.dx;
     d_in = dd;
   }
-  if (int e = launch_backward_v2(at(L.qp), at(L.kp), v, lambda, g, lse, o_maps, at(L.dqp), at(L.dkp), dv, dlambda,
-                                 B, 2 * H, Hkv, Lq, Lk, causal, w + L.bw, ws_bytes - L.bw, s, 64, d_in))
-    return e;
-  if (nq + nk > 0) {
-    V1UnpackArgs ua{at(L.dqp), at(L.dkp), static_cast<__nv_bfloat16*>(dq1), static_cast<__nv_bfloat16*>(dq2),
-                    static_cast<__nv_bfloat16*>(dk1), static_cast<__nv_bfloat16*>(dk2), nq, nk, Lq};
-    v1_unpack_kernel<<<stream_grid(dev, (nq + nk) * 8, V1A_THREADS), V1A_THREADS, 0, s>>>(ua);
-    CUDA_TRY(cudaGetLastError());
-  }
-  return ok();
+  return launch_backward(q1, q2, k1, k2, v, lambda, g, lse, o_maps, dq1, dq2, dk1, dk2, dv, dlambda, B, 2 * H, Hkv,
+                         Lq, Lk, causal, w + L.bw, ws_bytes - L.bw, s, true, d_in);
 }
 
 // Low-rank forward workspace: the per-head single-map outputs A1 V
@@ -732,8 +738,8 @@ int diffattn_bwd_v2(const void* q, const void* k, const void* v, const float* la
     return fail(DIFFATTN_ERR_INVALID_ARG, "null pointer");
   for (const void* p : std::initializer_list<const void*>{q, k, v, dout, o_maps, dq, dk, dv})
     if (p && !aligned16(p)) return fail(DIFFATTN_ERR_MISALIGNED, "bf16 tensor pointer %p is not 16-byte aligned", p);
-  return launch_backward_v2(q, k, v, lambda, dout, lse, o_maps, dq, dk, dv, dlambda, B, Hq, Hkv, Lq, Lk, causal,
-                            ws, ws_bytes, static_cast<cudaStream_t>(stream));
+  return launch_backward(q, nullptr, k, nullptr, v, lambda, dout, lse, o_maps, dq, nullptr, dk, nullptr, dv, dlambda,
+                         B, Hq, Hkv, Lq, Lk, causal, ws, ws_bytes, static_cast<cudaStream_t>(stream), false);
 }
 
 int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,

@@ -1,26 +1,12 @@
-// v1_adapter.cuh -- the V1-layout backward as a layout change around the V2 kernels.
+// v1_adapter.cuh -- the RMSNorm pass of the V1-layout backward.
 //
-// ("差分注意力" tutorial, section V1 到 V2 的 diff): head h of the V1 layout
-// scores Q1 K1^T and Q2 K2^T, each of width d, against one value tensor of
-// width 2d.  With d = 64 the pair (Q1, K1), (Q2, K2) is an exact instance of
-// the V2 pair (two Q heads over one 128-wide KV head):
-//
-//     Q'_1 = [Q1 | 0],   Q'_2 = [0 | Q2],   K' = [K1 | K2]
-//     Q'_1 K'^T = Q1 K1^T,   Q'_2 K'^T = Q2 K2^T            (the zeros add exact zeros)
-//
-// and the V2 gradients of the packed tensors hold the V1 ones in fixed halves:
-//
-//     dQ'_1 = s dS1 K' = [dQ1 | s dS1 K2]      -> dQ1 = dQ'_1[:, :64]
-//     dQ'_2 = s dS2 K' = [s dS2 K1 | dQ2]      -> dQ2 = dQ'_2[:, 64:]
-//     dK'   = s (dS1^T Q'_1 + dS2^T Q'_2) = [dK1 | dK2]
-//
-// with s = 1/sqrt(64).  The kernels here are the packing, the unpacking and
-// the gradient of the per-head RMSNorm that the V1 head applies to the
-// difference output (same section; unit weight, eps):
+// ("差分注意力" tutorial, section V1 到 V2 的 diff): a V1 head applies a
+// per-head RMSNorm (unit weight, eps) to its difference output x,
 //
 //     y = r x,  r = 1 / sqrt(mean(x^2) + eps)   =>   dX = r (dY - y <y, dY> / n)
 //
-// All three are HBM-bound streams of 16-byte (or 8-byte) vectors.
+// and the attention backward (backward_sm100.cuh, V1 instantiations) then
+// runs on dX.  This pass is an HBM-bound stream of 8-byte vectors.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -29,70 +15,6 @@
 namespace da {
 
 constexpr int V1A_THREADS = 256;
-
-// q1, q2 [B*H*Lq, 64] -> qp [B*2H*Lq, 128]; k1, k2 [B*Hkv*Lk, 64] -> kp [B*Hkv*Lk, 128].
-// Work item i < nq*8: chunk c = i % 8 (8 bf16) of Q row R = i / 8; then the K rows.
-struct V1PackArgs {
-  const __nv_bfloat16 *q1, *q2, *k1, *k2;
-  __nv_bfloat16 *qp, *kp;
-  long long nq, nk;   // Q rows (B*H*Lq), K rows (B*Hkv*Lk)
-  int Lq;
-};
-
-__global__ void __launch_bounds__(V1A_THREADS) v1_pack_kernel(V1PackArgs a) {
-  const long long total = (a.nq + a.nk) * 8;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int c = (int)(i & 7);
-    const long long R = i >> 3;
-    if (R < a.nq) {
-      const long long bh = R / a.Lq, l = R - bh * a.Lq;
-      const uint4 x1 = reinterpret_cast<const uint4*>(a.q1 + R * 64)[c];
-      const uint4 x2 = reinterpret_cast<const uint4*>(a.q2 + R * 64)[c];
-      uint4* r1 = reinterpret_cast<uint4*>(a.qp + ((2 * bh) * a.Lq + l) * 128);
-      uint4* r2 = reinterpret_cast<uint4*>(a.qp + ((2 * bh + 1) * a.Lq + l) * 128);
-      r1[c] = x1;
-      r1[c + 8] = zero;
-      r2[c] = zero;
-      r2[c + 8] = x2;
-    } else {
-      const long long K = R - a.nq;
-      uint4* r = reinterpret_cast<uint4*>(a.kp + K * 128);
-      r[c] = reinterpret_cast<const uint4*>(a.k1 + K * 64)[c];
-      r[c + 8] = reinterpret_cast<const uint4*>(a.k2 + K * 64)[c];
-    }
-  }
-}
-
-// The inverse selection: dq1 = dqp[2bh][:64], dq2 = dqp[2bh+1][64:], dk1 = dkp[:64], dk2 = dkp[64:].
-struct V1UnpackArgs {
-  const __nv_bfloat16 *dqp, *dkp;
-  __nv_bfloat16 *dq1, *dq2, *dk1, *dk2;
-  long long nq, nk;
-  int Lq;
-};
-
-__global__ void __launch_bounds__(V1A_THREADS) v1_unpack_kernel(V1UnpackArgs a) {
-  const long long total = (a.nq + a.nk) * 8;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int c = (int)(i & 7);
-    const long long R = i >> 3;
-    if (R < a.nq) {
-      const long long bh = R / a.Lq, l = R - bh * a.Lq;
-      reinterpret_cast<uint4*>(a.dq1 + R * 64)[c] =
-          reinterpret_cast<const uint4*>(a.dqp + ((2 * bh) * a.Lq + l) * 128)[c];
-      reinterpret_cast<uint4*>(a.dq2 + R * 64)[c] =
-          reinterpret_cast<const uint4*>(a.dqp + ((2 * bh + 1) * a.Lq + l) * 128)[c + 8];
-    } else {
-      const long long K = R - a.nq;
-      const uint4* r = reinterpret_cast<const uint4*>(a.dkp + K * 128);
-      reinterpret_cast<uint4*>(a.dk1 + K * 64)[c] = r[c];
-      reinterpret_cast<uint4*>(a.dk2 + K * 64)[c] = r[c + 8];
-    }
-  }
-}
 
 // dX = r (dY - y <y, dY> / 128) per 128-wide row, one warp per row, 4 elements
 // a lane.  y is the normalised forward output, r its saved 1/rms (0 for a row

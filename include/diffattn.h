@@ -272,11 +272,10 @@ DIFFATTN_API size_t diffattn_bwd_v1_workspace_size(int B, int H, int Hkv, int Lq
  *   dv              : bf16 [B, Hkv, Lk, 128]; dlambda : f32 [H]    (device)
  *   ws              : diffattn_bwd_v1_workspace_size bytes, 16-byte aligned.
  * The maps are those of diffattn_bwd_v2 with Q_1 K_1^T and Q_2 K_2^T as the
- * scores.  The call packs [Q1 | 0], [0 | Q2] and [K1 | K2] into 128-wide
- * tensors in the workspace, runs the V2 backward on them at scale 1/sqrt(64)
- * (the zero halves leave every score unchanged) and takes dQ1, dQ2, dK1 and
- * dK2 back out of the fixed halves of the packed gradients.  dK1, dK2 and dV
- * sum over the heads of a KV group.  With rmsnorm != 0 the RMSNorm pass also
+ * scores (scale 1/sqrt(64)), computed by V1 instances of the same kernels:
+ * the scores contract over the 64-wide Q_m, K_m read from their own tensors,
+ * and dQ_m, dK_m are 64-wide products.  dK1, dK2 and dV sum over the heads of
+ * a KV group.  With rmsnorm != 0 the RMSNorm pass also
  * forms the row terms D_m = dX·O_m from its f32 dX, D_2 as
  * dX·o_maps[.., 1, ..] + o2_coef <y, dY> (see diffattn_fwd_v1_train). */
 DIFFATTN_API int diffattn_bwd_v1(const void* q1, const void* k1, const void* q2, const void* k2, const void* v,

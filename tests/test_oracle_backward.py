@@ -146,10 +146,11 @@ def test_zero_upstream_gives_zero_gradients_and_linearity():
 
 
 def test_v1_gradients_are_v2_gradients_of_the_packed_layout():
-    """The library's V1 backward runs the V2 backward on [Q1|0], [0|Q2] and
-    [K1|K2].  Check that identity on the oracle: with d = 64 and the V2 scale
-    1/sqrt(128), Q' is multiplied by sqrt(2) so that the scores are Q_m K_m^T / 8;
-    the V1 gradients are then fixed halves of the packed ones."""
+    """The V1 and V2 oracle backwards agree through the packing identity: a V1
+    head is the V2 pair [Q1|0], [0|Q2] over [K1|K2].  With d = 64 and the V2
+    scale 1/sqrt(128), Q' is multiplied by sqrt(2) so that the scores are
+    Q_m K_m^T / 8; the V1 gradients are then fixed halves of the packed ones.
+    (Each backward is pinned on its own elsewhere; this ties the two.)"""
     rng = np.random.default_rng(29)
     B, H, Hkv, Lq, Lk, d = 1, 4, 2, 7, 9, 64
     q1, q2 = _rand((B, H, Lq, d), rng, 0.3), _rand((B, H, Lq, d), rng, 0.3)
@@ -182,3 +183,21 @@ def test_dlambda_terms_sum_to_dlambda(rms):
     if not rms:
         _, A2 = orc.maps(q1, k1, q2, k2, True)
         assert np.allclose(t, dout * (A2 @ v), rtol=1e-13, atol=0)
+
+
+def test_dlambda_orthogonal_terms_sum_to_dlambda_up_to_eps():
+    """With RMSNorm, the terms dX * (O_2 - c X) sum to -dlambda up to
+    c dX . X = c <y, dY> eps r^2, which vanishes with eps; and they are
+    smaller than dX * O_2 when the maps are alike."""
+    rng = np.random.default_rng(37)
+    q1, k1 = _rand((40, 8), rng, 0.05), _rand((40, 8), rng, 0.05)     # small scores: near-uniform maps
+    q2, k2 = _rand((40, 8), rng, 0.05), _rand((40, 8), rng, 0.05)
+    v, dout = _rand((40, 6), rng), _rand((40, 6), rng)
+    for eps in (1e-5, 0.0):
+        full = bwd.dlambda_terms(q1, k1, q2, k2, v, 0.5, dout, True, rms=True, eps=eps)
+        perp = bwd.dlambda_terms(q1, k1, q2, k2, v, 0.5, dout, True, rms=True, eps=eps, orthogonal=True)
+        dlam = bwd.head_backward(q1, k1, q2, k2, v, 0.5, dout, True, rms=True, eps=eps)[5]
+        assert np.isclose(-full.sum(), dlam, rtol=1e-12)
+        tol = 1e-12 if eps == 0.0 else 1e-3
+        assert abs(-perp.sum() - dlam) <= tol * np.abs(full).sum()
+        assert np.linalg.norm(perp) < 0.5 * np.linalg.norm(full)
