@@ -851,7 +851,7 @@ int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const floa
     CUDA_TRY(cudaMemsetAsync(a.tot, 0, sizeof(float) * (size_t)BH * (L.nc + 1) * r * LR_DV, s));
     CUDA_TRY(cudaMemsetAsync(a.ztot, 0, sizeof(float) * (size_t)BH * (L.nc + 1) * r, s));
   }
-  lr_prefix_kernel<<<BH, LR_DV, 0, s>>>(a);
+  lr_prefix_kernel<<<dim3((unsigned)r, BH), LR_DV, 0, s>>>(a);
   CUDA_TRY(cudaGetLastError());
   lr_emit_kernel<<<dim3((unsigned)((Lq + LR_C - 1) / LR_C), BH), LR_DV, 0, s>>>(a);
   CUDA_TRY(cudaGetLastError());

@@ -37,10 +37,13 @@
 // bf16-only P) would leave an error of A1 V's own rounding scale in it.  The
 // subtraction here is then the only rounding to bf16.
 //
-// One thread owns one of the 128 value columns and r <= LR_RMAX accumulators;
-// there is no shared memory and no wait.  Each kernel body is a host-device
-// function of (chunk, head, column), so the same code can be run over every
-// index on the host.
+// One thread owns one of the 128 value columns and r <= LR_RMAX accumulators.
+// The CTA first stages the factor rows its loop reads (the same for every
+// column) in shared memory; keys and rows are then taken several at a time
+// with their global loads issued first, so the passes are not bound by load
+// latency.  Each kernel body is a host-device function of (chunk, head,
+// column) that takes those rows as pointers, so the same code can be run over
+// every index on the host.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -99,28 +102,52 @@ __host__ __device__ inline void lr_key_range(const LowrankArgs& a, int c, long l
   }
 }
 
-__host__ __device__ inline void lr_add_key(const LowrankArgs& a, const __nv_bfloat16* vcol, const float* gh, long long j,
-                                           float (&S)[LR_RMAX], float (&z)[LR_RMAX]) {
-  const float vj = __bfloat162float(vcol[j * LR_DV]);
+// Adds keys [ks, ke) of one value column: S[t] += g_j[t] v_j, z[t] += g_j[t].
+// vcol: the column (keys LR_DV apart); gk: the G rows of these keys, gk[(j -
+// ks) r + t].  Keys in ascending order, U at a time with their V loads issued
+// first, so U loads are in flight per thread.
+__host__ __device__ inline void lr_add_keys(int r, const __nv_bfloat16* vcol, const float* gk, long long ks,
+                                            long long ke, float (&S)[LR_RMAX], float (&z)[LR_RMAX]) {
+  constexpr int U = 8;
+  long long j = ks;
+  for (; j + U <= ke; j += U) {
+    float vj[U];
 #pragma unroll
-  for (int t = 0; t < LR_RMAX; ++t)
-    if (t < a.r) {
-      const float gj = gh[j * a.r + t];
-      S[t] = fmaf(gj, vj, S[t]);
-      z[t] += gj;
+    for (int u = 0; u < U; ++u) vj[u] = __bfloat162float(vcol[(j + u) * LR_DV]);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float* g = gk + (j - ks + u) * r;
+#pragma unroll
+      for (int t = 0; t < LR_RMAX; ++t)
+        if (t < r) {
+          S[t] = fmaf(g[t], vj[u], S[t]);
+          z[t] += g[t];
+        }
     }
+  }
+  for (; j < ke; ++j) {
+    const float vj = __bfloat162float(vcol[j * LR_DV]);
+    const float* g = gk + (j - ks) * r;
+#pragma unroll
+    for (int t = 0; t < LR_RMAX; ++t)
+      if (t < r) {
+        S[t] = fmaf(g[t], vj, S[t]);
+        z[t] += g[t];
+      }
+  }
 }
 
-__host__ __device__ inline void lr_totals_body(const LowrankArgs& a, int c, int bh, int col) {
-  const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
+// Slot c of head bh, value column col; gk: the G rows of the slot's keys
+// [ks, ke) (lr_key_range), gk[(j - ks) r + t].
+__host__ __device__ inline void lr_totals_body(const LowrankArgs& a, int c, int bh, int col, const float* gk) {
+  const int b = bh / a.H, g = (bh % a.H) / (a.H / a.Hkv);
   long long ks, ke;
   lr_key_range(a, c, ks, ke);
   float S[LR_RMAX], z[LR_RMAX];
 #pragma unroll
   for (int t = 0; t < LR_RMAX; ++t) S[t] = z[t] = 0.f;
   const __nv_bfloat16* vcol = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lk * LR_DV + col;
-  const float* gh = a.G + (size_t)h * a.Lk * a.r;
-  for (long long j = ks; j < ke; ++j) lr_add_key(a, vcol, gh, j, S, z);
+  lr_add_keys(a.r, vcol, gk, ks, ke, S, z);
   const size_t slot = (size_t)bh * (a.nc + 1) + c;
 #pragma unroll
   for (int t = 0; t < LR_RMAX; ++t)
@@ -130,30 +157,52 @@ __host__ __device__ inline void lr_totals_body(const LowrankArgs& a, int c, int 
     }
 }
 
-__host__ __device__ inline void lr_prefix_body(const LowrankArgs& a, int bh, int col) {
-  for (int t = 0; t < a.r; ++t) {
-    float run = 0.f, zrun = 0.f;
-    for (int c = 0; c < a.nc; ++c) {
-      const size_t slot = (size_t)bh * (a.nc + 1) + c;
-      float* p = a.tot + (slot * a.r + t) * LR_DV + col;
-      const float x = *p;
-      *p = run;
-      run += x;
-      if (col == 0) {
-        float* q = a.ztot + slot * a.r + t;
-        const float y = *q;
-        *q = zrun;
-        zrun += y;
+// Exclusive prefix over the slots of head bh, rank index t, value column col
+// (and, for col == 0, of the z sums), plus the grand total in slot nc.  Eight
+// slots' values are loaded before their prefix is formed.
+__host__ __device__ inline void lr_prefix_body(const LowrankArgs& a, int bh, int t, int col) {
+  constexpr int U = 8;
+  float run = 0.f, zrun = 0.f;
+  const size_t s0 = (size_t)bh * (a.nc + 1);
+  for (int c0 = 0; c0 < a.nc; c0 += U) {
+    float x[U], y[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (c0 + u < a.nc) {
+        x[u] = a.tot[((s0 + c0 + u) * a.r + t) * LR_DV + col];
+        if (col == 0) y[u] = a.ztot[(s0 + c0 + u) * a.r + t];
       }
-    }
-    const size_t last = (size_t)bh * (a.nc + 1) + a.nc;
-    a.tot[(last * a.r + t) * LR_DV + col] = run;
-    if (col == 0) a.ztot[last * a.r + t] = zrun;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (c0 + u < a.nc) {
+        a.tot[((s0 + c0 + u) * a.r + t) * LR_DV + col] = run;
+        run += x[u];
+        if (col == 0) {
+          a.ztot[(s0 + c0 + u) * a.r + t] = zrun;
+          zrun += y[u];
+        }
+      }
   }
+  a.tot[((s0 + a.nc) * a.r + t) * LR_DV + col] = run;
+  if (col == 0) a.ztot[(s0 + a.nc) * a.r + t] = zrun;
 }
 
-// Row chunk c (rows [c LR_C, min(Lq, (c+1) LR_C))) of head bh, value column col.
-__host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh, int col) {
+// The rows of row chunk c and the keys they add (causal: row i adds key
+// i + Lk - Lq; none when unmasked), clamped to the tensors.
+__host__ __device__ inline void lr_emit_range(const LowrankArgs& a, int c, long long& r0, long long& r1,
+                                              long long& k0, long long& k1) {
+  r0 = (long long)c * LR_C;
+  r1 = r0 + LR_C < a.Lq ? r0 + LR_C : a.Lq;
+  const long long off = (long long)a.Lk - a.Lq;
+  k0 = a.causal ? lr_clamp(r0 + off, a.Lk) : 0;
+  k1 = a.causal ? lr_clamp(r1 + off, a.Lk) : 0;
+}
+
+// Row chunk c (rows [r0, r1)) of head bh, value column col.  fk: the F rows
+// of the chunk, fk[(i - r0) r + t]; gk: the G rows of the keys the rows add,
+// gk[(j - k0) r + t] (lr_emit_range).
+__host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh, int col, const float* fk,
+                                             const float* gk) {
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
   const size_t slot = (size_t)bh * (a.nc + 1) + (a.causal ? a.n_lead + c : a.nc);
   float S[LR_RMAX], z[LR_RMAX];
@@ -162,42 +211,77 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
     S[t] = t < a.r ? a.tot[(slot * a.r + t) * LR_DV + col] : 0.f;
     z[t] = t < a.r ? a.ztot[slot * a.r + t] : 0.f;
   }
+  long long r0, r1, k0, k1;
+  lr_emit_range(a, c, r0, r1, k0, k1);
   const long long off = (long long)a.Lk - a.Lq;
   const __nv_bfloat16* vcol = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lk * LR_DV + col;
-  const float* gh = a.G + (size_t)h * a.Lk * a.r;
-  const long long r0 = (long long)c * LR_C;
-  const long long r1 = r0 + LR_C < a.Lq ? r0 + LR_C : a.Lq;
   const float lam = a.lambda[h];
-  const float* fh = a.F + (size_t)h * a.Lq * a.r;
   const float* arow = a.a1v + (size_t)bh * a.Lq * LR_DV + col;
   __nv_bfloat16* orow = a.out + (size_t)bh * a.Lq * LR_DV + col;
-  for (long long i = r0; i < r1; ++i) {
-    if (a.causal) {
-      const long long j = i + off;
-      if (j >= 0 && j < a.Lk) lr_add_key(a, vcol, gh, j, S, z);
-    }
-    float num = 0.f, den = 0.f;
+  constexpr int U = 4;
+  for (long long i0 = r0; i0 < r1; i0 += U) {
+    // this group's loads first: A1 V of each row and the V value of the key it adds
+    float av[U], vj[U];
 #pragma unroll
-    for (int t = 0; t < LR_RMAX; ++t)
-      if (t < a.r) {
-        const float f = fh[i * a.r + t];
-        num = fmaf(f, S[t], num);
-        den = fmaf(f, z[t], den);
+    for (int u = 0; u < U; ++u) {
+      const long long i = i0 + u, j = i + off;
+      av[u] = i < r1 ? arow[i * LR_DV] : 0.f;
+      vj[u] = (a.causal && i < r1 && j >= 0 && j < a.Lk) ? __bfloat162float(vcol[j * LR_DV]) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = i0 + u, j = i + off;
+      if (i >= r1) break;
+      if (a.causal && j >= 0 && j < a.Lk) {
+        const float* gj = gk + (j - k0) * a.r;
+#pragma unroll
+        for (int t = 0; t < LR_RMAX; ++t)
+          if (t < a.r) {
+            S[t] = fmaf(gj[t], vj[u], S[t]);
+            z[t] += gj[t];
+          }
       }
-    const float nv = den > 0.f ? num / den : 0.f;
-    orow[i * LR_DV] = __float2bfloat16_rn(arow[i * LR_DV] - lam * nv);
+      const float* fi = fk + (i - r0) * a.r;
+      float num = 0.f, den = 0.f;
+#pragma unroll
+      for (int t = 0; t < LR_RMAX; ++t)
+        if (t < a.r) {
+          num = fmaf(fi[t], S[t], num);
+          den = fmaf(fi[t], z[t], den);
+        }
+      const float nv = den > 0.f ? num / den : 0.f;
+      orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * nv);
+    }
   }
 }
 
 #ifdef __CUDACC__
+// Copies n floats from global memory into shared memory, all threads of the CTA.
+__device__ __forceinline__ void lr_stage(float* dst, const float* src, long long n) {
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src[i];
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(LR_DV) lr_totals_kernel(LowrankArgs a) {
-  lr_totals_body(a, (int)blockIdx.x, (int)blockIdx.y, (int)threadIdx.x);
+  __shared__ float sg[LR_C * LR_RMAX];
+  const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
+  long long ks, ke;
+  lr_key_range(a, c, ks, ke);
+  lr_stage(sg, a.G + ((size_t)h * a.Lk + ks) * a.r, (ke - ks) * a.r);
+  lr_totals_body(a, c, bh, (int)threadIdx.x, sg);
 }
 __global__ void __launch_bounds__(LR_DV) lr_prefix_kernel(LowrankArgs a) {
-  lr_prefix_body(a, (int)blockIdx.x, (int)threadIdx.x);
+  lr_prefix_body(a, (int)blockIdx.y, (int)blockIdx.x, (int)threadIdx.x);
 }
 __global__ void __launch_bounds__(LR_DV) lr_emit_kernel(LowrankArgs a) {
-  lr_emit_body(a, (int)blockIdx.x, (int)blockIdx.y, (int)threadIdx.x);
+  __shared__ float sf[LR_C * LR_RMAX];
+  __shared__ float sg[LR_C * LR_RMAX];
+  const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
+  long long r0, r1, k0, k1;
+  lr_emit_range(a, c, r0, r1, k0, k1);
+  for (long long i = threadIdx.x; i < (r1 - r0) * a.r; i += blockDim.x) sf[i] = a.F[((size_t)h * a.Lq + r0) * a.r + i];
+  lr_stage(sg, a.G + ((size_t)h * a.Lk + k0) * a.r, (k1 - k0) * a.r);
+  lr_emit_body(a, c, bh, (int)threadIdx.x, sf, sg);
 }
 #endif
 

@@ -54,16 +54,28 @@ int main(int argc, char** argv) {
   a.tot = tot.data();
   a.ztot = ztot.data();
 
+  // The kernels stage the factor rows a CTA reads in shared memory; here the
+  // bodies read them in place, through pointers at the same offsets.
   if (a.nc > 0 && Lk > 0)
     for (int bh = 0; bh < (int)BH; ++bh)
-      for (int c = 0; c < a.nc; ++c)
-        for (int col = 0; col < da::LR_DV; ++col) da::lr_totals_body(a, c, bh, col);
+      for (int c = 0; c < a.nc; ++c) {
+        long long ks, ke;
+        da::lr_key_range(a, c, ks, ke);
+        const float* gk = G.data() + ((size_t)(bh % H) * Lk + ks) * r;
+        for (int col = 0; col < da::LR_DV; ++col) da::lr_totals_body(a, c, bh, col, gk);
+      }
   for (int bh = 0; bh < (int)BH; ++bh)
-    for (int col = 0; col < da::LR_DV; ++col) da::lr_prefix_body(a, bh, col);
+    for (int t = 0; t < r; ++t)
+      for (int col = 0; col < da::LR_DV; ++col) da::lr_prefix_body(a, bh, t, col);
   const int nrc = (Lq + da::LR_C - 1) / da::LR_C;
   for (int bh = 0; bh < (int)BH; ++bh)
-    for (int c = 0; c < nrc; ++c)
-      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col);
+    for (int c = 0; c < nrc; ++c) {
+      long long r0, r1, k0, k1;
+      da::lr_emit_range(a, c, r0, r1, k0, k1);
+      const float* fk = F.data() + ((size_t)(bh % H) * Lq + r0) * r;
+      const float* gk = G.data() + ((size_t)(bh % H) * Lk + k0) * r;
+      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, fk, gk);
+    }
 
   FILE* g = fopen(argv[2], "wb");
   if (!g) return 6;
