@@ -247,16 +247,16 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
   if (o_f32 != nullptr)               // single-map outputs (V2 layout)
-    prefill_kernel<128, PF_SINGLE><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv,
+    prefill_kernel<128, PF_SINGLE><<<(unsigned)units, pf_threads(PF_SINGLE), prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv,
                                                                                            a);
   else if (lse != nullptr && dqk == 128)   // training forward (V2)
-    prefill_kernel<128, PF_TRAIN><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<128, PF_TRAIN><<<(unsigned)units, pf_threads(PF_TRAIN), prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (lse != nullptr)            // training forward (V1, d = 64)
-    prefill_kernel<64, PF_TRAIN><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<64, PF_TRAIN><<<(unsigned)units, pf_threads(PF_TRAIN), prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (dqk == 64)
-    prefill_kernel<64><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<64><<<(unsigned)units, pf_threads(PF_INFER), prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else
-    prefill_kernel<128><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<128><<<(unsigned)units, pf_threads(PF_INFER), prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   CUDA_TRY(cudaGetLastError());
   return ok();
 }

@@ -218,12 +218,14 @@ def test_v1_training_forward_statistics():
         r = 1.0 / np.sqrt(np.mean(x * x, axis=1) + 1e-5)
         assert np.max(np.abs(rstd[0, h].cpu().numpy() - r) / r) <= 1e-2
         assert _rel(om[0, h, 0], A[0] @ vd) <= BF16_TOL
-        # map 2 is stored as its part orthogonal to x, with c eps r^2 per row
+        # map 2 is stored as its part orthogonal to x, with c eps r^2 per row.
+        # That part is a small difference of the kernel's own O_2 and x, which
+        # carry the bf16 rounding of P: its error is on the scale of O_2.
         o2 = A[1] @ vd
         c = np.sum(o2 * x, axis=1) / np.sum(x * x, axis=1)
         perp = o2 - c[:, None] * x
-        assert _rel(om[0, h, 1], perp) <= BF16_TOL
         got_perp = om[0, h, 1].double().cpu().numpy()
+        assert np.max(np.abs(got_perp - perp)) <= BF16_TOL * np.max(np.abs(o2))
         assert np.max(np.abs(np.sum(got_perp * x, axis=1))) <= 2e-2 * np.max(np.abs(np.sum(o2 * x, axis=1)))
         assert _rel(o2c[0, h], c * 1e-5 * r * r) <= BF16_TOL
 
