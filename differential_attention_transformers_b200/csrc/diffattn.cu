@@ -124,6 +124,7 @@ int device_setup(DeviceInfo** out) {
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_paged_smem()));
+    CUDA_TRY(cudaFuncSetAttribute(lr_emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LR_EMIT_SMEM));
     CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)bwd_dq_smem()));
     CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -247,16 +248,16 @@ int launch_prefill(const void* q1, const void* q2, const void* k1, const void* k
   const long long units = (long long)a.n_rb * B * Hout;
   if (units > 0x7fffffffLL) return fail(DIFFATTN_ERR_UNSUPPORTED, "too many row blocks");
   if (o_f32 != nullptr)               // single-map outputs (V2 layout)
-    prefill_kernel<128, PF_SINGLE><<<(unsigned)units, pf_threads(PF_SINGLE), prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv,
+    prefill_kernel<128, PF_SINGLE><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv,
                                                                                            a);
   else if (lse != nullptr && dqk == 128)   // training forward (V2)
-    prefill_kernel<128, PF_TRAIN><<<(unsigned)units, pf_threads(PF_TRAIN), prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<128, PF_TRAIN><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (lse != nullptr)            // training forward (V1, d = 64)
-    prefill_kernel<64, PF_TRAIN><<<(unsigned)units, pf_threads(PF_TRAIN), prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<64, PF_TRAIN><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else if (dqk == 64)
-    prefill_kernel<64><<<(unsigned)units, pf_threads(PF_INFER), prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<64><<<(unsigned)units, PF_THREADS, prefill_smem<64>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   else
-    prefill_kernel<128><<<(unsigned)units, pf_threads(PF_INFER), prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
+    prefill_kernel<128><<<(unsigned)units, PF_THREADS, prefill_smem<128>(), s>>>(mq1, mq2, mk1, mk2, mv, a);
   CUDA_TRY(cudaGetLastError());
   return ok();
 }
@@ -853,7 +854,7 @@ int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const floa
   }
   lr_prefix_kernel<<<dim3((unsigned)r, BH), LR_DV, 0, s>>>(a);
   CUDA_TRY(cudaGetLastError());
-  lr_emit_kernel<<<dim3((unsigned)((Lq + LR_C - 1) / LR_C), BH), LR_DV, 0, s>>>(a);
+  lr_emit_kernel<<<dim3((unsigned)((Lq + LR_C - 1) / LR_C), BH), LR_DV, LR_EMIT_SMEM, s>>>(a);
   CUDA_TRY(cudaGetLastError());
   return ok();
 }

@@ -10,13 +10,12 @@
 // serves both maps: in V2 both maps share K and V; in V1 the tile holds K1,
 // K2 and the shared V.
 //
-// Warp roles (416 threads; 384 in the training and single-map kernels):
+// Warp roles (352 threads):
 //   warps 0-3  softmax of map 1 (thread i <-> query row i <-> TMEM lane i)
 //   warps 4-7  softmax of map 2
 //   warp  8    TMA producer; allocates / frees TMEM
-//   warps 9-10 PV issuers of map 1 and map 2 (one thread each)
-//   warps 11-12 QK issuers of map 1 and map 2 (one thread each); the
-//              training and single-map kernels have one, warp 11, for both
+//   warp  9    PV issuer (one thread)
+//   warp 10    QK issuer (one thread)
 // Keys are processed in tiles of 64.  TMEM (512 columns) holds two S buffers
 // per map -- S1[0] [0,64) S1[1] [64,128) S2[0] [128,192) S2[1] [192,256) --
 // and the accumulators O1 [256,384) O2 [384,512).  While a map's softmax works
@@ -25,10 +24,10 @@
 // S_m(j) as bf16 P_hi in the buffer's columns [0,32) and, for heads that need
 // it, the bf16 residual P_lo = P - P_hi in [32,64); both accumulate into O_m.
 // The tensor pipe takes MMAs from a very shallow queue, so a single issuing
-// thread that stops to test a barrier leaves it idle.  Separate issuers keep
-// it fed: PV_m(j) is issued when P_m(j) is stored, S_m(j+2) into the buffer
-// PV_m(j) read once that PV has completed (s_free); each issuer's waits
-// overlap the others' MMAs.
+// thread that stops to test a barrier leaves it idle.  Two issuers keep it
+// fed: one issues PV_m(j) when P_m(j) is stored, the other issues S_m(j+2)
+// into the buffer PV_m(j) read, once that PV has completed (s_free); each
+// one's waits overlap the other's MMAs.
 // Shared memory: Q1, Q2 tiles (128 rows), then NS stages of {K tile(s), V
 // tile} of 64 keys; every tile is a set of boxes of 128-byte rows in the TMA
 // 128-byte swizzle, which is the canonical K-major (Q, K) / MN-major (V) UMMA
@@ -43,13 +42,7 @@ constexpr int PF_BM = 128;         // query rows per CTA
 constexpr int PF_BN = 64;          // keys per tile
 constexpr int PF_DV = 128;         // value width
 constexpr int PF_NS = 4;           // K/V pipeline stages
-// Threads: 8 softmax warps, the producer, two PV issuers and, for the
-// inference kernel, two QK issuers (one per map); the training and
-// single-map kernels keep one QK issuer for both maps, because a 13th warp
-// puts 4 warps on one SM sub-partition and caps them at 128 registers, below
-// what their epilogues hold.
-constexpr int pf_qk_issuers(int mode) { return mode == 0 ? 2 : 1; }
-constexpr int pf_threads(int mode) { return 32 * (11 + pf_qk_issuers(mode)); }
+constexpr int PF_THREADS = 352;
 constexpr int PF_QBOX = 128 * 128; // bytes of one 128-row x 64-element bf16 box (Q)
 constexpr int PF_KBOX = 64 * 128;  // bytes of one 64-row x 64-element bf16 box (K, V)
 constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -122,7 +115,7 @@ struct PfSmem {
   uint64_t o_final;
   uint64_t xl;      // epilogue exchange of l (256 arrivals)
   uint64_t xs;      // epilogue exchange of RMS partial sums (256 arrivals)
-  uint64_t drain[4];      // per issuer: all its MMAs complete
+  uint64_t drain[2];      // per issuer: all its MMAs complete
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -228,7 +221,7 @@ __device__ __forceinline__ void pf_store_rows_f32(uint8_t* st, const float (&y)[
 // PF_SINGLE (single-map outputs in f32); a template argument so the inference
 // kernel carries none of the other modes' code.
 template <int DQK, int MODE = PF_INFER>
-__global__ void __launch_bounds__(pf_threads(MODE), 1)
+__global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
                const __grid_constant__ CUtensorMap tmV, PrefillArgs a) {
@@ -273,8 +266,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
   kend = max(0LL, min(kend, (long long)a.Lk));
   const int nT = (int)((kend + PF_BN - 1) / PF_BN);
   // Residual choice per map: one lambda per output head, or in single-map
-  // mode each head's own.
-  const bool resid1 = fabsf(1.f - a.lambda[SINGLE ? 2 * h : h]) < a.resid_tau;
+  // mode each head's own.  The training forward with RMSNorm keeps it for
+  // every head: the backward's dlambda = -sum dX . O_2 is then a small
+  // remainder of terms (dX is orthogonal to X, O_2 nearly parallel to it
+  // when the maps are alike), and the 2^-9 rounding of a bf16-only P in O_2
+  // would not be orthogonal to X.
+  const bool all_resid = TRAIN && a.rms;
+  const bool resid1 = all_resid || fabsf(1.f - a.lambda[SINGLE ? 2 * h : h]) < a.resid_tau;
   const bool resid2 = SINGLE ? fabsf(1.f - a.lambda[2 * h + 1]) < a.resid_tau : resid1;
 
   if (threadIdx.x == 0) {
@@ -282,7 +280,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     for (int i = 0; i < PF_NS; ++i) {
       mbar_init(smem_u32(&S.k_full[i]), 1);
       mbar_init(smem_u32(&S.v_full[i]), 1);
-      mbar_init(smem_u32(&S.kv_empty[i]), 2);   // both maps' PV issuers
+      mbar_init(smem_u32(&S.kv_empty[i]), 1);
     }
     for (int m = 0; m < 2; ++m) {
       for (int bb = 0; bb < 2; ++bb) {
@@ -291,9 +289,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
         mbar_init(smem_u32(&S.s_free[m][bb]), 1);
       }
       mbar_init(smem_u32(&S.o_done[m]), 1);
+      mbar_init(smem_u32(&S.drain[m]), 1);
     }
-    for (int i = 0; i < 2 + pf_qk_issuers(MODE); ++i) mbar_init(smem_u32(&S.drain[i]), 1);
-    mbar_init(smem_u32(&S.o_final), 2);         // both maps' PV issuers
+    mbar_init(smem_u32(&S.o_final), 1);
     mbar_init(smem_u32(&S.xl), 256);
     mbar_init(smem_u32(&S.xs), 256);
     S.abort_flag = 0;
@@ -350,77 +348,65 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     }
   } else if (warp >= 9) {
     // --------------------------------------------------------- MMA issuers --
-    // One issuing thread per map for PV and, in the inference kernel, one per
-    // map for QK: PV of map 0, PV of map 1, QK of map 0, QK of map 1.  Each
-    // map's chain -- P_m(j) stored -> PV_m(j) -> S_m(j+2) -> softmax -- then
-    // runs at its own pace.  With one issuer per product serving both maps in
-    // turn, the map that finished first waited for the other one's P (or S
-    // buffer) before its own MMA was issued: in-kernel clock traces showed P
-    // waiting a median 1.5k cycles for its PV, a tile period of 1.8k cycles
-    // against a softmax of 1.2k.
     if (lane == 0 && nT > 0) {
       // Descriptor words computed once; per MMA only the low word moves.
       constexpr uint32_t HI = umma_desc_hi(1024);
       constexpr uint32_t KSTAGE = (2 * PF_KBOX) >> 4;          // stage stride in 16-byte units
-      const int issuer = warp - 9;                             // 0, 1: PV of map 0, 1; 2, 3: QK of map 0, 1
-      const int m = issuer & 1;
+      const int issuer = warp - 9;                             // 0: PV, 1: QK
       bool ok = true;
-      if (issuer < 2) {
-        // PV_m(j) as soon as the softmax has stored P_m(j).
+      if (issuer == 0) {
+        // PV_1(j), PV_2(j) as soon as the softmax has stored each map's P.
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, PF_DV, true);
         const uint32_t v_lo0 = umma_desc_lo(smem_u32(S.v[0]), PF_KBOX);
-        const bool resid = m ? resid2 : resid1;
-        const uint32_t o = tmem + 256 + m * 128;
         for (int j = 0; ok && j < nT; ++j) {
           const int bb = j & 1, ph = (j >> 1) & 1;
           const uint32_t vlo = v_lo0 + (uint32_t)(j % PF_NS) * KSTAGE;
           if (!(ok = wait_bar(smem_u32(&S.v_full[j % PF_NS]), (j / PF_NS) & 1, abort_flag, a.watch))) break;
-          if (!(ok = wait_bar(smem_u32(&S.p_full[m][bb]), ph, abort_flag, a.watch))) break;
-          tc_fence_after();
-          const uint32_t p = tmem + (uint32_t)(m * 128 + bb * 64);
+          for (int m = 0; m < 2; ++m) {
+            if (!(ok = wait_bar(smem_u32(&S.p_full[m][bb]), ph, abort_flag, a.watch))) break;
+            tc_fence_after();
+            const uint32_t p = tmem + (uint32_t)(m * 128 + bb * 64), o = tmem + 256 + m * 128;
 #pragma unroll
-          for (int s = 0; s < PF_BN / 16; ++s)
-            mma_ts_w(o, p + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, (j > 0 || s > 0));
-          if (resid) {
+            for (int s = 0; s < PF_BN / 16; ++s)
+              mma_ts_w(o, p + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, (j > 0 || s > 0));
+            if (m ? resid2 : resid1) {
 #pragma unroll
-            for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
-              mma_ts_w(o, p + 32 + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, 1);
+              for (int s = 0; s < PF_BN / 16; ++s)   // residual part of P
+                mma_ts_w(o, p + 32 + s * 8, vlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_PV, 1);
+            }
+            mma_commit(smem_u32(&S.o_done[m]));
+            mma_commit(smem_u32(&S.s_free[m][bb]));
           }
-          mma_commit(smem_u32(&S.o_done[m]));
-          mma_commit(smem_u32(&S.s_free[m][bb]));
-          // The stage is free once both maps' PV(j) are complete (kv_empty
-          // counts two arrivals); its K was read by S_m(j), complete before
-          // P_m(j) existed.
+          if (!ok) break;
+          // The stage's K was read by S(j), complete before P(j) existed.
           mma_commit(smem_u32(&S.kv_empty[j % PF_NS]));
         }
         if (ok) mma_commit(smem_u32(&S.o_final));
       } else {
         // S_m(j) once K(j) has landed and, for j >= 2, PV_m(j-2) -- the last
-        // reader of the buffer -- has completed: for map m alone, or for both
-        // maps in turn with one QK issuer.
+        // reader of the buffer -- has completed.
         constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, PF_BN, false);
-        constexpr bool PER_MAP = pf_qk_issuers(MODE) == 2;
-        const int m0 = PER_MAP ? m : 0, m1 = PER_MAP ? m + 1 : 2;
+        const uint32_t q_lo0 = umma_desc_lo(smem_u32(S.q[0]), 16), q_lo1 = umma_desc_lo(smem_u32(S.q[1]), 16);
         const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16);
+        const uint32_t km_off = a.v1 ? (PF_KBOX >> 4) : 0u;         // V1: K2 box follows the K1 box
         ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
         for (int j = 0; ok && j < nT; ++j) {
           const int bb = j & 1;
           if (!(ok = wait_bar(smem_u32(&S.k_full[j % PF_NS]), (j / PF_NS) & 1, abort_flag, a.watch))) break;
-          for (int mm = m0; mm < m1; ++mm) {
-            if (j >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[mm][bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch)))
+          for (int m = 0; m < 2; ++m) {
+            if (j >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[m][bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch)))
               break;
             tc_fence_after();
-            const uint32_t qlo = umma_desc_lo(smem_u32(S.q[mm]), 16);
-            const uint32_t km_off = (a.v1 && mm) ? (PF_KBOX >> 4) : 0u;   // V1: K2 box follows the K1 box
-            const uint32_t klo = k_lo0 + (uint32_t)(j % PF_NS) * KSTAGE + km_off;
-            const uint32_t d = tmem + (uint32_t)(mm * 128 + bb * 64);
+            const uint32_t klo = k_lo0 + (uint32_t)(j % PF_NS) * KSTAGE + (m ? km_off : 0u);
+            const uint32_t qlo = m ? q_lo1 : q_lo0;
+            const uint32_t d = tmem + (uint32_t)(m * 128 + bb * 64);
 #pragma unroll
             for (int s = 0; s < DQK / 16; ++s) {
               const uint32_t qo = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
               const uint32_t ko = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
               mma_ss_w(d, qlo + qo, HI, klo + ko, HI, IDESC_QK, s > 0);
             }
-            mma_commit(smem_u32(&S.s_full[mm][bb]));
+            mma_commit(smem_u32(&S.s_full[m][bb]));
           }
         }
       }

@@ -250,7 +250,10 @@ DIFFATTN_API int diffattn_bwd_v2(const void* q, const void* k, const void* v, co
  * orthogonal to X, to which O_2 is nearly parallel when the two maps are
  * alike; the sum is then a small remainder of large terms, and a bf16 O_2
  * would leave an error of the terms' size.  With X·dX = <y, dY> eps r^2,
- * dX·O_2 = dX·(O_2 - c X) + o2_coef <y, dY> needs only the small part. */
+ * dX·O_2 = dX·(O_2 - c X) + o2_coef <y, dY> needs only the small part.  For
+ * the same reason, with rmsnorm != 0 every head keeps the bf16 residual of P
+ * (the inference forward keeps it only for |1 - λ| < 0.15), so that O_2 has
+ * no 2^-9 rounding along X either. */
 DIFFATTN_API int diffattn_fwd_v1_train(const void* q1, const void* k1, const void* q2, const void* k2,
                                        const void* v, const float* lambda, void* out, float* lse, void* o_maps,
                                        float* rstd, float* o2_coef, diffattn_dtype dtype, int B, int H, int Hkv,
