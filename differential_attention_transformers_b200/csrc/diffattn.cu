@@ -124,7 +124,6 @@ int device_setup(DeviceInfo** out) {
                                   (int)decode_smem()));
     CUDA_TRY(cudaFuncSetAttribute(decode_split_kernel<kDecNst, true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_paged_smem()));
-    CUDA_TRY(cudaFuncSetAttribute(lr_emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LR_EMIT_SMEM));
     CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)bwd_dq_smem()));
     CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -854,7 +853,7 @@ int diffattn_fwd_lowrank(const void* q, const void* k, const void* v, const floa
   }
   lr_prefix_kernel<<<dim3((unsigned)r, BH), LR_DV, 0, s>>>(a);
   CUDA_TRY(cudaGetLastError());
-  lr_emit_kernel<<<dim3((unsigned)((Lq + LR_C - 1) / LR_C), BH), LR_DV, LR_EMIT_SMEM, s>>>(a);
+  lr_emit_kernel<<<dim3((unsigned)((Lq + LR_C - 1) / LR_C), BH), LR_DV, 0, s>>>(a);
   CUDA_TRY(cudaGetLastError());
   return ok();
 }

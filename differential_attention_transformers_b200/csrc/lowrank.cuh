@@ -102,12 +102,12 @@ __host__ __device__ inline void lr_key_range(const LowrankArgs& a, int c, long l
   }
 }
 
-// Adds keys [ks, ke) of one value column: S[t] += g_j[t] v_j.  vcol: the
-// column (keys LR_DV apart); gk: the G rows of these keys, gk[(j - ks) r + t].
-// Keys in ascending order, U at a time with their V loads issued first, so U
-// loads are in flight per thread.
+// Adds keys [ks, ke) of one value column: S[t] += g_j[t] v_j, z[t] += g_j[t].
+// vcol: the column (keys LR_DV apart); gk: the G rows of these keys, gk[(j -
+// ks) r + t].  Keys in ascending order, U at a time with their V loads issued
+// first, so U loads are in flight per thread.
 __host__ __device__ inline void lr_add_keys(int r, const __nv_bfloat16* vcol, const float* gk, long long ks,
-                                            long long ke, float (&S)[LR_RMAX]) {
+                                            long long ke, float (&S)[LR_RMAX], float (&z)[LR_RMAX]) {
   constexpr int U = 8;
   long long j = ks;
   for (; j + U <= ke; j += U) {
@@ -119,7 +119,10 @@ __host__ __device__ inline void lr_add_keys(int r, const __nv_bfloat16* vcol, co
       const float* g = gk + (j - ks + u) * r;
 #pragma unroll
       for (int t = 0; t < LR_RMAX; ++t)
-        if (t < r) S[t] = fmaf(g[t], vj[u], S[t]);
+        if (t < r) {
+          S[t] = fmaf(g[t], vj[u], S[t]);
+          z[t] += g[t];
+        }
     }
   }
   for (; j < ke; ++j) {
@@ -127,31 +130,31 @@ __host__ __device__ inline void lr_add_keys(int r, const __nv_bfloat16* vcol, co
     const float* g = gk + (j - ks) * r;
 #pragma unroll
     for (int t = 0; t < LR_RMAX; ++t)
-      if (t < r) S[t] = fmaf(g[t], vj, S[t]);
+      if (t < r) {
+        S[t] = fmaf(g[t], vj, S[t]);
+        z[t] += g[t];
+      }
   }
 }
 
 // Slot c of head bh, value column col; gk: the G rows of the slot's keys
-// [ks, ke) (lr_key_range), gk[(j - ks) r + t].  The sums of g do not depend
-// on the column: column t < r sums component t of them.
+// [ks, ke) (lr_key_range), gk[(j - ks) r + t].
 __host__ __device__ inline void lr_totals_body(const LowrankArgs& a, int c, int bh, int col, const float* gk) {
   const int b = bh / a.H, g = (bh % a.H) / (a.H / a.Hkv);
   long long ks, ke;
   lr_key_range(a, c, ks, ke);
-  float S[LR_RMAX];
+  float S[LR_RMAX], z[LR_RMAX];
 #pragma unroll
-  for (int t = 0; t < LR_RMAX; ++t) S[t] = 0.f;
+  for (int t = 0; t < LR_RMAX; ++t) S[t] = z[t] = 0.f;
   const __nv_bfloat16* vcol = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lk * LR_DV + col;
-  lr_add_keys(a.r, vcol, gk, ks, ke, S);
+  lr_add_keys(a.r, vcol, gk, ks, ke, S, z);
   const size_t slot = (size_t)bh * (a.nc + 1) + c;
 #pragma unroll
   for (int t = 0; t < LR_RMAX; ++t)
-    if (t < a.r) a.tot[(slot * a.r + t) * LR_DV + col] = S[t];
-  if (col < a.r) {
-    float z = 0.f;
-    for (long long j = ks; j < ke; ++j) z += gk[(j - ks) * a.r + col];
-    a.ztot[slot * a.r + col] = z;
-  }
+    if (t < a.r) {
+      a.tot[(slot * a.r + t) * LR_DV + col] = S[t];
+      if (col == 0) a.ztot[slot * a.r + t] = z[t];
+    }
 }
 
 // Exclusive prefix over the slots of head bh, rank index t, value column col
@@ -195,45 +198,19 @@ __host__ __device__ inline void lr_emit_range(const LowrankArgs& a, int c, long 
   k1 = a.causal ? lr_clamp(r1 + off, a.Lk) : 0;
 }
 
-// Normaliser of N's rows in chunk c of head bh, which does not depend on the
-// value column: rden[i - r0] = 1 / f_i^T z_i, or 0 when the row has no mass.
-// Component t of z_i is a running sum over the keys the rows add; this body
-// computes it for one t, and den_i = sum_t f_i[t] z_i[t] is then formed by
-// lr_emit_den_finish.  fk, gk as for lr_emit_body; zrow[(i - r0) r + t].
-__host__ __device__ inline void lr_emit_den_part(const LowrankArgs& a, int c, int bh, int t, const float* gk,
-                                                 float* zrow) {
-  const size_t slot = (size_t)bh * (a.nc + 1) + (a.causal ? a.n_lead + c : a.nc);
-  long long r0, r1, k0, k1;
-  lr_emit_range(a, c, r0, r1, k0, k1);
-  const long long off = (long long)a.Lk - a.Lq;
-  float z = a.ztot[slot * a.r + t];
-  for (long long i = r0; i < r1; ++i) {
-    const long long j = i + off;
-    if (a.causal && j >= 0 && j < a.Lk) z += gk[(j - k0) * a.r + t];
-    zrow[(i - r0) * a.r + t] = z;
-  }
-}
-__host__ __device__ inline void lr_emit_den_finish(const LowrankArgs& a, int c, int row, const float* fk,
-                                                   const float* zrow, float* rden) {
-  long long r0, r1, k0, k1;
-  lr_emit_range(a, c, r0, r1, k0, k1);
-  if (row >= r1 - r0) return;
-  float den = 0.f;
-  for (int t = 0; t < a.r; ++t) den = fmaf(fk[row * a.r + t], zrow[row * a.r + t], den);
-  rden[row] = den > 0.f ? 1.f / den : 0.f;
-}
-
 // Row chunk c (rows [r0, r1)) of head bh, value column col.  fk: the F rows
 // of the chunk, fk[(i - r0) r + t]; gk: the G rows of the keys the rows add,
-// gk[(j - k0) r + t] (lr_emit_range); rden: the rows' 1 / den
-// (lr_emit_den_part, lr_emit_den_finish).
+// gk[(j - k0) r + t] (lr_emit_range).
 __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh, int col, const float* fk,
-                                             const float* gk, const float* rden) {
+                                             const float* gk) {
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
   const size_t slot = (size_t)bh * (a.nc + 1) + (a.causal ? a.n_lead + c : a.nc);
-  float S[LR_RMAX];
+  float S[LR_RMAX], z[LR_RMAX];
 #pragma unroll
-  for (int t = 0; t < LR_RMAX; ++t) S[t] = t < a.r ? a.tot[(slot * a.r + t) * LR_DV + col] : 0.f;
+  for (int t = 0; t < LR_RMAX; ++t) {
+    S[t] = t < a.r ? a.tot[(slot * a.r + t) * LR_DV + col] : 0.f;
+    z[t] = t < a.r ? a.ztot[slot * a.r + t] : 0.f;
+  }
   long long r0, r1, k0, k1;
   lr_emit_range(a, c, r0, r1, k0, k1);
   const long long off = (long long)a.Lk - a.Lq;
@@ -259,14 +236,21 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
         const float* gj = gk + (j - k0) * a.r;
 #pragma unroll
         for (int t = 0; t < LR_RMAX; ++t)
-          if (t < a.r) S[t] = fmaf(gj[t], vj[u], S[t]);
+          if (t < a.r) {
+            S[t] = fmaf(gj[t], vj[u], S[t]);
+            z[t] += gj[t];
+          }
       }
       const float* fi = fk + (i - r0) * a.r;
-      float num = 0.f;
+      float num = 0.f, den = 0.f;
 #pragma unroll
       for (int t = 0; t < LR_RMAX; ++t)
-        if (t < a.r) num = fmaf(fi[t], S[t], num);
-      orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * (num * rden[i - r0]));
+        if (t < a.r) {
+          num = fmaf(fi[t], S[t], num);
+          den = fmaf(fi[t], z[t], den);
+        }
+      const float nv = den > 0.f ? num / den : 0.f;
+      orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * nv);
     }
   }
 }
@@ -289,22 +273,15 @@ __global__ void __launch_bounds__(LR_DV) lr_totals_kernel(LowrankArgs a) {
 __global__ void __launch_bounds__(LR_DV) lr_prefix_kernel(LowrankArgs a) {
   lr_prefix_body(a, (int)blockIdx.y, (int)blockIdx.x, (int)threadIdx.x);
 }
-// Dynamic shared memory: F rows, G rows, z rows (LR_C x LR_RMAX floats each)
-// and the rows' 1 / den.
-constexpr size_t LR_EMIT_SMEM = (3 * LR_C * LR_RMAX + LR_C) * sizeof(float);
 __global__ void __launch_bounds__(LR_DV) lr_emit_kernel(LowrankArgs a) {
-  extern __shared__ float lr_sm[];
-  float *sf = lr_sm, *sg = lr_sm + LR_C * LR_RMAX, *sz = lr_sm + 2 * LR_C * LR_RMAX, *rd = lr_sm + 3 * LR_C * LR_RMAX;
+  __shared__ float sf[LR_C * LR_RMAX];
+  __shared__ float sg[LR_C * LR_RMAX];
   const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
   long long r0, r1, k0, k1;
   lr_emit_range(a, c, r0, r1, k0, k1);
   for (long long i = threadIdx.x; i < (r1 - r0) * a.r; i += blockDim.x) sf[i] = a.F[((size_t)h * a.Lq + r0) * a.r + i];
   lr_stage(sg, a.G + ((size_t)h * a.Lk + k0) * a.r, (k1 - k0) * a.r);
-  if ((int)threadIdx.x < a.r) lr_emit_den_part(a, c, bh, (int)threadIdx.x, sg, sz);
-  __syncthreads();
-  for (int row = (int)threadIdx.x; row < LR_C; row += blockDim.x) lr_emit_den_finish(a, c, row, sf, sz, rd);
-  __syncthreads();
-  lr_emit_body(a, c, bh, (int)threadIdx.x, sf, sg, rd);
+  lr_emit_body(a, c, bh, (int)threadIdx.x, sf, sg);
 }
 #endif
 

@@ -74,10 +74,7 @@ int main(int argc, char** argv) {
       da::lr_emit_range(a, c, r0, r1, k0, k1);
       const float* fk = F.data() + ((size_t)(bh % H) * Lq + r0) * r;
       const float* gk = G.data() + ((size_t)(bh % H) * Lk + k0) * r;
-      std::vector<float> zrow((size_t)da::LR_C * r), rden(da::LR_C);
-      for (int t = 0; t < r; ++t) da::lr_emit_den_part(a, c, bh, t, gk, zrow.data());
-      for (int row = 0; row < da::LR_C; ++row) da::lr_emit_den_finish(a, c, row, fk, zrow.data(), rden.data());
-      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, fk, gk, rden.data());
+      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, fk, gk);
     }
 
   FILE* g = fopen(argv[2], "wb");

@@ -182,7 +182,12 @@ CASES_V1 = [
 def test_v1_backward_matches_oracle(B, H, Hkv, Lq, Lk, causal, rms):
     q1, k1, q2, k2, v, dout, lam = _case_v1(B, H, Hkv, Lq, Lk, seed=3 * Lq + Lk + H)
     out, lse, om, rstd, o2c = da.fwd_v1_train(q1, k1, q2, k2, v, lam, causal=causal, rmsnorm=rms)
-    assert torch.equal(out, da.fwd_v1(q1, k1, q2, k2, v, lam, causal=causal, rmsnorm=rms))
+    inf = da.fwd_v1(q1, k1, q2, k2, v, lam, causal=causal, rmsnorm=rms)
+    if rms:   # the training forward keeps P's residual on every head: equal up to P's rounding
+        assert _rel(out, orc.diffattn_v1(q1, k1, q2, k2, v, lam.cpu().numpy(), causal=causal, rms=True)) <= BF16_TOL
+        assert _rel(out, inf.double().cpu().numpy()) <= BF16_TOL
+    else:     # the training forward is the forward
+        assert torch.equal(out, inf)
     grads = da.bwd_v1(q1, k1, q2, k2, v, lam, dout, out, lse, om, rstd, o2c, causal=causal, rmsnorm=rms)
     torch.cuda.synchronize()
     assert da.last_status() == da.OK
@@ -235,8 +240,11 @@ def test_v1_dlambda_rmsnorm_alike_maps(lam_value):
     """dlambda with RMSNorm when the two maps are alike (near-uniform maps from
     small scores, the V1 workload's input scale): X = O_1 - lambda O_2 is then
     nearly parallel to O_2, and the sum of dX . O_2 is a small remainder of
-    terms over 5x larger in 2-norm.  With map 2's orthogonal part stored, the
-    error is within the plain output tolerance, 2e-2 |dlambda|."""
+    terms over 5x larger in 2-norm.  With map 2's orthogonal part stored (and
+    P's residual kept), the error scales with the terms dX * (O_2 - c X): it
+    stays within the output tolerance plus ten roundings of their 2-norm (at
+    least five times smaller than the terms dX * O_2 here), and within the
+    plain 2e-2 |dlambda| wherever |dlambda| is above twice their 2-norm."""
     q1, k1, q2, k2, v, dout, _ = _case_v1(1, 2, 1, 1024, 1024, seed=int(lam_value * 100) + 9)
     lam = torch.full((2,), lam_value, device=DEV)
     out, lse, om, rstd, o2c = da.fwd_v1_train(q1, k1, q2, k2, v, lam, causal=True, rmsnorm=True)
@@ -249,6 +257,10 @@ def test_v1_dlambda_rmsnorm_alike_maps(lam_value):
         full = bwd.dlambda_terms(q1[0, h], k1[0, 0], q2[0, h], k2[0, 0], v[0, 0], lr[h], dout[0, h], True, rms=True)
         perp = bwd.dlambda_terms(q1[0, h], k1[0, 0], q2[0, h], k2[0, 0], v[0, 0], lr[h], dout[0, h], True, rms=True,
                                  orthogonal=True)
-        assert np.sqrt(np.sum(perp ** 2)) < 0.2 * np.sqrt(np.sum(full ** 2))   # the case is ill-conditioned
+        n_full, n_perp = np.sqrt(np.sum(full ** 2)), np.sqrt(np.sum(perp ** 2))
+        assert n_perp < 0.2 * n_full   # the case is ill-conditioned for the terms dX * O_2
         err = abs(float(grads[5][h]) - ref[5][h])
-        assert err <= BF16_TOL * abs(ref[5][h]), (h, err, ref[5][h])
+        bound = BF16_TOL * abs(ref[5][h]) + DLAM_ROUND * n_perp
+        assert err <= bound, (h, err, bound)
+        if abs(ref[5][h]) > 2 * n_perp:
+            assert err <= BF16_TOL * abs(ref[5][h]), (h, err, ref[5][h])
