@@ -15,7 +15,8 @@
 //
 // Three kernels:
 //   bwd_prep_kernel  D_m per row from dO and the forward's normalised map
-//                    outputs, the log-sum-exp copied into a padded layout, and
+//                    outputs, and the log-sum-exp, both negated into a padded
+//                    layout (so the kernels below add them), and
 //                    per-block partial sums of dlambda (reduced in a fixed
 //                    order by bwd_dlambda_kernel, so the result is
 //                    deterministic).
@@ -53,8 +54,8 @@ constexpr int BW_RB = 64;         // rows per step of the key-stationary kernel
 
 struct BwdArgs {
   const float* lambda;   // [Hp]
-  const float* lse_p;    // [B, Hp, 2, Lp] log-sum-exp (log2 units), +inf past Lq
-  const float* dd;       // [B, Hp, 2, Lp] D_m, 0 past Lq
+  const float* nlse;     // [B, Hp, 2, Lp] minus the log-sum-exp (log2 units), -inf past Lq
+  const float* ndd;      // [B, Hp, 2, Lp] -D_m, 0 past Lq
   __nv_bfloat16* dq;     // [B, Hq, Lq, 128]; V1: dQ1 [B, Hq/2, Lq, 64]
   __nv_bfloat16* dk;     // [B, Hkv, Lk, 128]; V1: dK1 [B, Hkv, Lk, 64]
   __nv_bfloat16* dv;     // [B, Hkv, Lk, 128]
@@ -77,8 +78,8 @@ struct BwdPrepArgs {
   const __nv_bfloat16* dout;    // [B, Hp, Lq, 128]
   const __nv_bfloat16* o_maps;  // [B, Hp, 2, Lq, 128]
   const float* lse;             // [B, Hp, 2, Lq]
-  float* lse_p;                 // [B, Hp, 2, Lp]
-  float* dd;                    // [B, Hp, 2, Lp]
+  float* nlse;                  // [B, Hp, 2, Lp] -lse, -inf past Lq
+  float* ndd;                   // [B, Hp, 2, Lp] -D_m, 0 past Lq
   float* part;                  // [B * Hp, Lp / 64] partial sums of -D_2
   int B, Hp, Lq, Lp;
   const float* d_in;            // [B, Hp, 2, Lq] D_m formed upstream (V1 with RMSNorm), or null
@@ -119,8 +120,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
     }
     if (lane < 2) {
       const size_t at = ((size_t)bh * 2 + lane) * a.Lp + row;
-      a.dd[at] = d[lane];
-      a.lse_p[at] = row < a.Lq ? a.lse[((size_t)bh * 2 + lane) * a.Lq + row] : INFINITY;
+      a.ndd[at] = -d[lane];
+      a.nlse[at] = row < a.Lq ? -a.lse[((size_t)bh * 2 + lane) * a.Lq + row] : -INFINITY;
     }
     acc -= d[1];
   }
@@ -168,6 +169,27 @@ __device__ __forceinline__ uint32_t bw_slice(int s) { return (uint32_t)((s >> 1)
 // 64-wide tensor (tmQ for map 1, tmQ2 for map 2; tmK, tmK2 likewise), and dQ
 // of map 2 goes to dq2.  The scores then contract over 64 dimensions and dQ
 // is 64 wide; dO, V and everything else are as in V2.
+// One step of the query-stationary kernel for this thread's row and this
+// warp's 32-key chunk: dS = c P (dP - D) with P = 2^(S scale_log2 - lse), in
+// f32x2 pairs (each operation rounds as its scalar form would).  With MASK,
+// columns past lim (-1..31) are masked.
+template <bool MASK>
+__device__ __forceinline__ void bw_q_elementwise(const uint32_t (&sv)[32], const uint32_t (&pv)[32], uint32_t (&ds)[16],
+                                                 int lim, float2 sl2, float2 nl2, float2 nd2, float2 c2) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2, nl2);
+    if (MASK) {
+      if (2 * i > lim) x.x = -INFINITY;
+      if (2 * i + 1 > lim) x.y = -INFINITY;
+    }
+    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+    const float2 t = __fadd2_rn(make_float2(__uint_as_float(pv[2 * i]), __uint_as_float(pv[2 * i + 1])), nd2);
+    const float2 d = __fmul2_rn(__fmul2_rn(c2, p), t);
+    ds[i] = pack_bf16(d.x, d.y);
+  }
+}
+
 template <bool V1>
 __global__ void __maxnreg__(168)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ2,
@@ -309,8 +331,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int rg = r0 + r;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const size_t stat = (((size_t)b * Hp + h) * 2 + m) * a.Lp + rg;
-    const float lse = a.lse_p[stat], dsum = a.dd[stat];
     const float c = a.scale * (m == 0 ? 1.f : -a.lambda[h]);
+    const float2 nl2 = make_float2(a.nlse[stat], a.nlse[stat]), nd2 = make_float2(a.ndd[stat], a.ndd[stat]);
+    const float2 sl2 = make_float2(a.scale_log2, a.scale_log2), c2 = make_float2(c, c);
     const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
     bool ok = true;
     for (int j = 0; j < nT; ++j) {
@@ -322,17 +345,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
       tmem_wait_ld();
       const long long lim = lastk - (long long)j * PF_BN - ch * 32;   // columns > lim are masked
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float dsv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 2 * i + e;
-          const float x = col > lim ? -INFINITY : fmaf(__uint_as_float(sv[col]), a.scale_log2, -lse);
-          dsv[e] = c * ex2(x) * (__uint_as_float(pv[col]) - dsum);
-        }
-        ds[i] = pack_bf16(dsv[0], dsv[1]);
-      }
+      // warp-uniform, so that the tcgen05.st below runs convergently
+      if (__all_sync(0xffffffffu, lim >= 31))
+        bw_q_elementwise<false>(sv, pv, ds, 0, sl2, nl2, nd2, c2);
+      else
+        bw_q_elementwise<true>(sv, pv, ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
       tmem_st16p(tmem + lane_off + bb * 64 + ch * 32, ds);   // the chunk's own columns
       tmem_wait_st();
       tc_fence_before();
@@ -374,8 +391,8 @@ struct BwKSmem {
   alignas(1024) uint8_t v[2 * PF_QBOX];             // V tile, same layout
   alignas(1024) uint8_t q[BW_NS][2 * PF_KBOX];      // Q rows: 64, two boxes
   alignas(1024) uint8_t o[BW_NS][2 * PF_KBOX];      // dO rows
-  alignas(16) float lse[BW_NS][BW_RB];
-  alignas(16) float dd[BW_NS][BW_RB];
+  alignas(16) float nlse[BW_NS][BW_RB];
+  alignas(16) float ndd[BW_NS][BW_RB];
   alignas(16) uint8_t stage[8][16 * 128];
   alignas(8) uint64_t kv_full;
   uint64_t st_full[BW_NS], st_empty[BW_NS];
@@ -403,46 +420,49 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   return v;
 }
 
-// lse_s, dd_s: shared-window addresses of the chunk's 32 log-sum-exp and D
-// values (one per row, the same for every key).  They are read half a chunk
-// at a time as 16-byte vectors before that half's arithmetic: read one by one
-// through a generic pointer inside the loop, each element waited on its load
-// (an in-kernel trace measured 1.5k cycles for the 32 elements).
-template <bool RESID>
-__device__ __forceinline__ void bw_kv_elementwise(uint32_t tS, uint32_t tP, int row0, int kg, int rfirst, int Lk,
-                                                  float w, float cd, float sl, uint32_t lse_s, uint32_t dd_s) {
+// nl_s, nd_s: shared-window addresses of the chunk's 32 negated log-sum-exp
+// and D values (one per row, the same for every key), read as 16-byte vectors
+// half a chunk at a time.  The arithmetic runs on f32x2 pairs (each operation
+// rounds as its scalar form would).  vis0: the first visible column (0..32);
+// with MASK, columns before it give P = 0.
+template <bool RESID, bool MASK>
+__device__ __forceinline__ void bw_kv_elementwise(uint32_t tS, uint32_t tP, int vis0, float2 w2, float2 cd2, float2 sl2,
+                                                  uint32_t nl_s, uint32_t nd_s) {
   uint32_t sv[32], pv[32], pw[16], ds[16];
   tmem_ld32p(tS, sv);
   tmem_ld32p(tP, pv);
   tmem_wait_ld();
   uint32_t rpw[RESID ? 16 : 1], rds[RESID ? 16 : 1];
-  float lse[16], dd[16];
+  const float2 neg1 = make_float2(-1.f, -1.f);
+  float2 nl[8], nd[8];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    if ((j & 7) == 0) {   // this half's 16 log-sum-exp and D values
+    if ((j & 7) == 0) {   // this half's 16 values of each
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float4 l4 = lds_f4(lse_s + (uint32_t)((j * 2 + q * 4) * 4));
-        const float4 d4 = lds_f4(dd_s + (uint32_t)((j * 2 + q * 4) * 4));
-        lse[4 * q] = l4.x; lse[4 * q + 1] = l4.y; lse[4 * q + 2] = l4.z; lse[4 * q + 3] = l4.w;
-        dd[4 * q] = d4.x; dd[4 * q + 1] = d4.y; dd[4 * q + 2] = d4.z; dd[4 * q + 3] = d4.w;
+        const float4 l4 = lds_f4(nl_s + (uint32_t)((j * 2 + q * 4) * 4));
+        const float4 d4 = lds_f4(nd_s + (uint32_t)((j * 2 + q * 4) * 4));
+        nl[2 * q] = make_float2(l4.x, l4.y); nl[2 * q + 1] = make_float2(l4.z, l4.w);
+        nd[2 * q] = make_float2(d4.x, d4.y); nd[2 * q + 1] = make_float2(d4.z, d4.w);
       }
     }
-    float p2[2], d2[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int col = 2 * j + e, hc = col & 15;
-      const bool vis = kg < Lk && row0 + col >= rfirst;
-      const float x = vis ? fmaf(__uint_as_float(sv[col]), sl, -lse[hc]) : -INFINITY;
-      const float p = ex2(x);
-      p2[e] = w * p;
-      d2[e] = cd * p * (__uint_as_float(pv[col]) - dd[hc]);
+    float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sl2, nl[j & 7]);
+    if (MASK) {
+      if (2 * j < vis0) x.x = -INFINITY;
+      if (2 * j + 1 < vis0) x.y = -INFINITY;
     }
-    pw[j] = pack_bf16(p2[0], p2[1]);
-    ds[j] = pack_bf16(d2[0], d2[1]);
+    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+    const float2 p2 = __fmul2_rn(w2, p);
+    const float2 t = __fadd2_rn(make_float2(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1])), nd[j & 7]);
+    const float2 d2 = __fmul2_rn(__fmul2_rn(cd2, p), t);
+    pw[j] = pack_bf16(p2.x, p2.y);
+    ds[j] = pack_bf16(d2.x, d2.y);
     if constexpr (RESID) {   // x - bf16(x), exact in f32
-      rpw[j] = pack_bf16(p2[0] - __uint_as_float(pw[j] << 16), p2[1] - __uint_as_float(pw[j] & 0xFFFF0000u));
-      rds[j] = pack_bf16(d2[0] - __uint_as_float(ds[j] << 16), d2[1] - __uint_as_float(ds[j] & 0xFFFF0000u));
+      const float2 ph = make_float2(__uint_as_float(pw[j] << 16), __uint_as_float(pw[j] & 0xFFFF0000u));
+      const float2 dh = make_float2(__uint_as_float(ds[j] << 16), __uint_as_float(ds[j] & 0xFFFF0000u));
+      const float2 rp = __ffma2_rn(ph, neg1, p2), rd = __ffma2_rn(dh, neg1, d2);
+      rpw[j] = pack_bf16(rp.x, rp.y);
+      rds[j] = pack_bf16(rd.x, rd.y);
     }
   }
   tmem_st16p(tS, pw);
@@ -538,8 +558,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         for (int x = 0; x < 2; ++x)
           tma_load_3d(smem_u32(S.o[st]) + x * PF_KBOX, &tmO, fb, 64 * x, rb * BW_RB, b * Hp + hq);
         const size_t stat = (((size_t)b * Hp + hq) * 2 + mq) * a.Lp + (size_t)rb * BW_RB;
-        bulk_load(smem_u32(S.lse[st]), a.lse_p + stat, BW_RB * 4, fb);
-        bulk_load(smem_u32(S.dd[st]), a.dd + stat, BW_RB * 4, fb);
+        bulk_load(smem_u32(S.nlse[st]), a.nlse + stat, BW_RB * 4, fb);
+        bulk_load(smem_u32(S.ndd[st]), a.ndd + stat, BW_RB * 4, fb);
         last_use[st] = use;
       }
       drain_bar(kvb, 0, a.watch.status);
@@ -629,6 +649,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     // ------------------------------------------- elementwise (thread = key) --
     const int wq = warp & 3, ch = warp >> 2, kr = threadIdx.x & 127;
     const int kg = k0 + kr;   // this thread's key
+    const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     bool ok = true;
     for (int i = 0; i < nS; ++i) {
@@ -636,22 +657,27 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       const int qh = step_head(i), rb = step_rb(i);
       const int mq = qh & 1;
       const float w = mq == 0 ? 1.f : -a.lambda[qh / 2];   // weight of this map in A_1 - lambda A_2
-      const float cd = a.scale * w;
+      const float2 w2 = make_float2(w, w), cd2 = make_float2(a.scale * w, a.scale * w);
       // The stage's log-sum-exp and D values came by bulk copy: wait for them here too.
       if (!(ok = warp_wait(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
       if (!(ok = warp_wait(smem_u32(&S.s_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
       tc_fence_after();
       // rows r = rb*64 + col see this key iff kg < Lk and (not causal or kg <= r + off)
-      const int rfirst = a.causal ? kg - off : 0;   // first row that sees kg (causal)
+      const int row0 = rb * BW_RB + ch * 32;
+      const int vis0 = kg >= a.Lk ? 32 : (a.causal ? min(32, max(0, kg - off - row0)) : 0);
       const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
       const uint32_t tS = tmem + lane_off + bb * 64 + ch * 32, tP = tmem + lane_off + 128 + bb * 64 + ch * 32;
-      const int row0 = rb * BW_RB + ch * 32;
-      // branch once per step: each variant's loop is one straight-line block
-      const uint32_t lse_s = smem_u32(S.lse[st] + ch * 32), dd_s = smem_u32(S.dd[st] + ch * 32);
-      if (resid)
-        bw_kv_elementwise<true>(tS, tP, row0, kg, rfirst, a.Lk, w, cd, a.scale_log2, lse_s, dd_s);
-      else
-        bw_kv_elementwise<false>(tS, tP, row0, kg, rfirst, a.Lk, w, cd, a.scale_log2, lse_s, dd_s);
+      // branch once per step, warp-uniformly (the TMEM stores inside are
+      // warp-collective): each variant's loop is one straight-line block
+      const bool full = __all_sync(0xffffffffu, vis0 == 0);
+      const uint32_t nl_s = smem_u32(S.nlse[st] + ch * 32), nd_s = smem_u32(S.ndd[st] + ch * 32);
+      if (resid) {
+        if (full) bw_kv_elementwise<true, false>(tS, tP, 0, w2, cd2, sl2, nl_s, nd_s);
+        else bw_kv_elementwise<true, true>(tS, tP, vis0, w2, cd2, sl2, nl_s, nd_s);
+      } else {
+        if (full) bw_kv_elementwise<false, false>(tS, tP, 0, w2, cd2, sl2, nl_s, nd_s);
+        else bw_kv_elementwise<false, true>(tS, tP, vis0, w2, cd2, sl2, nl_s, nd_s);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&S.p_full[bb]));

@@ -357,19 +357,19 @@ int launch_backward(const void* q, const void* q2, const void* k, const void* k2
   if (!aligned16(ws)) return fail(DIFFATTN_ERR_MISALIGNED, "workspace not 16-byte aligned");
   const int Hp = Hq / 2, Lp = bwd_rows_padded(Lq);
   const int w = v1 ? 64 : 128;   // QK width
-  float* lse_p = static_cast<float*>(ws);
-  float* dd = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)B * Hp * 2 * Lp * 4));
+  float* nlse = static_cast<float*>(ws);
+  float* ndd = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)B * Hp * 2 * Lp * 4));
   float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + 2 * align256((size_t)B * Hp * 2 * Lp * 4));
   if (Lp > 0) {
     BwdPrepArgs pa{static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o_maps), lse,
-                   lse_p, dd, part, B, Hp, Lq, Lp, d_in};
+                   nlse, ndd, part, B, Hp, Lq, Lp, d_in};
     bwd_prep_kernel<<<dim3((unsigned)(Lp / 64), (unsigned)(B * Hp)), 256, 0, s>>>(pa);
     CUDA_TRY(cudaGetLastError());
   }
   bwd_dlambda_kernel<<<(Hp + 127) / 128, 128, 0, s>>>(part, dlambda, B, Hp, Lp / 64);
   CUDA_TRY(cudaGetLastError());
   BwdArgs a{};
-  a.lambda = lambda; a.lse_p = lse_p; a.dd = dd;
+  a.lambda = lambda; a.nlse = nlse; a.ndd = ndd;
   a.dq = static_cast<__nv_bfloat16*>(dq);
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
