@@ -22,8 +22,11 @@
 //                    deterministic).
 //   bwd_dq_kernel    query-stationary: one CTA per 128 rows of one Q head (one
 //                    map).  Per 64-key tile: S = Q K^T and dP = dO V^T into
-//                    TMEM, dS = c P (dP - D) written over S as bf16, then
-//                    dQ += dS K with dS as the TMEM operand.
+//                    TMEM, dS = c P (dP - D) written to shared memory as bf16,
+//                    then dQ += dS K with dS as the shared A operand.  The
+//                    score buffer is then free as soon as the elementwise
+//                    warps have loaded it, so S of tile j + 2 waits only for
+//                    that load and for its K/V stage (four stages).
 //   bwd_dkv_kernel   key-stationary: one CTA per 128 keys of one KV head.  Per
 //                    64-row step of each Q head of the group: S^T = K Q^T and
 //                    dP^T = V dO^T into TMEM, then w P^T (w = 1 or -lambda)
@@ -49,7 +52,9 @@ namespace da {
 // the next 16 -- so no warp overwrites scores another warp has yet to load.
 constexpr int BW_THREADS = 352;
 constexpr int BW_EW = 256;        // elementwise threads
-constexpr int BW_NS = 3;          // pipeline stages
+constexpr int BW_EW_WARPS = BW_EW / 32;   // arrivals on the elementwise warps' barriers: one per warp
+constexpr int BW_NS = 3;          // pipeline stages of the key-stationary kernel
+constexpr int BWQ_NS = 4;         // K/V stages of the query-stationary kernel
 constexpr int BW_RB = 64;         // rows per step of the key-stationary kernel
 
 struct BwdArgs {
@@ -148,12 +153,15 @@ __global__ void bwd_dlambda_kernel(const float* part, float* dlambda, int B, int
 struct BwQSmem {
   alignas(1024) uint8_t q[2 * PF_QBOX];            // Q tile of the head: 128 rows, dims 0-63 box, 64-127 box
   alignas(1024) uint8_t o[2 * PF_QBOX];            // dO tile of the pair, same layout
-  alignas(1024) uint8_t k[BW_NS][2 * PF_KBOX];     // K tile: 64 keys, two boxes
-  alignas(1024) uint8_t v[BW_NS][2 * PF_KBOX];     // V tile
-  alignas(16) uint8_t stage[8][16 * 128];          // epilogue staging, per elementwise warp
+  alignas(1024) uint8_t k[BWQ_NS][2 * PF_KBOX];    // K tile: 64 keys, two boxes
+  alignas(1024) uint8_t v[BWQ_NS][2 * PF_KBOX];    // V tile
+  // dS, bf16 [128 rows][64 keys], K-major with the 128-byte swizzle (the A
+  // operand of dQ += dS K); ds[0] doubles as the epilogue's staging once
+  // every product has completed
+  alignas(1024) uint8_t ds[2][PF_QBOX];
   alignas(8) uint64_t q_full;
-  uint64_t k_full[BW_NS], v_full[BW_NS], kv_empty[BW_NS];
-  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t k_full[BWQ_NS], v_full[BWQ_NS], kv_empty[BWQ_NS];
+  uint64_t s_full[2], p_full[2], s_free[2], ds_free[2];
   uint64_t fin;
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -214,15 +222,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&S.q_full), 1);
-    for (int i = 0; i < BW_NS; ++i) {
+    for (int i = 0; i < BWQ_NS; ++i) {
       mbar_init(smem_u32(&S.k_full[i]), 1);
       mbar_init(smem_u32(&S.v_full[i]), 1);
       mbar_init(smem_u32(&S.kv_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&S.s_full[i]), 1);
-      mbar_init(smem_u32(&S.p_full[i]), BW_EW);
-      mbar_init(smem_u32(&S.s_free[i]), 1);
+      mbar_init(smem_u32(&S.p_full[i]), BW_EW_WARPS);
+      mbar_init(smem_u32(&S.s_free[i]), BW_EW_WARPS);
+      mbar_init(smem_u32(&S.ds_free[i]), 1);
       mbar_init(smem_u32(&S.drain[i]), 1);
     }
     mbar_init(smem_u32(&S.fin), 1);
@@ -237,6 +246,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;   // S [0,128), dP [128,256), dQ [256,384)
+  constexpr uint32_t DS_BUF = (uint32_t)sizeof(S.ds[0]);
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
@@ -247,10 +257,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_expect_tx(qb, (QB + 2) * PF_QBOX);
       for (int x = 0; x < QB; ++x) tma_load_3d(smem_u32(S.q) + x * PF_QBOX, tq, qb, 64 * x, r0, V1 ? b * Hp + h : b * a.Hq + qh);
       for (int x = 0; x < 2; ++x) tma_load_3d(smem_u32(S.o) + x * PF_QBOX, &tmO, qb, 64 * x, r0, b * Hp + h);
-      int last_use[BW_NS];
-      for (int i = 0; i < BW_NS; ++i) last_use[i] = -1;
+      int last_use[BWQ_NS];
+      for (int i = 0; i < BWQ_NS; ++i) last_use[i] = -1;
       for (int j = 0; j < nT; ++j) {
-        const int st = j % BW_NS, use = j / BW_NS;
+        const int st = j % BWQ_NS, use = j / BWQ_NS;
         if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
         const uint32_t kb = smem_u32(&S.k_full[st]), vb = smem_u32(&S.v_full[st]);
         mbar_expect_tx(kb, QB * PF_KBOX);
@@ -262,7 +272,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         last_use[st] = use;
       }
       drain_bar(qb, 0, a.watch.status);
-      for (int i = 0; i < BW_NS; ++i) {
+      for (int i = 0; i < BWQ_NS; ++i) {
         if (last_use[i] >= 0) {
           drain_bar(smem_u32(&S.k_full[i]), last_use[i] & 1, a.watch.status);
           drain_bar(smem_u32(&S.v_full[i]), last_use[i] & 1, a.watch.status);
@@ -279,19 +289,21 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (issuer == 0) {
         constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 64 * QB, true);
         const uint32_t k_mn0 = umma_desc_lo(smem_u32(S.k[0]), PF_KBOX);   // K as the N-major B operand
+        const uint32_t ds_lo0 = umma_desc_lo(smem_u32(S.ds[0]), 16);       // dS as the K-major A operand
         for (int j = 0; ok && j < nT; ++j) {
           const int bb = j & 1;
           // this thread reads the K stage too: acquire it here
-          if (!(ok = wait_bar(smem_u32(&S.k_full[j % BW_NS]), (j / BW_NS) & 1, abort_flag, a.watch))) break;
+          if (!(ok = wait_bar(smem_u32(&S.k_full[j % BWQ_NS]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
           if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
           tc_fence_after();
-          const uint32_t klo = k_mn0 + (uint32_t)(j % BW_NS) * KSTAGE;
+          const uint32_t klo = k_mn0 + (uint32_t)(j % BWQ_NS) * KSTAGE;
+          const uint32_t dlo = ds_lo0 + (uint32_t)bb * (DS_BUF >> 4);
 #pragma unroll
           for (int s = 0; s < PF_BN / 16; ++s)
-            mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s), klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+            mma_ss_w(tmem + 256, dlo + (uint32_t)(s * 2), HI, klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
                      (j > 0 || s > 0));
-          mma_commit(smem_u32(&S.s_free[bb]));
-          mma_commit(smem_u32(&S.kv_empty[j % BW_NS]));
+          mma_commit(smem_u32(&S.ds_free[bb]));
+          mma_commit(smem_u32(&S.kv_empty[j % BWQ_NS]));
         }
         if (ok) mma_commit(smem_u32(&S.fin));
       } else {
@@ -300,9 +312,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16), v_lo0 = umma_desc_lo(smem_u32(S.v[0]), 16);
         ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
         for (int j = 0; ok && j < nT; ++j) {
-          const int bb = j & 1, st = j % BW_NS;
-          if (!(ok = wait_bar(smem_u32(&S.k_full[st]), (j / BW_NS) & 1, abort_flag, a.watch))) break;
-          if (!(ok = wait_bar(smem_u32(&S.v_full[st]), (j / BW_NS) & 1, abort_flag, a.watch))) break;
+          const int bb = j & 1, st = j % BWQ_NS;
+          if (!(ok = wait_bar(smem_u32(&S.k_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
+          if (!(ok = wait_bar(smem_u32(&S.v_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
           if (j >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch)))
             break;
           tc_fence_after();
@@ -330,6 +342,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int wq = warp & 3, ch = warp >> 2, r = threadIdx.x & 127;
     const int rg = r0 + r;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    // this thread's row of dS buffer 0: 128 bytes, its 16-byte chunks XOR-swizzled by row
+    const uint32_t ds_row = smem_u32(S.ds[0]) + (uint32_t)r * 128, sw = (uint32_t)(r & 7);
     const size_t stat = (((size_t)b * Hp + h) * 2 + m) * a.Lp + rg;
     const float c = a.scale * (m == 0 ? 1.f : -a.lambda[h]);
     const float2 nl2 = make_float2(a.nlse[stat], a.nlse[stat]), nd2 = make_float2(a.ndd[stat], a.ndd[stat]);
@@ -344,16 +358,24 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
       tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.s_free[bb]));   // in registers: S of tile j + 2 may overwrite them
       const long long lim = lastk - (long long)j * PF_BN - ch * 32;   // columns > lim are masked
-      // warp-uniform, so that the tcgen05.st below runs convergently
+      // warp-uniform: the warp runs one straight-line variant per tile
       if (__all_sync(0xffffffffu, lim >= 31))
         bw_q_elementwise<false>(sv, pv, ds, 0, sl2, nl2, nd2, c2);
       else
         bw_q_elementwise<true>(sv, pv, ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
-      tmem_st16p(tmem + lane_off + bb * 64 + ch * 32, ds);   // the chunk's own columns
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&S.p_full[bb]));
+      // dS buffer bb is free once dQ of tile j - 2 has completed
+      if (j >= 2 && !(ok = warp_wait(smem_u32(&S.ds_free[bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch))) break;
+      const uint32_t row_at = ds_row + (uint32_t)bb * DS_BUF;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)   // keys 32 ch + 8 q .. + 7: logical chunk 4 ch + q
+        sts_u4(row_at + ((((uint32_t)(4 * ch + q)) ^ sw) << 4), ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.p_full[bb]));
     }
     // ---- epilogue: dQ rows ----
     bool have = nT == 0;
@@ -373,7 +395,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
         for (int i = 0; i < 32; ++i) y[cc * 32 + i] = nT > 0 ? __uint_as_float(o[i]) : 0.f;
       }
-      pf_store_rows(S.stage[warp], y, base + ch * 64, r0 + wq * 32, a.Lq, lane, 64 * QB);
+      pf_store_rows(S.ds[0] + warp * 16 * 128, y, base + ch * 64, r0 + wq * 32, a.Lq, lane, 64 * QB);
     }
   }
 
@@ -517,7 +539,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&S.s_full[i]), 1);
-      mbar_init(smem_u32(&S.p_full[i]), BW_EW);
+      mbar_init(smem_u32(&S.p_full[i]), BW_EW_WARPS);
       mbar_init(smem_u32(&S.s_free[i]), 1);
       mbar_init(smem_u32(&S.drain[i]), 1);
     }
@@ -680,7 +702,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&S.p_full[bb]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.p_full[bb]));
     }
     // ---- epilogue: dV and dK rows of this tile's keys ----
     bool have = nS == 0;

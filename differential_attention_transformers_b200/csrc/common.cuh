@@ -216,6 +216,16 @@ __device__ __forceinline__ uint32_t umma_desc_lo(uint32_t saddr, uint32_t lbo_by
 __host__ __device__ constexpr uint32_t umma_desc_hi(uint32_t sbo_bytes) {
   return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
+// 16-byte shared-memory store (addr: a shared-window address).
+__device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (a tcgen05.mma operand): issue it after the
+// writes and before the barrier arrival that hands the buffer over.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 // D[tmem] (+)= A[smem desc] * B[smem desc], descriptors as {lo, hi} words.
 __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi,
                                          uint32_t idesc, uint32_t accumulate) {

@@ -89,6 +89,12 @@ constexpr size_t decode_smem() { return sizeof(DecSmem<kDecNst>) + 1024; }
 constexpr size_t decode_paged_smem() { return sizeof(DecSmem<kDecNst, true>) + 1024; }
 constexpr size_t bwd_dq_smem() { return sizeof(BwQSmem) + 1024; }
 constexpr size_t bwd_dkv_smem() { return sizeof(BwKSmem) + 1024; }
+static_assert(bwd_dq_smem() <= 227 * 1024 && bwd_dkv_smem() <= 227 * 1024,
+              "backward shared memory above the 227 KB a block may use");
+// each dS buffer holds 128 rows of 64 bf16 keys (128 bytes), and buffer 0
+// also the epilogue's staging (8 warps x 16 rows x 128 bytes)
+static_assert(sizeof(BwQSmem::ds[0]) == 128 * 128 && sizeof(BwQSmem::ds[0]) >= 8 * 16 * 128,
+              "dS buffer size");
 constexpr int kDecCtasPerSm = 2;
 
 // Per-device set-up: SM count, status word address, kernel attributes,
