@@ -418,7 +418,7 @@ struct BwKSmem {
   alignas(16) uint8_t stage[8][16 * 128];
   alignas(8) uint64_t kv_full;
   uint64_t st_full[BW_NS], st_empty[BW_NS];
-  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t s_full[2], p_full[2], sv_free[2], sd_free[2];
   uint64_t fin;
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -540,7 +540,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&S.s_full[i]), 1);
       mbar_init(smem_u32(&S.p_full[i]), BW_EW_WARPS);
-      mbar_init(smem_u32(&S.s_free[i]), 1);
+      mbar_init(smem_u32(&S.sv_free[i]), 1);
+      mbar_init(smem_u32(&S.sd_free[i]), 1);
       mbar_init(smem_u32(&S.drain[i]), 1);
     }
     mbar_init(smem_u32(&S.fin), 1);
@@ -613,25 +614,32 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           // first head); V2: one dK for both maps
           const uint32_t dk_t = tmem + 384 + (V1 ? (uint32_t)((qh & 1) * 64) : 0u);
           const bool dk_acc = V1 ? i > 1 : i > 0;
+          // dV += (w P)^T dO, with the bf16 residual 16 columns after each
+          // chunk's hi part; then S^T of step i + 2 may overwrite buffer bb
 #pragma unroll
-          for (int s = 0; s < BW_RB / 16; ++s)   // dV += (w P)^T dO
+          for (int s = 0; s < BW_RB / 16; ++s)
             mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s), olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
                      (i > 0 || s > 0));
-#pragma unroll
-          for (int s = 0; s < BW_RB / 16; ++s)   // dK += dS^T Q
-            mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_DK,
-                     (dk_acc || s > 0));
-          if (resid) {   // the bf16 residuals, 16 columns after each chunk's hi part
+          if (resid) {
 #pragma unroll
             for (int s = 0; s < BW_RB / 16; ++s)
               mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s) + 16, olo + (uint32_t)(s * (2048 >> 4)), HI,
                        IDESC_ACC, 1);
+          }
+          mma_commit(smem_u32(&S.sv_free[bb]));
+          // dK += dS^T Q and its residual; then dP^T of step i + 2 may
+          // overwrite buffer bb, and the stage is free
+#pragma unroll
+          for (int s = 0; s < BW_RB / 16; ++s)
+            mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_DK,
+                     (dk_acc || s > 0));
+          if (resid) {
 #pragma unroll
             for (int s = 0; s < BW_RB / 16; ++s)
               mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s) + 16, qlo + (uint32_t)(s * (2048 >> 4)), HI,
                        IDESC_DK, 1);
           }
-          mma_commit(smem_u32(&S.s_free[bb]));
+          mma_commit(smem_u32(&S.sd_free[bb]));
           mma_commit(smem_u32(&S.st_empty[st]));
         }
         if (ok) mma_commit(smem_u32(&S.fin));
@@ -643,7 +651,9 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         for (int i = 0; ok && i < nS; ++i) {
           const int bb = i & 1, st = i % BW_NS;
           if (!(ok = wait_bar(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
-          if (i >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[bb]), ((i - 2) >> 1) & 1, abort_flag, a.watch)))
+          // S^T(i) overwrites what dV(i - 2) read, dP^T(i) what dK(i - 2)
+          // read: each waits for its own reader
+          if (i >= 2 && !(ok = wait_bar(smem_u32(&S.sv_free[bb]), ((i - 2) >> 1) & 1, abort_flag, a.watch)))
             break;
           tc_fence_after();
           const uint32_t qlo = q_lo0 + (uint32_t)st * QSTAGE, olo = o_lo0 + (uint32_t)st * QSTAGE;
@@ -655,6 +665,9 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
             mma_ss_w(tmem + bb * 64, k_lo + kmo + ao, HI, qlo + bo, HI, IDESC_S, s > 0);
           }
+          if (i >= 2 && !(ok = wait_bar(smem_u32(&S.sd_free[bb]), ((i - 2) >> 1) & 1, abort_flag, a.watch)))
+            break;
+          tc_fence_after();
 #pragma unroll
           for (int s = 0; s < 8; ++s) {
             const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
