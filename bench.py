@@ -346,8 +346,8 @@ class Backward:
             self.out, self.lse, self.om, self.rstd, self.o2c = da.fwd_v1_train(x["q1"], x["k1"], x["q2"], x["k2"], x["v"],
                                                                      self.lam, causal=w.causal, rmsnorm=w.rmsnorm)
             nws = da.load().diffattn_bwd_v1_workspace_size(w.B, w.H, w.Hkv, w.Lq, w.Lk, int(w.rmsnorm))
-            # lambda, pack, [RMSNorm gradient], prep, dlambda, dQ, dK/dV, unpack, lambda's parameter gradients
-            self.launches_per_step = 9 if w.rmsnorm else 8
+            # lambda, [RMSNorm gradient], prep, dlambda, dQ, dK/dV, lambda's parameter gradients
+            self.launches_per_step = 7 if w.rmsnorm else 6
         self.ws = torch.empty(int(nws), dtype=torch.uint8, device=device)
 
     def step(self, ev=None):
