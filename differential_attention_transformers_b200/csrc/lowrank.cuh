@@ -39,9 +39,10 @@
 //
 // One thread owns one of the 128 value columns and r <= LR_RMAX accumulators.
 // The CTA first stages the factor rows its loop reads (the same for every
-// column) in shared memory; keys and rows are then taken several at a time
-// with their global loads issued first, so the passes are not bound by load
-// latency.  Each kernel body is a host-device function of (chunk, head,
+// column) in shared memory, each padded with zeros to LR_RMAX floats, so a row
+// is four 16-byte loads and the rank loops run to LR_RMAX without a test (the
+// padded ranks add exact zeros).  Keys and rows are then taken several at a
+// time with their global loads issued first.  Each kernel body is a host-device function of (chunk, head,
 // column) that takes those rows as pointers, so the same code can be run over
 // every index on the host.
 #pragma once
@@ -84,6 +85,22 @@ __host__ __device__ inline void lr_slots(int Lq, int Lk, int causal, int& n_lead
 
 __host__ __device__ inline long long lr_clamp(long long x, long long hi) { return x < 0 ? 0 : (x > hi ? hi : x); }
 
+// Element e of the padded copy of n rows of r factors (rows LR_RMAX apart,
+// ranks >= r zero); src: the rows, r apart.
+__host__ __device__ inline float lr_padded(const float* src, int r, long long e) {
+  const int t = (int)(e % LR_RMAX);
+  return t < r ? src[(e / LR_RMAX) * r + t] : 0.f;
+}
+
+// The LR_RMAX factors of one padded row (16-byte aligned).
+__host__ __device__ inline void lr_row(const float* row, float (&x)[LR_RMAX]) {
+#pragma unroll
+  for (int q = 0; q < LR_RMAX / 4; ++q) {
+    const float4 v = reinterpret_cast<const float4*>(row)[q];
+    x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+  }
+}
+
 // Keys whose sums slot c contributes (see the header).
 __host__ __device__ inline void lr_key_range(const LowrankArgs& a, int c, long long& ks, long long& ke) {
   if (a.causal) {
@@ -102,59 +119,55 @@ __host__ __device__ inline void lr_key_range(const LowrankArgs& a, int c, long l
   }
 }
 
-// Adds keys [ks, ke) of one value column: S[t] += g_j[t] v_j, z[t] += g_j[t].
-// vcol: the column (keys LR_DV apart); gk: the G rows of these keys, gk[(j -
-// ks) r + t].  Keys in ascending order, U at a time with their V loads issued
-// first, so U loads are in flight per thread.
-__host__ __device__ inline void lr_add_keys(int r, const __nv_bfloat16* vcol, const float* gk, long long ks,
-                                            long long ke, float (&S)[LR_RMAX], float (&z)[LR_RMAX]) {
+// Adds keys [ks, ke) of one value column: S[t] += g_j[t] v_j.  vcol: the
+// column (keys LR_DV apart); gk: the padded G rows of these keys, row j - ks
+// at gk + (j - ks) LR_RMAX.
+// Keys in ascending order, U at a time; the V loads of the next U keys are
+// issued before this group's arithmetic, so a group's memory latency overlaps
+// the one before it.
+__host__ __device__ inline void lr_add_keys(const __nv_bfloat16* vcol, const float* gk, long long ks, long long ke,
+                                            float (&S)[LR_RMAX]) {
   constexpr int U = 8;
-  long long j = ks;
-  for (; j + U <= ke; j += U) {
-    float vj[U];
+  float vj[U], vn[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) vj[u] = __bfloat162float(vcol[(j + u) * LR_DV]);
+  for (int u = 0; u < U; ++u) vj[u] = ks + u < ke ? __bfloat162float(vcol[(ks + u) * LR_DV]) : 0.f;
+  for (long long j = ks; j < ke; j += U) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) vn[u] = j + U + u < ke ? __bfloat162float(vcol[(j + U + u) * LR_DV]) : 0.f;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const float* g = gk + (j - ks + u) * r;
+      if (j + u >= ke) break;
+      float g[LR_RMAX];
+      lr_row(gk + (j - ks + u) * LR_RMAX, g);
 #pragma unroll
-      for (int t = 0; t < LR_RMAX; ++t)
-        if (t < r) {
-          S[t] = fmaf(g[t], vj[u], S[t]);
-          z[t] += g[t];
-        }
+      for (int t = 0; t < LR_RMAX; ++t) S[t] = fmaf(g[t], vj[u], S[t]);
     }
-  }
-  for (; j < ke; ++j) {
-    const float vj = __bfloat162float(vcol[j * LR_DV]);
-    const float* g = gk + (j - ks) * r;
 #pragma unroll
-    for (int t = 0; t < LR_RMAX; ++t)
-      if (t < r) {
-        S[t] = fmaf(g[t], vj, S[t]);
-        z[t] += g[t];
-      }
+    for (int u = 0; u < U; ++u) vj[u] = vn[u];
   }
 }
 
-// Slot c of head bh, value column col; gk: the G rows of the slot's keys
-// [ks, ke) (lr_key_range), gk[(j - ks) r + t].
+// Slot c of head bh, value column col; gk: the padded G rows of the slot's
+// keys [ks, ke) (lr_key_range).  The sums of g do not depend on the column:
+// column t < r forms the one of rank t.
 __host__ __device__ inline void lr_totals_body(const LowrankArgs& a, int c, int bh, int col, const float* gk) {
   const int b = bh / a.H, g = (bh % a.H) / (a.H / a.Hkv);
   long long ks, ke;
   lr_key_range(a, c, ks, ke);
-  float S[LR_RMAX], z[LR_RMAX];
+  float S[LR_RMAX];
 #pragma unroll
-  for (int t = 0; t < LR_RMAX; ++t) S[t] = z[t] = 0.f;
+  for (int t = 0; t < LR_RMAX; ++t) S[t] = 0.f;
   const __nv_bfloat16* vcol = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lk * LR_DV + col;
-  lr_add_keys(a.r, vcol, gk, ks, ke, S, z);
+  lr_add_keys(vcol, gk, ks, ke, S);
   const size_t slot = (size_t)bh * (a.nc + 1) + c;
 #pragma unroll
   for (int t = 0; t < LR_RMAX; ++t)
-    if (t < a.r) {
-      a.tot[(slot * a.r + t) * LR_DV + col] = S[t];
-      if (col == 0) a.ztot[slot * a.r + t] = z[t];
-    }
+    if (t < a.r) a.tot[(slot * a.r + t) * LR_DV + col] = S[t];
+  if (col < a.r) {
+    float z = 0.f;
+    for (long long j = ks; j < ke; ++j) z += gk[(j - ks) * LR_RMAX + col];
+    a.ztot[slot * a.r + col] = z;
+  }
 }
 
 // Exclusive prefix over the slots of head bh, rank index t, value column col
@@ -198,9 +211,10 @@ __host__ __device__ inline void lr_emit_range(const LowrankArgs& a, int c, long 
   k1 = a.causal ? lr_clamp(r1 + off, a.Lk) : 0;
 }
 
-// Row chunk c (rows [r0, r1)) of head bh, value column col.  fk: the F rows
-// of the chunk, fk[(i - r0) r + t]; gk: the G rows of the keys the rows add,
-// gk[(j - k0) r + t] (lr_emit_range).
+// Row chunk c (rows [r0, r1)) of head bh, value column col.  fk: the padded F
+// rows of the chunk, row i - r0 at fk + (i - r0) LR_RMAX; gk: the padded G
+// rows of the keys the rows add, row j - k0 at gk + (j - k0) LR_RMAX
+// (lr_emit_range).
 __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh, int col, const float* fk,
                                              const float* gk) {
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
@@ -233,22 +247,22 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
       const long long i = i0 + u, j = i + off;
       if (i >= r1) break;
       if (a.causal && j >= 0 && j < a.Lk) {
-        const float* gj = gk + (j - k0) * a.r;
+        float gj[LR_RMAX];
+        lr_row(gk + (j - k0) * LR_RMAX, gj);
 #pragma unroll
-        for (int t = 0; t < LR_RMAX; ++t)
-          if (t < a.r) {
-            S[t] = fmaf(gj[t], vj[u], S[t]);
-            z[t] += gj[t];
-          }
+        for (int t = 0; t < LR_RMAX; ++t) {
+          S[t] = fmaf(gj[t], vj[u], S[t]);
+          z[t] += gj[t];
+        }
       }
-      const float* fi = fk + (i - r0) * a.r;
+      float fi[LR_RMAX];
+      lr_row(fk + (i - r0) * LR_RMAX, fi);
       float num = 0.f, den = 0.f;
 #pragma unroll
-      for (int t = 0; t < LR_RMAX; ++t)
-        if (t < a.r) {
-          num = fmaf(fi[t], S[t], num);
-          den = fmaf(fi[t], z[t], den);
-        }
+      for (int t = 0; t < LR_RMAX; ++t) {
+        num = fmaf(fi[t], S[t], num);
+        den = fmaf(fi[t], z[t], den);
+      }
       const float nv = den > 0.f ? num / den : 0.f;
       orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * nv);
     }
@@ -256,31 +270,32 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
 }
 
 #ifdef __CUDACC__
-// Copies n floats from global memory into shared memory, all threads of the CTA.
-__device__ __forceinline__ void lr_stage(float* dst, const float* src, long long n) {
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src[i];
+// Stages n padded factor rows (lr_padded) into shared memory, all threads of the CTA.
+__device__ __forceinline__ void lr_stage(float* dst, const float* src, int r, long long n) {
+  for (long long e = threadIdx.x; e < n * LR_RMAX; e += blockDim.x) dst[e] = lr_padded(src, r, e);
   __syncthreads();
 }
 
 __global__ void __launch_bounds__(LR_DV) lr_totals_kernel(LowrankArgs a) {
-  __shared__ float sg[LR_C * LR_RMAX];
+  __shared__ alignas(16) float sg[LR_C * LR_RMAX];
   const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
   long long ks, ke;
   lr_key_range(a, c, ks, ke);
-  lr_stage(sg, a.G + ((size_t)h * a.Lk + ks) * a.r, (ke - ks) * a.r);
+  lr_stage(sg, a.G + ((size_t)h * a.Lk + ks) * a.r, a.r, ke - ks);
   lr_totals_body(a, c, bh, (int)threadIdx.x, sg);
 }
 __global__ void __launch_bounds__(LR_DV) lr_prefix_kernel(LowrankArgs a) {
   lr_prefix_body(a, (int)blockIdx.y, (int)blockIdx.x, (int)threadIdx.x);
 }
 __global__ void __launch_bounds__(LR_DV) lr_emit_kernel(LowrankArgs a) {
-  __shared__ float sf[LR_C * LR_RMAX];
-  __shared__ float sg[LR_C * LR_RMAX];
+  __shared__ alignas(16) float sf[LR_C * LR_RMAX];
+  __shared__ alignas(16) float sg[LR_C * LR_RMAX];
   const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
   long long r0, r1, k0, k1;
   lr_emit_range(a, c, r0, r1, k0, k1);
-  for (long long i = threadIdx.x; i < (r1 - r0) * a.r; i += blockDim.x) sf[i] = a.F[((size_t)h * a.Lq + r0) * a.r + i];
-  lr_stage(sg, a.G + ((size_t)h * a.Lk + k0) * a.r, (k1 - k0) * a.r);
+  for (long long e = threadIdx.x; e < (r1 - r0) * LR_RMAX; e += blockDim.x)
+    sf[e] = lr_padded(a.F + ((size_t)h * a.Lq + r0) * a.r, a.r, e);
+  lr_stage(sg, a.G + ((size_t)h * a.Lk + k0) * a.r, a.r, k1 - k0);
   lr_emit_body(a, c, bh, (int)threadIdx.x, sf, sg);
 }
 #endif

@@ -54,15 +54,20 @@ int main(int argc, char** argv) {
   a.tot = tot.data();
   a.ztot = ztot.data();
 
-  // The kernels stage the factor rows a CTA reads in shared memory; here the
-  // bodies read them in place, through pointers at the same offsets.
+  // The kernels stage the factor rows a CTA reads in shared memory, padded to
+  // LR_RMAX floats a row; here the same padded rows are built per CTA.
+  std::vector<float> pf, pg;
+  auto pad = [&](std::vector<float>& dst, const float* src, long long n) {
+    dst.assign((size_t)(n > 0 ? n : 0) * da::LR_RMAX, 0.f);
+    for (long long e = 0; e < n * da::LR_RMAX; ++e) dst[e] = da::lr_padded(src, r, e);
+  };
   if (a.nc > 0 && Lk > 0)
     for (int bh = 0; bh < (int)BH; ++bh)
       for (int c = 0; c < a.nc; ++c) {
         long long ks, ke;
         da::lr_key_range(a, c, ks, ke);
-        const float* gk = G.data() + ((size_t)(bh % H) * Lk + ks) * r;
-        for (int col = 0; col < da::LR_DV; ++col) da::lr_totals_body(a, c, bh, col, gk);
+        pad(pg, G.data() + ((size_t)(bh % H) * Lk + ks) * r, ke - ks);
+        for (int col = 0; col < da::LR_DV; ++col) da::lr_totals_body(a, c, bh, col, pg.data());
       }
   for (int bh = 0; bh < (int)BH; ++bh)
     for (int t = 0; t < r; ++t)
@@ -72,9 +77,9 @@ int main(int argc, char** argv) {
     for (int c = 0; c < nrc; ++c) {
       long long r0, r1, k0, k1;
       da::lr_emit_range(a, c, r0, r1, k0, k1);
-      const float* fk = F.data() + ((size_t)(bh % H) * Lq + r0) * r;
-      const float* gk = G.data() + ((size_t)(bh % H) * Lk + k0) * r;
-      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, fk, gk);
+      pad(pf, F.data() + ((size_t)(bh % H) * Lq + r0) * r, r1 - r0);
+      pad(pg, G.data() + ((size_t)(bh % H) * Lk + k0) * r, k1 - k0);
+      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, pf.data(), pg.data());
     }
 
   FILE* g = fopen(argv[2], "wb");
