@@ -232,16 +232,22 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
   const float lam = a.lambda[h];
   const float* arow = a.a1v + (size_t)bh * a.Lq * LR_DV + col;
   __nv_bfloat16* orow = a.out + (size_t)bh * a.Lq * LR_DV + col;
+  // Rows U at a time; the loads of the next group (A1 V of each row and the
+  // V value of the key it adds) are issued before this group's arithmetic,
+  // so a group's memory latency overlaps the one before it.
   constexpr int U = 4;
-  for (long long i0 = r0; i0 < r1; i0 += U) {
-    // this group's loads first: A1 V of each row and the V value of the key it adds
-    float av[U], vj[U];
+  float av[U], vj[U], an[U], vn[U];
+  auto load = [&](long long i0, float (&A)[U], float (&W)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const long long i = i0 + u, j = i + off;
-      av[u] = i < r1 ? arow[i * LR_DV] : 0.f;
-      vj[u] = (a.causal && i < r1 && j >= 0 && j < a.Lk) ? __bfloat162float(vcol[j * LR_DV]) : 0.f;
+      A[u] = i < r1 ? arow[i * LR_DV] : 0.f;
+      W[u] = (a.causal && i < r1 && j >= 0 && j < a.Lk) ? __bfloat162float(vcol[j * LR_DV]) : 0.f;
     }
+  };
+  load(r0, av, vj);
+  for (long long i0 = r0; i0 < r1; i0 += U) {
+    load(i0 + U, an, vn);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const long long i = i0 + u, j = i + off;
@@ -266,6 +272,11 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
       const float nv = den > 0.f ? num / den : 0.f;
       orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * nv);
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      av[u] = an[u];
+      vj[u] = vn[u];
+    }
   }
 }
 
@@ -287,7 +298,9 @@ __global__ void __launch_bounds__(LR_DV) lr_totals_kernel(LowrankArgs a) {
 __global__ void __launch_bounds__(LR_DV) lr_prefix_kernel(LowrankArgs a) {
   lr_prefix_body(a, (int)blockIdx.y, (int)blockIdx.x, (int)threadIdx.x);
 }
-__global__ void __launch_bounds__(LR_DV) lr_emit_kernel(LowrankArgs a) {
+// Six CTAs per SM: the 32 KB of staged factor rows allow no more, and the
+// register budget keeps the prefetched group within it.
+__global__ void __launch_bounds__(LR_DV, 6) lr_emit_kernel(LowrankArgs a) {
   __shared__ alignas(16) float sf[LR_C * LR_RMAX];
   __shared__ alignas(16) float sg[LR_C * LR_RMAX];
   const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
