@@ -699,7 +699,12 @@ def compact(name, r, total_ms, kern_ms, steps, rf):
             round(rf["frac_of_8tbs"], 4) if "frac_of_8tbs" in rf else None]
 
 
-SECONDARY_COLS = ["value", "unit", "ms_per_step", "kernel_ms", "frac", "frac_of_8tbs"]
+SECONDARY_COLS = ["value", "unit", "ms_per_step", "kernel_ms", "frac", "frac_of_8tbs", "sm_mhz"]
+
+# Idle time before each secondary row's warm-up, so that its timed region
+# starts from the regime of the headline one (a launch timed on its own, the
+# burst clock) rather than from the power-capped clock the rows before it left.
+SETTLE_S = 1.0
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
@@ -985,16 +990,23 @@ def main():
         names = ["v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged", "v2_decode_serving",
                  "v1_decode", "v1_decode_unfused", "lowrank_prefill", "snr_sweep", "v2_prefill"]
         n2 = max(3, args.steps // 2)
-        for name in names:
-            if name == args.workload:
-                continue
-            r2 = make_runner(name, device)
-            t2, k2 = time_runner(r2, n2, args.warmup, False)
-            secondary[name] = compact(name, r2, t2, k2, n2, roofline(r2, k2, peaks, capped, name))
-            if isinstance(r2, SnrSweep):
-                snr = r2.compact_summary()
-            del r2
-            torch.cuda.empty_cache()
+        with ClockSampler(torch.cuda.current_device()) as clk2:
+            for name in names:
+                if name == args.workload:
+                    continue
+                r2 = make_runner(name, device)
+                torch.cuda.synchronize()
+                time.sleep(SETTLE_S)
+                w2 = []
+                t2, k2 = time_runner(r2, n2, args.warmup, False, w2)
+                c2 = clk2.summary(*w2)
+                rf2 = roofline(r2, k2, peaks, "sw_power_cap" in c2["reasons"], name)
+                mhz = c2["sm_mhz"]
+                secondary[name] = compact(name, r2, t2, k2, n2, rf2) + [None if mhz is None else int(round(mhz))]
+                if isinstance(r2, SnrSweep):
+                    snr = r2.compact_summary()
+                del r2
+                torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:

@@ -33,9 +33,9 @@ def test_default_line_has_every_key_and_secondary():
     assert set(line["secondary"]) == {"v1_prefill", "v2_backward", "v1_backward", "v2_decode", "v2_decode_paged",
                                       "v2_decode_serving", "v1_decode", "v1_decode_unfused", "lowrank_prefill",
                                       "snr_sweep"}
-    assert line["secondary_cols"] == ["value", "unit", "ms_per_step", "kernel_ms", "frac", "frac_of_8tbs"]
+    assert line["secondary_cols"] == ["value", "unit", "ms_per_step", "kernel_ms", "frac", "frac_of_8tbs", "sm_mhz"]
     for name, row in line["secondary"].items():
-        assert len(row) == 6 and row[1] in ("TFLOP/s", "GB/s"), name
+        assert len(row) == 7 and row[1] in ("TFLOP/s", "GB/s"), name
         assert (row[5] is None) == (row[1] == "TFLOP/s"), name
     assert [r[0] for r in line["snr"]] == [1024, 2048]
     # the rows come last and the whole line stays short, so the end of the
