@@ -194,31 +194,47 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
       long long issued_last[NST];
       for (int i = 0; i < NST; ++i) issued_last[i] = -1;
       bool ok = true;
+      // Paged mode: where block x lies -- its KV head, first key and page
+      // ids.  The sequence index only moves forward as x does, and the page
+      // ids of block x + 1 are read before the wait for block x's stage, so
+      // the block-table reads are in flight while this thread waits.
+      struct PagedBlk {
+        int pg, pkey0, pparts, pages[4];
+      };
+      int bcur = PAGED ? dec_find_seq(S.cu, a.B, lo) : 0;
+      auto locate = [&](long long x) {
+        PagedBlk r{0, 0, 1, {0, 0, 0, 0}};
+        if constexpr (PAGED) {
+          while (S.cu[bcur + 1] <= x) ++bcur;   // skips empty sequences; x < cu[B]
+          const int b = bcur;
+          const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
+          const int within = (int)(x - S.cu[b]);
+          r.pg = within / nb;
+          r.pkey0 = (within % nb) * DEC_KB;
+          const int* row = a.block_table + (size_t)b * a.max_pages + (r.pkey0 >> a.page_shift);
+          if (a.page_size >= DEC_KB) {
+            r.pages[0] = row[0];
+          } else {
+            // page parts of the block that hold a key of the sequence (>= 1);
+            // parts wholly past it are not loaded (masked, V rows zeroed)
+            r.pparts = min(DEC_KB, S.len[b] - r.pkey0 + a.page_size - 1) / a.page_size;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (i < r.pparts) r.pages[i] = row[i];
+          }
+        }
+        return r;
+      };
+      PagedBlk nxt{0, 0, 1, {0, 0, 0, 0}};
+      if (PAGED && lo < hi) nxt = locate(lo);
       for (long long x = lo; x < hi; ++x) {
         const long long it = x - lo;
         const int st = (int)(it % NST);
         const long long use = it / NST;
-        // Paged mode: locate the block and read its page ids before waiting
-        // for the stage, so the table reads overlap the wait.
-        int pg = 0, pkey0 = 0, pparts = 1, pages[4] = {0, 0, 0, 0};
-        if constexpr (PAGED) {
-          const int b = dec_find_seq(S.cu, a.B, x);
-          const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
-          const int within = (int)(x - S.cu[b]);
-          pg = within / nb;
-          pkey0 = (within % nb) * DEC_KB;
-          const int* row = a.block_table + (size_t)b * a.max_pages + (pkey0 >> a.page_shift);
-          if (a.page_size >= DEC_KB) {
-            pages[0] = row[0];
-          } else {
-            // page parts of the block that hold a key of the sequence (>= 1);
-            // parts wholly past it are not loaded (masked, V rows zeroed)
-            pparts = min(DEC_KB, S.len[b] - pkey0 + a.page_size - 1) / a.page_size;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (i < pparts) pages[i] = row[i];
-          }
-        }
+        const PagedBlk cur = nxt;
+        if (PAGED && x + 1 < hi) nxt = locate(x + 1);
+        const int pg = cur.pg, pkey0 = cur.pkey0, pparts = cur.pparts;
+        const int pages[4] = {cur.pages[0], cur.pages[1], cur.pages[2], cur.pages[3]};
         if (use > 0 && !wait_bar(smem_u32(&S.empty[st]), (uint32_t)((use - 1) & 1), abort_flag, a.watch)) {
           ok = false;
           break;
