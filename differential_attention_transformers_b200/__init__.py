@@ -201,7 +201,7 @@ def compute_lambda(lq1, lk1, lq2, lk2, lam_init: float, out=None):
 # ----------------------------------------------------------------------------
 # end-to-end prefill on host tensors: chunked, with copies overlapping kernels
 _PIPELINE_MIN_BYTES = 64 << 20     # smaller inputs take the plain copy-compute-copy path
-_PIPELINE_CHUNK_UNITS = 1024       # 128-row blocks per chunk kernel: several waves of CTAs
+_PIPELINE_CHUNK_UNITS = 256        # 128-row blocks per chunk kernel
 _pipe_streams = {}
 
 
