@@ -59,6 +59,7 @@ CASES = [
     (1, 4, 1, 200, 200, True),      # ragged tails, one KV head for both pairs
     (2, 8, 2, 300, 300, False),     # non-causal, GQA groups of 4 Q heads
     (1, 4, 2, 130, 257, True),      # Lq < Lk: bottom-right causal offset
+    (1, 4, 2, 257, 130, True),      # Lq > Lk: the first rows see no key (a row block with no key tile)
     (1, 8, 1, 64, 64, True),        # a single tile
 ]
 
