@@ -285,7 +285,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     for (int m = 0; m < 2; ++m) {
       for (int bb = 0; bb < 2; ++bb) {
         mbar_init(smem_u32(&S.s_full[m][bb]), 1);
-        mbar_init(smem_u32(&S.p_full[m][bb]), 128);
+        mbar_init(smem_u32(&S.p_full[m][bb]), 4);   // one arrival per softmax warp of the map
         mbar_init(smem_u32(&S.s_free[m][bb]), 1);
       }
       mbar_init(smem_u32(&S.o_done[m]), 1);
@@ -494,7 +494,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&S.p_full[m][bb]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.p_full[m][bb]));
     }
 
     // --------------------------------------------------------- epilogue --
