@@ -602,13 +602,14 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         const uint32_t o_mn0 = umma_desc_lo(smem_u32(S.o[0]), PF_KBOX), q_mn0 = umma_desc_lo(smem_u32(S.q[0]), PF_KBOX);
         for (int i = 0; ok && i < nS; ++i) {
           const int bb = i & 1, st = i % BW_NS;
+          const int qh = step_head(i);
+          // read before the waits, so the load is not on the issue path
+          const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
           // this thread reads the stage's Q and dO too: acquire them here
           if (!(ok = wait_bar(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
           if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
           tc_fence_after();
           const uint32_t olo = o_mn0 + (uint32_t)st * QSTAGE, qlo = q_mn0 + (uint32_t)st * QSTAGE;
-          const int qh = step_head(i);
-          const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
           // V1: map m's dK lives in its own 64 columns and first receives a
           // value at step m (steps 0 and 1 are the two maps of the group's
           // first head); V2: one dK for both maps
@@ -691,7 +692,10 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       const int bb = i & 1, st = i % BW_NS;
       const int qh = step_head(i), rb = step_rb(i);
       const int mq = qh & 1;
-      const float w = mq == 0 ? 1.f : -a.lambda[qh / 2];   // weight of this map in A_1 - lambda A_2
+      // lambda read once, before the waits, so its load is not on the step's path
+      const float lam = a.lambda[qh / 2];
+      const float w = mq == 0 ? 1.f : -lam;   // weight of this map in A_1 - lambda A_2
+      const bool resid = fabsf(1.f - lam) < a.resid_tau;
       const float2 w2 = make_float2(w, w), cd2 = make_float2(a.scale * w, a.scale * w);
       // The stage's log-sum-exp and D values came by bulk copy: wait for them here too.
       if (!(ok = warp_wait(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
@@ -700,7 +704,6 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       // rows r = rb*64 + col see this key iff kg < Lk and (not causal or kg <= r + off)
       const int row0 = rb * BW_RB + ch * 32;
       const int vis0 = kg >= a.Lk ? 32 : (a.causal ? min(32, max(0, kg - off - row0)) : 0);
-      const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
       const uint32_t tS = tmem + lane_off + bb * 64 + ch * 32, tP = tmem + lane_off + 128 + bb * 64 + ch * 32;
       // branch once per step, warp-uniformly (the TMEM stores inside are
       // warp-collective): each variant's loop is one straight-line block
