@@ -90,46 +90,65 @@ struct BwdPrepArgs {
   const float* d_in;            // [B, Hp, 2, Lq] D_m formed upstream (V1 with RMSNorm), or null
 };
 
-// grid (Lp / 64, B * Hp), 256 threads: warp w handles rows 8w .. 8w+7 of the block.
+// grid (Lp / 64, B * Hp), 256 threads: warp w handles rows 8w .. 8w+7 of the
+// block, four lanes a row (lane l: row 8w + l/4, columns 32 (l%4) .. +31), so
+// the loads of all eight rows are in flight at once.
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
   __shared__ float wsum[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  float acc = 0.f;
-  for (int i = 0; i < 8; ++i) {
-    const int row = blockIdx.x * 64 + warp * 8 + i;
-    float d[2] = {0.f, 0.f};
-    if (row < a.Lq && a.d_in != nullptr) {
+  const int row = blockIdx.x * 64 + warp * 8 + (lane >> 2), part = lane & 3;
+  float d[2] = {0.f, 0.f};
+  if (a.d_in != nullptr) {
+    if (row < a.Lq) {
       d[0] = a.d_in[((size_t)bh * 2) * a.Lq + row];
       d[1] = a.d_in[((size_t)bh * 2 + 1) * a.Lq + row];
-    } else if (row < a.Lq) {
-      const __nv_bfloat16* go = a.dout + ((size_t)bh * a.Lq + row) * 128 + lane * 4;
-      const uint2 gv = *reinterpret_cast<const uint2*>(go);
+    }
+  } else {
+    float s[2] = {0.f, 0.f};
+    if (row < a.Lq) {
+      const size_t col = (size_t)part * 32;
+      const uint4* go = reinterpret_cast<const uint4*>(a.dout + ((size_t)bh * a.Lq + row) * 128 + col);
+      const uint4* o1 = reinterpret_cast<const uint4*>(a.o_maps + (((size_t)bh * 2) * a.Lq + row) * 128 + col);
+      const uint4* o2 = reinterpret_cast<const uint4*>(a.o_maps + (((size_t)bh * 2 + 1) * a.Lq + row) * 128 + col);
+      uint4 gv[4], v1[4], v2[4];
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint2 ov =
-            *reinterpret_cast<const uint2*>(a.o_maps + (((size_t)bh * 2 + m) * a.Lq + row) * 128 + lane * 4);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
-        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-        float s = 0.f;
+      for (int q = 0; q < 4; ++q) {
+        gv[q] = go[q];
+        v1[q] = o1[q];
+        v2[q] = o2[q];
+      }
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float2 gf = __bfloat1622float2(g2[j]), of = __bfloat1622float2(o2[j]);
-          s = fmaf(gf.x, of.x, s);
-          s = fmaf(gf.y, of.y, s);
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[q]);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&v1[q]);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v2[q]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 gf = __bfloat1622float2(g2[e]), af = __bfloat1622float2(a2[e]), bf = __bfloat1622float2(b2[e]);
+          s[0] = fmaf(gf.x, af.x, s[0]);
+          s[0] = fmaf(gf.y, af.y, s[0]);
+          s[1] = fmaf(gf.x, bf.x, s[1]);
+          s[1] = fmaf(gf.y, bf.y, s[1]);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        d[m] = s;
       }
     }
-    if (lane < 2) {
-      const size_t at = ((size_t)bh * 2 + lane) * a.Lp + row;
-      a.ndd[at] = -d[lane];
-      a.nlse[at] = row < a.Lq ? -a.lse[((size_t)bh * 2 + lane) * a.Lq + row] : -INFINITY;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {   // the row's four lanes; rows past Lq add zeros
+      s[m] += __shfl_xor_sync(0xffffffffu, s[m], 1);
+      s[m] += __shfl_xor_sync(0xffffffffu, s[m], 2);
+      d[m] = s[m];
     }
-    acc -= d[1];
   }
+  if (part < 2) {   // lane part m of the row writes map m's values
+    const size_t at = ((size_t)bh * 2 + part) * a.Lp + row;
+    a.ndd[at] = -d[part];
+    a.nlse[at] = row < a.Lq ? -a.lse[((size_t)bh * 2 + part) * a.Lq + row] : -INFINITY;
+  }
+  // dlambda partial: the sum of -D_2 over the warp's eight rows, then the block's
+  float acc = part == 0 ? -d[1] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) wsum[warp] = acc;
   __syncthreads();
   if (threadIdx.x == 0) {
