@@ -498,15 +498,17 @@ struct CombineArgs {
   const int* cu;       // paged mode: block prefix written by the split kernel (null otherwise)
 };
 
-// One CTA (128 threads = the value width) per (batch, output head).
+// One CTA (128 threads = the value width) per (batch, KV head): the output
+// heads of a KV head share one walk over the split CTAs' records.  Each
+// output keeps the order of operations of a walk of its own, so the result
+// does not depend on how many heads share it.
 __global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
+  constexpr int MAXO = 4;   // output heads of a KV head: V2 (8 Q columns) / 2, V1 (4 + 4 columns)
   const int t = threadIdx.x;
   const int Hout = a.v1 ? a.Hq : a.Hq / 2;
-  const int b = blockIdx.x / Hout, h = blockIdx.x % Hout;
   const int grp = a.Hq / a.Hkv;
-  int g, c1, c2;
-  if (a.v1) { g = h / grp; c1 = h % grp; c2 = 4 + h % grp; }
-  else { g = (2 * h) / grp; c1 = (2 * h) % grp; c2 = c1 + 1; }
+  const int opg = a.v1 ? grp : grp / 2;
+  const int b = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
   const long long bg = (long long)b * a.Hkv + g;
   long long x0, x1, total = a.total;
   if (a.cu) {   // paged: this sequence's blocks per KV head from the prefix
@@ -518,6 +520,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
     x0 = bg * a.nblk;
     x1 = x0 + a.nblk;
   }
+  // query column of output head oh and map mp: V2 pair oh = columns 2 oh,
+  // 2 oh + 1; V1 head oh = column oh (map 1) and 4 + oh (map 2)
+  auto col = [&](int oh, int mp) { return a.v1 ? (mp ? 4 + oh : oh) : 2 * oh + mp; };
 
   // The CTAs whose ranges overlap [x0, x1), in ascending order: start at the
   // owner of x0, then jump to the owner of the block after each range.  Only
@@ -530,33 +535,49 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(CombineArgs a) {
     return a.cu ? base + ((size_t)i + (size_t)bg) * DEC_REC
                 : base + ((size_t)i * a.maxseg + (size_t)(bg - s / a.nblk)) * DEC_REC;
   };
-  const int cc[2] = {c1, c2};
-  float M[2] = {-INFINITY, -INFINITY};
+  float M[MAXO][2];
+#pragma unroll
+  for (int oh = 0; oh < MAXO; ++oh) M[oh][0] = M[oh][1] = -INFINITY;
   for (long long x = x0; x < x1;) {
     const long long i = dec_owner(x, total, a.grid);
     const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
 #pragma unroll
-    for (int mp = 0; mp < 2; ++mp) M[mp] = fmaxf(M[mp], record(i, s, mp)[cc[mp]]);
+    for (int oh = 0; oh < MAXO; ++oh)
+      if (oh < opg) {
+#pragma unroll
+        for (int mp = 0; mp < 2; ++mp) M[oh][mp] = fmaxf(M[oh][mp], record(i, s, mp)[col(oh, mp)]);
+      }
     x = e;
   }
-  float o[2] = {0.f, 0.f}, l[2] = {0.f, 0.f};
+  float o[MAXO][2], l[MAXO][2];
+#pragma unroll
+  for (int oh = 0; oh < MAXO; ++oh) o[oh][0] = o[oh][1] = l[oh][0] = l[oh][1] = 0.f;
   for (long long x = x0; x < x1;) {
     const long long i = dec_owner(x, total, a.grid);
     const long long s = dec_blk_start(i, total, a.grid), e = dec_blk_start(i + 1, total, a.grid);
 #pragma unroll
-    for (int mp = 0; mp < 2; ++mp) {
-      const float* rec = record(i, s, mp);
-      const float f = ex2(rec[cc[mp]] - (M[mp] == -INFINITY ? 0.f : M[mp]));
-      o[mp] += rec[16 + cc[mp] * 128 + t] * f;
-      l[mp] += rec[8 + cc[mp]] * f;
+    for (int oh = 0; oh < MAXO; ++oh)
+      if (oh < opg) {
+#pragma unroll
+        for (int mp = 0; mp < 2; ++mp) {
+          const int c = col(oh, mp);
+          const float* rec = record(i, s, mp);
+          const float f = ex2(rec[c] - (M[oh][mp] == -INFINITY ? 0.f : M[oh][mp]));
+          o[oh][mp] += rec[16 + c * 128 + t] * f;
+          l[oh][mp] += rec[8 + c] * f;
+        }
+      }
+    x = e;
+  }
+#pragma unroll
+  for (int oh = 0; oh < MAXO; ++oh)
+    if (oh < opg) {
+      const int h = g * opg + oh;
+      const float r0 = l[oh][0] > 0.f ? o[oh][0] / l[oh][0] : 0.f;
+      const float r1 = l[oh][1] > 0.f ? o[oh][1] / l[oh][1] : 0.f;
+      const float lam = a.lambda[h];
+      a.out[((size_t)b * Hout + h) * 128 + t] = __float2bfloat16_rn(__fsub_rn(r0, __fmul_rn(lam, r1)));
     }
-    x = e;
-  }
-  float res[2];
-#pragma unroll
-  for (int mp = 0; mp < 2; ++mp) res[mp] = l[mp] > 0.f ? o[mp] / l[mp] : 0.f;
-  const float lam = a.lambda[h];
-  a.out[((size_t)b * Hout + h) * 128 + t] = __float2bfloat16_rn(__fsub_rn(res[0], __fmul_rn(lam, res[1])));
 }
 
 }  // namespace da

@@ -330,8 +330,7 @@ int launch_decode(const void* q1, const void* q2, const void* k1, const void* k2
   c.two_pass = passes == 2 ? 1 : 0;
   c.half_floats = p.bytes_per_pass / sizeof(float);
   c.cu = nullptr;
-  const int Hout = v1 ? Hq : Hq / 2;
-  decode_combine_kernel<<<(unsigned)(B * Hout), 128, 0, s>>>(c);
+  decode_combine_kernel<<<(unsigned)(B * Hkv), 128, 0, s>>>(c);   // one CTA per (batch, KV head)
   CUDA_TRY(cudaGetLastError());
   return ok();
 }
@@ -539,7 +538,7 @@ int launch_decode_paged(const void* q, const void* kp, const void* vp, const int
   c.grid = a.grid; c.maxseg = 0; c.nblk = 0; c.total = 0;
   c.two_pass = 0; c.half_floats = 0;
   c.cu = cu;
-  decode_combine_kernel<<<(unsigned)(B * (Hq / 2)), 128, 0, s>>>(c);
+  decode_combine_kernel<<<(unsigned)(B * Hkv), 128, 0, s>>>(c);   // one CTA per (batch, KV head)
   CUDA_TRY(cudaGetLastError());
   return ok();
 }
