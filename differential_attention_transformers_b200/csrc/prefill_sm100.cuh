@@ -292,8 +292,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       mbar_init(smem_u32(&S.drain[m]), 1);
     }
     mbar_init(smem_u32(&S.o_final), 1);
-    mbar_init(smem_u32(&S.xl), 256);
-    mbar_init(smem_u32(&S.xs), 256);
+    mbar_init(smem_u32(&S.xl), 8);   // one arrival per softmax warp
+    mbar_init(smem_u32(&S.xs), 8);
     S.abort_flag = 0;
     mbar_fence_init();
   }
@@ -506,7 +506,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     float kx = 0.f;   // training with RMSNorm: c / rs, so that c X = kx y once y holds rs X
     if (ok && nT > 0) {
       S.l[m][r] = l_run;
-      mbar_arrive(smem_u32(&S.xl));
+      // the warp's stores, then one arrival for it
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.xl));
       ok = warp_wait(smem_u32(&S.xl), 0, abort_flag, a.watch) &&
            warp_wait(smem_u32(&S.o_final), 0, abort_flag, a.watch);
       if (ok && SINGLE) {
@@ -538,7 +541,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           for (int i = 0; i < 64; ++i) ss = fmaf(y[i], y[i], ss);
           S.ss[m][r] = ss;
           if (TRAIN) S.sp[m][r] = sp;
-          mbar_arrive(smem_u32(&S.xs));
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&S.xs));
           ok = warp_wait(smem_u32(&S.xs), 0, abort_flag, a.watch);
           have = ok;
           if (ok) {
