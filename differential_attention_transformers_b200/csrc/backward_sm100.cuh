@@ -21,19 +21,20 @@
 //                    order by bwd_dlambda_kernel, so the result is
 //                    deterministic).
 //   bwd_dq_kernel    query-stationary: one CTA per 128 rows of one Q head (one
-//                    map).  Per 64-key tile: S = Q K^T and dP = dO V^T into
-//                    TMEM, dS = c P (dP - D) written to shared memory as bf16,
-//                    then dQ += dS K with dS as the shared A operand.  The
-//                    score buffer is then free as soon as the elementwise
-//                    warps have loaded it, so S of tile j + 2 waits only for
-//                    that load and for its K/V stage (four stages).
+//                    map).  Per 128-key tile: S = Q K^T and dP = dO V^T into
+//                    TMEM (N = 128 products, with Q and dO in TMEM as their A
+//                    operands), dS = c P (dP - D) written to shared memory as
+//                    bf16, then dQ += dS K with dS as the shared A operand.
+//                    The one score buffer is free as soon as the elementwise
+//                    warps have loaded it, so the products of tile j + 1 run
+//                    while tile j's elementwise phase does.
 //   bwd_dkv_kernel   key-stationary: one CTA per 128 keys of one KV head.  Per
 //                    64-row step of each Q head of the group: S^T = K Q^T and
 //                    dP^T = V dO^T into TMEM, then w P^T (w = 1 or -lambda)
 //                    and dS^T written back as bf16, and dV += (w P)^T dO,
 //                    dK += dS^T Q with those as the TMEM operands.
 // Computing dQ apart from dK/dV recomputes S and dP once more but needs no
-// atomics, and each kernel fits TMEM: dQ 384 columns, dK/dV 512.
+// atomics, and each kernel fits TMEM (512 columns each).
 // Both MMA kernels use the forward's pipeline: a TMA producer warp, one
 // issuing thread for the S-type products and one for the accumulating ones,
 // and eight warps (two per TMEM lane quadrant, one per 32-column chunk)
@@ -54,7 +55,8 @@ constexpr int BW_THREADS = 352;
 constexpr int BW_EW = 256;        // elementwise threads
 constexpr int BW_EW_WARPS = BW_EW / 32;   // arrivals on the elementwise warps' barriers: one per warp
 constexpr int BW_NS = 3;          // pipeline stages of the key-stationary kernel
-constexpr int BWQ_NS = 4;         // K/V stages of the query-stationary kernel
+constexpr int BWQ_NS = 3;         // K/V stages of the query-stationary kernel
+constexpr int BWQ_BN = 128;       // keys per tile of the query-stationary kernel
 constexpr int BW_RB = 64;         // rows per step of the key-stationary kernel
 
 struct BwdArgs {
@@ -170,17 +172,18 @@ __global__ void bwd_dlambda_kernel(const float* part, float* dlambda, int B, int
 
 // ------------------------------------------------------------ dQ (Q-stationary) --
 struct BwQSmem {
-  alignas(1024) uint8_t q[2 * PF_QBOX];            // Q tile of the head: 128 rows, dims 0-63 box, 64-127 box
-  alignas(1024) uint8_t o[2 * PF_QBOX];            // dO tile of the pair, same layout
-  alignas(1024) uint8_t k[BWQ_NS][2 * PF_KBOX];    // K tile: 64 keys, two boxes
-  alignas(1024) uint8_t v[BWQ_NS][2 * PF_KBOX];    // V tile
-  // dS, bf16 [128 rows][64 keys], K-major with the 128-byte swizzle (the A
-  // operand of dQ += dS K); ds[0] doubles as the epilogue's staging once
-  // every product has completed
-  alignas(1024) uint8_t ds[2][PF_QBOX];
-  alignas(8) uint64_t q_full;
+  // K/V stage st: the K tile (two [128 keys][64] boxes of the QK width; V1
+  // one), then the V tile (two boxes).  Stage 2 first holds the Q tile (two
+  // [128 rows][64] boxes; V1 one) and the dO tile: the elementwise warps copy
+  // them into TMEM (qt_full) before a K/V tile is loaded there.
+  alignas(1024) uint8_t kv[BWQ_NS][4 * PF_QBOX];
+  // dS, bf16 [128 rows][128 keys]: two K-major, 128-byte-swizzled boxes of 64
+  // keys (the A operand of dQ += dS K); the epilogue's staging once every
+  // product has completed
+  alignas(1024) uint8_t ds[2 * PF_QBOX];
+  alignas(8) uint64_t q_full, qt_full;
   uint64_t k_full[BWQ_NS], v_full[BWQ_NS], kv_empty[BWQ_NS];
-  uint64_t s_full[2], p_full[2], s_free[2], ds_free[2];
+  uint64_t s_full, s_free, p_full, ds_free;
   uint64_t fin;
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -191,12 +194,7 @@ struct BwQSmem {
 // bf16 buffer (slices 0, 1 in chunk 0; 2, 3 in chunk 1).
 __device__ __forceinline__ uint32_t bw_slice(int s) { return (uint32_t)((s >> 1) * 32 + (s & 1) * 8); }
 
-// V1: the V1 layout ("差分注意力" tutorial, section V1 到 V2 的 diff): Q head
-// qh of the Hq = 2H heads is map qh & 1 of V1 head qh / 2, read from its own
-// 64-wide tensor (tmQ for map 1, tmQ2 for map 2; tmK, tmK2 likewise), and dQ
-// of map 2 goes to dq2.  The scores then contract over 64 dimensions and dQ
-// is 64 wide; dO, V and everything else are as in V2.
-// One step of the query-stationary kernel for this thread's row and this
+// One half-step of the query-stationary kernel for this thread's row and this
 // warp's 32-key chunk: dS = c P (dP - D) with P = 2^(S scale_log2 - lse), in
 // f32x2 pairs (each operation rounds as its scalar form would).  With MASK,
 // columns past lim (-1..31) are masked.
@@ -217,6 +215,19 @@ __device__ __forceinline__ void bw_q_elementwise(const uint32_t (&sv)[32], const
   }
 }
 
+// V1: the V1 layout ("差分注意力" tutorial, section V1 到 V2 的 diff): Q head
+// qh of the Hq = 2H heads is map qh & 1 of V1 head qh / 2, read from its own
+// 64-wide tensor (tmQ for map 1, tmQ2 for map 2; tmK, tmK2 likewise), and dQ
+// of map 2 goes to dq2.  The scores then contract over 64 dimensions and dQ
+// is an N = 64 product.
+//
+// Tiles are 128 keys, so the score products S = Q K^T and dP = dO V^T are
+// N = 128 (a tcgen05.mma of N = 64 runs at about two-thirds of the tensor
+// rate, one of N = 128 at the full rate).  Q and dO, the same for every tile,
+// sit in TMEM as their A operands.  S and dP have one TMEM buffer: the
+// elementwise warps release it (s_free) once they have loaded both of its
+// 64-key halves, and write dS to shared memory, so the products of tile j + 1
+// run while tile j's elementwise phase does.
 template <bool V1>
 __global__ void __maxnreg__(168)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ2,
@@ -237,22 +248,21 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int r0 = rb * PF_BM;
   long long kend = a.causal ? (long long)min(r0 + PF_BM, a.Lq) - 1 + (a.Lk - a.Lq) + 1 : a.Lk;
   kend = max(0LL, min(kend, (long long)a.Lk));
-  const int nT = (int)((kend + PF_BN - 1) / PF_BN);
+  const int nT = (int)((kend + BWQ_BN - 1) / BWQ_BN);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&S.q_full), 1);
+    mbar_init(smem_u32(&S.qt_full), BW_EW_WARPS);
     for (int i = 0; i < BWQ_NS; ++i) {
       mbar_init(smem_u32(&S.k_full[i]), 1);
       mbar_init(smem_u32(&S.v_full[i]), 1);
       mbar_init(smem_u32(&S.kv_empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&S.s_full[i]), 1);
-      mbar_init(smem_u32(&S.p_full[i]), BW_EW_WARPS);
-      mbar_init(smem_u32(&S.s_free[i]), BW_EW_WARPS);
-      mbar_init(smem_u32(&S.ds_free[i]), 1);
-      mbar_init(smem_u32(&S.drain[i]), 1);
-    }
+    mbar_init(smem_u32(&S.s_full), 1);
+    mbar_init(smem_u32(&S.s_free), BW_EW_WARPS);
+    mbar_init(smem_u32(&S.p_full), BW_EW_WARPS);
+    mbar_init(smem_u32(&S.ds_free), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&S.drain[i]), 1);
     mbar_init(smem_u32(&S.fin), 1);
     S.abort_flag = 0;
     mbar_fence_init();
@@ -264,30 +274,33 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = S.tmem_base;   // S [0,128), dP [128,256), dQ [256,384)
-  constexpr uint32_t DS_BUF = (uint32_t)sizeof(S.ds[0]);
+  const uint32_t tmem = S.tmem_base;
+  // S [0,128), dP [128,256), dQ [256, 256 + 64 QB), Q [384, 384 + 32 QB), dO [448,512)
+  constexpr uint32_t T_S = 0, T_P = 128, T_DQ = 256, T_Q = 384, T_O = 448;
+  constexpr uint32_t HI = umma_desc_hi(1024);
+  constexpr int QO = BWQ_NS - 1;   // the stage that first holds Q and dO
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
     if (lane == 0 && nT > 0) {
-      const uint32_t qb = smem_u32(&S.q_full);
+      const uint32_t qb = smem_u32(&S.q_full), qo = smem_u32(S.kv[QO]);
       const CUtensorMap* tq = (V1 && m) ? &tmQ2 : &tmQ;
       const CUtensorMap* tk = (V1 && m) ? &tmK2 : &tmK;
       mbar_expect_tx(qb, (QB + 2) * PF_QBOX);
-      for (int x = 0; x < QB; ++x) tma_load_3d(smem_u32(S.q) + x * PF_QBOX, tq, qb, 64 * x, r0, V1 ? b * Hp + h : b * a.Hq + qh);
-      for (int x = 0; x < 2; ++x) tma_load_3d(smem_u32(S.o) + x * PF_QBOX, &tmO, qb, 64 * x, r0, b * Hp + h);
+      for (int x = 0; x < QB; ++x) tma_load_3d(qo + x * PF_QBOX, tq, qb, 64 * x, r0, V1 ? b * Hp + h : b * a.Hq + qh);
+      for (int x = 0; x < 2; ++x) tma_load_3d(qo + (2 + x) * PF_QBOX, &tmO, qb, 64 * x, r0, b * Hp + h);
       int last_use[BWQ_NS];
       for (int i = 0; i < BWQ_NS; ++i) last_use[i] = -1;
       for (int j = 0; j < nT; ++j) {
         const int st = j % BWQ_NS, use = j / BWQ_NS;
         if (use > 0 && !wait_bar(smem_u32(&S.kv_empty[st]), (use - 1) & 1, abort_flag, a.watch)) break;
-        const uint32_t kb = smem_u32(&S.k_full[st]), vb = smem_u32(&S.v_full[st]);
-        mbar_expect_tx(kb, QB * PF_KBOX);
-        for (int x = 0; x < QB; ++x)
-          tma_load_3d(smem_u32(S.k[st]) + x * PF_KBOX, tk, kb, 64 * x, j * PF_BN, b * a.Hkv + g);
-        mbar_expect_tx(vb, 2 * PF_KBOX);
-        tma_load_3d(smem_u32(S.v[st]), &tmV, vb, 0, j * PF_BN, b * a.Hkv + g);
-        tma_load_3d(smem_u32(S.v[st]) + PF_KBOX, &tmV, vb, 64, j * PF_BN, b * a.Hkv + g);
+        // the first tile into the Q / dO stage waits for their copy into TMEM
+        if (j == QO && !wait_bar(smem_u32(&S.qt_full), 0, abort_flag, a.watch)) break;
+        const uint32_t kb = smem_u32(&S.k_full[st]), vb = smem_u32(&S.v_full[st]), base = smem_u32(S.kv[st]);
+        mbar_expect_tx(kb, QB * PF_QBOX);
+        for (int x = 0; x < QB; ++x) tma_load_3d(base + x * PF_QBOX, tk, kb, 64 * x, j * BWQ_BN, b * a.Hkv + g);
+        mbar_expect_tx(vb, 2 * PF_QBOX);
+        for (int x = 0; x < 2; ++x) tma_load_3d(base + (2 + x) * PF_QBOX, &tmV, vb, 64 * x, j * BWQ_BN, b * a.Hkv + g);
         last_use[st] = use;
       }
       drain_bar(qb, 0, a.watch.status);
@@ -298,103 +311,129 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
-  } else if (warp >= 9) {
-    // --------------------------------------------------------- MMA issuers --
+  } else if (warp == 9) {
+    // ------------------------------------------------------- dQ issuer --
     if (lane == 0 && nT > 0) {
-      constexpr uint32_t HI = umma_desc_hi(1024);
-      constexpr uint32_t KSTAGE = (2 * PF_KBOX) >> 4;
-      const int issuer = warp - 9;   // 0: dQ += dS K, 1: S = Q K^T and dP = dO V^T
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 64 * QB, true);
+      const uint32_t ds_lo = umma_desc_lo(smem_u32(S.ds), 16);   // dS as the K-major A operand
       bool ok = true;
-      if (issuer == 0) {
-        constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 64 * QB, true);
-        const uint32_t k_mn0 = umma_desc_lo(smem_u32(S.k[0]), PF_KBOX);   // K as the N-major B operand
-        const uint32_t ds_lo0 = umma_desc_lo(smem_u32(S.ds[0]), 16);       // dS as the K-major A operand
-        for (int j = 0; ok && j < nT; ++j) {
-          const int bb = j & 1;
-          // this thread reads the K stage too: acquire it here
-          if (!(ok = wait_bar(smem_u32(&S.k_full[j % BWQ_NS]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
-          if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
-          tc_fence_after();
-          const uint32_t klo = k_mn0 + (uint32_t)(j % BWQ_NS) * KSTAGE;
-          const uint32_t dlo = ds_lo0 + (uint32_t)bb * (DS_BUF >> 4);
+      for (int j = 0; ok && j < nT; ++j) {
+        const int st = j % BWQ_NS;
+        // this thread reads the K stage too: acquire it here
+        if (!(ok = wait_bar(smem_u32(&S.k_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
+        if (!(ok = wait_bar(smem_u32(&S.p_full), j & 1, abort_flag, a.watch))) break;
+        tc_fence_after();
+        // K as the N-major B operand: keys down the rows, 64-wide dimension boxes PF_QBOX apart
+        const uint32_t klo = umma_desc_lo(smem_u32(S.kv[st]), PF_QBOX);
 #pragma unroll
-          for (int s = 0; s < PF_BN / 16; ++s)
-            mma_ss_w(tmem + 256, dlo + (uint32_t)(s * 2), HI, klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
-                     (j > 0 || s > 0));
-          mma_commit(smem_u32(&S.ds_free[bb]));
-          mma_commit(smem_u32(&S.kv_empty[j % BWQ_NS]));
+        for (int s = 0; s < BWQ_BN / 16; ++s) {   // dQ += dS K over the tile's 128 keys
+          const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+          mma_ss_w(tmem + T_DQ, ds_lo + ao, HI, klo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC, (j > 0 || s > 0));
         }
-        if (ok) mma_commit(smem_u32(&S.fin));
-      } else {
-        constexpr uint32_t IDESC_S = idesc_bf16_f32(128, PF_BN, false);
-        const uint32_t q_lo = umma_desc_lo(smem_u32(S.q), 16), o_lo = umma_desc_lo(smem_u32(S.o), 16);
-        const uint32_t k_lo0 = umma_desc_lo(smem_u32(S.k[0]), 16), v_lo0 = umma_desc_lo(smem_u32(S.v[0]), 16);
-        ok = wait_bar(smem_u32(&S.q_full), 0, abort_flag, a.watch);
-        for (int j = 0; ok && j < nT; ++j) {
-          const int bb = j & 1, st = j % BWQ_NS;
-          if (!(ok = wait_bar(smem_u32(&S.k_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
-          if (!(ok = wait_bar(smem_u32(&S.v_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
-          if (j >= 2 && !(ok = wait_bar(smem_u32(&S.s_free[bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch)))
-            break;
-          tc_fence_after();
-          const uint32_t klo = k_lo0 + (uint32_t)st * KSTAGE, vlo = v_lo0 + (uint32_t)st * KSTAGE;
-#pragma unroll
-          for (int s = 0; s < 4 * QB; ++s) {   // S = Q K^T over the QK width
-            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
-            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
-            mma_ss_w(tmem + bb * 64, q_lo + ao, HI, klo + bo, HI, IDESC_S, s > 0);
-          }
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {        // dP = dO V^T over the value width
-            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
-            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
-            mma_ss_w(tmem + 128 + bb * 64, o_lo + ao, HI, vlo + bo, HI, IDESC_S, s > 0);
-          }
-          mma_commit(smem_u32(&S.s_full[bb]));
-        }
+        mma_commit(smem_u32(&S.ds_free));
+        mma_commit(smem_u32(&S.kv_empty[st]));
       }
-      mma_commit(smem_u32(&S.drain[issuer]));
-      drain_bar(smem_u32(&S.drain[issuer]), 0, a.watch.status);
+      if (ok) mma_commit(smem_u32(&S.fin));
+      mma_commit(smem_u32(&S.drain[0]));
+      drain_bar(smem_u32(&S.drain[0]), 0, a.watch.status);
     }
-  } else {
+  } else if (warp == 10) {
+    // --------------------------------------------- S and dP issuer --
+    if (lane == 0 && nT > 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BWQ_BN, false);
+      bool ok = wait_bar(smem_u32(&S.qt_full), 0, abort_flag, a.watch);
+      for (int j = 0; ok && j < nT; ++j) {
+        const int st = j % BWQ_NS;
+        if (!(ok = wait_bar(smem_u32(&S.k_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
+        if (!(ok = wait_bar(smem_u32(&S.v_full[st]), (j / BWQ_NS) & 1, abort_flag, a.watch))) break;
+        // the one S / dP buffer: the elementwise warps have loaded tile j - 1's
+        if (j >= 1 && !(ok = wait_bar(smem_u32(&S.s_free), (j - 1) & 1, abort_flag, a.watch))) break;
+        tc_fence_after();
+        const uint32_t base = smem_u32(S.kv[st]);
+        const uint32_t klo = umma_desc_lo(base, 16), vlo = umma_desc_lo(base + 2 * PF_QBOX, 16);
+#pragma unroll
+        for (int s = 0; s < 4 * QB; ++s) {   // S = Q K^T over the QK width, Q from TMEM
+          const uint32_t bo = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+          mma_ts_w(tmem + T_S, tmem + T_Q + (uint32_t)(s * 8), klo + bo, HI, IDESC_S, s > 0);
+        }
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {        // dP = dO V^T over the value width, dO from TMEM
+          const uint32_t bo = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+          mma_ts_w(tmem + T_P, tmem + T_O + (uint32_t)(s * 8), vlo + bo, HI, IDESC_S, s > 0);
+        }
+        mma_commit(smem_u32(&S.s_full));
+      }
+      mma_commit(smem_u32(&S.drain[1]));
+      drain_bar(smem_u32(&S.drain[1]), 0, a.watch.status);
+    }
+  } else if (warp < 8) {
     // ------------------------------------------- elementwise (thread = row) --
     const int wq = warp & 3, ch = warp >> 2, r = threadIdx.x & 127;
     const int rg = r0 + r;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    // this thread's row of dS buffer 0: 128 bytes, its 16-byte chunks XOR-swizzled by row
-    const uint32_t ds_row = smem_u32(S.ds[0]) + (uint32_t)r * 128, sw = (uint32_t)(r & 7);
+    const uint32_t ds_base = smem_u32(S.ds);
     const size_t stat = (((size_t)b * Hp + h) * 2 + m) * a.Lp + rg;
     const float c = a.scale * (m == 0 ? 1.f : -a.lambda[h]);
     const float2 nl2 = make_float2(a.nlse[stat], a.nlse[stat]), nd2 = make_float2(a.ndd[stat], a.ndd[stat]);
     const float2 sl2 = make_float2(a.scale_log2, a.scale_log2), c2 = make_float2(c, c);
     const long long lastk = a.causal ? min((long long)a.Lk - 1, (long long)rg + (a.Lk - a.Lq)) : (long long)a.Lk - 1;
     bool ok = true;
-    for (int j = 0; j < nT; ++j) {
-      const int bb = j & 1;
-      if (!(ok = warp_wait(smem_u32(&S.s_full[bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
-      tc_fence_after();
-      uint32_t sv[32], pv[32], ds[16];
-      tmem_ld32p(tmem + lane_off + bb * 64 + ch * 32, sv);
-      tmem_ld32p(tmem + lane_off + 128 + bb * 64 + ch * 32, pv);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&S.s_free[bb]));   // in registers: S of tile j + 2 may overwrite them
-      const long long lim = lastk - (long long)j * PF_BN - ch * 32;   // columns > lim are masked
-      // warp-uniform: the warp runs one straight-line variant per tile
-      if (__all_sync(0xffffffffu, lim >= 31))
-        bw_q_elementwise<false>(sv, pv, ds, 0, sl2, nl2, nd2, c2);
-      else
-        bw_q_elementwise<true>(sv, pv, ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
-      // dS buffer bb is free once dQ of tile j - 2 has completed
-      if (j >= 2 && !(ok = warp_wait(smem_u32(&S.ds_free[bb]), ((j - 2) >> 1) & 1, abort_flag, a.watch))) break;
-      const uint32_t row_at = ds_row + (uint32_t)bb * DS_BUF;
+    if (nT > 0) {
+      // This row of Q (chunk 0's warps) or of dO (chunk 1's) into TMEM: each
+      // 64-element box row from its 128-byte-swizzled tile, two bf16 a column.
+      if ((ok = warp_wait(smem_u32(&S.q_full), 0, abort_flag, a.watch))) {
+        const uint8_t* tile = S.kv[QO] + (ch == 0 ? 0 : 2 * PF_QBOX);
+        const int nbox = ch == 0 ? QB : 2;
+        const uint32_t tdst = tmem + lane_off + (ch == 0 ? T_Q : T_O);
+        for (int x = 0; x < nbox; ++x) {
+          uint32_t wv[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)   // keys 32 ch + 8 q .. + 7: logical chunk 4 ch + q
-        sts_u4(row_at + ((((uint32_t)(4 * ch + q)) ^ sw) << 4), ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + x * PF_QBOX + r * 128 + ((cc ^ (r & 7)) << 4));
+            wv[4 * cc] = v.x; wv[4 * cc + 1] = v.y; wv[4 * cc + 2] = v.z; wv[4 * cc + 3] = v.w;
+          }
+          tmem_st32p(tdst + (uint32_t)(x * 32), wv);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        fence_proxy_async_smem();   // these reads come before the TMA writes of K/V tiles there
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S.qt_full));
+      }
+    }
+    for (int j = 0; ok && j < nT; ++j) {
+      if (!(ok = warp_wait(smem_u32(&S.s_full), j & 1, abort_flag, a.watch))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {   // the tile's two 64-key halves
+        uint32_t sv[32], pv[32], ds[16];
+        tmem_ld32p(tmem + lane_off + T_S + hh * 64 + ch * 32, sv);
+        tmem_ld32p(tmem + lane_off + T_P + hh * 64 + ch * 32, pv);
+        tmem_wait_ld();
+        if (hh == 1) {   // both halves are in registers: tile j + 1's products may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&S.s_free));
+        }
+        const long long lim = lastk - (long long)j * BWQ_BN - hh * 64 - ch * 32;   // columns > lim are masked
+        // warp-uniform: the warp runs one straight-line variant per half
+        if (__all_sync(0xffffffffu, lim >= 31))
+          bw_q_elementwise<false>(sv, pv, ds, 0, sl2, nl2, nd2, c2);
+        else
+          bw_q_elementwise<true>(sv, pv, ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
+        // the dS buffer is free once dQ of tile j - 1 has completed
+        if (hh == 0 && j >= 1 && !(ok = warp_wait(smem_u32(&S.ds_free), (j - 1) & 1, abort_flag, a.watch))) break;
+        // row r of box hh, keys 32 ch + 8 q .. + 7 of the box: logical chunk 4 ch + q
+        const uint32_t row_at = ds_base + (uint32_t)hh * PF_QBOX + (uint32_t)r * 128, sw = (uint32_t)(r & 7);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          sts_u4(row_at + ((((uint32_t)(4 * ch + q)) ^ sw) << 4), ds[4 * q], ds[4 * q + 1], ds[4 * q + 2],
+                 ds[4 * q + 3]);
+      }
+      if (!ok) break;
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&S.p_full[bb]));
+      if (lane == 0) mbar_arrive(smem_u32(&S.p_full));
     }
     // ---- epilogue: dQ rows ----
     bool have = nT == 0;
@@ -408,13 +447,14 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
         if (nT > 0) {
-          tmem_ld32p(tmem + lane_off + 256 + ch * 64 + cc * 32, o);
+          tmem_ld32p(tmem + lane_off + T_DQ + ch * 64 + cc * 32, o);
           tmem_wait_ld();
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) y[cc * 32 + i] = nT > 0 ? __uint_as_float(o[i]) : 0.f;
       }
-      pf_store_rows(S.ds[0] + warp * 16 * 128, y, base + ch * 64, r0 + wq * 32, a.Lq, lane, 64 * QB);
+      // staging: the dS buffer, free once every product has completed (or never used)
+      pf_store_rows(S.ds + warp * 16 * 128, y, base + ch * 64, r0 + wq * 32, a.Lq, lane, 64 * QB);
     }
   }
 

@@ -91,10 +91,9 @@ constexpr size_t bwd_dq_smem() { return sizeof(BwQSmem) + 1024; }
 constexpr size_t bwd_dkv_smem() { return sizeof(BwKSmem) + 1024; }
 static_assert(bwd_dq_smem() <= 227 * 1024 && bwd_dkv_smem() <= 227 * 1024,
               "backward shared memory above the 227 KB a block may use");
-// each dS buffer holds 128 rows of 64 bf16 keys (128 bytes), and buffer 0
-// also the epilogue's staging (8 warps x 16 rows x 128 bytes)
-static_assert(sizeof(BwQSmem::ds[0]) == 128 * 128 && sizeof(BwQSmem::ds[0]) >= 8 * 16 * 128,
-              "dS buffer size");
+// the dS buffer holds 128 rows of 128 bf16 keys as two 16 KB boxes, and also
+// the epilogue's staging (8 warps x 16 rows x 128 bytes)
+static_assert(sizeof(BwQSmem::ds) == 2 * 128 * 128 && sizeof(BwQSmem::ds) >= 8 * 16 * 128, "dS buffer size");
 constexpr int kDecCtasPerSm = 2;
 
 // Per-device set-up: SM count, status word address, kernel attributes,
@@ -395,9 +394,9 @@ int launch_backward(const void* q, const void* q2, const void* k, const void* k2
     if (int e = make_map(&mq, q, w, Lq_map, zq, PF_BM)) return e;
     if (int e = make_map(&mq2, q2, w, Lq_map, zq, PF_BM)) return e;
     if (int e = make_map(&mo, dout, 128, Lq_map, (long long)B * Hp, PF_BM)) return e;
-    if (int e = make_map(&mk, Lk > 0 ? k : q, w, Lk_map, (long long)B * Hkv, PF_BN)) return e;
-    if (int e = make_map(&mk2, Lk > 0 ? k2 : q, w, Lk_map, (long long)B * Hkv, PF_BN)) return e;
-    if (int e = make_map(&mv, Lk > 0 ? v : dout, 128, Lk_map, (long long)B * Hkv, PF_BN)) return e;
+    if (int e = make_map(&mk, Lk > 0 ? k : q, w, Lk_map, (long long)B * Hkv, BWQ_BN)) return e;
+    if (int e = make_map(&mk2, Lk > 0 ? k2 : q, w, Lk_map, (long long)B * Hkv, BWQ_BN)) return e;
+    if (int e = make_map(&mv, Lk > 0 ? v : dout, 128, Lk_map, (long long)B * Hkv, BWQ_BN)) return e;
     const long long units = (long long)((Lq + PF_BM - 1) / PF_BM) * B * Hq;
     if (v1)
       bwd_dq_kernel<true><<<(unsigned)units, BW_THREADS, bwd_dq_smem(), s>>>(mq, mq2, mo, mk, mk2, mv, a);
