@@ -404,23 +404,27 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     for (int j = 0; ok && j < nT; ++j) {
       if (!(ok = warp_wait(smem_u32(&S.s_full), j & 1, abort_flag, a.watch))) break;
       tc_fence_after();
+      // both halves into registers at once, then the buffer is released:
+      // tile j + 1's products overlap all of this tile's arithmetic
+      uint32_t sv[2][32], pv[2][32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32p(tmem + lane_off + T_S + hh * 64 + ch * 32, sv[hh]);
+        tmem_ld32p(tmem + lane_off + T_P + hh * 64 + ch * 32, pv[hh]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.s_free));
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {   // the tile's two 64-key halves
-        uint32_t sv[32], pv[32], ds[16];
-        tmem_ld32p(tmem + lane_off + T_S + hh * 64 + ch * 32, sv);
-        tmem_ld32p(tmem + lane_off + T_P + hh * 64 + ch * 32, pv);
-        tmem_wait_ld();
-        if (hh == 1) {   // both halves are in registers: tile j + 1's products may overwrite them
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&S.s_free));
-        }
+        uint32_t ds[16];
         const long long lim = lastk - (long long)j * BWQ_BN - hh * 64 - ch * 32;   // columns > lim are masked
         // warp-uniform: the warp runs one straight-line variant per half
         if (__all_sync(0xffffffffu, lim >= 31))
-          bw_q_elementwise<false>(sv, pv, ds, 0, sl2, nl2, nd2, c2);
+          bw_q_elementwise<false>(sv[hh], pv[hh], ds, 0, sl2, nl2, nd2, c2);
         else
-          bw_q_elementwise<true>(sv, pv, ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
+          bw_q_elementwise<true>(sv[hh], pv[hh], ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
         // the dS buffer is free once dQ of tile j - 1 has completed
         if (hh == 0 && j >= 1 && !(ok = warp_wait(smem_u32(&S.ds_free), (j - 1) & 1, abort_flag, a.watch))) break;
         // row r of box hh, keys 32 ch + 8 q .. + 7 of the box: logical chunk 4 ch + q
