@@ -29,10 +29,12 @@
 //                    warps have loaded it, so the products of tile j + 1 run
 //                    while tile j's elementwise phase does.
 //   bwd_dkv_kernel   key-stationary: one CTA per 128 keys of one KV head.  Per
-//                    64-row step of each Q head of the group: S^T = K Q^T and
-//                    dP^T = V dO^T into TMEM, then w P^T (w = 1 or -lambda)
-//                    and dS^T written back as bf16, and dV += (w P)^T dO,
-//                    dK += dS^T Q with those as the TMEM operands.
+//                    64-row block, the two maps of each diff pair of the
+//                    group in turn: S_m^T = K Q_m^T into TMEM, and once per
+//                    pair dP^T = V dO^T (the maps share dO).  dS_m^T and
+//                    (P_1 - lambda P_2)^T are written back as bf16, and
+//                    dK += dS_m^T Q_m, dV += (P_1 - lambda P_2)^T dO take
+//                    them as the TMEM operands.
 // Computing dQ apart from dK/dV recomputes S and dP once more but needs no
 // atomics, and each kernel fits TMEM (512 columns each).
 // Both MMA kernels use the forward's pipeline: a TMA producer warp, one
@@ -71,11 +73,12 @@ struct BwdArgs {
   int B, Hq, Hkv, Lq, Lk, Lp;
   int causal;
   float scale, scale_log2;
-  // Heads with |1 - lambda| < resid_tau keep the bf16 residual of w P and of
-  // dS in the key-stationary kernel (a second MMA for dV and for dK): with
-  // alike maps, dV = sum (A_1 - lambda A_2)^T dO and dK = sum dS_m^T Q_m
-  // cancel, and the separate bf16 roundings of the two maps' operands would be
-  // amplified as in the forward.
+  // V2 heads with |1 - lambda| < resid_tau keep the bf16 residual of dS in
+  // the key-stationary kernel (a second MMA for dK): with alike maps the sum
+  // dK = sum over the pair's maps of dS_m^T Q_m cancels, and the separate bf16
+  // roundings of the two maps' operands would be amplified as in the forward.
+  // dV needs none: its operand is (P_1 - lambda P_2)^T, formed in f32 and
+  // rounded once.  V1 keeps dK_1 and dK_2 apart, so it needs none either.
   float resid_tau;
   Watch watch;
 };
@@ -494,10 +497,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
-// One step of the key-stationary kernel for this thread's key and this warp's
-// 32-row chunk: from S^T and dP^T (the chunk's columns at tS, tP) write w P^T
-// and dS^T back as bf16 into the chunk's first 16 columns and, with RESID,
-// their bf16 residuals into its next 16.
 // 16-byte load from shared memory (addr: a shared-window address).
 __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   float4 v;
@@ -505,57 +504,97 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   return v;
 }
 
-// nl_s, nd_s: shared-window addresses of the chunk's 32 negated log-sum-exp
-// and D values (one per row, the same for every key), read as 16-byte vectors
-// half a chunk at a time.  The arithmetic runs on f32x2 pairs (each operation
-// rounds as its scalar form would).  vis0: the first visible column (0..32);
-// with MASK, columns before it give P = 0.
+// The stage's 16 negated log-sum-exp and D values of half h of a 32-row chunk
+// (one per row, the same for every key), as f32 pairs.
+__device__ __forceinline__ void bw_kv_stats(uint32_t nl_s, uint32_t nd_s, int h, float2 (&nl)[8], float2 (&nd)[8]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 l4 = lds_f4(nl_s + (uint32_t)((h * 16 + q * 4) * 4));
+    const float4 d4 = lds_f4(nd_s + (uint32_t)((h * 16 + q * 4) * 4));
+    nl[2 * q] = make_float2(l4.x, l4.y); nl[2 * q + 1] = make_float2(l4.z, l4.w);
+    nd[2 * q] = make_float2(d4.x, d4.y); nd[2 * q + 1] = make_float2(d4.z, d4.w);
+  }
+}
+
+// The two steps of a diff pair in the key-stationary kernel, for this
+// thread's key and this warp's 32-row chunk.  The pair's maps share dO, so
+// dP^T = V dO^T is computed once, in the map-1 step, and the map-2 step takes
+// it from registers; P_1 waits there too, so that dV's operand is the
+// difference (P_1 - lambda P_2)^T formed in f32 and rounded once.  The
+// arithmetic runs on f32x2 pairs (each operation rounds as its scalar form
+// would).  vis0: the first visible row of the chunk (0..32); with MASK, rows
+// before it give P = 0.  With RESID, dS^T's bf16 residual goes 16 columns
+// after its hi part.
+//
+// Map 1: from S_1^T (tS) and dP^T (tP) write dS_1^T = c P_1 (dP - D_1) back
+// over S_1^T, and keep P_1 and dP.
 template <bool RESID, bool MASK>
-__device__ __forceinline__ void bw_kv_elementwise(uint32_t tS, uint32_t tP, int vis0, float2 w2, float2 cd2, float2 sl2,
-                                                  uint32_t nl_s, uint32_t nd_s) {
-  uint32_t sv[32], pv[32], pw[16], ds[16];
+__device__ __forceinline__ void bw_kv_map1(uint32_t tS, uint32_t tP, int vis0, float2 cd2, float2 sl2, uint32_t nl_s,
+                                           uint32_t nd_s, float2 (&p1)[16], float2 (&dp)[16]) {
+  uint32_t sv[32], pv[32], ds[16];
   tmem_ld32p(tS, sv);
   tmem_ld32p(tP, pv);
   tmem_wait_ld();
-  uint32_t rpw[RESID ? 16 : 1], rds[RESID ? 16 : 1];
+  uint32_t rds[RESID ? 16 : 1];
   const float2 neg1 = make_float2(-1.f, -1.f);
   float2 nl[8], nd[8];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    if ((j & 7) == 0) {   // this half's 16 values of each
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 l4 = lds_f4(nl_s + (uint32_t)((j * 2 + q * 4) * 4));
-        const float4 d4 = lds_f4(nd_s + (uint32_t)((j * 2 + q * 4) * 4));
-        nl[2 * q] = make_float2(l4.x, l4.y); nl[2 * q + 1] = make_float2(l4.z, l4.w);
-        nd[2 * q] = make_float2(d4.x, d4.y); nd[2 * q + 1] = make_float2(d4.z, d4.w);
-      }
-    }
+    if ((j & 7) == 0) bw_kv_stats(nl_s, nd_s, j >> 3, nl, nd);
     float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sl2, nl[j & 7]);
     if (MASK) {
       if (2 * j < vis0) x.x = -INFINITY;
       if (2 * j + 1 < vis0) x.y = -INFINITY;
     }
     const float2 p = make_float2(ex2(x.x), ex2(x.y));
-    const float2 p2 = __fmul2_rn(w2, p);
-    const float2 t = __fadd2_rn(make_float2(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1])), nd[j & 7]);
-    const float2 d2 = __fmul2_rn(__fmul2_rn(cd2, p), t);
-    pw[j] = pack_bf16(p2.x, p2.y);
+    p1[j] = p;
+    dp[j] = make_float2(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1]));
+    const float2 d2 = __fmul2_rn(__fmul2_rn(cd2, p), __fadd2_rn(dp[j], nd[j & 7]));
     ds[j] = pack_bf16(d2.x, d2.y);
     if constexpr (RESID) {   // x - bf16(x), exact in f32
-      const float2 ph = make_float2(__uint_as_float(pw[j] << 16), __uint_as_float(pw[j] & 0xFFFF0000u));
       const float2 dh = make_float2(__uint_as_float(ds[j] << 16), __uint_as_float(ds[j] & 0xFFFF0000u));
-      const float2 rp = __ffma2_rn(ph, neg1, p2), rd = __ffma2_rn(dh, neg1, d2);
-      rpw[j] = pack_bf16(rp.x, rp.y);
+      const float2 rd = __ffma2_rn(dh, neg1, d2);
       rds[j] = pack_bf16(rd.x, rd.y);
     }
   }
-  tmem_st16p(tS, pw);
-  tmem_st16p(tP, ds);
-  if constexpr (RESID) {
-    tmem_st16p(tS + 16, rpw);
-    tmem_st16p(tP + 16, rds);
+  tmem_st16p(tS, ds);
+  if constexpr (RESID) tmem_st16p(tS + 16, rds);
+}
+
+// Map 2: from S_2^T (tS) and the map-1 step's P_1 and dP, write
+// (P_1 - lambda P_2)^T over S_2^T and dS_2^T = c P_2 (dP - D_2) at tD.
+template <bool RESID, bool MASK>
+__device__ __forceinline__ void bw_kv_map2(uint32_t tS, uint32_t tD, int vis0, float2 nlam2, float2 cd2, float2 sl2,
+                                           uint32_t nl_s, uint32_t nd_s, const float2 (&p1)[16],
+                                           const float2 (&dp)[16]) {
+  uint32_t sv[32], cw[16], ds[16];
+  tmem_ld32p(tS, sv);
+  tmem_wait_ld();
+  uint32_t rds[RESID ? 16 : 1];
+  const float2 neg1 = make_float2(-1.f, -1.f);
+  float2 nl[8], nd[8];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if ((j & 7) == 0) bw_kv_stats(nl_s, nd_s, j >> 3, nl, nd);
+    float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sl2, nl[j & 7]);
+    if (MASK) {
+      if (2 * j < vis0) x.x = -INFINITY;
+      if (2 * j + 1 < vis0) x.y = -INFINITY;
+    }
+    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+    const float2 c = __ffma2_rn(nlam2, p, p1[j]);
+    cw[j] = pack_bf16(c.x, c.y);
+    const float2 d2 = __fmul2_rn(__fmul2_rn(cd2, p), __fadd2_rn(dp[j], nd[j & 7]));
+    ds[j] = pack_bf16(d2.x, d2.y);
+    if constexpr (RESID) {
+      const float2 dh = make_float2(__uint_as_float(ds[j] << 16), __uint_as_float(ds[j] & 0xFFFF0000u));
+      const float2 rd = __ffma2_rn(dh, neg1, d2);
+      rds[j] = pack_bf16(rd.x, rd.y);
+    }
   }
+  tmem_st16p(tS, cw);
+  tmem_st16p(tD, ds);
+  if constexpr (RESID) tmem_st16p(tD + 16, rds);
 }
 
 // V1: as for bwd_dq_kernel.  The CTA holds K1 and K2 side by side in its
@@ -618,7 +657,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = S.tmem_base;   // S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512)
+  // TMEM: S_1^T [0,64), S_2^T [64,128), dP^T [128,192), dS_2^T [192,256), dV [256,384), dK [384,512)
+  const uint32_t tmem = S.tmem_base;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
@@ -666,8 +706,10 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         for (int i = 0; ok && i < nS; ++i) {
           const int bb = i & 1, st = i % BW_NS;
           const int qh = step_head(i);
-          // read before the waits, so the load is not on the issue path
-          const bool resid = fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
+          // dK's residual: V2 sums dK over the pair's maps, which cancel when
+          // they are alike; V1 keeps dK_1 and dK_2 apart.  lambda is read
+          // before the waits, so its load is not on the issue path.
+          const bool resid = !V1 && fabsf(1.f - a.lambda[qh / 2]) < a.resid_tau;
           // this thread reads the stage's Q and dO too: acquire them here
           if (!(ok = wait_bar(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
           if (!(ok = wait_bar(smem_u32(&S.p_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
@@ -676,34 +718,32 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           // V1: map m's dK lives in its own 64 columns and first receives a
           // value at step m (steps 0 and 1 are the two maps of the group's
           // first head); V2: one dK for both maps
-          const uint32_t dk_t = tmem + 384 + (V1 ? (uint32_t)((qh & 1) * 64) : 0u);
+          const uint32_t dk_t = tmem + 384 + (V1 ? (uint32_t)(bb * 64) : 0u);
           const bool dk_acc = V1 ? i > 1 : i > 0;
-          // dV += (w P)^T dO, with the bf16 residual 16 columns after each
-          // chunk's hi part; then S^T of step i + 2 may overwrite buffer bb
+          // map 1: dS_1^T over S_1^T at [0, 64); map 2: (P_1 - lambda P_2)^T
+          // over S_2^T at [64, 128) and dS_2^T at [192, 256)
+          const uint32_t ds_t = tmem + (bb ? 192u : 0u);
+          if (bb) {
+            // dV += (P_1 - lambda P_2)^T dO; then S_2^T of the next pair may
+            // overwrite [64, 128)
+#pragma unroll
+            for (int s = 0; s < BW_RB / 16; ++s)
+              mma_ts_w(tmem + 256, tmem + 64 + bw_slice(s), olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
+                       (i > 1 || s > 0));
+            mma_commit(smem_u32(&S.sv_free[1]));
+          }
+          // dK += dS_m^T Q_m and its residual
 #pragma unroll
           for (int s = 0; s < BW_RB / 16; ++s)
-            mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s), olo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_ACC,
-                     (i > 0 || s > 0));
+            mma_ts_w(dk_t, ds_t + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_DK, (dk_acc || s > 0));
           if (resid) {
 #pragma unroll
             for (int s = 0; s < BW_RB / 16; ++s)
-              mma_ts_w(tmem + 256, tmem + bb * 64 + bw_slice(s) + 16, olo + (uint32_t)(s * (2048 >> 4)), HI,
-                       IDESC_ACC, 1);
+              mma_ts_w(dk_t, ds_t + bw_slice(s) + 16, qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_DK, 1);
           }
-          mma_commit(smem_u32(&S.sv_free[bb]));
-          // dK += dS^T Q and its residual; then dP^T of step i + 2 may
-          // overwrite buffer bb, and the stage is free
-#pragma unroll
-          for (int s = 0; s < BW_RB / 16; ++s)
-            mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s), qlo + (uint32_t)(s * (2048 >> 4)), HI, IDESC_DK,
-                     (dk_acc || s > 0));
-          if (resid) {
-#pragma unroll
-            for (int s = 0; s < BW_RB / 16; ++s)
-              mma_ts_w(dk_t, tmem + 128 + bb * 64 + bw_slice(s) + 16, qlo + (uint32_t)(s * (2048 >> 4)), HI,
-                       IDESC_DK, 1);
-          }
-          mma_commit(smem_u32(&S.sd_free[bb]));
+          // map 1: the next pair's S_1^T and dP^T may overwrite [0, 64) and
+          // [128, 192); map 2: its dS_2^T may overwrite [192, 256)
+          mma_commit(smem_u32(bb ? &S.sd_free[1] : &S.sv_free[0]));
           mma_commit(smem_u32(&S.st_empty[st]));
         }
         if (ok) mma_commit(smem_u32(&S.fin));
@@ -715,28 +755,33 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         for (int i = 0; ok && i < nS; ++i) {
           const int bb = i & 1, st = i % BW_NS;
           if (!(ok = wait_bar(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
-          // S^T(i) overwrites what dV(i - 2) read, dP^T(i) what dK(i - 2)
-          // read: each waits for its own reader
+          // S_m^T(i) overwrites what the accumulating products of step i - 2
+          // read (dK_1 for map 1, dV for map 2)
           if (i >= 2 && !(ok = wait_bar(smem_u32(&S.sv_free[bb]), ((i - 2) >> 1) & 1, abort_flag, a.watch)))
             break;
           tc_fence_after();
           const uint32_t qlo = q_lo0 + (uint32_t)st * QSTAGE, olo = o_lo0 + (uint32_t)st * QSTAGE;
           // V1: the step's map m scores against K_m, box m of the K tile
-          const uint32_t kmo = V1 ? (uint32_t)((step_head(i) & 1) * (PF_QBOX >> 4)) : 0u;
+          const uint32_t kmo = V1 ? (uint32_t)(bb * (PF_QBOX >> 4)) : 0u;
 #pragma unroll
           for (int s = 0; s < 4 * QB; ++s) {   // S^T = K Q^T over the QK width
             const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
             const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
             mma_ss_w(tmem + bb * 64, k_lo + kmo + ao, HI, qlo + bo, HI, IDESC_S, s > 0);
           }
-          if (i >= 2 && !(ok = wait_bar(smem_u32(&S.sd_free[bb]), ((i - 2) >> 1) & 1, abort_flag, a.watch)))
-            break;
-          tc_fence_after();
+          if (bb == 0) {
+            // dP^T = V dO^T, once per pair, into [128, 192): the elementwise
+            // warps loaded it at step i - 2, before dK_1(i - 2) (sv_free[0])
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
-            const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
-            mma_ss_w(tmem + 128 + bb * 64, v_lo + ao, HI, olo + bo, HI, IDESC_S, s > 0);
+            for (int s = 0; s < 8; ++s) {
+              const uint32_t ao = (uint32_t)((s >> 2) * (PF_QBOX >> 4) + (s & 3) * 2);
+              const uint32_t bo = (uint32_t)((s >> 2) * (PF_KBOX >> 4) + (s & 3) * 2);
+              mma_ss_w(tmem + 128, v_lo + ao, HI, olo + bo, HI, IDESC_S, s > 0);
+            }
+          } else if (i >= 3 && !(ok = wait_bar(smem_u32(&S.sd_free[1]), ((i - 2) >> 1) & 1, abort_flag, a.watch))) {
+            // map 2's elementwise step writes dS_2^T over [192, 256), which
+            // dK_2(i - 2) read: the commit below follows this wait
+            break;
           }
           mma_commit(smem_u32(&S.s_full[bb]));
         }
@@ -751,15 +796,15 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     bool ok = true;
+    float2 p1[16], dp[16];   // P_1 and dP of this thread's key and chunk, from the map-1 step to the map-2 step
     for (int i = 0; i < nS; ++i) {
+      // the group's heads are innermost and come in pairs, so step i is map
+      // i & 1 of a pair, and steps 2k, 2k + 1 share their rows
       const int bb = i & 1, st = i % BW_NS;
       const int qh = step_head(i), rb = step_rb(i);
-      const int mq = qh & 1;
       // lambda read once, before the waits, so its load is not on the step's path
       const float lam = a.lambda[qh / 2];
-      const float w = mq == 0 ? 1.f : -lam;   // weight of this map in A_1 - lambda A_2
-      const bool resid = fabsf(1.f - lam) < a.resid_tau;
-      const float2 w2 = make_float2(w, w), cd2 = make_float2(a.scale * w, a.scale * w);
+      const bool resid = !V1 && fabsf(1.f - lam) < a.resid_tau;
       // The stage's log-sum-exp and D values came by bulk copy: wait for them here too.
       if (!(ok = warp_wait(smem_u32(&S.st_full[st]), (i / BW_NS) & 1, abort_flag, a.watch))) break;
       if (!(ok = warp_wait(smem_u32(&S.s_full[bb]), (i >> 1) & 1, abort_flag, a.watch))) break;
@@ -767,17 +812,29 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       // rows r = rb*64 + col see this key iff kg < Lk and (not causal or kg <= r + off)
       const int row0 = rb * BW_RB + ch * 32;
       const int vis0 = kg >= a.Lk ? 32 : (a.causal ? min(32, max(0, kg - off - row0)) : 0);
-      const uint32_t tS = tmem + lane_off + bb * 64 + ch * 32, tP = tmem + lane_off + 128 + bb * 64 + ch * 32;
       // branch once per step, warp-uniformly (the TMEM stores inside are
       // warp-collective): each variant's loop is one straight-line block
       const bool full = __all_sync(0xffffffffu, vis0 == 0);
       const uint32_t nl_s = smem_u32(S.nlse[st] + ch * 32), nd_s = smem_u32(S.ndd[st] + ch * 32);
-      if (resid) {
-        if (full) bw_kv_elementwise<true, false>(tS, tP, 0, w2, cd2, sl2, nl_s, nd_s);
-        else bw_kv_elementwise<true, true>(tS, tP, vis0, w2, cd2, sl2, nl_s, nd_s);
+      const uint32_t t0 = tmem + lane_off + ch * 32;
+      if (bb == 0) {
+        const float2 cd2 = make_float2(a.scale, a.scale);
+        if (resid) {
+          if (full) bw_kv_map1<true, false>(t0, t0 + 128, 0, cd2, sl2, nl_s, nd_s, p1, dp);
+          else bw_kv_map1<true, true>(t0, t0 + 128, vis0, cd2, sl2, nl_s, nd_s, p1, dp);
+        } else {
+          if (full) bw_kv_map1<false, false>(t0, t0 + 128, 0, cd2, sl2, nl_s, nd_s, p1, dp);
+          else bw_kv_map1<false, true>(t0, t0 + 128, vis0, cd2, sl2, nl_s, nd_s, p1, dp);
+        }
       } else {
-        if (full) bw_kv_elementwise<false, false>(tS, tP, 0, w2, cd2, sl2, nl_s, nd_s);
-        else bw_kv_elementwise<false, true>(tS, tP, vis0, w2, cd2, sl2, nl_s, nd_s);
+        const float2 nlam2 = make_float2(-lam, -lam), cd2 = make_float2(-a.scale * lam, -a.scale * lam);
+        if (resid) {
+          if (full) bw_kv_map2<true, false>(t0 + 64, t0 + 192, 0, nlam2, cd2, sl2, nl_s, nd_s, p1, dp);
+          else bw_kv_map2<true, true>(t0 + 64, t0 + 192, vis0, nlam2, cd2, sl2, nl_s, nd_s, p1, dp);
+        } else {
+          if (full) bw_kv_map2<false, false>(t0 + 64, t0 + 192, 0, nlam2, cd2, sl2, nl_s, nd_s, p1, dp);
+          else bw_kv_map2<false, true>(t0 + 64, t0 + 192, vis0, nlam2, cd2, sl2, nl_s, nd_s, p1, dp);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
