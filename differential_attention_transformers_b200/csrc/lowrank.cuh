@@ -211,23 +211,52 @@ __host__ __device__ inline void lr_emit_range(const LowrankArgs& a, int c, long 
   k1 = a.causal ? lr_clamp(r1 + off, a.Lk) : 0;
 }
 
+// Slot of row chunk c of head bh: the prefix sums the chunk starts from.
+__host__ __device__ inline size_t lr_emit_slot(const LowrankArgs& a, int c, int bh) {
+  return (size_t)bh * (a.nc + 1) + (a.causal ? a.n_lead + c : a.nc);
+}
+
+// The key row i of a causal chunk adds (its G row at gk + (key - k0) LR_RMAX),
+// or -1 when it adds none.
+__host__ __device__ inline long long lr_row_key(const LowrankArgs& a, long long i, long long r1) {
+  const long long j = i + ((long long)a.Lk - a.Lq);
+  return (a.causal && i < r1 && j >= 0 && j < a.Lk) ? j : -1;
+}
+
+// The row normaliser of row chunk c of head bh, serially: rd[i - r0] =
+// 1 / (f_i . z_i), or 0 when that is not positive, with z_i = the chunk's
+// starting z plus the G rows of the keys rows r0..i add.  fk, gk as for
+// lr_emit_body.  (The kernel forms the same sums in parallel, lr_emit_norm.)
+__host__ __device__ inline void lr_emit_norm_serial(const LowrankArgs& a, int c, int bh, const float* fk,
+                                                    const float* gk, float* rd) {
+  const size_t slot = lr_emit_slot(a, c, bh);
+  long long r0, r1, k0, k1;
+  lr_emit_range(a, c, r0, r1, k0, k1);
+  float z[LR_RMAX];
+  for (int t = 0; t < LR_RMAX; ++t) z[t] = t < a.r ? a.ztot[slot * a.r + t] : 0.f;
+  for (long long i = r0; i < r1; ++i) {
+    const long long j = lr_row_key(a, i, r1);
+    if (j >= 0)
+      for (int t = 0; t < LR_RMAX; ++t) z[t] += gk[(j - k0) * LR_RMAX + t];
+    float den = 0.f;
+    for (int t = 0; t < LR_RMAX; ++t) den = fmaf(fk[(i - r0) * LR_RMAX + t], z[t], den);
+    rd[i - r0] = den > 0.f ? 1.f / den : 0.f;
+  }
+}
+
 // Row chunk c (rows [r0, r1)) of head bh, value column col.  fk: the padded F
 // rows of the chunk, row i - r0 at fk + (i - r0) LR_RMAX; gk: the padded G
 // rows of the keys the rows add, row j - k0 at gk + (j - k0) LR_RMAX
-// (lr_emit_range).
+// (lr_emit_range); rd: the chunk's row normalisers (lr_emit_norm_serial).
 __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh, int col, const float* fk,
-                                             const float* gk) {
+                                             const float* gk, const float* rd) {
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
-  const size_t slot = (size_t)bh * (a.nc + 1) + (a.causal ? a.n_lead + c : a.nc);
-  float S[LR_RMAX], z[LR_RMAX];
+  const size_t slot = lr_emit_slot(a, c, bh);
+  float S[LR_RMAX];
 #pragma unroll
-  for (int t = 0; t < LR_RMAX; ++t) {
-    S[t] = t < a.r ? a.tot[(slot * a.r + t) * LR_DV + col] : 0.f;
-    z[t] = t < a.r ? a.ztot[slot * a.r + t] : 0.f;
-  }
+  for (int t = 0; t < LR_RMAX; ++t) S[t] = t < a.r ? a.tot[(slot * a.r + t) * LR_DV + col] : 0.f;
   long long r0, r1, k0, k1;
   lr_emit_range(a, c, r0, r1, k0, k1);
-  const long long off = (long long)a.Lk - a.Lq;
   const __nv_bfloat16* vcol = a.v + ((size_t)b * a.Hkv + g) * (size_t)a.Lk * LR_DV + col;
   const float lam = a.lambda[h];
   const float* arow = a.a1v + (size_t)bh * a.Lq * LR_DV + col;
@@ -240,9 +269,9 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
   auto load = [&](long long i0, float (&A)[U], float (&W)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const long long i = i0 + u, j = i + off;
+      const long long i = i0 + u, j = lr_row_key(a, i, r1);
       A[u] = i < r1 ? arow[i * LR_DV] : 0.f;
-      W[u] = (a.causal && i < r1 && j >= 0 && j < a.Lk) ? __bfloat162float(vcol[j * LR_DV]) : 0.f;
+      W[u] = j >= 0 ? __bfloat162float(vcol[j * LR_DV]) : 0.f;
     }
   };
   load(r0, av, vj);
@@ -250,27 +279,20 @@ __host__ __device__ inline void lr_emit_body(const LowrankArgs& a, int c, int bh
     load(i0 + U, an, vn);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const long long i = i0 + u, j = i + off;
+      const long long i = i0 + u, j = lr_row_key(a, i, r1);
       if (i >= r1) break;
-      if (a.causal && j >= 0 && j < a.Lk) {
+      if (j >= 0) {
         float gj[LR_RMAX];
         lr_row(gk + (j - k0) * LR_RMAX, gj);
 #pragma unroll
-        for (int t = 0; t < LR_RMAX; ++t) {
-          S[t] = fmaf(gj[t], vj[u], S[t]);
-          z[t] += gj[t];
-        }
+        for (int t = 0; t < LR_RMAX; ++t) S[t] = fmaf(gj[t], vj[u], S[t]);
       }
       float fi[LR_RMAX];
       lr_row(fk + (i - r0) * LR_RMAX, fi);
-      float num = 0.f, den = 0.f;
+      float num = 0.f;
 #pragma unroll
-      for (int t = 0; t < LR_RMAX; ++t) {
-        num = fmaf(fi[t], S[t], num);
-        den = fmaf(fi[t], z[t], den);
-      }
-      const float nv = den > 0.f ? num / den : 0.f;
-      orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * nv);
+      for (int t = 0; t < LR_RMAX; ++t) num = fmaf(fi[t], S[t], num);
+      orow[i * LR_DV] = __float2bfloat16_rn(av[u] - lam * (num * rd[i - r0]));
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -298,18 +320,57 @@ __global__ void __launch_bounds__(LR_DV) lr_totals_kernel(LowrankArgs a) {
 __global__ void __launch_bounds__(LR_DV) lr_prefix_kernel(LowrankArgs a) {
   lr_prefix_body(a, (int)blockIdx.y, (int)blockIdx.x, (int)threadIdx.x);
 }
-// Six CTAs per SM: the 32 KB of staged factor rows allow no more, and the
-// register budget keeps the prefetched group within it.
+// The row normalisers of a chunk (as lr_emit_norm_serial), by the CTA's 128
+// threads: thread t takes rank component t % 16 of the rows in segment t / 16
+// (LR_C / 8 rows each).  The segments' sums of the added G rows go to seg;
+// each thread then runs its component's prefix down its segment, and the 16
+// threads of a segment (a half-warp) add their f_i[t] z_i[t] by shuffles.
+// Every lane runs the same trip count, so the shuffles are warp-uniform.
+constexpr int LR_SEGS = LR_DV / LR_RMAX;
+constexpr int LR_SEG_ROWS = LR_C / LR_SEGS;
+static_assert(LR_SEGS * LR_RMAX == LR_DV && LR_SEG_ROWS * LR_SEGS == LR_C, "normaliser thread layout");
+__device__ __forceinline__ void lr_emit_norm(const LowrankArgs& a, int c, int bh, const float* fk, const float* gk,
+                                             float* rd, float (*seg)[LR_RMAX]) {
+  const int t = (int)threadIdx.x, q = t % LR_RMAX, sg = t / LR_RMAX;
+  long long r0, r1, k0, k1;
+  lr_emit_range(a, c, r0, r1, k0, k1);
+  const long long i_beg = r0 + (long long)sg * LR_SEG_ROWS;
+  float part = 0.f;
+  for (int u = 0; u < LR_SEG_ROWS; ++u) {
+    const long long j = lr_row_key(a, i_beg + u, r1);
+    if (j >= 0) part += gk[(j - k0) * LR_RMAX + q];
+  }
+  seg[sg][q] = part;
+  __syncthreads();
+  const size_t slot = lr_emit_slot(a, c, bh);
+  float z = q < a.r ? a.ztot[slot * a.r + q] : 0.f;
+  for (int s2 = 0; s2 < sg; ++s2) z += seg[s2][q];
+  for (int u = 0; u < LR_SEG_ROWS; ++u) {
+    const long long i = i_beg + u, j = lr_row_key(a, i, r1);
+    if (j >= 0) z += gk[(j - k0) * LR_RMAX + q];
+    float p = i < r1 ? fk[(i - r0) * LR_RMAX + q] * z : 0.f;
+#pragma unroll
+    for (int o = LR_RMAX / 2; o >= 1; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+    if (q == 0 && i < r1) rd[i - r0] = p > 0.f ? 1.f / p : 0.f;
+  }
+  __syncthreads();
+}
+
+// Six CTAs per SM: the 33.5 KB of staged factor rows and normalisers allow no
+// more, and the register budget keeps the prefetched group within it.
 __global__ void __launch_bounds__(LR_DV, 6) lr_emit_kernel(LowrankArgs a) {
   __shared__ alignas(16) float sf[LR_C * LR_RMAX];
   __shared__ alignas(16) float sg[LR_C * LR_RMAX];
+  __shared__ float srd[LR_C];
+  __shared__ float sseg[LR_SEGS][LR_RMAX];
   const int c = (int)blockIdx.x, bh = (int)blockIdx.y, h = bh % a.H;
   long long r0, r1, k0, k1;
   lr_emit_range(a, c, r0, r1, k0, k1);
   for (long long e = threadIdx.x; e < (r1 - r0) * LR_RMAX; e += blockDim.x)
     sf[e] = lr_padded(a.F + ((size_t)h * a.Lq + r0) * a.r, a.r, e);
   lr_stage(sg, a.G + ((size_t)h * a.Lk + k0) * a.r, a.r, k1 - k0);
-  lr_emit_body(a, c, bh, (int)threadIdx.x, sf, sg);
+  lr_emit_norm(a, c, bh, sf, sg, srd, sseg);
+  lr_emit_body(a, c, bh, (int)threadIdx.x, sf, sg, srd);
 }
 #endif
 

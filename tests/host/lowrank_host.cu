@@ -79,7 +79,9 @@ int main(int argc, char** argv) {
       da::lr_emit_range(a, c, r0, r1, k0, k1);
       pad(pf, F.data() + ((size_t)(bh % H) * Lq + r0) * r, r1 - r0);
       pad(pg, G.data() + ((size_t)(bh % H) * Lk + k0) * r, k1 - k0);
-      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, pf.data(), pg.data());
+      float rd[da::LR_C];
+      da::lr_emit_norm_serial(a, c, bh, pf.data(), pg.data(), rd);
+      for (int col = 0; col < da::LR_DV; ++col) da::lr_emit_body(a, c, bh, col, pf.data(), pg.data(), rd);
     }
 
   FILE* g = fopen(argv[2], "wb");
