@@ -384,7 +384,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (nT > 0) {
       // This row of Q (chunk 0's warps) or of dO (chunk 1's) into TMEM: each
       // 64-element box row from its 128-byte-swizzled tile, two bf16 a column.
-      if ((ok = warp_wait(smem_u32(&S.q_full), 0, abort_flag, a.watch))) {
+      if ((ok = warp_wait<true>(smem_u32(&S.q_full), 0, abort_flag, a.watch))) {
         const uint8_t* tile = S.kv[QO] + (ch == 0 ? 0 : 2 * PF_QBOX);
         const int nbox = ch == 0 ? QB : 2;
         const uint32_t tdst = tmem + lane_off + (ch == 0 ? T_Q : T_O);
@@ -405,7 +405,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
     for (int j = 0; ok && j < nT; ++j) {
-      if (!(ok = warp_wait(smem_u32(&S.s_full), j & 1, abort_flag, a.watch))) break;
+      if (!(ok = warp_wait<true>(smem_u32(&S.s_full), j & 1, abort_flag, a.watch))) break;
       tc_fence_after();
       // both halves into registers at once, then the buffer is released:
       // tile j + 1's products overlap all of this tile's arithmetic
@@ -429,7 +429,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         else
           bw_q_elementwise<true>(sv[hh], pv[hh], ds, (int)max(-1LL, min(lim, 31LL)), sl2, nl2, nd2, c2);
         // the dS buffer is free once dQ of tile j - 1 has completed
-        if (hh == 0 && j >= 1 && !(ok = warp_wait(smem_u32(&S.ds_free), (j - 1) & 1, abort_flag, a.watch))) break;
+        if (hh == 0 && j >= 1 && !(ok = warp_wait<true>(smem_u32(&S.ds_free), (j - 1) & 1, abort_flag, a.watch))) break;
         // row r of box hh, keys 32 ch + 8 q .. + 7 of the box: logical chunk 4 ch + q
         const uint32_t row_at = ds_base + (uint32_t)hh * PF_QBOX + (uint32_t)r * 128, sw = (uint32_t)(r & 7);
 #pragma unroll
@@ -445,7 +445,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // ---- epilogue: dQ rows ----
     bool have = nT == 0;
     float y[64];
-    if (nT > 0 && ok) have = warp_wait(smem_u32(&S.fin), 0, abort_flag, a.watch);
+    if (nT > 0 && ok) have = warp_wait<true>(smem_u32(&S.fin), 0, abort_flag, a.watch);
     if (have && ch < QB) {   // chunk ch writes dQ columns [64 ch, 64 ch + 64) of its rows
       if (nT > 0) tc_fence_after();
       __nv_bfloat16* base = V1 ? (m ? a.dq2 : a.dq) + ((size_t)b * Hp + h) * a.Lq * 64

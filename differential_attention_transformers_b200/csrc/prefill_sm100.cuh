@@ -120,8 +120,16 @@ struct PfSmem {
   int abort_flag;
 };
 
+// Bounded wait of a whole warp: lane 0 waits, then broadcasts the outcome.
+// With VOTE, every lane first tests the phase and the warp votes, so a phase
+// that is already complete costs one test and one vote, with no divergence.
+// Measured per kernel: the vote helps the prefill's softmax warps (V1 +3 %)
+// and is neutral in the query-stationary backward kernel; the key-stationary
+// one runs 8 % slower with it and keeps the plain form.
+template <bool VOTE = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           const Watch& w) {
+  if (VOTE && __all_sync(0xffffffffu, mbar_test(bar, parity))) return true;
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, w);
   return __shfl_sync(0xffffffffu, ok, 0);
@@ -430,7 +438,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
     for (int j = 0; j < nT; ++j) {
       const int bb = j & 1;
       const uint32_t tS = tmem + lane_off + m * 128 + bb * 64;
-      if (!(ok = warp_wait(smem_u32(&S.s_full[m][bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
+      if (!(ok = warp_wait<true>(smem_u32(&S.s_full[m][bb]), (j >> 1) & 1, abort_flag, a.watch))) break;
       tc_fence_after();
       float s[PF_BN];
       {
@@ -480,7 +488,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       // S_m(j) was issued only after s_free showed it, so the parity is
       // unambiguous).
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!(ok = warp_wait(smem_u32(&S.o_done[m]), (j - 1) & 1, abort_flag, a.watch))) break;
+        if (!(ok = warp_wait<true>(smem_u32(&S.o_done[m]), (j - 1) & 1, abort_flag, a.watch))) break;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < PF_DV / 32; ++c) {
@@ -510,8 +518,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
       __threadfence_block();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.xl));
-      ok = warp_wait(smem_u32(&S.xl), 0, abort_flag, a.watch) &&
-           warp_wait(smem_u32(&S.o_final), 0, abort_flag, a.watch);
+      ok = warp_wait<true>(smem_u32(&S.xl), 0, abort_flag, a.watch) &&
+           warp_wait<true>(smem_u32(&S.o_final), 0, abort_flag, a.watch);
       if (ok && SINGLE) {
         tc_fence_after();
         have = true;
@@ -544,7 +552,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__
           __threadfence_block();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&S.xs));
-          ok = warp_wait(smem_u32(&S.xs), 0, abort_flag, a.watch);
+          ok = warp_wait<true>(smem_u32(&S.xs), 0, abort_flag, a.watch);
           have = ok;
           if (ok) {
             const float xx = S.ss[0][r] + S.ss[1][r];
