@@ -155,8 +155,8 @@ class ClockSampler:
 # launch is scaled by B / captured B.  None where no capture of the current
 # kernel exists.
 MEASURED_TRAFFIC = {
-    "v2_prefill": (168.4e6 + 44.7e6, 1),       # prefill_kernel<128, PF_INFER>, B1
-    "v1_prefill": (151.4e6 + 16.3e6, 2),       # prefill_kernel<64, PF_INFER>, B2, 4-row-block groups
+    "v2_prefill": (168.1e6 + 45.3e6, 1),       # prefill_kernel<128, PF_INFER>, B1
+    "v1_prefill": (144.5e6 + 16.6e6, 2),       # prefill_kernel<64, PF_INFER>, B2, 4-row-block groups
     "v2_decode": (537.0e6 + 3.3e6, 2),         # decode_split_kernel<2, false>, B2
     "v2_decode_paged": (537.1e6 + 5.9e6, 2),   # decode_split_kernel<2, true>, B2, 16-token pages
 }
