@@ -298,54 +298,78 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
   // V1 single-map passes load only one K half: skip the other half's k-steps.
   const int kk_lo = (a.v1 && !load_k1) ? 4 : 0;
   const int kk_hi = (a.v1 && !load_k2) ? 4 : 8;
-  bool aborted = false;
-  long long x = lo;
-  while (x < hi) {
-    long long bg, seg_end, seg_x0;   // segment (b, g), its end in this range, its first block
+  // The segment (b, g) holding block xx, its first block and its end within
+  // this CTA's range.
+  struct Seg {
+    long long bg, x0, end;
     int b, g, len;
+  };
+  auto seg_at = [&](long long xx) {
+    Seg sg;
     if constexpr (PAGED) {
-      b = dec_find_seq(S.cu, a.B, x);
-      const int nb = (S.cu[b + 1] - S.cu[b]) / a.Hkv;
-      g = (int)(x - S.cu[b]) / nb;
-      bg = (long long)b * a.Hkv + g;
-      seg_x0 = S.cu[b] + (long long)g * nb;
-      seg_end = min(hi, seg_x0 + nb);
-      len = S.len[b];
+      sg.b = dec_find_seq(S.cu, a.B, xx);
+      const int nb = (S.cu[sg.b + 1] - S.cu[sg.b]) / a.Hkv;
+      sg.g = (int)(xx - S.cu[sg.b]) / nb;
+      sg.bg = (long long)sg.b * a.Hkv + sg.g;
+      sg.x0 = S.cu[sg.b] + (long long)sg.g * nb;
+      sg.end = min(hi, sg.x0 + nb);
+      sg.len = S.len[sg.b];
     } else {
-      bg = x / a.nblk;
-      seg_x0 = bg * a.nblk;
-      seg_end = min(hi, (bg + 1) * a.nblk);
-      b = (int)(bg / a.Hkv);
-      g = (int)(bg % a.Hkv);
-      len = a.T;
+      sg.bg = xx / a.nblk;
+      sg.x0 = sg.bg * a.nblk;
+      sg.end = min(hi, (sg.bg + 1) * a.nblk);
+      sg.b = (int)(sg.bg / a.Hkv);
+      sg.g = (int)(sg.bg % a.Hkv);
+      sg.len = a.T;
     }
-
-    // query operand (B fragments) for the 8 columns: n = lane / 4
-    uint32_t qb[8][2];
-    {
-      const int n = lane >> 2;
+    return sg;
+  };
+  // query operand (B fragments) of segment (b, g) for the 8 columns: n = lane / 4
+  auto load_q = [&](int b, int g, uint32_t (&q)[8][2]) {
+    const int n = lane >> 2;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        uint32_t v0 = 0u, v1r = 0u;
-        const int dim = 16 * (kk & 3) + 2 * (lane & 3);
-        if (a.v1) {
-          // columns 0..3: map 1 (dims of K1 = k-steps 0..3); 4..7: map 2 (k-steps 4..7)
-          const bool m2 = n >= 4;
-          const int hl = n & 3;
-          const bool active = (kk >= 4) == m2 && hl < grp && (m2 ? (a.maps & 2) : (a.maps & 1));
-          if (active) {
-            const __nv_bfloat16* qp = (m2 ? a.q2 : a.q1) + ((size_t)b * a.Hq + g * grp + hl) * 64;
-            v0 = *reinterpret_cast<const uint32_t*>(qp + dim);
-            v1r = *reinterpret_cast<const uint32_t*>(qp + dim + 8);
-          }
-        } else if (n < grp) {
-          const __nv_bfloat16* qp = a.q1 + ((size_t)b * a.Hq + g * grp + n) * 128 + 64 * (kk >> 2);
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t v0 = 0u, v1r = 0u;
+      const int dim = 16 * (kk & 3) + 2 * (lane & 3);
+      if (a.v1) {
+        // columns 0..3: map 1 (dims of K1 = k-steps 0..3); 4..7: map 2 (k-steps 4..7)
+        const bool m2 = n >= 4;
+        const int hl = n & 3;
+        const bool active = (kk >= 4) == m2 && hl < grp && (m2 ? (a.maps & 2) : (a.maps & 1));
+        if (active) {
+          const __nv_bfloat16* qp = (m2 ? a.q2 : a.q1) + ((size_t)b * a.Hq + g * grp + hl) * 64;
           v0 = *reinterpret_cast<const uint32_t*>(qp + dim);
           v1r = *reinterpret_cast<const uint32_t*>(qp + dim + 8);
         }
-        qb[kk][0] = v0;
-        qb[kk][1] = v1r;
+      } else if (n < grp) {
+        const __nv_bfloat16* qp = a.q1 + ((size_t)b * a.Hq + g * grp + n) * 128 + 64 * (kk >> 2);
+        v0 = *reinterpret_cast<const uint32_t*>(qp + dim);
+        v1r = *reinterpret_cast<const uint32_t*>(qp + dim + 8);
       }
+      q[kk][0] = v0;
+      q[kk][1] = v1r;
+    }
+  };
+
+  bool aborted = false;
+  long long x = lo;
+  Seg cur{};
+  uint32_t qb[8][2];
+  if (x < hi) {
+    cur = seg_at(x);
+    load_q(cur.b, cur.g, qb);
+  }
+  while (x < hi) {
+    const long long bg = cur.bg, seg_end = cur.end, seg_x0 = cur.x0;
+    const int len = cur.len;
+    // The next segment's queries are loaded now, while this segment's
+    // blocks stream, so they are in registers when it starts.
+    const bool more = seg_end < hi;
+    Seg nxt = cur;
+    uint32_t qn[8][2];
+    if (more) {
+      nxt = seg_at(seg_end);
+      load_q(nxt.b, nxt.g, qn);
     }
 
     float m_run[2] = {-INFINITY, -INFINITY};
@@ -357,9 +381,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
     for (; x < seg_end; ++x) {
       const long long it = x - lo;
       const int st = (int)(it % NST);
-      bool ok = true;
-      if (lane == 0) ok = wait_bar(smem_u32(&S.full[st]), (uint32_t)((it / NST) & 1), abort_flag, a.watch);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // a stage already full costs one test and one vote; otherwise lane 0 waits
+      const uint32_t fbar = smem_u32(&S.full[st]), fpar = (uint32_t)((it / NST) & 1);
+      bool ok = __all_sync(0xffffffffu, mbar_test(fbar, fpar));
+      if (!ok) {
+        if (lane == 0) ok = wait_bar(fbar, fpar, abort_flag, a.watch);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
       if (!ok) { aborted = true; break; }
 
       const uint32_t kb = smem_u32(S.k[st]), vb = smem_u32(S.v[st]);
@@ -483,6 +511,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK1, const __grid_const
       }
     }
     if (bar_any(false)) break;  // records read from smem before the next segment overwrites it
+    if (more) {
+      cur = nxt;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        qb[kk][0] = qn[kk][0];
+        qb[kk][1] = qn[kk][1];
+      }
+    }
   }
 }
 
