@@ -157,8 +157,8 @@ class ClockSampler:
 MEASURED_TRAFFIC = {
     "v2_prefill": (168.1e6 + 45.3e6, 1),       # prefill_kernel<128, PF_INFER>, B1
     "v1_prefill": (144.5e6 + 16.6e6, 2),       # prefill_kernel<64, PF_INFER>, B2, 4-row-block groups
-    "v2_decode": (537.0e6 + 3.3e6, 2),         # decode_split_kernel<2, false>, B2
-    "v2_decode_paged": (537.1e6 + 5.9e6, 2),   # decode_split_kernel<2, true>, B2, 16-token pages
+    "v2_decode": (537.0e6 + 3.2e6, 2),         # decode_split_kernel<2, false>, B2
+    "v2_decode_paged": (537.0e6 + 3.2e6, 2),   # decode_split_kernel<2, true>, B2, 16-token pages
 }
 
 
