@@ -118,6 +118,9 @@ def test_argument_errors_before_any_device_call(L):
     # (q, k, v, lambda, dout, lse, o_maps, dq, dk, dv, dlambda, dtype, B, Hq, Hkv, Lq, Lk, D, causal, ws, bytes, s)
     assert bw(P, P, P, P, P, P, P, P, P, P, P, da.F32, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_UNSUPPORTED
     assert bw(P, P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 4, 3, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
+    # Hq/Hkv odd: a diff pair's two maps must share a KV head (the key-stationary kernel takes them in
+    # consecutive steps and shares dP between them)
+    assert bw(P, P, P, P, P, P, P, P, P, P, P, da.BF16, 1, 6, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
     assert bw(P, P, P, P, P, None, P, P, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_INVALID_ARG
     assert bw(P, P, P, P, P, P, P, Pm, P, P, P, da.BF16, 1, 4, 2, 8, 8, 128, 1, P, 1 << 20, s) == da.ERR_MISALIGNED
     assert L.diffattn_bwd_v2_workspace_size(2, 64, 8192) > 0
